@@ -312,6 +312,16 @@ def test_norm_layer_special_cases():
     plain = oracle.Model(synthetic.Shape(1, 256, 16, 4, 64, 64, zipf_s=1.0), layers).layer(0, h)
     assert np.array_equal(out["sel"], plain["sel"])
     assert np.allclose(out["h_out"] - h, plain["y"], rtol=1e-12, atol=1e-12)
+    # with a non-uniform power-of-two gain g on the same unit-RMS h, the norm reduces to
+    # x = g * h exactly, so the update equals the plain layer on g * h
+    g = np.where(np.arange(s.hidden) % 3 == 0, 2.0, 0.5).astype(np.float32)
+    lw_g = [synthetic.LayerWeights(layers[0].experts, layers[0].shared, layers[0].router,
+                                   layers[0].bias, g)]
+    out_g = oracle.Model(s, lw_g).layer(0, h)
+    plain_g = oracle.Model(synthetic.Shape(1, 256, 16, 4, 64, 64, zipf_s=1.0), lw_g).layer(0, g * h)
+    assert np.array_equal(out_g["z"], plain_g["z"])
+    assert np.array_equal(out_g["sel"], plain_g["sel"])
+    assert np.allclose(out_g["h_out"] - h, plain_g["y"], rtol=1e-12, atol=1e-12)
     # scale invariance of RMSNorm (eps = 0): y(4h) == y(h) and routing is unchanged
     h = rng.standard_normal(s.hidden).astype(np.float32)
     a, b = m.layer(0, h), m.layer(0, 4 * h)
