@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Decode throughput of the expert-cache MoE path on B200.
+
+Workload (one "step" = one batch-1 decode token through the whole hot path): a 40-layer
+pre-norm MoE stack, hidden 2048, 256 experts, top-8, SwiGLU 512 plus a 512-wide shared
+expert, GGUF Q4_0 expert weights, Zipf(1.0)-biased router over seeded per-layer
+permutations, tokens x ~ N(0, 1).  Timed at 100% expert residency (the value) and at
+60% residency with the hot set pinned from a 128-token calibration histogram plus an
+8-slot LRU ring per layer, cold experts in pinned host memory (Luce Spark write-up,
+theneuralfeed.com, key components), and with a uniform 60% placement for contrast.
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "MoE decode tok/s at 100%/60% expert residency; fraction of HBM/PCIe roofline"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
+            "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
+            "residency + 8-slot LRU ring (residency_60)")
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def active_bytes_per_token(s) -> int:
+    """Algorithmic expert bytes of one token: L * (k + shared) experts' Q4_0 weights."""
+    per = 3 * s.hidden * s.inter * 18 // 32
+    sh = 3 * s.hidden * s.shared_inter * 18 // 32
+    return s.n_layers * (s.top_k * per + sh)
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the GPU is busy."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def reduce_over_ranks(value_ms: float, units: float, world: int):
+    """Max of the per-rank times and sum of the per-rank units (replicas)."""
+    if world == 1:
+        return value_ms, units
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+
+def oracle_tokens_per_s(shape, n_layers: int, n_tokens: int, warmup: int = 0):
+    """The oracle, as it stands, on n_tokens tokens through the first n_layers layers;
+    returns (tok/s scaled to the full stack, seconds, threads)."""
+    import oracle
+    sub = synthetic.Shape(n_layers, shape.hidden, shape.n_experts, shape.top_k, shape.inter,
+                          shape.shared_inter, shape.ring_slots, shape.use_rmsnorm, shape.zipf_s)
+    layers = [synthetic.layer_weights(l, shape) for l in range(n_layers)]
+    m = oracle.Model(sub, layers)
+    for i in range(warmup):
+        m.decode(synthetic.token(i, shape.hidden))
+    t0 = time.perf_counter()
+    for i in range(n_tokens):
+        m.decode(synthetic.token(warmup + i, shape.hidden))
+    dt = time.perf_counter() - t0
+    return n_tokens * n_layers / shape.n_layers / dt, dt, 1
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    shape = synthetic.FULL_STACK
+    sample_layers = 4
+    tps, dt, cores = oracle_tokens_per_s(shape, sample_layers, args.steps, args.warmup)
+    sample = (f"{args.steps} timed steps (after {args.warmup} warm-up), each one token through "
+              f"{sample_layers} of the 40 layers, scaled to full tokens")
+    line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "layers": 40},
+            "cpu_baseline": {"value": tps, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tps, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args):
+    import torch
+
+    import expert_cache_host_router_b200 as moe
+    from expert_cache_host_router_b200 import build as libbuild
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if rank == 0:
+        libbuild.build()
+    if world > 1:
+        dist.barrier()
+    shape = synthetic.FULL_STACK
+    dev = torch.device("cuda", local)
+    keep_layers = rank == 0 and world == 1 and not args.no_cpu_baseline
+    m = moe.ExpertCacheMoE(shape, device=local, log_steps=max(4096, args.steps + args.warmup + 16))
+    t0 = time.time()
+    for l in range(shape.n_layers):
+        m.load_layer(l, synthetic.layer_weights(l, shape))
+    load_s = time.time() - t0
+
+    stream = torch.cuda.current_stream(dev)
+    n_tok = args.warmup + args.steps
+    xs = torch.from_numpy(synthetic.tokens(0, n_tok, shape.hidden)).to(dev)
+    y = torch.empty(shape.hidden, dtype=torch.float32, device=dev)
+
+    # calibration histogram: 128 tokens of a separate stream at full residency
+    m.set_residency(1.0)
+    calib = torch.from_numpy(synthetic.tokens(0, args.calib_steps, shape.hidden, synthetic.SEED_CALIB)).to(dev)
+    for i in range(args.calib_steps):
+        m.decode(calib[i], y)
+    m.sync()
+    _, hist, _ = m.stats(reset=True)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+            torch.cuda.synchronize()
+
+    def timed():
+        for i in range(args.warmup):
+            m.decode(xs[i], y)
+        m.sync()
+        m.stats(reset=True)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            m.decode(xs[args.warmup + i], y)
+            ends[i].record(stream)
+        e1.record(stream)
+        barrier()
+        total = e0.elapsed_time(e1)
+        per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        m.sync()
+        st, _, _ = m.stats(reset=True)
+        return total, per, st
+
+    peak, peak_kind = measured_peaks()
+    bytes_tok = active_bytes_per_token(shape)
+    slot_bytes = 3 * shape.hidden * shape.inter * 18 // 32
+
+    with ClockSampler(local) as clk:
+        m.set_residency(1.0)
+        t100, per100, st100 = timed()
+        m.set_residency(0.6, hist, moe.MOE_PLACE_CALIBRATED)
+        t60, per60, st60 = timed()
+        m.set_residency(0.6, hist, moe.MOE_PLACE_UNIFORM)
+        t60u, per60u, st60u = timed()
+
+    # host-to-device bandwidth for one expert slot from pinned memory (the miss copy)
+    src = torch.empty(slot_bytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(slot_bytes, dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.stream(side):
+        for _ in range(5):
+            dst.copy_(src, non_blocking=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(side)
+        for _ in range(100):
+            dst.copy_(src, non_blocking=True)
+        b.record(side)
+    side.synchronize()
+    h2d_gbs = 100 * slot_bytes / (a.elapsed_time(b) * 1e-3) / 1e9
+
+    # end to end through the host-buffer entry point at full residency
+    m.set_residency(1.0)
+    xh = synthetic.tokens(0, n_tok, shape.hidden)
+    for i in range(args.warmup):
+        m.decode_host(xh[i])
+    barrier()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        m.decode_host(xh[args.warmup + i])
+    e2e_s = time.perf_counter() - t0
+    e2e_ms, e2e_units = reduce_over_ranks(1e3 * e2e_s, args.steps, world)
+
+    t100_max, units100 = reduce_over_ranks(t100, args.steps, world)
+    t60_max, units60 = reduce_over_ranks(t60, args.steps, world)
+    value100 = units100 / (t100_max * 1e-3)
+    value60 = units60 / (t60_max * 1e-3)
+    value60u = args.steps * world / (max(t60u, 1e-9) * 1e-3)
+    kern_ms = statistics.mean(per100)
+    achieved = bytes_tok / (kern_ms * 1e-3) / 1e9
+
+    def cache_summary(st):
+        acc = max(st["accesses"], 1)
+        return {"cold_hit_rate": (st["ring_hits"] + st["misses"]) / acc, "miss_rate": st["misses"] / acc,
+                "misses_per_token": st["misses"] / args.steps,
+                "staged_misses": st["staged_misses"]}
+
+    c60 = cache_summary(st60)
+    miss_bytes = c60["misses_per_token"] * slot_bytes
+    roof60_s = max(bytes_tok / (peak * 1e9), miss_bytes / (h2d_gbs * 1e9))
+    line = {
+        "metric": METRIC, "value": value100, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t100_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "q4_0 x int16 codes, int32 dot, fp32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": shape.n_layers, "hidden": shape.hidden,
+                   "experts": shape.n_experts, "top_k": shape.top_k, "inter": shape.inter,
+                   "shared_inter": shape.shared_inter, "ring_slots": shape.ring_slots,
+                   "calibration_tokens": args.calib_steps, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 637 MB of expert weights streamed per token"},
+        "residency_60": {"value": value60, "unit": "tok/s", "ratio_to_100": value60 / value100,
+                         "roofline_frac": roof60_s / (t60_max * 1e-3 / args.steps),
+                         "roofline_us_per_token": roof60_s * 1e6, "h2d_gbs": h2d_gbs,
+                         **c60,
+                         "uniform_placement": {"value": value60u, **cache_summary(st60u)}},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "moe_decode_kernel", "bytes_per_launch": bytes_tok,
+                     "mean_launch_ms": kern_ms},
+        "e2e": {"value": e2e_units / (e2e_ms * 1e-3), "unit": "tok/s",
+                "h2d_bytes_per_step": 4 * shape.hidden, "d2h_bytes_per_step": 4 * shape.hidden + 4},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "setup": {"load_s": load_s},
+    }
+    m.close()
+    del m
+    if keep_layers:
+        tps, dt, cores = oracle_tokens_per_s(shape, shape.n_layers, args.cpu_tokens)
+        line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{args.cpu_tokens} tokens through all 40 layers ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--calib-steps", type=int, default=128)
+    ap.add_argument("--cpu-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

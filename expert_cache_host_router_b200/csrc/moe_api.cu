@@ -1,0 +1,668 @@
+// moe_api.cu -- host runtime and C ABI of libmoe (see include/moe_cache.h).
+//
+// Owns: the pinned host tier holding every routed expert in the slot layout (the
+// write-up's "long tail lives in system RAM", baguaai.com event core; "copied
+// asynchronously from pinned host memory", theneuralfeed.com key components item 2),
+// the device slot pool (pinned experts, ring slots, staging slots), the cache tables,
+// the exchange scratch of the decode kernel, the event log and histogram, the
+// per-token CUDA graphs (key components item 3), and the miss proxy: a host thread
+// that watches the host-mapped mailbox the kernel writes on a miss, issues the
+// copy-engine transfer pinned host -> ring slot on a non-blocking side stream, and then
+// signals the kernel with a stream memory write, so the slot is refilled by the copy
+// engine in stream order after its last reader (the kernel issues the request only
+// after the layer's routing, when no reader of the victim slot is left).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <chrono>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <thread>
+#include <vector>
+
+#include "../../include/moe_cache.h"
+#include "moe_internal.h"
+
+namespace moe {
+uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is);
+cudaError_t decode_configure(int H, int E, int K, int I, int Is);
+cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int* out);
+cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream);
+}  // namespace moe
+
+using namespace moe;
+
+typedef CUresult (*PfnWriteValue32)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+
+struct moe_ctx {
+  moe_config cfg{};
+  int L = 0, H = 0, E = 0, K = 0, I = 0, Is = 0, R = 0;
+  int nsm = 0, grid = 0;
+  SlotLayout lay{}, slay{};
+  uint64_t slot_bytes = 0, shared_slot_bytes = 0;
+  // host tier
+  uint8_t* host_tier = nullptr;
+  std::vector<uint8_t> loaded;
+  // device
+  uint8_t* shared_pool = nullptr;
+  std::atomic<uint8_t*> pool{nullptr};
+  int64_t pool_slots = 0;
+  uint16_t* router = nullptr;
+  float* bias = nullptr;
+  float* gain = nullptr;
+  bool has_bias = false, has_gain = false;
+  int32_t *pin_slot = nullptr, *layer_base = nullptr, *n_pinned = nullptr, *ring_owner = nullptr;
+  uint32_t *ring_stamp = nullptr, *ring_clock = nullptr;
+  float *h = nullptr, *part = nullptr, *sq = nullptr, *z = nullptr;
+  uint8_t* acodes = nullptr;
+  uint32_t* hist = nullptr;
+  int32_t* log = nullptr;
+  int log_steps = 0;
+  Ctrl* ctrl = nullptr;
+  uint32_t* done_seq = nullptr;
+  float *x_buf = nullptr, *y_buf = nullptr;
+  float *x_pin = nullptr, *y_pin = nullptr;
+  int32_t* err_pin = nullptr;
+  MissReq *mbox_host = nullptr, *mbox_dev = nullptr;
+  // residency
+  bool resident = false;
+  float residency = 0.0f;
+  int placement = 0, P = 0, staging_base = 0;
+  // streams and graphs
+  cudaStream_t side = nullptr, own = nullptr;
+  cudaGraphExec_t g_dev = nullptr, g_host = nullptr;
+  const float* g_x = nullptr;
+  float* g_y = nullptr;
+  // proxy
+  std::thread proxy;
+  std::atomic<bool> stop{false};
+  std::atomic<uint32_t> proxy_next{1};
+  std::atomic<int> drop{0};
+  std::atomic<int> proxy_err{0};
+  PfnWriteValue32 write_value32 = nullptr;
+  // tracing and log reading
+  float *h_trace = nullptr, *w_trace = nullptr;
+  uint64_t log_read_step = 0, log_dropped = 0;
+};
+
+#define CK(call)                                  \
+  do {                                            \
+    cudaError_t e_ = (call);                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_);  \
+  } while (0)
+
+static int cuda_fail(cudaError_t e) {
+  if (e == cudaErrorMemoryAllocation) return MOE_ERR_NOMEM;
+  return MOE_ERR_CUDA;
+}
+
+static int deverr_status(int32_t e) {
+  if (e == 0) return MOE_OK;
+  if (e == MOE_DEVERR_BARRIER || e == MOE_DEVERR_MISS || e == MOE_DEVERR_TMA) return MOE_ERR_TIMEOUT;
+  return MOE_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------ proxy
+
+static void cpu_relax() {
+#if defined(__x86_64__)
+  __builtin_ia32_pause();
+#endif
+}
+
+static void proxy_main(moe_ctx* c) {
+  cudaSetDevice(c->cfg.device);
+  auto last_work = std::chrono::steady_clock::now();
+  while (!c->stop.load(std::memory_order_relaxed)) {
+    const uint32_t next = c->proxy_next.load(std::memory_order_relaxed);
+    volatile MissReq* q = &c->mbox_host[next % kMboxCap];
+    if (q->seq != next) {
+      cpu_relax();
+      if (std::chrono::steady_clock::now() - last_work > std::chrono::milliseconds(20))
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+      continue;
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    const uint32_t layer = q->layer, expert = q->expert, dst = q->dst_slot;
+    uint8_t* pool = c->pool.load(std::memory_order_acquire);
+    if (layer >= (uint32_t)c->L || expert >= (uint32_t)c->E || (int64_t)dst >= c->pool_slots || !pool) {
+      c->proxy_err.store(1);  // leave it unsignalled: the kernel's bounded wait reports it
+    } else {
+      cudaMemcpyAsync(pool + (size_t)dst * c->slot_bytes,
+                      c->host_tier + ((size_t)layer * c->E + expert) * c->slot_bytes, c->slot_bytes,
+                      cudaMemcpyHostToDevice, c->side);
+      if (c->drop.load() > 0) {
+        c->drop.fetch_sub(1);
+      } else {
+        c->write_value32((CUstream)c->side, (CUdeviceptr)c->done_seq, next, 0);
+      }
+    }
+    c->proxy_next.store(next + 1, std::memory_order_release);
+    last_work = std::chrono::steady_clock::now();
+  }
+}
+
+// ------------------------------------------------------------------ helpers
+
+static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
+  DecodeParams p{};
+  p.L = c->L;
+  p.H = c->H;
+  p.E = c->E;
+  p.K = c->K;
+  p.I = c->I;
+  p.Is = c->Is;
+  p.R = c->R;
+  p.use_norm = c->cfg.use_rmsnorm;
+  p.eps = c->cfg.rms_eps;
+  p.nch = c->H / kChunk;
+  p.n_units = c->K * (c->I / 32) + c->Is / 32;
+  p.n_exp = c->K + (c->Is > 0 ? 1 : 0);
+  p.pool = c->pool.load();
+  p.slot_bytes = c->slot_bytes;
+  p.lay = c->lay;
+  p.shared_pool = c->shared_pool;
+  p.shared_slot_bytes = c->shared_slot_bytes;
+  p.slay = c->slay;
+  p.router = c->router;
+  p.bias = c->has_bias ? c->bias : nullptr;
+  p.gain = c->has_gain ? c->gain : nullptr;
+  p.pin_slot = c->pin_slot;
+  p.layer_base = c->layer_base;
+  p.n_pinned = c->n_pinned;
+  p.ring_owner = c->ring_owner;
+  p.ring_stamp = c->ring_stamp;
+  p.ring_clock = c->ring_clock;
+  p.staging_base = c->staging_base;
+  p.x = x;
+  p.y = y;
+  p.h_trace = c->h_trace;
+  p.w_trace = c->w_trace;
+  p.h = c->h;
+  p.part = c->part;
+  p.sq = c->sq;
+  p.z = c->z;
+  p.acodes = c->acodes;
+  p.hist = c->hist;
+  p.log = c->log;
+  p.log_steps = c->log_steps;
+  p.ctrl = c->ctrl;
+  p.mbox = c->mbox_dev;
+  p.done_seq = c->done_seq;
+  p.timeout_ns = (unsigned long long)c->cfg.wait_timeout_ms * 1000000ull;
+  return p;
+}
+
+static void drop_graphs(moe_ctx* c) {
+  if (c->g_dev) cudaGraphExecDestroy(c->g_dev);
+  if (c->g_host) cudaGraphExecDestroy(c->g_host);
+  c->g_dev = c->g_host = nullptr;
+  c->g_x = nullptr;
+  c->g_y = nullptr;
+}
+
+// Capture one token: [optional H2D of x] -> decode kernel -> [optional D2H of y, error].
+static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cudaGraphExec_t* out) {
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = cudaSuccess;
+  if (host_io) e = cudaMemcpyAsync(c->x_buf, c->x_pin, sizeof(float) * c->H, cudaMemcpyHostToDevice, c->own);
+  if (e == cudaSuccess) e = decode_launch(make_params(c, x, y), c->grid, c->own);
+  if (e == cudaSuccess && host_io)
+    e = cudaMemcpyAsync(c->y_pin, c->y_buf, sizeof(float) * c->H, cudaMemcpyDeviceToHost, c->own);
+  if (e == cudaSuccess && host_io)
+    e = cudaMemcpyAsync(c->err_pin, &c->ctrl->error, sizeof(int32_t), cudaMemcpyDeviceToHost, c->own);
+  cudaError_t e2 = cudaStreamEndCapture(c->own, &graph);
+  if (e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    return cuda_fail(e);
+  }
+  if (e2 != cudaSuccess) return cuda_fail(e2);
+  e = cudaGraphInstantiate(out, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
+}
+
+template <typename T>
+static cudaError_t dalloc(T** p, size_t count) {
+  return cudaMalloc((void**)p, sizeof(T) * (count ? count : 1));
+}
+
+static void repack_matrix(const uint8_t* src, uint8_t* dst, const MatView& mv, int64_t rows, int64_t cols) {
+  const int64_t nb = rows * cols / 32;
+  uint8_t* qs = dst + mv.qs;
+  uint8_t* d = dst + mv.d;
+  for (int64_t b = 0; b < nb; ++b) {
+    memcpy(d + 2 * b, src + 18 * b, 2);
+    memcpy(qs + 16 * b, src + 18 * b + 2, 16);
+  }
+}
+
+static void repack_expert(const uint8_t* src, uint8_t* dst, const SlotLayout& s, int H, int I) {
+  const uint64_t gu = q4_bytes(I, H);
+  repack_matrix(src, dst, s.gate, I, H);
+  repack_matrix(src + gu, dst, s.up, I, H);
+  repack_matrix(src + 2 * gu, dst, s.down, H, I);
+}
+
+// ------------------------------------------------------------------ C ABI
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument or configuration";
+    case MOE_ERR_NOMEM: return "out of memory";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case MOE_ERR_STATE: return "call out of order";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or feature";
+    case MOE_ERR_DEVICE: return "the kernel flagged a bad route or slot";
+    default: return "unknown status";
+  }
+}
+
+void moe_destroy(moe_ctx* c) {
+  if (!c) return;
+  if (c->proxy.joinable()) {
+    c->stop.store(true);
+    c->proxy.join();
+  }
+  cudaSetDevice(c->cfg.device);
+  cudaDeviceSynchronize();
+  drop_graphs(c);
+  if (c->side) cudaStreamDestroy(c->side);
+  if (c->own) cudaStreamDestroy(c->own);
+  void* dev[] = {c->shared_pool, c->pool.load(), c->router, c->bias, c->gain, c->pin_slot,
+                 c->layer_base, c->n_pinned, c->ring_owner, c->ring_stamp, c->ring_clock,
+                 c->h, c->part, c->sq, c->z, c->acodes, c->hist, c->log, c->ctrl, c->done_seq,
+                 c->x_buf, c->y_buf};
+  for (void* p : dev)
+    if (p) cudaFree(p);
+  void* hst[] = {c->host_tier, c->x_pin, c->y_pin, c->err_pin, c->mbox_host};
+  for (void* p : hst)
+    if (p) cudaFreeHost(p);
+  delete c;
+}
+
+int moe_load_layer(moe_ctx* c, int32_t l, const uint8_t* const* experts, const uint8_t* shared,
+                   const uint16_t* router_bf16, const float* bias, const float* gain) {
+  if (!c || l < 0 || l >= c->L || !experts || !router_bf16) return MOE_ERR_INVALID;
+  if (c->Is > 0 && !shared) return MOE_ERR_INVALID;
+  for (int e = 0; e < c->E; ++e)
+    if (!experts[e]) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  // routed experts -> pinned host tier (slot layout), in parallel over experts
+  {
+    const int nthr = std::max(1, std::min(16, (int)std::thread::hardware_concurrency()));
+    std::vector<std::thread> th;
+    for (int t = 0; t < nthr; ++t)
+      th.emplace_back([=]() {
+        for (int e = t; e < c->E; e += nthr)
+          repack_expert(experts[e], c->host_tier + ((size_t)l * c->E + e) * c->slot_bytes, c->lay, c->H, c->I);
+      });
+    for (auto& t : th) t.join();
+  }
+  if (c->Is > 0) {
+    std::vector<uint8_t> tmp(c->shared_slot_bytes, 0);
+    repack_expert(shared, tmp.data(), c->slay, c->H, c->Is);
+    CK(cudaMemcpy(c->shared_pool + (size_t)l * c->shared_slot_bytes, tmp.data(), c->shared_slot_bytes,
+                  cudaMemcpyHostToDevice));
+  }
+  {  // router [E][H] -> [H/16][E][16]
+    const int nch = c->H / kChunk;
+    std::vector<uint16_t> tmp((size_t)c->E * c->H);
+    for (int ch = 0; ch < nch; ++ch)
+      for (int e = 0; e < c->E; ++e)
+        memcpy(&tmp[((size_t)ch * c->E + e) * kChunk], router_bf16 + (size_t)e * c->H + ch * kChunk,
+               kChunk * sizeof(uint16_t));
+    CK(cudaMemcpy(c->router + (size_t)l * c->E * c->H, tmp.data(), tmp.size() * 2, cudaMemcpyHostToDevice));
+  }
+  if (bias) {
+    CK(cudaMemcpy(c->bias + (size_t)l * c->E, bias, sizeof(float) * c->E, cudaMemcpyHostToDevice));
+    c->has_bias = true;
+  } else {
+    CK(cudaMemset(c->bias + (size_t)l * c->E, 0, sizeof(float) * c->E));
+  }
+  if (gain) {
+    CK(cudaMemcpy(c->gain + (size_t)l * c->H, gain, sizeof(float) * c->H, cudaMemcpyHostToDevice));
+    c->has_gain = true;
+  } else {
+    std::vector<float> ones(c->H, 1.0f);
+    CK(cudaMemcpy(c->gain + (size_t)l * c->H, ones.data(), sizeof(float) * c->H, cudaMemcpyHostToDevice));
+  }
+  c->loaded[l] = 1;
+  c->resident = false;
+  drop_graphs(c);
+  return MOE_OK;
+}
+
+int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
+  if (!cfg_in || !out) return MOE_ERR_INVALID;
+  moe_config cfg = *cfg_in;
+  if (cfg.n_layers < 1 || cfg.hidden < 32 || cfg.hidden % 32 || cfg.hidden > kMaxH) return MOE_ERR_INVALID;
+  if (cfg.top_k < 1 || cfg.top_k > kMaxK || cfg.n_experts < cfg.top_k || cfg.n_experts > kMaxE)
+    return MOE_ERR_INVALID;
+  if (cfg.inter < 32 || cfg.inter % 32 || cfg.shared_inter < 0 || cfg.shared_inter % 32) return MOE_ERR_INVALID;
+  if (cfg.ring_slots < 0 || cfg.ring_slots > kMaxR) return MOE_ERR_INVALID;
+  if (cfg.use_rmsnorm != 0 && cfg.use_rmsnorm != 1) return MOE_ERR_INVALID;
+  if (!(cfg.rms_eps >= 0.0f)) return MOE_ERR_INVALID;
+  if (cfg.log_steps < 0) return MOE_ERR_INVALID;
+  if (cfg.log_steps == 0) cfg.log_steps = 4096;
+  if (cfg.wait_timeout_ms == 0) cfg.wait_timeout_ms = 2000;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || cfg.device < 0 || cfg.device >= ndev) return MOE_ERR_INVALID;
+
+  moe_ctx* c = new (std::nothrow) moe_ctx();
+  if (!c) return MOE_ERR_NOMEM;
+  c->cfg = cfg;
+  c->L = cfg.n_layers;
+  c->H = cfg.hidden;
+  c->E = cfg.n_experts;
+  c->K = cfg.top_k;
+  c->I = cfg.inter;
+  c->Is = cfg.shared_inter;
+  c->R = cfg.ring_slots;
+  c->lay = slot_layout(c->H, c->I);
+  c->slay = slot_layout(c->H, c->Is > 0 ? c->Is : 32);
+  c->slot_bytes = c->lay.bytes;
+  c->shared_slot_bytes = c->Is > 0 ? c->slay.bytes : 0;
+  c->log_steps = cfg.log_steps;
+  c->loaded.assign(c->L, 0);
+  int st = MOE_OK;
+  auto fail = [&](int s) {
+    moe_destroy(c);
+    return s;
+  };
+#define CKC(call)                                       \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return fail(cuda_fail(e_));  \
+  } while (0)
+  CKC(cudaSetDevice(cfg.device));
+  CKC(cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, cfg.device));
+  int smem_optin = 0, coop = 0;
+  CKC(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, cfg.device));
+  CKC(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, cfg.device));
+  if (!coop || decode_smem_bytes(c->H, c->E, c->K, c->I, c->Is) > (uint32_t)smem_optin)
+    return fail(MOE_ERR_UNSUPPORTED);
+  CKC(decode_configure(c->H, c->E, c->K, c->I, c->Is));
+  int per_sm = 0;
+  CKC(decode_max_blocks_per_sm(c->H, c->E, c->K, c->I, c->Is, &per_sm));
+  if (per_sm < 1) return fail(MOE_ERR_UNSUPPORTED);
+  c->grid = c->nsm;  // one persistent CTA per SM
+
+  const size_t nch = c->H / kChunk;
+  const int n_exp = c->K + (c->Is > 0);
+  const int imax = std::max(c->I, c->Is);
+  CKC(dalloc(&c->router, (size_t)c->L * c->E * c->H));
+  CKC(dalloc(&c->bias, (size_t)c->L * c->E));
+  CKC(dalloc(&c->gain, (size_t)c->L * c->H));
+  if (c->Is > 0) CKC(dalloc(&c->shared_pool, (size_t)c->L * c->shared_slot_bytes));
+  CKC(dalloc(&c->pin_slot, (size_t)c->L * c->E));
+  CKC(dalloc(&c->layer_base, c->L));
+  CKC(dalloc(&c->n_pinned, c->L));
+  CKC(dalloc(&c->ring_owner, (size_t)2 * c->L * std::max(c->R, 1)));
+  CKC(dalloc(&c->ring_stamp, (size_t)2 * c->L * std::max(c->R, 1)));
+  CKC(dalloc(&c->ring_clock, (size_t)2 * c->L));
+  CKC(dalloc(&c->h, c->H));
+  CKC(dalloc(&c->part, (size_t)c->E * nch));
+  CKC(dalloc(&c->sq, nch));
+  CKC(dalloc(&c->z, c->E));
+  CKC(dalloc(&c->acodes, (size_t)n_exp * (imax / 32) * kACodeBytes));
+  CKC(dalloc(&c->hist, (size_t)c->L * c->E));
+  CKC(dalloc(&c->log, (size_t)c->log_steps * c->L * c->K * 7));
+  CKC(dalloc(&c->ctrl, 1));
+  CKC(dalloc(&c->done_seq, 1));
+  CKC(dalloc(&c->x_buf, c->H));
+  CKC(dalloc(&c->y_buf, c->H));
+  CKC(cudaMemset(c->hist, 0, sizeof(uint32_t) * c->L * c->E));
+  CKC(cudaMemset(c->ctrl, 0, sizeof(Ctrl)));
+  CKC(cudaMemset(c->done_seq, 0, sizeof(uint32_t)));
+  CKC(cudaMemset(c->acodes, 0, (size_t)n_exp * (imax / 32) * kACodeBytes));
+  CKC(cudaHostAlloc((void**)&c->host_tier, (size_t)c->L * c->E * c->slot_bytes, cudaHostAllocPortable));
+  CKC(cudaHostAlloc((void**)&c->x_pin, sizeof(float) * c->H, cudaHostAllocPortable));
+  CKC(cudaHostAlloc((void**)&c->y_pin, sizeof(float) * c->H, cudaHostAllocPortable));
+  CKC(cudaHostAlloc((void**)&c->err_pin, sizeof(int32_t), cudaHostAllocPortable));
+  CKC(cudaHostAlloc((void**)&c->mbox_host, sizeof(MissReq) * kMboxCap, cudaHostAllocMapped | cudaHostAllocPortable));
+  memset(c->mbox_host, 0, sizeof(MissReq) * kMboxCap);
+  CKC(cudaHostGetDevicePointer((void**)&c->mbox_dev, c->mbox_host, 0));
+  CKC(cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking));
+  CKC(cudaStreamCreateWithFlags(&c->own, cudaStreamNonBlocking));
+  {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    CKC(cudaGetDriverEntryPointByVersion("cuStreamWriteValue32", &fn, 12000, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return fail(MOE_ERR_UNSUPPORTED);
+    c->write_value32 = (PfnWriteValue32)fn;
+  }
+  c->proxy = std::thread(proxy_main, c);
+  if (w) {
+    if (!w->expert_q4_0 || !w->router_bf16 || (c->Is > 0 && !w->shared_q4_0)) return fail(MOE_ERR_INVALID);
+    for (int l = 0; l < c->L; ++l) {
+      st = moe_load_layer(c, l, w->expert_q4_0 + (size_t)l * c->E, c->Is > 0 ? w->shared_q4_0[l] : nullptr,
+                          w->router_bf16 + (size_t)l * c->E * c->H,
+                          w->router_bias ? w->router_bias + (size_t)l * c->E : nullptr,
+                          w->rms_gain ? w->rms_gain + (size_t)l * c->H : nullptr);
+      if (st != MOE_OK) return fail(st);
+    }
+  }
+#undef CKC
+  *out = c;
+  return MOE_OK;
+}
+
+int moe_set_residency(moe_ctx* c, float fraction, const uint32_t* hist, int32_t placement) {
+  if (!c || !(fraction >= 0.0f && fraction <= 1.0f)) return MOE_ERR_INVALID;
+  if (placement != MOE_PLACE_CALIBRATED && placement != MOE_PLACE_UNIFORM) return MOE_ERR_INVALID;
+  for (int l = 0; l < c->L; ++l)
+    if (!c->loaded[l]) return MOE_ERR_STATE;
+  const int P = (int)std::lround((double)fraction * c->E);
+  if (P < c->E && c->R == 0) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  std::vector<uint32_t> h((size_t)c->L * c->E, 0);
+  if (hist) {
+    memcpy(h.data(), hist, h.size() * sizeof(uint32_t));
+  } else {
+    CK(cudaMemcpy(h.data(), c->hist, h.size() * sizeof(uint32_t), cudaMemcpyDeviceToHost));
+  }
+  // slot pool: per layer P pinned + R ring slots, then k staging slots
+  const int64_t need = (int64_t)c->L * (P + c->R) + c->K;
+  if (need > c->pool_slots) {
+    drop_graphs(c);
+    uint8_t* old = c->pool.exchange(nullptr);
+    if (old) cudaFree(old);
+    c->pool_slots = 0;
+    uint8_t* np = nullptr;
+    CK(cudaMalloc((void**)&np, (size_t)need * c->slot_bytes));
+    c->pool.store(np);
+    c->pool_slots = need;
+  }
+  uint8_t* pool = c->pool.load();
+  std::vector<int32_t> pin((size_t)c->L * c->E, -1), base(c->L), npin(c->L, P);
+  std::vector<int> order(c->E);
+  for (int l = 0; l < c->L; ++l) {
+    base[l] = l * (P + c->R);
+    std::vector<uint8_t> mask(c->E, 0);
+    if (placement == MOE_PLACE_UNIFORM) {
+      for (int e = 0; e < P; ++e) mask[e] = 1;
+    } else {
+      for (int e = 0; e < c->E; ++e) order[e] = e;
+      const uint32_t* hl = h.data() + (size_t)l * c->E;
+      std::stable_sort(order.begin(), order.end(), [hl](int a, int b) { return hl[a] > hl[b]; });
+      for (int p = 0; p < P; ++p) mask[order[p]] = 1;
+    }
+    int p = 0;
+    for (int e = 0; e < c->E; ++e)
+      if (mask[e]) {
+        pin[(size_t)l * c->E + e] = p;
+        CK(cudaMemcpyAsync(pool + (size_t)(base[l] + p) * c->slot_bytes,
+                           c->host_tier + ((size_t)l * c->E + e) * c->slot_bytes, c->slot_bytes,
+                           cudaMemcpyHostToDevice, c->own));
+        ++p;
+      }
+  }
+  c->staging_base = c->L * (P + c->R);
+  CK(cudaMemcpyAsync(c->pin_slot, pin.data(), pin.size() * 4, cudaMemcpyHostToDevice, c->own));
+  CK(cudaMemcpyAsync(c->layer_base, base.data(), base.size() * 4, cudaMemcpyHostToDevice, c->own));
+  CK(cudaMemcpyAsync(c->n_pinned, npin.data(), npin.size() * 4, cudaMemcpyHostToDevice, c->own));
+  const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);
+  CK(cudaMemsetAsync(c->ring_owner, 0xff, nr * 4, c->own));
+  CK(cudaMemsetAsync(c->ring_stamp, 0, nr * 4, c->own));
+  CK(cudaMemsetAsync(c->ring_clock, 0, (size_t)2 * c->L * 4, c->own));
+  CK(cudaStreamSynchronize(c->own));
+  c->P = P;
+  c->residency = fraction;
+  c->placement = placement;
+  c->resident = true;
+  drop_graphs(c);
+  return MOE_OK;
+}
+
+int moe_decode_step(moe_ctx* c, const float* x_dev, float* y_dev, void* stream) {
+  if (!c || !x_dev || !y_dev) return MOE_ERR_INVALID;
+  if (!c->resident) return MOE_ERR_STATE;
+  if (!c->g_dev || c->g_x != x_dev || c->g_y != y_dev) {
+    if (c->g_dev) cudaGraphExecDestroy(c->g_dev);
+    c->g_dev = nullptr;
+    const int st = capture_token(c, x_dev, y_dev, false, &c->g_dev);
+    if (st != MOE_OK) return st;
+    c->g_x = x_dev;
+    c->g_y = y_dev;
+  }
+  CK(cudaGraphLaunch(c->g_dev, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+int moe_decode_step_host(moe_ctx* c, const float* x_host, float* y_host) {
+  if (!c || !x_host || !y_host) return MOE_ERR_INVALID;
+  if (!c->resident) return MOE_ERR_STATE;
+  if (!c->g_host) {
+    const int st = capture_token(c, c->x_buf, c->y_buf, true, &c->g_host);
+    if (st != MOE_OK) return st;
+  }
+  memcpy(c->x_pin, x_host, sizeof(float) * c->H);
+  CK(cudaGraphLaunch(c->g_host, c->own));
+  CK(cudaStreamSynchronize(c->own));
+  memcpy(y_host, c->y_pin, sizeof(float) * c->H);
+  return deverr_status(*c->err_pin);
+}
+
+int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, void* stream) {
+  (void)x_dev;
+  (void)n_tokens;
+  (void)y_dev;
+  (void)stream;
+  if (!c) return MOE_ERR_INVALID;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+int moe_sync(moe_ctx* c) {
+  if (!c) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  int32_t err = 0;
+  CK(cudaMemcpy(&err, &c->ctrl->error, sizeof(err), cudaMemcpyDeviceToHost));
+  return deverr_status(err);
+}
+
+int moe_clear_error(moe_ctx* c) {
+  if (!c) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  // let the proxy drain every request the failed launch published
+  for (int spin = 0; spin < 2000; ++spin) {
+    const uint32_t next = c->proxy_next.load();
+    if (c->mbox_host[next % kMboxCap].seq != next) break;
+    std::this_thread::sleep_for(std::chrono::microseconds(500));
+  }
+  CK(cudaStreamSynchronize(c->side));
+  Ctrl ctl;
+  CK(cudaMemcpy(&ctl, c->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  const uint32_t last = c->proxy_next.load() - 1;
+  ctl.req_seq = last;
+  ctl.error = 0;
+  ctl.bar_count = 0;
+  CK(cudaMemcpy(c->ctrl, &ctl, sizeof(Ctrl), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(c->done_seq, &last, sizeof(uint32_t), cudaMemcpyHostToDevice));
+  const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);
+  CK(cudaMemset(c->ring_owner, 0xff, nr * 4));
+  CK(cudaMemset(c->ring_stamp, 0, nr * 4));
+  CK(cudaMemset(c->ring_clock, 0, (size_t)2 * c->L * 4));
+  c->proxy_err.store(0);
+  return MOE_OK;
+}
+
+int moe_stats(moe_ctx* c, moe_stats_t* out, uint32_t* hist_out, moe_event* log_out, size_t log_cap,
+              size_t* log_n, int32_t reset) {
+  if (!c) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  Ctrl ctl;
+  CK(cudaMemcpy(&ctl, c->ctrl, sizeof(Ctrl), cudaMemcpyDeviceToHost));
+  if (out) {
+    memset(out, 0, sizeof(*out));
+    out->steps = ctl.step;
+    out->pin_hits = ctl.pin_hits;
+    out->ring_hits = ctl.ring_hits;
+    out->misses = ctl.misses;
+    out->evictions = ctl.evictions;
+    out->accesses = ctl.pin_hits + ctl.ring_hits + ctl.misses;
+    out->bytes_copied = ctl.misses * c->slot_bytes;
+    out->staged_misses = ctl.staged;
+    out->device_error = ctl.error;
+    out->n_pinned = c->P;
+    out->residency = c->residency;
+    out->placement = c->placement;
+  }
+  if (hist_out)
+    CK(cudaMemcpy(hist_out, c->hist, sizeof(uint32_t) * c->L * c->E, cudaMemcpyDeviceToHost));
+  const uint64_t step = ctl.step;
+  if (step > c->log_read_step + (uint64_t)c->log_steps) {
+    c->log_dropped += (step - c->log_read_step - c->log_steps) * (uint64_t)c->L * c->K;
+    c->log_read_step = step - c->log_steps;
+  }
+  size_t n = 0;
+  if (log_out) {
+    const size_t per_step = (size_t)c->L * c->K;
+    while (c->log_read_step < step && n + per_step <= log_cap) {
+      const size_t slot = (size_t)(c->log_read_step % (uint64_t)c->log_steps);
+      CK(cudaMemcpy(log_out + n, c->log + slot * per_step * 7, per_step * sizeof(moe_event),
+                    cudaMemcpyDeviceToHost));
+      n += per_step;
+      ++c->log_read_step;
+    }
+  }
+  if (log_n) *log_n = n;
+  if (out) out->log_dropped = c->log_dropped;
+  if (reset) {
+    ctl.pin_hits = ctl.ring_hits = ctl.misses = ctl.evictions = ctl.staged = 0;
+    CK(cudaMemcpy(&c->ctrl->pin_hits, &ctl.pin_hits, 5 * sizeof(unsigned long long), cudaMemcpyHostToDevice));
+    CK(cudaMemset(c->hist, 0, sizeof(uint32_t) * c->L * c->E));
+  }
+  return MOE_OK;
+}
+
+int moe_set_trace(moe_ctx* c, float* h_trace_dev, float* w_trace_dev) {
+  if (!c) return MOE_ERR_INVALID;
+  c->h_trace = h_trace_dev;
+  c->w_trace = w_trace_dev;
+  drop_graphs(c);
+  return MOE_OK;
+}
+
+int moe_debug_drop_signals(moe_ctx* c, int32_t n) {
+  if (!c || n < 0) return MOE_ERR_INVALID;
+  c->drop.store(n);
+  return MOE_OK;
+}
+
+}  // extern "C"

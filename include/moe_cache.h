@@ -1,0 +1,191 @@
+/*
+ * moe_cache.h -- C ABI of libmoe: the sparse Mixture-of-Experts FFN step of batch-1
+ * decode with a bounded GPU expert cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method is Luce Spark as described on theneuralfeed.com ("Luce Spark runs 35B MoE
+ * models on 16GB GPU without speed loss", key-components paragraph): an A3B MoE routes
+ * each token to about 8 of 256 experts; (1) calibrated placement accumulates per-expert
+ * routing frequencies and pins the most-used set on the GPU; (2) a bounded asynchronous
+ * cache with a fixed ring of spare GPU slots copies a cold expert from pinned host
+ * memory into a spare slot while evicting the least recently used entry; (3) the whole
+ * token runs as one graph instead of one per layer; at full residency the output is
+ * bit-identical to all-GPU.  The baguaai.com summary ("Luce Spark: Shattering the VRAM
+ * Ceiling ...", event core) adds that the long tail lives in system RAM and is swapped
+ * in on demand.
+ *
+ * The MoE layer these calls compute (the pages do not spell it out; the library takes
+ * the plainest reading): router z = W_r x + b (W_r bf16, fp32 accumulation), softmax,
+ * top-k, renormalise; expert i: a = silu(G_i x) * (U_i x), o_i = D_i a with Q4_0 weights
+ * (GGUF block: fp16 scale d, 16 bytes of nibbles, weight = (q - 8) d); y = sum_i w_i o_i
+ * + o_shared; stacks are pre-norm residual: h <- h + MoE(RMSNorm(h)).  Routing
+ * decisions, routing histograms and the cache event log are exact; outputs are fp32.
+ *
+ * Conventions for every call:
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  No exception and no
+ *     abort crosses the ABI.  Calls on a NULL context return MOE_ERR_INVALID.
+ *   - Host pointers are read during the call only; the library copies what it keeps.
+ *   - Device pointers (suffix _dev) are CUDA device addresses on cfg.device, owned by
+ *     the caller, stream-ordered on the stream passed (a cudaStream_t, NULL = legacy).
+ *   - One context is not thread-safe: serialise calls on it.  Distinct contexts are
+ *     independent.
+ */
+#ifndef MOE_CACHE_H
+#define MOE_CACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID (-1)     /* bad argument or configuration */
+#define MOE_ERR_NOMEM (-2)       /* device or pinned-host allocation failed */
+#define MOE_ERR_CUDA (-3)        /* a CUDA runtime/driver call failed */
+#define MOE_ERR_TIMEOUT (-4)     /* a bounded device-side wait ran out (see moe_sync) */
+#define MOE_ERR_STATE (-5)       /* call out of order (e.g. decode before residency) */
+#define MOE_ERR_UNSUPPORTED (-6) /* shape or feature outside this build's limits */
+#define MOE_ERR_DEVICE (-7)      /* the kernel flagged a bad route or slot (see moe_sync) */
+
+/* Cache event kinds (key-components item 2 of the Luce Spark write-up). */
+#define MOE_PIN_HIT 0  /* expert is in the calibrated pinned set */
+#define MOE_RING_HIT 1 /* expert is resident in the layer's ring; recency refreshed */
+#define MOE_MISS 2     /* expert copied from pinned host memory into a ring slot */
+
+/* Placement policies for moe_set_residency. */
+#define MOE_PLACE_CALIBRATED 0 /* top-P experts by routing count, ties -> lower index */
+#define MOE_PLACE_UNIFORM 1    /* experts 0..P-1 (the write-up's naive offload) */
+
+typedef struct moe_ctx moe_ctx; /* opaque; owned by the library */
+
+typedef struct {
+  int32_t n_layers;       /* L >= 1 */
+  int32_t hidden;         /* H, multiple of 32, <= 4096 */
+  int32_t n_experts;      /* E, top_k <= E <= 1024 */
+  int32_t top_k;          /* k, 1..32 */
+  int32_t inter;          /* expert SwiGLU width I, multiple of 32 */
+  int32_t shared_inter;   /* shared expert width, multiple of 32; 0 = no shared expert */
+  int32_t ring_slots;     /* R spare slots per layer, 0..32 (0 only with full residency) */
+  int32_t use_rmsnorm;    /* 1: pre-norm residual stack h += MoE(RMSNorm(h)); 0: h = MoE(h) */
+  float rms_eps;          /* RMSNorm epsilon (1e-6 for the pages' A3B shape) */
+  int32_t device;         /* CUDA device ordinal */
+  int32_t log_steps;      /* event-log capacity in decode steps; 0 -> 4096 */
+  uint32_t wait_timeout_ms; /* bound on every device-side wait; 0 -> 2000 */
+} moe_config;
+
+/* Weights, canonical layouts (caller-owned, read during the call):
+ *   expert_q4_0[l*E + e]: gate [I x H] | up [I x H] | down [H x I], each row-major with
+ *     K = the column count contiguous, as GGUF Q4_0 blocks (18 bytes per 32 weights);
+ *   shared_q4_0[l]: the same for the shared expert with width shared_inter (NULL if 0);
+ *   router_bf16: [L][E][H] bf16 bit patterns; router_bias: [L][E] fp32 or NULL (zero);
+ *   rms_gain: [L][H] fp32 or NULL (ones). */
+typedef struct {
+  const uint8_t *const *expert_q4_0;
+  const uint8_t *const *shared_q4_0;
+  const uint16_t *router_bf16;
+  const float *router_bias;
+  const float *rms_gain;
+} moe_weights;
+
+/* One cache event.  step counts decode steps since moe_create; rank is the position
+ * in the token's top-k (descending logit); slot numbers pinned experts 0..P-1 in
+ * ascending expert order and ring slot r as P + r; evicted is the expert a miss
+ * displaced, or -1. */
+typedef struct {
+  int32_t step, layer, rank, expert, kind, slot, evicted;
+} moe_event;
+
+typedef struct {
+  uint64_t steps;        /* decode steps completed since create */
+  uint64_t accesses;     /* expert selections (steps * L * k) since the last reset */
+  uint64_t pin_hits, ring_hits, misses, evictions;
+  uint64_t bytes_copied; /* host-to-device bytes moved by misses since the last reset */
+  uint64_t staged_misses; /* misses whose ring slot was still read in the same layer */
+  uint64_t log_dropped;  /* events lost because the log wrapped before being read */
+  int32_t device_error;  /* 0, or the kernel's error word (MOE_DEVERR_*) */
+  int32_t n_pinned;      /* P of the current residency */
+  float residency;       /* fraction passed to the last moe_set_residency */
+  int32_t placement;     /* policy of the last moe_set_residency */
+} moe_stats_t;
+
+#define MOE_DEVERR_BARRIER 1 /* grid barrier wait ran out */
+#define MOE_DEVERR_MISS 2    /* wait for a miss copy ran out */
+#define MOE_DEVERR_TMA 3     /* wait for a bulk shared-memory load ran out */
+#define MOE_DEVERR_ROUTE 4   /* a logit was NaN: no valid top-k */
+#define MOE_DEVERR_SLOT 5    /* an expert had no slot (cold with an empty ring) */
+
+/* Create a context on cfg->device: allocates the pinned host tier (all experts), the
+ * device tables and the proxy thread that serves miss copies.  weights may be NULL
+ * (then load layers with moe_load_layer).  *out is set only on MOE_OK. */
+MOE_API int moe_create(const moe_config *cfg, const moe_weights *weights, moe_ctx **out);
+
+/* Load (or replace) one layer's weights.  Experts go to the pinned host tier in the
+ * library's slot layout; the shared expert, router, bias and gain go to the device.
+ * Invalidates the residency: call moe_set_residency before decoding. */
+MOE_API int moe_load_layer(moe_ctx *ctx, int32_t layer, const uint8_t *const *expert_q4_0,
+                   const uint8_t *shared_q4_0, const uint16_t *router_bf16,
+                   const float *router_bias, const float *rms_gain);
+
+/* Choose the resident set (Luce Spark key components (1) and (2)).  fraction in [0, 1]
+ * gives P = round(fraction * E) pinned experts per layer, chosen by placement from
+ * hist ([L][E] counts; NULL = the library's own accumulated histogram); every layer
+ * also gets ring_slots spare slots, emptied here.  Copies the pinned experts to the
+ * device and synchronises the device.  fraction < 1 needs ring_slots >= 1. */
+MOE_API int moe_set_residency(moe_ctx *ctx, float fraction, const uint32_t *hist, int32_t placement);
+
+/* One decode step (one token through all L layers) as one graph launch on stream:
+ * reads x_dev [H] fp32, writes y_dev [H] fp32 (h_L of the stack, or MoE(x) when
+ * use_rmsnorm = 0).  Routing, the histogram, the cache and the event log advance.
+ * Asynchronous: device-side failures surface at moe_sync / moe_stats. */
+MOE_API int moe_decode_step(moe_ctx *ctx, const float *x_dev, float *y_dev, void *stream);
+
+/* The same step on host buffers, synchronously: x_host [H] fp32 is staged to the
+ * device, the step runs, y_host [H] receives the result.  Returns the step's status. */
+MOE_API int moe_decode_step_host(moe_ctx *ctx, const float *x_host, float *y_host);
+
+/* Batched prefill of T tokens (x_dev [T][H] -> y_dev [T][H]).  Not in this build:
+ * returns MOE_ERR_UNSUPPORTED. */
+MOE_API int moe_prefill(moe_ctx *ctx, const float *x_dev, int32_t n_tokens, float *y_dev, void *stream);
+
+/* Wait for all work of the context and report a device-side failure as an error code
+ * (MOE_ERR_TIMEOUT for a wait that ran out, MOE_ERR_DEVICE otherwise). */
+MOE_API int moe_sync(moe_ctx *ctx);
+
+/* Clear a device-side failure so decoding can resume: empties every ring (its state
+ * may be torn), resynchronises the miss queue and the grid barrier. */
+MOE_API int moe_clear_error(moe_ctx *ctx);
+
+/* Counters, histogram and event log.  Synchronises the device.  hist_out: [L][E] or
+ * NULL.  log_out: room for log_cap events or NULL; receives the events of the steps
+ * not yet read, oldest first, and *log_n their count.  reset != 0 zeroes the counters
+ * and the histogram after reading. */
+MOE_API int moe_stats(moe_ctx *ctx, moe_stats_t *out, uint32_t *hist_out, moe_event *log_out,
+              size_t log_cap, size_t *log_n, int32_t reset);
+
+/* Tracing: when h_trace_dev is non-NULL, every decode step writes its input and each
+ * layer's output ([(L+1)][H] fp32) there; w_trace_dev ([L][k] fp32, or NULL) receives
+ * the routing weights.  Pass NULLs to stop.  Device pointers owned by the caller. */
+MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
+
+/* Fault injection for tests: the miss proxy issues the next n copies but never
+ * signals them, so the kernel's bounded wait runs out (no GPU fault involved). */
+MOE_API int moe_debug_drop_signals(moe_ctx *ctx, int32_t n);
+
+/* Free everything.  NULL is a no-op. */
+MOE_API void moe_destroy(moe_ctx *ctx);
+
+/* Static description of a status code. */
+MOE_API const char *moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_CACHE_H */

@@ -158,9 +158,19 @@ class LayerWeights:
 
 
 def layer_weights(layer: int, shape: Shape, gain_kind: str = "ones",
-                  bias_seed: int = SEED_PERM) -> LayerWeights:
+                  bias_seed: int = SEED_PERM, threads: int = 8) -> LayerWeights:
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(e):
+        return expert_q4_0(layer, e, shape.hidden, shape.inter)
+
+    if threads > 1 and shape.n_experts >= 16:
+        with ThreadPoolExecutor(threads) as ex:
+            experts = list(ex.map(one, range(shape.n_experts)))
+    else:
+        experts = [one(e) for e in range(shape.n_experts)]
     return LayerWeights(
-        experts=[expert_q4_0(layer, e, shape.hidden, shape.inter) for e in range(shape.n_experts)],
+        experts=experts,
         shared=shared_q4_0(layer, shape),
         router=router_bf16(layer, shape.n_experts, shape.hidden),
         bias=zipf_bias(layer, shape.n_experts, shape.zipf_s, bias_seed),
