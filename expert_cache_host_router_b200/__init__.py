@@ -86,6 +86,7 @@ _SIGS = {
     "moe_stats": (ctypes.c_int, [_P, ctypes.POINTER(Stats), _P, _P, ctypes.c_size_t,
                                  ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
     "moe_set_trace": (ctypes.c_int, [_P, _P, _P]),
+    "moe_set_phase_trace": (ctypes.c_int, [_P, _P]),
     "moe_debug_drop_signals": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_destroy": (None, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -192,6 +193,10 @@ def moe_set_trace(ctx: int, h_trace_dev: int | None, w_trace_dev: int | None) ->
     _check(lib().moe_set_trace(ctx, h_trace_dev, w_trace_dev), "moe_set_trace")
 
 
+def moe_set_phase_trace(ctx: int, stamps_dev: int | None) -> None:
+    _check(lib().moe_set_phase_trace(ctx, stamps_dev), "moe_set_phase_trace")
+
+
 def moe_debug_drop_signals(ctx: int, n: int) -> None:
     _check(lib().moe_debug_drop_signals(ctx, n), "moe_debug_drop_signals")
 
@@ -252,6 +257,10 @@ class ExpertCacheMoE:
 
     def sync(self):
         moe_sync(self.ctx)
+
+    def set_phase_trace(self, stamps=None):
+        """stamps: torch int64 [(L+1), 8] on the device, or None."""
+        moe_set_phase_trace(self.ctx, None if stamps is None else stamps.data_ptr())
 
     def set_trace(self, h_trace=None, w_trace=None):
         moe_set_trace(self.ctx, None if h_trace is None else h_trace.data_ptr(),

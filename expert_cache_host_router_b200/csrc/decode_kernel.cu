@@ -143,13 +143,51 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-// Canonical fold of n partials (stride 1) by one warp; every lane returns the total.
+// Canonical fold of n partials (n <= 256, stride 1) by one warp; every lane returns
+// the total.  Lane l adds parts l, l+32, ... from +0 in that order, then the lanes
+// combine by xor-butterfly offsets 16, 8, 4, 2, 1.
 __device__ __forceinline__ float canonical_fold(const float* parts, int n, int lane) {
+  float v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = lane + 32 * k < n ? __ldcg(parts + lane + 32 * k) : 0.0f;
   float acc = 0.0f;
-  for (int m = lane; m < n; m += 32) acc = __fadd_rn(acc, __ldcg(parts + m));
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (lane + 32 * k < n) acc = __fadd_rn(acc, v[k]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
   return acc;
+}
+
+// Quantise one 32-value block held one value per lane to int16 codes:
+// code = rint(v * 32767 / amax); scale16 = amax / (32767 * 16) reconstructs 16 * v / code;
+// csum = sum of the block's codes.  Same arithmetic in every CTA: deterministic.
+__device__ __forceinline__ int quant_block(float v, float& scale16, int& csum) {
+  const float amax = warp_max(fabsf(v));
+  int code = 0;
+  if (amax > 0.0f) {
+    code = __float2int_rn(v * (32767.0f * __frcp_rn(amax)));
+    code = max(-32767, min(32767, code));
+  }
+  scale16 = amax * (1.0f / (32767.0f * 16.0f));
+  csum = warp_sum_int(code);
+  return code;
+}
+
+// Orderable 64-bit routing key: larger logit first, then lower expert index; -0 == +0;
+// a NaN logit gets key 0 and is never preferred.
+__device__ __forceinline__ uint64_t route_key(float v, int e) {
+  if (v == 0.0f) v = 0.0f;
+  const uint32_t u = __float_as_uint(v);
+  uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  if (v != v) o = 0;
+  return ((uint64_t)o << 32) | (uint32_t)(~(uint32_t)e);
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int off) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, off);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), off);
+  return ((uint64_t)hi << 32) | lo;
 }
 
 __host__ __device__ inline int pow2_ceil_le32(int n) {
@@ -161,28 +199,37 @@ __host__ __device__ inline int pow2_ceil_le32(int n) {
 // ------------------------------------------------------------------ shared memory plan
 
 struct Misc {
-  uint64_t bar[2];
+  uint64_t bar_u[4];  // gate/up unit, four 16-row stages
+  uint64_t bar_d;     // down rows of the owned chunk
+  uint64_t bar_r;     // next layer's router columns of the owned chunks
   const uint8_t* src[kMaxK + 1];  // slot base of each active expert (rank order, then shared)
   uint32_t miss_seq[kMaxK + 1];   // copy to wait for (0: resident)
   int32_t sel[kMaxK];
   float w[kMaxK];
   int32_t fix_dst[kMaxR], fix_src[kMaxR];  // deferred ring fills (pool indices)
   int32_t n_fix;
-  float hchunk[kChunk];
+  int32_t ring_owner[kMaxR];
+  uint32_t ring_stamp[kMaxR];
+  uint32_t ring_clock;
+  float hown[kMaxOwn][kChunk];   // this CTA's rows of the residual stream
+  float gnext[kMaxOwn][kChunk];  // next layer's RMSNorm gain on those rows
   float u[kChunk];
   float gu[2 * kUnitRows];
   float inv;
   uint32_t step, seq_base, n_miss, gen;
   int32_t flag;
+  int32_t P_l, base_l;  // pinned count and pool base of the current layer
+  int32_t unit_ok;   // first gate/up unit issued
+  int32_t d_issued;  // down rows of the first owned chunk issued during routing
 };
 
 struct SmemPlan {
-  uint32_t unit, dchunk, z, xcodes, xs, xc, acodes, o, misc, total;
+  uint32_t unit, dchunk, rchunk, hbuf, gbuf, pinrow, z, xcodes, xs, xc, acodes, o, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is) {
+__host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is, int nown) {
   SmemPlan s;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) {
@@ -193,8 +240,12 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
   };
   const int n_exp = K + (Is > 0);
   const int imax = I > Is ? I : Is;
-  s.unit = take(36u * H);                       // gate qs|d, up qs|d for 32 rows
-  s.dchunk = take(9u * (uint32_t)(K * I + Is)); // down rows of one chunk, all experts
+  s.unit = take(36u * H);                        // gate qs|d, up qs|d for 32 rows
+  s.dchunk = take(9u * (uint32_t)(K * I + Is));  // down rows of one chunk, all experts
+  s.rchunk = take(32u * E * nown);               // router columns of the owned chunks
+  s.hbuf = take(4u * H);
+  s.gbuf = take(4u * H);
+  s.pinrow = take(4u * E);
   s.z = take(4u * E);
   s.xcodes = take(2u * H);
   s.xs = take(4u * (H / 32));
@@ -208,39 +259,42 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
 
 // ------------------------------------------------------------------ barriers and waits
 
-// Grid barrier over all CTAs (co-resident by cooperative launch).  Returns false when
-// the wait ran out or another CTA flagged an error.
+// Grid barrier over all CTAs (co-resident by cooperative launch).  The arrival counter
+// only grows during a launch (the graph zeroes it before the kernel), so barrier b of
+// the launch completes when it reaches (b + 1) * gridDim.x.  Returns false when the
+// wait ran out or another CTA flagged an error.
 __device__ bool grid_sync(const DecodeParams& p, Misc& m) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    const uint32_t gen = m.gen;
-    __threadfence();
-    const uint32_t arrived = atomicAdd(&p.ctrl->bar_count, 1u);
-    if (arrived == gridDim.x - 1) {
-      atomicExch(&p.ctrl->bar_count, 0u);
-      __threadfence();
-      atomicExch(&p.ctrl->bar_gen, gen + 1);
-    } else {
+    const uint32_t target = (m.gen + 1) * gridDim.x;
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
+    if (ld_acquire(&p.ctrl->bar_count) < target) {
       const uint64_t t0 = gtimer();
-      while (ld_acquire(&p.ctrl->bar_gen) == gen) {
-        if (has_error(p.ctrl)) {
-          ok = 0;
-          break;
-        }
-        if (gtimer() - t0 > p.timeout_ns) {
-          set_error(p.ctrl, MOE_DEVERR_BARRIER);
-          ok = 0;
-          break;
+      uint32_t polls = 0;
+      while (ld_acquire(&p.ctrl->bar_count) < target) {
+        if ((++polls & 63u) == 0) {
+          if (has_error(p.ctrl)) {
+            ok = 0;
+            break;
+          }
+          if (gtimer() - t0 > p.timeout_ns) {
+            set_error(p.ctrl, MOE_DEVERR_BARRIER);
+            ok = 0;
+            break;
+          }
         }
       }
     }
-    __threadfence();
-    m.gen = gen + 1;
-    m.flag = ok && !has_error(p.ctrl);
+    m.gen += 1;
+    m.flag = ok;
   }
   __syncthreads();
   return m.flag != 0;
+}
+
+__device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
+  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 16 + k] = gtimer();
 }
 
 // Thread 0: wait until the proxy has signalled miss copy seq (0: nothing to wait for).
@@ -262,7 +316,7 @@ __device__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
   return true;
 }
 
-// All threads: wait for the bulk copies counted on bar to land (bounded).
+// Wait for the bulk copies counted on bar to land (bounded).
 __device__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtimer();
@@ -277,20 +331,19 @@ __device__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity)
 
 // ------------------------------------------------------------------ phases
 
-// Router partials of layer l over chunk c (16 columns of h held in m.hchunk), and the
-// chunk's sum of squares for the RMSNorm of layer l.
-__device__ void router_partials(const DecodeParams& p, Misc& m, int l, int c) {
+// Router partials of layer l over chunk c (16 columns): every thread e folds
+// w[e][t] * u_t, u_t = g_t * h_t (g = 1 without a gain; u = h without the norm), from
+// +0 in ascending column order; plus the chunk's sum of squares of h.  wrow(e) points
+// at the 16 bf16 weights of expert e for this chunk (global or shared memory).
+template <typename WRow>
+__device__ void router_partials(const DecodeParams& p, Misc& m, int c, const float* hv, const float* gv,
+                                WRow wrow) {
   const int tid = threadIdx.x;
-  if (tid < kChunk) {
-    const float hv = m.hchunk[tid];
-    float u = hv;
-    if (p.use_norm && p.gain) u = __fmul_rn(p.gain[(size_t)l * p.H + c * kChunk + tid], hv);
-    m.u[tid] = u;
-  }
+  if (tid < kChunk) m.u[tid] = (p.use_norm && gv) ? __fmul_rn(gv[tid], hv[tid]) : hv[tid];
   __syncthreads();
   for (int e = tid; e < p.E; e += kThreads) {
-    const uint4* wp = reinterpret_cast<const uint4*>(p.router + (((size_t)l * p.nch + c) * p.E + e) * kChunk);
-    const uint4 w0 = __ldg(wp), w1 = __ldg(wp + 1);
+    const uint4* wp = wrow(e);
+    const uint4 w0 = wp[0], w1 = wp[1];
     const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
     float acc = 0.0f;
 #pragma unroll
@@ -303,80 +356,95 @@ __device__ void router_partials(const DecodeParams& p, Misc& m, int l, int c) {
   if (tid == 0 && p.use_norm) {
     float s = 0.0f;
 #pragma unroll
-    for (int t = 0; t < kChunk; ++t) s = fmaf(m.hchunk[t], m.hchunk[t], s);
+    for (int t = 0; t < kChunk; ++t) s = fmaf(hv[t], hv[t], s);
     __stcg(p.sq + c, s);
   }
 }
 
 // Warp 0: top-k of z (value desc, index asc) and the renormalised softmax weights.
-__device__ void topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
+// Keys live in registers (E <= 256: 8 per lane); each round is a lane-local max and a
+// 64-bit butterfly max.  Lane i returns the expert of rank i (and m.sel / m.w are set).
+__device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
   const int lane = threadIdx.x & 31;
-  uint32_t taken = 0;
-  for (int i = 0; i < p.K; ++i) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-    for (int mb = 0; lane + 32 * mb < p.E; ++mb) {
-      const int e = lane + 32 * mb;
-      if ((taken >> mb) & 1u) continue;
-      const float v = zs[e];
-      if (v > bv || (v == bv && e < be)) {
-        bv = v;
-        be = e;
-      }
-    }
+  const int E = p.E;
+  int my_e = -1;
+  if (E <= 256) {
+    uint32_t ord[8];  // orderable logit bits; 0 marks a taken (or NaN) entry
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
+    for (int k = 0; k < 8; ++k) {
+      const int e = lane + 32 * k;
+      ord[k] = e < E ? (uint32_t)(route_key(zs[e], e) >> 32) : 0u;
+    }
+    for (int i = 0; i < p.K; ++i) {
+      uint32_t lv = ord[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k) lv = max(lv, ord[k]);
+      const uint32_t gv = __reduce_max_sync(0xffffffffu, lv);
+      uint32_t li = 0xffffffffu;
+#pragma unroll
+      for (int k = 7; k >= 0; --k)
+        if (ord[k] == gv) li = (uint32_t)(lane + 32 * k);
+      const int e = (int)__reduce_min_sync(0xffffffffu, li);
+      if (gv == 0u && lane == 0) set_error(p.ctrl, MOE_DEVERR_ROUTE);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (lane + 32 * k == e) ord[k] = 0u;
+      if (lane == i) my_e = e;
+    }
+  } else {  // large expert counts: keys re-read from shared memory every round
+    uint32_t taken = 0;
+    for (int i = 0; i < p.K; ++i) {
+      uint64_t best = 0;
+      for (int k = 0; lane + 32 * k < E; ++k)
+        if (!((taken >> k) & 1u)) {
+          const uint64_t kk = route_key(zs[lane + 32 * k], lane + 32 * k);
+          best = kk > best ? kk : best;
+        }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const uint64_t o = shfl_xor_u64(best, off);
+        best = o > best ? o : best;
       }
+      const int e = (int)(~(uint32_t)best);
+      if ((best >> 32) == 0ull && lane == 0) set_error(p.ctrl, MOE_DEVERR_ROUTE);
+      if ((e & 31) == lane) taken |= 1u << (e >> 5);
+      if (lane == i) my_e = e;
     }
-    if (be == 0x7fffffff) {
-      if (lane == 0) set_error(p.ctrl, MOE_DEVERR_ROUTE);
-      be = 0;
-    }
-    if (lane == (be & 31)) taken |= 1u << (be >> 5);
-    if (lane == 0) m.sel[i] = be;
+  }
+  if (my_e < 0 || my_e >= E) my_e = 0;  // lanes >= k (and a failed route)
+  const float zmax = __shfl_sync(0xffffffffu, zs[my_e], 0);
+  const float ex = lane < p.K ? expf(zs[my_e] - zmax) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < p.K) {
+    m.sel[lane] = my_e;
+    m.w[lane] = ex / sum;
   }
   __syncwarp();
-  if (lane == 0) {
-    const float zmax = zs[m.sel[0]];
-    float ex[kMaxK];
-    float s = 0.0f;
-    for (int i = 0; i < p.K; ++i) {
-      ex[i] = expf(zs[m.sel[i]] - zmax);
-      s += ex[i];
-    }
-    for (int i = 0; i < p.K; ++i) m.w[i] = ex[i] / s;
-  }
+  return my_e;
 }
 
-// Thread 0 of every CTA: the cache decision for layer l (identical in all CTAs).  CTA 0
-// also commits the next ring state, the event log, histogram, counters and requests.
-__device__ void cache_decide(const DecodeParams& p, Misc& m, int l) {
-  const int R = p.R, E = p.E, K = p.K;
+// Thread 0 of every CTA: the cache decision for layer l (identical in all CTAs), from
+// the layer's pinned-slot row and ring state staged in shared memory.  CTA 0 also
+// commits the next ring state, the event log, histogram, counters and miss requests.
+__device__ void cache_decide(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow) {
+  const int R = p.R, K = p.K;
   const int par = m.step & 1;
   const bool commit = blockIdx.x == 0;
-  const int P = p.n_pinned[l];
-  const int base = p.layer_base[l];
-  int32_t owner[kMaxR];
-  uint32_t stamp[kMaxR];
+  const int P = m.P_l;
+  const int base = m.base_l;
   bool busy[kMaxR];
   int32_t fix[kMaxR];
-  const size_t rs = ((size_t)par * p.L + l) * R;
-  uint32_t clock = __ldcg(p.ring_clock + (size_t)par * p.L + l);
+  uint32_t clock = m.ring_clock;
   for (int r = 0; r < R; ++r) {
-    owner[r] = __ldcg(p.ring_owner + rs + r);
-    stamp[r] = __ldcg(p.ring_stamp + rs + r);
     busy[r] = false;
     fix[r] = -1;
   }
   unsigned long long n_pin = 0, n_ring = 0, n_miss = 0, n_evict = 0, n_staged = 0;
   for (int i = 0; i < K; ++i) {
     const int e = m.sel[i];
-    const int ps = p.pin_slot[(size_t)l * E + e];
+    const int ps = pinrow[e];
     int kind, slot_log, evicted = -1, pool_idx;
     uint32_t seq = 0;
     if (ps >= 0) {
@@ -387,10 +455,10 @@ __device__ void cache_decide(const DecodeParams& p, Misc& m, int l) {
     } else {
       int r = -1;
       for (int rr = 0; rr < R; ++rr)
-        if (owner[rr] == e) r = rr;
+        if (m.ring_owner[rr] == e) r = rr;
       if (r >= 0) {
         kind = MOE_RING_HIT;
-        stamp[r] = ++clock;
+        m.ring_stamp[r] = ++clock;
         busy[r] = true;
         slot_log = P + r;
         pool_idx = base + P + r;
@@ -403,15 +471,15 @@ __device__ void cache_decide(const DecodeParams& p, Misc& m, int l) {
       } else {
         int v = -1;
         for (int rr = 0; rr < R && v < 0; ++rr)
-          if (owner[rr] < 0) v = rr;
+          if (m.ring_owner[rr] < 0) v = rr;
         if (v < 0) {
           v = 0;
           for (int rr = 1; rr < R; ++rr)
-            if (stamp[rr] < stamp[v]) v = rr;
+            if (m.ring_stamp[rr] < m.ring_stamp[v]) v = rr;
         }
-        evicted = owner[v];
-        owner[v] = e;
-        stamp[v] = ++clock;
+        evicted = m.ring_owner[v];
+        m.ring_owner[v] = e;
+        m.ring_stamp[v] = ++clock;
         kind = MOE_MISS;
         slot_log = P + v;
         seq = m.seq_base + 1 + m.n_miss++;
@@ -449,7 +517,7 @@ __device__ void cache_decide(const DecodeParams& p, Misc& m, int l) {
       ev[4] = kind;
       ev[5] = slot_log;
       ev[6] = evicted;
-      atomicAdd(p.hist + (size_t)l * E + e, 1u);
+      atomicAdd(p.hist + (size_t)l * p.E + e, 1u);
     }
   }
   if (p.Is > 0) {
@@ -466,25 +534,108 @@ __device__ void cache_decide(const DecodeParams& p, Misc& m, int l) {
   if (commit) {
     const size_t ws = ((size_t)(par ^ 1) * p.L + l) * R;
     for (int r = 0; r < R; ++r) {
-      p.ring_owner[ws + r] = owner[r];
-      p.ring_stamp[ws + r] = stamp[r];
+      p.ring_owner[ws + r] = m.ring_owner[r];
+      p.ring_stamp[ws + r] = m.ring_stamp[r];
     }
     p.ring_clock[(size_t)(par ^ 1) * p.L + l] = clock;
-    p.ctrl->pin_hits += n_pin;
-    p.ctrl->ring_hits += n_ring;
-    p.ctrl->misses += n_miss;
-    p.ctrl->evictions += n_evict;
-    p.ctrl->staged += n_staged;
+    atomicAdd(&p.ctrl->pin_hits, n_pin);
+    atomicAdd(&p.ctrl->ring_hits, n_ring);
+    atomicAdd(&p.ctrl->misses, n_miss);
+    atomicAdd(&p.ctrl->evictions, n_evict);
+    atomicAdd(&p.ctrl->staged, n_staged);
   }
+}
+
+// Warp 0: the common case where every selected expert is pinned; lane i handles rank
+// i.  Returns false (nothing written) when some expert is not pinned.
+__device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow, int my_e) {
+  const int lane = threadIdx.x & 31;
+  const int ps = lane < p.K ? pinrow[my_e] : 0;
+  if (!__all_sync(0xffffffffu, ps >= 0)) return false;
+  const bool commit = blockIdx.x == 0;
+  if (lane < p.K) {
+    m.src[lane] = p.pool + (size_t)(m.base_l + ps) * p.slot_bytes;
+    m.miss_seq[lane] = 0;
+    if (commit) {
+      int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * p.K + lane) * 7;
+      ev[0] = (int32_t)m.step;
+      ev[1] = l;
+      ev[2] = lane;
+      ev[3] = my_e;
+      ev[4] = MOE_PIN_HIT;
+      ev[5] = ps;
+      ev[6] = -1;
+      atomicAdd(p.hist + (size_t)l * p.E + my_e, 1u);
+    }
+  }
+  if (commit && lane < p.R) {  // the ring is untouched: carry it to the next token's copy
+    const int par = m.step & 1;
+    const size_t ws = ((size_t)(par ^ 1) * p.L + l) * p.R;
+    p.ring_owner[ws + lane] = m.ring_owner[lane];
+    p.ring_stamp[ws + lane] = m.ring_stamp[lane];
+  }
+  if (lane == 0) {
+    if (p.Is > 0) {
+      m.src[p.K] = p.shared_pool + (size_t)l * p.shared_slot_bytes;
+      m.miss_seq[p.K] = 0;
+    }
+    m.n_fix = 0;
+    if (commit) {
+      p.ring_clock[(size_t)((m.step & 1) ^ 1) * p.L + l] = m.ring_clock;
+      atomicAdd(&p.ctrl->pin_hits, (unsigned long long)p.K);
+    }
+  }
+  __syncwarp();
+  return true;
+}
+
+// Thread 0: bulk-load gate/up unit u (32 rows of gate and of up of one expert) into
+// shared memory as four 16-row tiles, one bulk copy each, after its miss copy (if any)
+// has landed.
+__device__ bool issue_unit(const DecodeParams& p, Misc& m, uint8_t* unit, int u) {
+  const int per = p.I / 32, routed = p.K * per;
+  const int i = u < routed ? u / per : p.K;
+  const int rb = u < routed ? u % per : u - routed;
+  const SlotLayout& L = i < p.K ? p.lay : p.slay;
+  if (!wait_miss(p, m.miss_seq[i])) return false;
+  const uint32_t tb = 9u * p.H;
+  const uint8_t* src = m.src[i] + L.gu + (size_t)rb * 4 * tb;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    mbar_expect_tx(&m.bar_u[st], tb);
+    bulk_g2s(unit + st * tb, src + st * tb, tb, &m.bar_u[st]);
+  }
+  return true;
+}
+
+// Thread 0: bulk-load the down tile of chunk c of every active expert (one copy each).
+__device__ bool issue_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c) {
+  for (int i = 0; i < p.n_exp; ++i)
+    if (!wait_miss(p, m.miss_seq[i])) return false;
+  uint32_t total = 0;
+  for (int i = 0; i < p.n_exp; ++i) total += 9u * (i < p.K ? p.I : p.Is);
+  mbar_expect_tx(&m.bar_d, total);
+  uint32_t off = 0;
+  for (int i = 0; i < p.n_exp; ++i) {
+    const int Ii = i < p.K ? p.I : p.Is;
+    const SlotLayout& L = i < p.K ? p.lay : p.slay;
+    const uint32_t tb = 9u * Ii;
+    bulk_g2s(dch + off, m.src[i] + L.down + (size_t)c * tb, tb, &m.bar_d);
+    off += tb;
+  }
+  return true;
 }
 
 // ------------------------------------------------------------------ the kernel
 
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const SmemPlan S = smem_plan(p.H, p.E, p.K, p.I, p.Is);
+  const SmemPlan S = smem_plan(p.H, p.E, p.K, p.I, p.Is, p.nown);
   Misc& m = *reinterpret_cast<Misc*>(smem + S.misc);
   float* zs = reinterpret_cast<float*>(smem + S.z);
+  float* hbuf = reinterpret_cast<float*>(smem + S.hbuf);
+  float* gbuf = reinterpret_cast<float*>(smem + S.gbuf);
+  int32_t* pinrow = reinterpret_cast<int32_t*>(smem + S.pinrow);
   int16_t* xcodes = reinterpret_cast<int16_t*>(smem + S.xcodes);
   float* xs = reinterpret_cast<float*>(smem + S.xs);
   int32_t* xc = reinterpret_cast<int32_t*>(smem + S.xc);
@@ -492,98 +643,206 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   float* os = reinterpret_cast<float*>(smem + S.o);
   uint8_t* unit = smem + S.unit;
   uint8_t* dch = smem + S.dchunk;
+  uint8_t* rch = smem + S.rchunk;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.H, nb = H / 32;
   const int imax = p.I > p.Is ? p.I : p.Is;
   const int rec_per_exp = imax / 32;
+  const bool has_gain = p.use_norm && p.gain;
+  int n_own = 0;  // chunks of h owned by this CTA
+  while (n_own < p.nown && (int)blockIdx.x + n_own * (int)gridDim.x < p.nch) ++n_own;
 
   if (tid == 0) {
-    mbar_init(&m.bar[0], 1);
-    mbar_init(&m.bar[1], 1);
+    for (int b = 0; b < 4; ++b) mbar_init(&m.bar_u[b], 1);
+    mbar_init(&m.bar_d, 1);
+    mbar_init(&m.bar_r, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     m.step = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->step);
     m.seq_base = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->req_seq);
-    m.gen = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->bar_gen);
+    m.gen = 0;
     m.n_miss = 0;
     m.flag = !has_error(p.ctrl);
   }
   __syncthreads();
   if (!m.flag) return;
-  uint32_t par0 = 0, par1 = 0;  // mbarrier phase parities (uniform across threads)
+  uint32_t par_u[4] = {0, 0, 0, 0}, par_d = 0, par_r = 0;  // mbarrier parities (uniform)
+  stamp(p, p.L, 0);
 
-  // ---- prologue: h = x, and layer 0's router partials
-  for (int c = blockIdx.x; c < p.nch; c += gridDim.x) {
+  // ---- prologue: h = x on the owned rows, and layer 0's router partials
+  for (int k = 0; k < n_own; ++k) {
+    const int c = blockIdx.x + k * gridDim.x;
     if (tid < kChunk) {
       const float v = p.x[c * kChunk + tid];
-      m.hchunk[tid] = v;
+      m.hown[k][tid] = v;
+      m.gnext[k][tid] = has_gain ? p.gain[c * kChunk + tid] : 1.0f;
       __stcg(p.h + c * kChunk + tid, v);
       if (p.h_trace) p.h_trace[c * kChunk + tid] = v;
     }
     __syncthreads();
-    router_partials(p, m, 0, c);
+    router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
+      return reinterpret_cast<const uint4*>(p.router + ((size_t)c * p.E + e) * kChunk);
+    });
     __syncthreads();
   }
   if (!grid_sync(p, m)) return;
+  stamp(p, p.L, 1);
 
   for (int l = 0; l < p.L; ++l) {
+    stamp(p, l, 0);
+    const bool next = l + 1 < p.L;
     // ---------------------------------------------------------------- R phase
-    if (warp == 0) {
+    // prefetch the next layer's router columns of the owned chunks (bulk copies)
+    if (tid == 0 && next && n_own > 0) {
+      mbar_expect_tx(&m.bar_r, 32u * p.E * n_own);
+      for (int k = 0; k < n_own; ++k) {
+        const int c = blockIdx.x + k * gridDim.x;
+        bulk_g2s(rch + (size_t)k * 32u * p.E, p.router + (((size_t)(l + 1) * p.nch + c) * p.E) * kChunk,
+                 32u * p.E, &m.bar_r);
+      }
+    }
+    // stage this layer's inputs: every load of the phase is issued before any is used
+    float4 hreg[4], greg[4];
+    int32_t preg[4];
+    {
+      const float4* h4 = reinterpret_cast<const float4*>(p.h);
+      const float4* g4 = has_gain ? reinterpret_cast<const float4*>(p.gain + (size_t)l * H) : nullptr;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = tid + q * kThreads;
+        if (t < H / 4) {
+          hreg[q] = __ldcg(h4 + t);
+          if (has_gain) greg[q] = __ldg(g4 + t);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = tid + q * kThreads;
+        if (e < p.E) preg[q] = __ldg(p.pin_slot + (size_t)l * p.E + e);
+      }
+      const int par = m.step & 1;
+      const size_t rs = ((size_t)par * p.L + l) * p.R;
+      if (tid < p.R) {
+        m.ring_owner[tid] = __ldcg(p.ring_owner + rs + tid);
+        m.ring_stamp[tid] = __ldcg(p.ring_stamp + rs + tid);
+      }
+      if (tid == kThreads - 1) m.ring_clock = __ldcg(p.ring_clock + (size_t)par * p.L + l);
+      if (tid == kThreads - 2) m.P_l = __ldg(p.n_pinned + l);
+      if (tid == kThreads - 3) m.base_l = __ldg(p.layer_base + l);
+      if (next && tid < n_own * kChunk) {
+        const int k = tid / kChunk, t = tid % kChunk;
+        const int c = blockIdx.x + k * gridDim.x;
+        m.gnext[k][t] = has_gain ? __ldg(p.gain + (size_t)(l + 1) * H + c * kChunk + t) : 1.0f;
+      }
+    }
+    // logits of this CTA's experts (and the norm scale, in every CTA)
+    {
       float inv = 1.0f;
       if (p.use_norm) {
         const float ss = canonical_fold(p.sq, p.nch, lane);
         inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), p.eps)));
       }
-      if (lane == 0) m.inv = inv;
-    }
-    __syncthreads();
-    {
-      const float inv = m.inv;
+      if (warp == 0 && lane == 0) m.inv = inv;
       for (int e = blockIdx.x * kWarps + warp; e < p.E; e += gridDim.x * kWarps) {
-        const float s = canonical_fold(p.part + (size_t)e * p.nch, p.nch, lane);
-        if (lane == 0) __stcg(p.z + e, fmaf(s, inv, p.bias ? p.bias[(size_t)l * p.E + e] : 0.0f));
+        const float sum = canonical_fold(p.part + (size_t)e * p.nch, p.nch, lane);
+        if (lane == 0) __stcg(p.z + e, fmaf(sum, inv, p.bias ? __ldg(p.bias + (size_t)l * p.E + e) : 0.0f));
       }
     }
+    {
+      float4* hb4 = reinterpret_cast<float4*>(hbuf);
+      float4* gb4 = reinterpret_cast<float4*>(gbuf);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = tid + q * kThreads;
+        if (t < H / 4) {
+          hb4[t] = hreg[q];
+          if (has_gain) gb4[t] = greg[q];
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = tid + q * kThreads;
+        if (e < p.E) pinrow[e] = preg[q];
+      }
+    }
+    __syncthreads();
+    // quantised activations x = RMSNorm(h) (or h): one lane per 32-block, int16 codes
+    if (tid < nb) {
+      const int b = tid;
+      const float inv = m.inv;
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 hv = reinterpret_cast<const float4*>(hbuf + b * 32)[q];
+        float4 xv = hv;
+        if (p.use_norm) {
+          xv.x = __fmul_rn(hv.x, inv);
+          xv.y = __fmul_rn(hv.y, inv);
+          xv.z = __fmul_rn(hv.z, inv);
+          xv.w = __fmul_rn(hv.w, inv);
+          if (has_gain) {
+            const float4 gv = reinterpret_cast<const float4*>(gbuf + b * 32)[q];
+            xv.x = __fmul_rn(xv.x, gv.x);
+            xv.y = __fmul_rn(xv.y, gv.y);
+            xv.z = __fmul_rn(xv.z, gv.z);
+            xv.w = __fmul_rn(xv.w, gv.w);
+          }
+        }
+        v[4 * q] = xv.x;
+        v[4 * q + 1] = xv.y;
+        v[4 * q + 2] = xv.z;
+        v[4 * q + 3] = xv.w;
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      const float mult = amax > 0.0f ? 32767.0f * __frcp_rn(amax) : 0.0f;
+      int csum = 0;
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c0 = max(-32767, min(32767, __float2int_rn(v[2 * j] * mult)));
+        const int c1 = max(-32767, min(32767, __float2int_rn(v[2 * j + 1] * mult)));
+        csum += c0 + c1;
+        w[j] = ((uint32_t)c0 & 0xffffu) | ((uint32_t)c1 << 16);
+      }
+      int4* dst = reinterpret_cast<int4*>(xcodes + b * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_int4((int)w[4 * q], (int)w[4 * q + 1], (int)w[4 * q + 2], (int)w[4 * q + 3]);
+      xs[b] = amax * (1.0f / (32767.0f * 16.0f));
+      xc[b] = csum;
+    }
     if (!grid_sync(p, m)) return;
+    stamp(p, l, 1);
 
     // ---------------------------------------------------------------- routing
     for (int e = tid; e < p.E; e += kThreads) zs[e] = __ldcg(p.z + e);
     __syncthreads();
-    if (warp == 0) topk_weights(p, m, zs);
-    __syncthreads();
-    if (tid == 0) cache_decide(p, m, l);
-    if (blockIdx.x == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
-    // quantised activations: x = RMSNorm(h) (or h), int16 codes per 32-block
-    {
-      const float inv = m.inv;
-      for (int b = warp; b < nb; b += kWarps) {
-        const int j = b * 32 + lane;
-        const float hv = __ldcg(p.h + j);
-        float xv = hv;
-        if (p.use_norm) {
-          xv = __fmul_rn(hv, inv);
-          if (p.gain) xv = __fmul_rn(xv, p.gain[(size_t)l * H + j]);
-        }
-        const float amax = warp_max(fabsf(xv));
-        int code = 0;
-        if (amax > 0.0f) {
-          code = __float2int_rn(xv * (32767.0f / amax));
-          code = max(-32767, min(32767, code));
-        }
-        const int csum = warp_sum_int(code);
-        xcodes[j] = (int16_t)code;
-        if (lane == 0) {
-          xs[b] = amax > 0.0f ? (amax / 32767.0f) * 0.0625f : 0.0f;
-          xc[b] = csum;
-        }
+    stamp(p, l, 8);
+    if (warp == 0) {
+      const int my_e = topk_weights(p, m, zs);
+      stamp(p, l, 9);
+      const bool fast = cache_all_pinned(p, m, l, pinrow, my_e);
+      if (lane == 0) {
+        if (!fast) cache_decide(p, m, l, pinrow);
+        stamp(p, l, 10);
+        m.unit_ok = (int)blockIdx.x < p.n_units ? issue_unit(p, m, unit, blockIdx.x) : 1;
+        stamp(p, l, 11);
+        m.d_issued = 0;
+        stamp(p, l, 12);
       }
     }
     __syncthreads();
+    if (!m.unit_ok) return;
+    if (blockIdx.x == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
+    stamp(p, l, 2);
 
     // ---------------------------------------------------------------- G phase
     {
       const int GS = pow2_ceil_le32(nb), RPW = 32 / GS, g = lane % GS, sub = lane / GS;
       const int bpl = (nb + GS - 1) / GS;
+      const int rows_per_lane = (2 * kUnitRows + kWarps * RPW - 1) / (kWarps * RPW);
       int4 xq[4][4];
       float xsc[4];
       int xsum[4];
@@ -604,68 +863,91 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           xsum[mb] = 0;
         }
       }
-      const int units_routed = p.K * (p.I / 32);
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-        const int i = u < units_routed ? u / (p.I / 32) : p.K;
-        const int rb = u < units_routed ? u % (p.I / 32) : u - units_routed;
-        const SlotLayout& L = i < p.K ? p.lay : p.slay;
-        if (tid == 0) {
-          int ok = wait_miss(p, m.miss_seq[i]);
-          if (ok) {
-            const uint8_t* s = m.src[i];
-            const uint32_t qb = 16u * H, db = 2u * H;  // 32 rows
-            mbar_expect_tx(&m.bar[0], 2 * (qb + db));
-            bulk_g2s(unit, s + L.gate.qs + (size_t)rb * qb, qb, &m.bar[0]);
-            bulk_g2s(unit + qb, s + L.gate.d + (size_t)rb * db, db, &m.bar[0]);
-            bulk_g2s(unit + qb + db, s + L.up.qs + (size_t)rb * qb, qb, &m.bar[0]);
-            bulk_g2s(unit + 2 * qb + db, s + L.up.d + (size_t)rb * db, db, &m.bar[0]);
-          }
-          m.flag = ok;
+      const int routed = p.K * (p.I / 32);
+      for (int u = blockIdx.x, k = 0; u < p.n_units; u += gridDim.x, ++k) {
+        const int i = u < routed ? u / (p.I / 32) : p.K;
+        const int rb = u < routed ? u % (p.I / 32) : u - routed;
+        if (k > 0) {
+          __syncthreads();  // the previous unit's buffer is free
+          if (tid == 0) m.flag = issue_unit(p, m, unit, u);
+          __syncthreads();
+          if (!m.flag) return;
         }
-        __syncthreads();
-        if (!m.flag) return;
-        if (!mbar_wait(p, &m.bar[0], par0)) return;
-        par0 ^= 1u;
-        for (int r = warp * RPW + sub; r < 2 * kUnitRows; r += kWarps * RPW) {
-          const uint8_t* qbase = unit + (r < kUnitRows ? 0 : 18u * H) + (size_t)(r % kUnitRows) * nb * 16;
-          const __half* dbase = reinterpret_cast<const __half*>(unit + (r < kUnitRows ? 0 : 18u * H) + 16u * H) +
-                                (size_t)(r % kUnitRows) * nb;
-          float acc = 0.0f;
+        uint32_t done = 0;
+        // four rows at a time per lane group, their dot products and reductions
+        // interleaved; row r of the unit: gate rows 0-31, then up rows 0-31
+        for (int k0 = 0; k0 < rows_per_lane; k0 += 4) {
+          int rows[4];
+          float acc[4];
+          bool live[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            rows[q] = warp * RPW + sub + (k0 + q) * kWarps * RPW;
+            live[q] = k0 + q < rows_per_lane && rows[q] < 2 * kUnitRows;
+            acc[q] = 0.0f;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (!live[q]) continue;
+            const int st = rows[q] / 16;
+            if (!((done >> st) & 1u)) {
+              if (!mbar_wait(p, &m.bar_u[st], par_u[st])) return;
+              done |= 1u << st;
+            }
+          }
+          stamp(p, l, 7);
 #pragma unroll
           for (int mb = 0; mb < 4; ++mb) {
             const int b = g + GS * mb;
-            if (mb < bpl && b < nb) {
-              const uint4 q = *reinterpret_cast<const uint4*>(qbase + b * 16);
-              const float d = __half2float(dbase[b]);
-              const int v = q4_block_dot16(q, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
-              acc = fmaf(d * xsc[mb], (float)v, acc);
+            if (!(mb < bpl && b < nb)) continue;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (!live[q]) continue;
+              const int r = rows[q];
+              const uint8_t* tile = unit + (r / 16) * 9u * H;
+              const uint4 qv = *reinterpret_cast<const uint4*>(tile + ((size_t)(r % 16) * nb + b) * 16);
+              const float d = __half2float(reinterpret_cast<const __half*>(tile + 8u * H)[(r % 16) * nb + b]);
+              const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
+              acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
             }
           }
-          for (int off = GS / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-          if (g == 0) m.gu[r] = acc;
+          for (int off = GS / 2; off >= 1; off >>= 1) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
+          }
+          if (g == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (live[q]) m.gu[rows[q]] = acc[q];
+          }
         }
+#pragma unroll
+        for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
         __syncthreads();
         if (warp == 0) {
           const float gv = m.gu[lane], uv = m.gu[kUnitRows + lane];
           const float a = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
-          const float amax = warp_max(fabsf(a));
-          int code = 0;
-          if (amax > 0.0f) {
-            code = __float2int_rn(a * (32767.0f / amax));
-            code = max(-32767, min(32767, code));
-          }
-          const int csum = warp_sum_int(code);
+          float sc;
+          int csum;
+          const int code = quant_block(a, sc, csum);
           uint8_t* rec = p.acodes + ((size_t)i * rec_per_exp + rb) * kACodeBytes;
-          reinterpret_cast<int16_t*>(rec)[lane] = (int16_t)code;
+          __stcg(reinterpret_cast<int16_t*>(rec) + lane, (int16_t)code);
           if (lane == 0) {
-            reinterpret_cast<float*>(rec + 64)[0] = amax > 0.0f ? (amax / 32767.0f) * 0.0625f : 0.0f;
-            reinterpret_cast<int32_t*>(rec + 68)[0] = csum;
+            __stcg(reinterpret_cast<float*>(rec + 64), sc);
+            __stcg(reinterpret_cast<int32_t*>(rec + 68), csum);
           }
         }
-        __syncthreads();
       }
     }
+    // the owned chunk's down tiles load while the grid waits for the slowest unit
+    if (tid == 0 && n_own > 0) {
+      bool layer_misses = false;
+      for (int i = 0; i < p.n_exp; ++i) layer_misses |= m.miss_seq[i] != 0;
+      if (!layer_misses) m.d_issued = issue_dchunk(p, m, dch, blockIdx.x) ? 1 : 0;
+    }
+    stamp(p, l, 3);
     if (!grid_sync(p, m)) return;
+    stamp(p, l, 4);
 
     // ---------------------------------------------------------------- D phase
     {
@@ -675,79 +957,67 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       for (int t = tid; t < n_rec; t += kThreads) dstr[t] = __ldcg(srcr + t);
     }
     __syncthreads();
-    for (int c = blockIdx.x; c < p.nch; c += gridDim.x) {
-      if (tid == 0) {
-        int ok = 1;
-        uint32_t total = 0;
-        for (int i = 0; i < p.n_exp; ++i) total += 9u * (i < p.K ? p.I : p.Is);
-        for (int i = 0; i < p.n_exp && ok; ++i) ok = wait_miss(p, m.miss_seq[i]);
-        if (ok) {
-          mbar_expect_tx(&m.bar[1], total);
-          uint32_t off = 0;
-          for (int i = 0; i < p.n_exp; ++i) {
-            const int Ii = i < p.K ? p.I : p.Is;
-            const SlotLayout& L = i < p.K ? p.lay : p.slay;
-            const uint32_t qb = 8u * Ii, db = (uint32_t)Ii;  // 16 rows
-            bulk_g2s(dch + off, m.src[i] + L.down.qs + (size_t)c * qb, qb, &m.bar[1]);
-            bulk_g2s(dch + off + qb, m.src[i] + L.down.d + (size_t)c * db, db, &m.bar[1]);
-            off += qb + db;
-          }
-        }
-        m.flag = ok;
-      }
+    stamp(p, l, 13);
+    for (int k = 0; k < n_own; ++k) {
+      const int c = blockIdx.x + k * gridDim.x;
+      if (tid == 0 && !(k == 0 && m.d_issued)) m.flag = issue_dchunk(p, m, dch, c);
       __syncthreads();
-      if (!m.flag) return;
-      if (!mbar_wait(p, &m.bar[1], par1)) return;
-      par1 ^= 1u;
-      // tasks: (expert i, row group); each warp handles whole row groups
+      if (!(k == 0 && m.d_issued) && !m.flag) return;
+      if (!mbar_wait(p, &m.bar_d, par_d)) return;
+      par_d ^= 1u;
+      stamp(p, l, 14);
+      // thread (row r, block column b0): every expert's blocks b0, b0+16, ... of row r
       {
-        int task = 0;
+        const int r = tid >> 4, b0 = tid & 15;
         uint32_t off = 0;
+#pragma unroll 3
         for (int i = 0; i < p.n_exp; ++i) {
           const int Ii = i < p.K ? p.I : p.Is;
-          const int nbd = Ii / 32, GS = pow2_ceil_le32(nbd), RPW = 32 / GS, g = lane % GS, sub = lane / GS;
-          const int passes = (kChunk + RPW - 1) / RPW;
-          const uint8_t* qbase0 = dch + off;
-          const __half* dbase0 = reinterpret_cast<const __half*>(dch + off + 8u * Ii);
-          for (int ps = 0; ps < passes; ++ps, ++task) {
-            if (task % kWarps != warp) continue;
-            const int r = ps * RPW + sub;
-            float acc = 0.0f;
-            if (r < kChunk) {
-              for (int b = g; b < nbd; b += GS) {
-                const uint8_t* rec = acs + ((size_t)i * rec_per_exp + b) * kACodeBytes;
-                const int4* ap = reinterpret_cast<const int4*>(rec);
-                const uint4 q = *reinterpret_cast<const uint4*>(qbase0 + ((size_t)r * nbd + b) * 16);
-                const float d = __half2float(dbase0[(size_t)r * nbd + b]);
-                const float sc = reinterpret_cast<const float*>(rec + 64)[0];
-                const int cs = reinterpret_cast<const int32_t*>(rec + 68)[0];
-                const int v = q4_block_dot16(q, ap[0], ap[1], ap[2], ap[3]) - 128 * cs;
-                acc = fmaf(d * sc, (float)v, acc);
-              }
-            }
-            for (int o2 = GS / 2; o2 >= 1; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
-            if (g == 0 && r < kChunk) os[i * kChunk + r] = acc;
+          const int nbd = Ii / 32;
+          const uint8_t* qbase = dch + off;
+          const __half* dbase = reinterpret_cast<const __half*>(dch + off + 8u * Ii);
+          float acc = 0.0f;
+          for (int b = b0; b < nbd; b += 16) {
+            const uint8_t* rec = acs + ((size_t)i * rec_per_exp + b) * kACodeBytes;
+            const int4* ap = reinterpret_cast<const int4*>(rec);
+            const uint4 qv = *reinterpret_cast<const uint4*>(qbase + ((size_t)r * nbd + b) * 16);
+            const float d = __half2float(dbase[(size_t)r * nbd + b]);
+            const float sc = reinterpret_cast<const float*>(rec + 64)[0];
+            const int cs = reinterpret_cast<const int32_t*>(rec + 68)[0];
+            const int v = q4_block_dot16(qv, ap[0], ap[1], ap[2], ap[3]) - 128 * cs;
+            acc = fmaf(d * sc, (float)v, acc);
           }
+#pragma unroll
+          for (int o2 = 8; o2 >= 1; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
+          if (b0 == 0) os[i * kChunk + r] = acc;
           off += 9u * Ii;
         }
       }
       __syncthreads();
+      stamp(p, l, 15);
       if (tid < kChunk) {
         const int j = c * kChunk + tid;
         float y = 0.0f;
         for (int i = 0; i < p.K; ++i) y = fmaf(m.w[i], os[i * kChunk + tid], y);
         if (p.Is > 0) y = __fadd_rn(y, os[p.K * kChunk + tid]);
-        const float hn = p.use_norm ? __fadd_rn(__ldcg(p.h + j), y) : y;
-        m.hchunk[tid] = hn;
+        const float hn = p.use_norm ? __fadd_rn(m.hown[k][tid], y) : y;
+        m.hown[k][tid] = hn;
         __stcg(p.h + j, hn);
         if (p.h_trace) p.h_trace[(size_t)(l + 1) * H + j] = hn;
         if (l == p.L - 1) p.y[j] = hn;
       }
-      __syncthreads();
-      if (l + 1 < p.L) router_partials(p, m, l + 1, c);
+      if (next) {
+        if (k == 0 && !mbar_wait(p, &m.bar_r, par_r)) return;
+        router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
+          return reinterpret_cast<const uint4*>(rch + (size_t)k * 32u * p.E + (size_t)e * 32u);
+        });
+      }
       __syncthreads();
     }
+    if (next && n_own > 0) par_r ^= 1u;
+    stamp(p, l, 5);
     if (!grid_sync(p, m)) return;
+    stamp(p, l, 6);
 
     // deferred ring fills (only when a layer misses more often than it has ring slots)
     for (int f = 0; f < m.n_fix; ++f) {
@@ -758,7 +1028,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         d[t] = __ldcg(s + t);
     }
   }
-  if (!grid_sync(p, m)) return;
+  stamp(p, p.L, 2);
   if (blockIdx.x == 0 && tid == 0) {
     p.ctrl->step = m.step + 1;
     p.ctrl->req_seq = m.seq_base + m.n_miss;
@@ -767,23 +1037,25 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
 
 // ------------------------------------------------------------------ host-side launch
 
-uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is) { return smem_plan(H, E, K, I, Is).total; }
+uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown) {
+  return smem_plan(H, E, K, I, Is, nown).total;
+}
 
-cudaError_t decode_configure(int H, int E, int K, int I, int Is) {
-  const uint32_t bytes = decode_smem_bytes(H, E, K, I, Is);
+cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown) {
+  const uint32_t bytes = decode_smem_bytes(H, E, K, I, Is, nown);
   return cudaFuncSetAttribute(moe_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int* out) {
+cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int nown, int* out) {
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, moe_decode_kernel, kThreads,
-                                                       decode_smem_bytes(H, E, K, I, Is));
+                                                       decode_smem_bytes(H, E, K, I, Is, nown));
 }
 
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, p.E, p.K, p.I, p.Is);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, p.E, p.K, p.I, p.Is, p.nown);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

@@ -28,9 +28,9 @@
 #include "moe_internal.h"
 
 namespace moe {
-uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is);
-cudaError_t decode_configure(int H, int E, int K, int I, int Is);
-cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int* out);
+uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown);
+cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown);
+cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int nown, int* out);
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream);
 }  // namespace moe
 
@@ -41,7 +41,7 @@ typedef CUresult (*PfnWriteValue32)(CUstream, CUdeviceptr, cuuint32_t, unsigned 
 struct moe_ctx {
   moe_config cfg{};
   int L = 0, H = 0, E = 0, K = 0, I = 0, Is = 0, R = 0;
-  int nsm = 0, grid = 0;
+  int nsm = 0, grid = 0, nown = 1;
   SlotLayout lay{}, slay{};
   uint64_t slot_bytes = 0, shared_slot_bytes = 0;
   // host tier
@@ -86,6 +86,7 @@ struct moe_ctx {
   PfnWriteValue32 write_value32 = nullptr;
   // tracing and log reading
   float *h_trace = nullptr, *w_trace = nullptr;
+  unsigned long long* phase_trace = nullptr;
   uint64_t log_read_step = 0, log_dropped = 0;
 };
 
@@ -162,6 +163,7 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
   p.nch = c->H / kChunk;
   p.n_units = c->K * (c->I / 32) + c->Is / 32;
   p.n_exp = c->K + (c->Is > 0 ? 1 : 0);
+  p.nown = c->nown;
   p.pool = c->pool.load();
   p.slot_bytes = c->slot_bytes;
   p.lay = c->lay;
@@ -194,6 +196,7 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
   p.mbox = c->mbox_dev;
   p.done_seq = c->done_seq;
   p.timeout_ns = (unsigned long long)c->cfg.wait_timeout_ms * 1000000ull;
+  p.phase_trace = c->phase_trace;
   return p;
 }
 
@@ -211,6 +214,7 @@ static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cud
   CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
   cudaError_t e = cudaSuccess;
   if (host_io) e = cudaMemcpyAsync(c->x_buf, c->x_pin, sizeof(float) * c->H, cudaMemcpyHostToDevice, c->own);
+  if (e == cudaSuccess) e = cudaMemsetAsync(&c->ctrl->bar_count, 0, sizeof(uint32_t), c->own);
   if (e == cudaSuccess) e = decode_launch(make_params(c, x, y), c->grid, c->own);
   if (e == cudaSuccess && host_io)
     e = cudaMemcpyAsync(c->y_pin, c->y_buf, sizeof(float) * c->H, cudaMemcpyDeviceToHost, c->own);
@@ -233,21 +237,29 @@ static cudaError_t dalloc(T** p, size_t count) {
   return cudaMalloc((void**)p, sizeof(T) * (count ? count : 1));
 }
 
-static void repack_matrix(const uint8_t* src, uint8_t* dst, const MatView& mv, int64_t rows, int64_t cols) {
-  const int64_t nb = rows * cols / 32;
-  uint8_t* qs = dst + mv.qs;
-  uint8_t* d = dst + mv.d;
-  for (int64_t b = 0; b < nb; ++b) {
-    memcpy(d + 2 * b, src + 18 * b, 2);
-    memcpy(qs + 16 * b, src + 18 * b + 2, 16);
+// Canonical Q4_0 rows [rows x cols] -> 16-row tiles; tile_of(row) gives the tile's offset.
+template <typename TileOf>
+static void repack_rows(const uint8_t* src, uint8_t* dst, int64_t rows, int64_t cols, TileOf tile_of) {
+  const int64_t nb = cols / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    uint8_t* tile = dst + tile_of(r);
+    const int64_t rr = r % 16;
+    uint8_t* qs = tile + rr * nb * 16;
+    uint8_t* d = tile + 16 * nb * 16 + rr * nb * 2;
+    for (int64_t b = 0; b < nb; ++b) {
+      const uint8_t* blk = src + (r * nb + b) * 18;
+      memcpy(d + 2 * b, blk, 2);
+      memcpy(qs + 16 * b, blk + 2, 16);
+    }
   }
 }
 
 static void repack_expert(const uint8_t* src, uint8_t* dst, const SlotLayout& s, int H, int I) {
   const uint64_t gu = q4_bytes(I, H);
-  repack_matrix(src, dst, s.gate, I, H);
-  repack_matrix(src + gu, dst, s.up, I, H);
-  repack_matrix(src + 2 * gu, dst, s.down, H, I);
+  const uint64_t t_gu = 9ull * H, t_d = 9ull * I;
+  repack_rows(src, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + (r % 32) / 16) * t_gu; });
+  repack_rows(src + gu, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + 2 + (r % 32) / 16) * t_gu; });
+  repack_rows(src + 2 * gu, dst, H, I, [&](int64_t r) { return s.down + (r / 16) * t_d; });
 }
 
 // ------------------------------------------------------------------ C ABI
@@ -391,13 +403,15 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   int smem_optin = 0, coop = 0;
   CKC(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, cfg.device));
   CKC(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, cfg.device));
-  if (!coop || decode_smem_bytes(c->H, c->E, c->K, c->I, c->Is) > (uint32_t)smem_optin)
-    return fail(MOE_ERR_UNSUPPORTED);
-  CKC(decode_configure(c->H, c->E, c->K, c->I, c->Is));
-  int per_sm = 0;
-  CKC(decode_max_blocks_per_sm(c->H, c->E, c->K, c->I, c->Is, &per_sm));
-  if (per_sm < 1) return fail(MOE_ERR_UNSUPPORTED);
   c->grid = c->nsm;  // one persistent CTA per SM
+  c->nown = (c->H / kChunk + c->grid - 1) / c->grid;
+  if (!coop || c->nown > kMaxOwn ||
+      decode_smem_bytes(c->H, c->E, c->K, c->I, c->Is, c->nown) > (uint32_t)smem_optin)
+    return fail(MOE_ERR_UNSUPPORTED);
+  CKC(decode_configure(c->H, c->E, c->K, c->I, c->Is, c->nown));
+  int per_sm = 0;
+  CKC(decode_max_blocks_per_sm(c->H, c->E, c->K, c->I, c->Is, c->nown, &per_sm));
+  if (per_sm < 1) return fail(MOE_ERR_UNSUPPORTED);
 
   const size_t nch = c->H / kChunk;
   const int n_exp = c->K + (c->Is > 0);
@@ -590,7 +604,7 @@ int moe_clear_error(moe_ctx* c) {
   const uint32_t last = c->proxy_next.load() - 1;
   ctl.req_seq = last;
   ctl.error = 0;
-  ctl.bar_count = 0;
+  ctl.bar_count = 0;  // (the graphs zero it before every launch as well)
   CK(cudaMemcpy(c->ctrl, &ctl, sizeof(Ctrl), cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->done_seq, &last, sizeof(uint32_t), cudaMemcpyHostToDevice));
   const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);
@@ -598,6 +612,7 @@ int moe_clear_error(moe_ctx* c) {
   CK(cudaMemset(c->ring_stamp, 0, nr * 4));
   CK(cudaMemset(c->ring_clock, 0, (size_t)2 * c->L * 4));
   c->proxy_err.store(0);
+  c->drop.store(0);
   return MOE_OK;
 }
 
@@ -655,6 +670,13 @@ int moe_set_trace(moe_ctx* c, float* h_trace_dev, float* w_trace_dev) {
   if (!c) return MOE_ERR_INVALID;
   c->h_trace = h_trace_dev;
   c->w_trace = w_trace_dev;
+  drop_graphs(c);
+  return MOE_OK;
+}
+
+int moe_set_phase_trace(moe_ctx* c, uint64_t* stamps_dev) {
+  if (!c) return MOE_ERR_INVALID;
+  c->phase_trace = reinterpret_cast<unsigned long long*>(stamps_dev);
   drop_graphs(c);
   return MOE_OK;
 }

@@ -1,13 +1,17 @@
 // moe_internal.h -- layouts shared by the host runtime and the decode kernel of libmoe.
 //
-// Expert slot layout (device slot pool and pinned host tier alike).  Q4_0 blocks
-// (GGUF convention: fp16 scale d + 16 bytes, byte j = weight j low nibble, weight j+16
-// high nibble) are split structure-of-arrays so that every 16-byte nibble group is
-// 16-byte aligned for vector and bulk (TMA) loads:
+// Expert slot layout (device slot pool and pinned host tier alike).  The canonical
+// Q4_0 blocks (GGUF convention: fp16 scale d + 16 bytes, byte j = weight j low nibble,
+// weight j+16 high nibble) are regrouped into tiles of 16 matrix rows, each tile one
+// contiguous run that a single bulk (TMA) copy brings into shared memory:
 //
-//   gate:  qs [I][H/32][16]  then  d [I][H/32] fp16
-//   up:    qs [I][H/32][16]  then  d [I][H/32] fp16
-//   down:  qs [H][I/32][16]  then  d [H][I/32] fp16
+//   tile = [ qs: 16 rows x (K/32 blocks) x 16 bytes ][ d: 16 rows x (K/32) fp16 ]
+//
+//   gate/up part: for every 32-row block rb of the expert's width I, four tiles:
+//     gate rows 32rb..+15, gate rows 32rb+16..+31, up rows 32rb..+15, up rows 32rb+16..+31
+//     (K = H, 9H bytes each)
+//   down part: for every 16-row chunk c of H, one tile of down rows 16c..16c+15
+//     (K = I, 9I bytes each)
 //
 // Values are the canonical blocks' bytes moved, never changed, so a slot is the same
 // expert wherever it lives and full residency stays bit-identical to partial residency.
@@ -25,6 +29,7 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxR = 32;
 constexpr int kMaxH = 4096;
 constexpr int kMboxCap = 256;  // miss-request mailbox entries
+constexpr int kMaxOwn = 4;     // chunks of h one CTA may own
 constexpr int kACodeBytes = 80;  // one quantised block of a: 32 int16, scale, sum, pad
 
 // Bytes of one Q4_0 matrix [rows x cols] in the slot layout (== canonical size).
@@ -32,30 +37,17 @@ inline constexpr uint64_t q4_bytes(uint64_t rows, uint64_t cols) {
   return rows * cols / 32 * 18;
 }
 
-struct MatView {  // offsets of one matrix inside a slot
-  uint64_t qs, d;
-};
-
 struct SlotLayout {
-  MatView gate, up, down;
+  uint64_t gu;     // offset of gate/up tile (rb, st): gu + (4 rb + st) * 9H
+  uint64_t down;   // offset of down tile c: down + c * 9I
   uint64_t bytes;  // rounded up to 256
 };
 
 inline SlotLayout slot_layout(int H, int I) {
   SlotLayout s;
-  uint64_t off = 0;
-  auto mat = [&](uint64_t rows, uint64_t cols) {
-    MatView m;
-    m.qs = off;
-    off += rows * cols / 2;
-    m.d = off;
-    off += rows * cols / 16;
-    return m;
-  };
-  s.gate = mat(I, H);
-  s.up = mat(I, H);
-  s.down = mat(H, I);
-  s.bytes = (off + 255) / 256 * 256;
+  s.gu = 0;
+  s.down = (uint64_t)(I / 32) * 4 * 9 * H;
+  s.bytes = (s.down + (uint64_t)(H / 16) * 9 * I + 255) / 256 * 256;
   return s;
 }
 
@@ -69,14 +61,16 @@ struct MissReq {
   uint32_t dst_slot;
 };
 
-// Device control block (one per context).
-struct Ctrl {
-  uint32_t step;        // decode steps completed
-  uint32_t req_seq;     // miss requests issued so far
-  int32_t error;        // MOE_DEVERR_* or 0
-  uint32_t bar_count;   // grid barrier arrivals
-  uint32_t bar_gen;     // grid barrier generation
-  uint32_t pad[3];
+// Device control block (one per context).  The words every CTA polls live on cache
+// lines of their own so that polling one does not slow the atomics on another.
+struct alignas(128) Ctrl {
+  uint32_t step;     // decode steps completed
+  uint32_t req_seq;  // miss requests issued so far
+  uint32_t pad0[30];
+  int32_t error;  // MOE_DEVERR_* or 0
+  uint32_t pad1[31];
+  uint32_t bar_count;  // grid barrier arrivals, zeroed before every launch
+  uint32_t pad2[31];
   unsigned long long pin_hits, ring_hits, misses, evictions, staged;
 };
 
@@ -87,6 +81,7 @@ struct DecodeParams {
   int nch;      // H / kChunk
   int n_units;  // K * I / 32 + Is / 32
   int n_exp;    // K + (Is > 0)
+  int nown;     // max chunks of h per CTA: ceil(nch / grid)
   // weights
   const uint8_t* pool;  // slot pool
   uint64_t slot_bytes;
@@ -125,6 +120,7 @@ struct DecodeParams {
   MissReq* mbox;                 // host-mapped, kMboxCap entries
   const uint32_t* done_seq;      // device word, written by the proxy's stream
   unsigned long long timeout_ns;
+  unsigned long long* phase_trace;  // [L+1][8] globaltimer stamps of CTA 0, or null
 };
 
 }  // namespace moe

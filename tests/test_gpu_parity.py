@@ -206,7 +206,8 @@ def test_host_buffer_entry_point_matches_device_entry_point():
 
 
 def test_lost_miss_signal_times_out_and_recovers():
-    """Failure detection without a GPU fault: the proxy drops one completion signal, the
+    """Failure detection without a GPU fault: the proxy stops signalling completed miss
+    copies (the completion word is monotonic, so every signal of the step is dropped), the
     kernel's bounded wait runs out, the step reports MOE_ERR_TIMEOUT, and after
     moe_clear_error decoding resumes with correct results."""
     import expert_cache_host_router_b200 as moe
@@ -218,7 +219,7 @@ def test_lost_miss_signal_times_out_and_recovers():
     xs = synthetic.tokens(0, 2, s.hidden)
     base, _, _ = _run_tokens(m, xs)
     m.set_residency(0.0)
-    moe.moe_debug_drop_signals(m.ctx, 1)
+    moe.moe_debug_drop_signals(m.ctx, 1000)
     m.decode(torch.from_numpy(xs[0]).to(DEV))
     with pytest.raises(moe.MoEError) as ei:
         m.sync()
