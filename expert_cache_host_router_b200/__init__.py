@@ -51,6 +51,12 @@ class Weights(ctypes.Structure):
                 ("rms_gain", ctypes.c_void_p)]
 
 
+class NoAllocWeights(ctypes.Structure):
+    _fields_ = [("experts_dev", ctypes.c_void_p), ("shared_dev", ctypes.c_void_p),
+                ("router_dev", ctypes.c_void_p), ("bias_dev", ctypes.c_void_p),
+                ("gain_dev", ctypes.c_void_p)]
+
+
 class Event(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("step", "layer", "rank", "expert", "kind", "slot", "evicted")]
@@ -88,6 +94,8 @@ _SIGS = {
     "moe_set_trace": (ctypes.c_int, [_P, _P, _P]),
     "moe_set_phase_trace": (ctypes.c_int, [_P, _P]),
     "moe_debug_drop_signals": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "moe_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(NoAllocWeights),
+                                                _P, _P, _P]),
     "moe_destroy": (None, [_P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -199,6 +207,12 @@ def moe_set_phase_trace(ctx: int, stamps_dev: int | None) -> None:
 
 def moe_debug_drop_signals(ctx: int, n: int) -> None:
     _check(lib().moe_debug_drop_signals(ctx, n), "moe_debug_drop_signals")
+
+
+def moe_decode_step_noalloc(cfg: Config, weights: NoAllocWeights, x_dev: int, y_dev: int,
+                            stream: int) -> None:
+    _check(lib().moe_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(weights), x_dev, y_dev, stream),
+           "moe_decode_step_noalloc")
 
 
 def moe_destroy(ctx: int) -> None:

@@ -188,6 +188,48 @@ MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev);
  * every signal of a step to make it time out.  moe_clear_error cancels the count. */
 MOE_API int moe_debug_drop_signals(moe_ctx *ctx, int32_t n);
 
+/* Weights for moe_decode_step_noalloc: device memory owned by the caller, every expert
+ * resident, in the library's own layouts (a byte regrouping of the canonical Q4_0
+ * blocks, values unchanged):
+ *   experts_dev: [L][E] routed experts, one slot each, slots slot_bytes(I) apart, where
+ *     slot_bytes(W) = 3 * H * W * 9 / 16 rounded up to a multiple of 256.  A slot is a
+ *     run of tiles; a tile is 16 matrix rows stored as [16 rows x K/32 blocks x 16
+ *     nibble bytes] followed by [16 rows x K/32 fp16 scales].  First, for each 32-row
+ *     block rb of the width W: gate rows 32rb..+15, gate rows 32rb+16..+31, up rows
+ *     32rb..+15, up rows 32rb+16..+31 (K = H); then, for each chunk c of 16 rows of H,
+ *     down rows 16c..16c+15 (K = W).
+ *   shared_dev: [L] shared experts in the same layout with W = shared_inter, slots
+ *     slot_bytes(shared_inter) apart; NULL when shared_inter = 0.
+ *   router_dev: [L][H/16][E][16] bf16, i.e. W_r[l][e][16 c + t] at ((l H/16 + c) E + e) 16 + t.
+ *   bias_dev: [L][E] fp32 or NULL; gain_dev: [L][H] fp32 or NULL. */
+typedef struct {
+  const uint8_t *experts_dev;
+  const uint8_t *shared_dev;
+  const uint16_t *router_dev;
+  const float *bias_dev;
+  const float *gain_dev;
+} moe_noalloc_weights;
+
+/* The decode step of moe_decode_step for callers that cannot allocate device memory:
+ * code that runs under a fixed memory budget or its own allocator, code inside a
+ * stream-capture region where cudaMalloc is not allowed, or a real-time path that must
+ * not take the implicit synchronisation an allocation can bring.  No paper passage
+ * corresponds to it; it is a deployment variant of the same kernel and arithmetic.
+ *
+ * It allocates nothing: no context, no graph, no cudaMalloc / cudaFree.  Its scratch
+ * (exchange buffers, grid-barrier word, slot tables, histogram, one step of event log)
+ * lives in a static 512 KiB device array that every GPU which loads the library holds
+ * until the process exits; the call rejects shapes whose scratch would not fit
+ * (MOE_ERR_UNSUPPORTED).  All experts must be resident (no cache, no miss path); cfg's
+ * ring_slots and log_steps are ignored.  Reads x_dev [H], writes y_dev [H] on stream
+ * (the current device must be cfg->device).  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) and sets the kernel's shared-memory
+ * limit: make that first call before any stream capture.  Every call shares the array
+ * and overwrites it (it is cleared at the start of each call): calls that overlap on
+ * the GPU, on any stream, race.  Asynchronous; returns the launch status. */
+MOE_API int moe_decode_step_noalloc(const moe_config *cfg, const moe_noalloc_weights *w,
+                                    const float *x_dev, float *y_dev, void *stream);
+
 /* Free everything.  NULL is a no-op. */
 MOE_API void moe_destroy(moe_ctx *ctx);
 
