@@ -183,8 +183,11 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     shape = synthetic.FULL_STACK
+    if args.layers != shape.n_layers:  # a shorter stack of the same layers (profiling cases)
+        import dataclasses
+        shape = dataclasses.replace(shape, n_layers=args.layers)
     dev = torch.device("cuda", local)
-    keep_layers = rank == 0 and world == 1 and not args.no_cpu_baseline
+    keep_layers = rank == 0 and world == 1 and not args.no_cpu_baseline and args.layers == 40
     m = moe.ExpertCacheMoE(shape, device=local, log_steps=max(4096, args.steps + args.warmup + 16))
     t0 = time.time()
     for l in range(shape.n_layers):
@@ -336,6 +339,7 @@ def main():
     ap.add_argument("--calib-steps", type=int, default=128)
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
