@@ -92,8 +92,34 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Same copy with an L2 cache policy: streamed expert and router weights are read once
+// per token, so they are marked evict-first and do not push the kernel's code and the
+// small exchange buffers out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  const uint64_t pol = l2_evict_first_policy();
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* ptr) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* ptr, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 
 // Two-way dot products: a holds two int16 (signed), b four uint8; .lo uses bytes 0-1,
@@ -166,7 +192,7 @@ __device__ __forceinline__ int quant_block(float v, float& scale16, int& csum) {
   const float amax = warp_max(fabsf(v));
   int code = 0;
   if (amax > 0.0f) {
-    code = __float2int_rn(v * (32767.0f * __frcp_rn(amax)));
+    code = __float2int_rn(v * __fdividef(32767.0f, amax));
     code = max(-32767, min(32767, code));
   }
   scale16 = amax * (1.0f / (32767.0f * 16.0f));
@@ -259,6 +285,26 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
 
 // ------------------------------------------------------------------ barriers and waits
 
+// Out-of-line slow paths of the bounded waits: the common case (already there) stays
+// inline and short; the spin loops live in separate functions so that the code each
+// layer runs through stays small enough for the SM instruction cache.
+
+// Spin until *count >= target (acquire), with back-off; false on timeout / error.
+__device__ __noinline__ bool spin_count(const DecodeParams& p, const uint32_t* count, uint32_t target) {
+  const uint64_t t0 = gtimer();
+  for (uint32_t polls = 1; ld_acquire(count) < target; ++polls) {
+    __nanosleep(32);
+    if ((polls & 31u) == 0) {
+      if (has_error(p.ctrl)) return false;
+      if (gtimer() - t0 > p.timeout_ns) {
+        set_error(p.ctrl, MOE_DEVERR_BARRIER);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 // Grid barrier over all CTAs (co-resident by cooperative launch).  The arrival counter
 // only grows during a launch (the graph zeroes it before the kernel), so barrier b of
 // the launch completes when it reaches (b + 1) * gridDim.x.  Returns false when the
@@ -266,26 +312,9 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
 __device__ bool grid_sync(const DecodeParams& p, Misc& m) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    int ok = 1;
     const uint32_t target = (m.gen + 1) * gridDim.x;
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
-    if (ld_acquire(&p.ctrl->bar_count) < target) {
-      const uint64_t t0 = gtimer();
-      uint32_t polls = 0;
-      while (ld_acquire(&p.ctrl->bar_count) < target) {
-        if ((++polls & 63u) == 0) {
-          if (has_error(p.ctrl)) {
-            ok = 0;
-            break;
-          }
-          if (gtimer() - t0 > p.timeout_ns) {
-            set_error(p.ctrl, MOE_DEVERR_BARRIER);
-            ok = 0;
-            break;
-          }
-        }
-      }
-    }
+    int ok = ld_acquire(&p.ctrl->bar_count) >= target || spin_count(p, &p.ctrl->bar_count, target);
     m.gen += 1;
     m.flag = ok;
   }
@@ -294,16 +323,28 @@ __device__ bool grid_sync(const DecodeParams& p, Misc& m) {
 }
 
 __device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 16 + k] = gtimer();
+  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = gtimer();
+}
+
+// Counted exchange: a producer CTA publishes with one release add after its stores;
+// a consumer CTA's thread 0 waits (with back-off) until the count reaches target, then
+// the CTA reads the data.  Only producers arrive and only consumers wait.
+__device__ __forceinline__ void publish(const DecodeParams& p, uint32_t* count) {
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+}
+
+__device__ bool await_count(const DecodeParams& p, Misc& m, const uint32_t* count, uint32_t target) {
+  if (threadIdx.x == 0) {
+    const int ok = ld_acquire(count) >= target || spin_count(p, count, target);
+    m.flag = ok && !has_error(p.ctrl);
+  }
+  __syncthreads();
+  return m.flag != 0;
 }
 
 // Thread 0: wait until the proxy has signalled miss copy seq (0: nothing to wait for).
-__device__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
-  if (seq == 0) return true;
-  if ((int32_t)(ld_acquire(p.done_seq) - seq) >= 0) {
-    fence_proxy_async();
-    return true;
-  }
+__device__ __noinline__ bool spin_miss(const DecodeParams& p, uint32_t seq) {
   const uint64_t t0 = gtimer();
   while ((int32_t)(ld_acquire(p.done_seq) - seq) < 0) {
     if (has_error(p.ctrl)) return false;
@@ -312,13 +353,18 @@ __device__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
       return false;
     }
   }
+  return true;
+}
+
+__device__ __forceinline__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
+  if (seq == 0) return true;
+  if ((int32_t)(ld_acquire(p.done_seq) - seq) < 0 && !spin_miss(p, seq)) return false;
   fence_proxy_async();
   return true;
 }
 
 // Wait for the bulk copies counted on bar to land (bounded).
-__device__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool spin_mbar(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = gtimer();
   while (!mbar_try_wait(bar, parity)) {
     if (gtimer() - t0 > p.timeout_ns) {
@@ -327,6 +373,19 @@ __device__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity)
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity) || spin_mbar(p, bar, parity);
+}
+
+// CTA-uniform check of the error word: one thread reads it, everyone acts on that read
+// (threads reading it themselves could disagree and split at the next barrier).
+__device__ __forceinline__ bool cta_ok(const DecodeParams& p, int32_t& flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) flag = !has_error(p.ctrl);
+  __syncthreads();
+  return flag != 0;
 }
 
 // ------------------------------------------------------------------ phases
@@ -361,6 +420,30 @@ __device__ void router_partials(const DecodeParams& p, Misc& m, int c, const flo
   }
 }
 
+// Top-k for more than 256 experts: keys re-read from shared memory every round.
+__device__ __noinline__ int topk_large(const DecodeParams& p, const float* zs) {
+  const int lane = threadIdx.x & 31;
+  int my_e = -1;
+  uint32_t taken = 0;
+  for (int i = 0; i < p.K; ++i) {
+    uint64_t best = 0;
+    for (int k = 0; lane + 32 * k < p.E; ++k)
+      if (!((taken >> k) & 1u)) {
+        const uint64_t kk = route_key(zs[lane + 32 * k], lane + 32 * k);
+        best = kk > best ? kk : best;
+      }
+    for (int off = 16; off >= 1; off >>= 1) {
+      const uint64_t o = shfl_xor_u64(best, off);
+      best = o > best ? o : best;
+    }
+    const int e = (int)(~(uint32_t)best);
+    if ((best >> 32) == 0ull && lane == 0) set_error(p.ctrl, MOE_DEVERR_ROUTE);
+    if ((e & 31) == lane) taken |= 1u << (e >> 5);
+    if (lane == i) my_e = e;
+  }
+  return my_e;
+}
+
 // Warp 0: top-k of z (value desc, index asc) and the renormalised softmax weights.
 // Keys live in registers (E <= 256: 8 per lane); each round is a lane-local max and a
 // 64-bit butterfly max.  Lane i returns the expert of rank i (and m.sel / m.w are set).
@@ -391,25 +474,8 @@ __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
         if (lane + 32 * k == e) ord[k] = 0u;
       if (lane == i) my_e = e;
     }
-  } else {  // large expert counts: keys re-read from shared memory every round
-    uint32_t taken = 0;
-    for (int i = 0; i < p.K; ++i) {
-      uint64_t best = 0;
-      for (int k = 0; lane + 32 * k < E; ++k)
-        if (!((taken >> k) & 1u)) {
-          const uint64_t kk = route_key(zs[lane + 32 * k], lane + 32 * k);
-          best = kk > best ? kk : best;
-        }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const uint64_t o = shfl_xor_u64(best, off);
-        best = o > best ? o : best;
-      }
-      const int e = (int)(~(uint32_t)best);
-      if ((best >> 32) == 0ull && lane == 0) set_error(p.ctrl, MOE_DEVERR_ROUTE);
-      if ((e & 31) == lane) taken |= 1u << (e >> 5);
-      if (lane == i) my_e = e;
-    }
+  } else {
+    my_e = topk_large(p, zs);
   }
   if (my_e < 0 || my_e >= E) my_e = 0;  // lanes >= k (and a failed route)
   const float zmax = __shfl_sync(0xffffffffu, zs[my_e], 0);
@@ -419,7 +485,7 @@ __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
   for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   if (lane < p.K) {
     m.sel[lane] = my_e;
-    m.w[lane] = ex / sum;
+    m.w[lane] = __fdividef(ex, sum);
   }
   __syncwarp();
   return my_e;
@@ -428,7 +494,7 @@ __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
 // Thread 0 of every CTA: the cache decision for layer l (identical in all CTAs), from
 // the layer's pinned-slot row and ring state staged in shared memory.  CTA 0 also
 // commits the next ring state, the event log, histogram, counters and miss requests.
-__device__ void cache_decide(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow) {
+__device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow) {
   const int R = p.R, K = p.K;
   const int par = m.step & 1;
   const bool commit = blockIdx.x == 0;
@@ -546,6 +612,13 @@ __device__ void cache_decide(const DecodeParams& p, Misc& m, int l, const int32_
   }
 }
 
+// Layer 0's router partials over chunk c from global router weights (once per launch).
+__device__ __noinline__ void prologue_partials(const DecodeParams& p, Misc& m, int c, int k, bool has_gain) {
+  router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
+    return reinterpret_cast<const uint4*>(p.router + ((size_t)c * p.E + e) * kChunk);
+  });
+}
+
 // Warp 0: the common case where every selected expert is pinned; lane i handles rank
 // i.  Returns false (nothing written) when some expert is not pinned.
 __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow, int my_e) {
@@ -603,7 +676,7 @@ __device__ bool issue_unit(const DecodeParams& p, Misc& m, uint8_t* unit, int u)
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
     mbar_expect_tx(&m.bar_u[st], tb);
-    bulk_g2s(unit + st * tb, src + st * tb, tb, &m.bar_u[st]);
+    bulk_g2s_stream(unit + st * tb, src + st * tb, tb, &m.bar_u[st]);
   }
   return true;
 }
@@ -620,7 +693,7 @@ __device__ bool issue_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c
     const int Ii = i < p.K ? p.I : p.Is;
     const SlotLayout& L = i < p.K ? p.lay : p.slay;
     const uint32_t tb = 9u * Ii;
-    bulk_g2s(dch + off, m.src[i] + L.down + (size_t)c * tb, tb, &m.bar_d);
+    bulk_g2s_stream(dch + off, m.src[i] + L.down + (size_t)c * tb, tb, &m.bar_d);
     off += tb;
   }
   return true;
@@ -628,6 +701,7 @@ __device__ bool issue_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c
 
 // ------------------------------------------------------------------ the kernel
 
+template <int BPL>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const SmemPlan S = smem_plan(p.H, p.E, p.K, p.I, p.Is, p.nown);
@@ -680,9 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (p.h_trace) p.h_trace[c * kChunk + tid] = v;
     }
     __syncthreads();
-    router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
-      return reinterpret_cast<const uint4*>(p.router + ((size_t)c * p.E + e) * kChunk);
-    });
+    prologue_partials(p, m, c, k, has_gain);
     __syncthreads();
   }
   if (!grid_sync(p, m)) return;
@@ -697,8 +769,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       mbar_expect_tx(&m.bar_r, 32u * p.E * n_own);
       for (int k = 0; k < n_own; ++k) {
         const int c = blockIdx.x + k * gridDim.x;
-        bulk_g2s(rch + (size_t)k * 32u * p.E, p.router + (((size_t)(l + 1) * p.nch + c) * p.E) * kChunk,
-                 32u * p.E, &m.bar_r);
+        bulk_g2s_stream(rch + (size_t)k * 32u * p.E, p.router + (((size_t)(l + 1) * p.nch + c) * p.E) * kChunk,
+                        32u * p.E, &m.bar_r);
       }
     }
     // stage this layer's inputs: every load of the phase is issued before any is used
@@ -748,6 +820,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         if (lane == 0) __stcg(p.z + e, fmaf(sum, inv, p.bias ? __ldg(p.bias + (size_t)l * p.E + e) : 0.0f));
       }
     }
+    const int n_folders = min((int)gridDim.x, (p.E + kWarps - 1) / kWarps);  // CTAs holding logits
+    if ((int)blockIdx.x < n_folders) publish(p, &p.ctrl->z_count);
     {
       float4* hb4 = reinterpret_cast<float4*>(hbuf);
       float4* gb4 = reinterpret_cast<float4*>(gbuf);
@@ -766,59 +840,59 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       }
     }
     __syncthreads();
-    // quantised activations x = RMSNorm(h) (or h): one lane per 32-block, int16 codes
+    // quantised activations x = RMSNorm(h) (or h): one lane per 32-block, int16 codes;
+    // a first pass finds the block's largest |x|, a second writes the codes
     if (tid < nb) {
       const int b = tid;
       const float inv = m.inv;
-      float v[32];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 hv = reinterpret_cast<const float4*>(hbuf + b * 32)[q];
-        float4 xv = hv;
+      const float4* h4 = reinterpret_cast<const float4*>(hbuf + b * 32);
+      const float4* g4 = reinterpret_cast<const float4*>(gbuf + b * 32);
+      auto xval = [&](float4 hv, int q) {
         if (p.use_norm) {
-          xv.x = __fmul_rn(hv.x, inv);
-          xv.y = __fmul_rn(hv.y, inv);
-          xv.z = __fmul_rn(hv.z, inv);
-          xv.w = __fmul_rn(hv.w, inv);
+          hv.x = __fmul_rn(hv.x, inv);
+          hv.y = __fmul_rn(hv.y, inv);
+          hv.z = __fmul_rn(hv.z, inv);
+          hv.w = __fmul_rn(hv.w, inv);
           if (has_gain) {
-            const float4 gv = reinterpret_cast<const float4*>(gbuf + b * 32)[q];
-            xv.x = __fmul_rn(xv.x, gv.x);
-            xv.y = __fmul_rn(xv.y, gv.y);
-            xv.z = __fmul_rn(xv.z, gv.z);
-            xv.w = __fmul_rn(xv.w, gv.w);
+            const float4 gv = g4[q];
+            hv.x = __fmul_rn(hv.x, gv.x);
+            hv.y = __fmul_rn(hv.y, gv.y);
+            hv.z = __fmul_rn(hv.z, gv.z);
+            hv.w = __fmul_rn(hv.w, gv.w);
           }
         }
-        v[4 * q] = xv.x;
-        v[4 * q + 1] = xv.y;
-        v[4 * q + 2] = xv.z;
-        v[4 * q + 3] = xv.w;
-      }
+        return hv;
+      };
       float amax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      const float mult = amax > 0.0f ? 32767.0f * __frcp_rn(amax) : 0.0f;
-      int csum = 0;
-      uint32_t w[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int c0 = max(-32767, min(32767, __float2int_rn(v[2 * j] * mult)));
-        const int c1 = max(-32767, min(32767, __float2int_rn(v[2 * j + 1] * mult)));
-        csum += c0 + c1;
-        w[j] = ((uint32_t)c0 & 0xffffu) | ((uint32_t)c1 << 16);
+#pragma unroll 2
+      for (int q = 0; q < 8; ++q) {
+        const float4 xv = xval(h4[q], q);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(xv.x), fabsf(xv.y)), fmaxf(fabsf(xv.z), fabsf(xv.w))));
       }
-      int4* dst = reinterpret_cast<int4*>(xcodes + b * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        dst[q] = make_int4((int)w[4 * q], (int)w[4 * q + 1], (int)w[4 * q + 2], (int)w[4 * q + 3]);
+      const float mult = amax > 0.0f ? __fdividef(32767.0f, amax) : 0.0f;
+      int csum = 0;
+      uint2* dst = reinterpret_cast<uint2*>(xcodes + b * 32);
+#pragma unroll 2
+      for (int q = 0; q < 8; ++q) {
+        const float4 xv = xval(h4[q], q);
+        const int c0 = max(-32767, min(32767, __float2int_rn(xv.x * mult)));
+        const int c1 = max(-32767, min(32767, __float2int_rn(xv.y * mult)));
+        const int c2 = max(-32767, min(32767, __float2int_rn(xv.z * mult)));
+        const int c3 = max(-32767, min(32767, __float2int_rn(xv.w * mult)));
+        csum += c0 + c1 + c2 + c3;
+        dst[q] = make_uint2(((uint32_t)c0 & 0xffffu) | ((uint32_t)c1 << 16),
+                            ((uint32_t)c2 & 0xffffu) | ((uint32_t)c3 << 16));
+      }
       xs[b] = amax * (1.0f / (32767.0f * 16.0f));
       xc[b] = csum;
     }
-    if (!grid_sync(p, m)) return;
+    __syncthreads();
     stamp(p, l, 1);
 
     // ---------------------------------------------------------------- routing
+    if (!await_count(p, m, &p.ctrl->z_count, (uint32_t)(l + 1) * n_folders)) return;
     for (int e = tid; e < p.E; e += kThreads) zs[e] = __ldcg(p.z + e);
-    __syncthreads();
+    if (!cta_ok(p, m.flag)) return;
     stamp(p, l, 8);
     if (warp == 0) {
       const int my_e = topk_weights(p, m, zs);
@@ -840,16 +914,16 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
 
     // ---------------------------------------------------------------- G phase
     {
+      // lane groups of GS lanes per row; each lane covers BPL blocks of the row
       const int GS = pow2_ceil_le32(nb), RPW = 32 / GS, g = lane % GS, sub = lane / GS;
-      const int bpl = (nb + GS - 1) / GS;
       const int rows_per_lane = (2 * kUnitRows + kWarps * RPW - 1) / (kWarps * RPW);
-      int4 xq[4][4];
-      float xsc[4];
-      int xsum[4];
+      int4 xq[BPL][4];
+      float xsc[BPL];
+      int xsum[BPL];
 #pragma unroll
-      for (int mb = 0; mb < 4; ++mb) {
+      for (int mb = 0; mb < BPL; ++mb) {
         const int b = g + GS * mb;
-        if (mb < bpl && b < nb) {
+        if (b < nb) {
           const int4* src = reinterpret_cast<const int4*>(xcodes + b * 32);
           xq[mb][0] = src[0];
           xq[mb][1] = src[1];
@@ -897,9 +971,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           }
           stamp(p, l, 7);
 #pragma unroll
-          for (int mb = 0; mb < 4; ++mb) {
+          for (int mb = 0; mb < BPL; ++mb) {
             const int b = g + GS * mb;
-            if (!(mb < bpl && b < nb)) continue;
+            if (b >= nb) continue;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               if (!live[q]) continue;
@@ -923,40 +997,49 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         }
 #pragma unroll
         for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
+        stamp(p, l, 16);
         __syncthreads();
+        stamp(p, l, 17);
         if (warp == 0) {
           const float gv = m.gu[lane], uv = m.gu[kUnitRows + lane];
-          const float a = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
+          const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+          stamp(p, l, 18);
           float sc;
           int csum;
           const int code = quant_block(a, sc, csum);
+          stamp(p, l, 19);
           uint8_t* rec = p.acodes + ((size_t)i * rec_per_exp + rb) * kACodeBytes;
           __stcg(reinterpret_cast<int16_t*>(rec) + lane, (int16_t)code);
           if (lane == 0) {
             __stcg(reinterpret_cast<float*>(rec + 64), sc);
             __stcg(reinterpret_cast<int32_t*>(rec + 68), csum);
           }
+          stamp(p, l, 20);
         }
       }
     }
-    // the owned chunk's down tiles load while the grid waits for the slowest unit
+    const int n_producers = min((int)gridDim.x, p.n_units);  // CTAs holding gate/up units
+    stamp(p, l, 21);
+    // the owned chunk's down tiles (resident experts) load while the other units finish
     if (tid == 0 && n_own > 0) {
       bool layer_misses = false;
       for (int i = 0; i < p.n_exp; ++i) layer_misses |= m.miss_seq[i] != 0;
       if (!layer_misses) m.d_issued = issue_dchunk(p, m, dch, blockIdx.x) ? 1 : 0;
     }
+    if ((int)blockIdx.x < n_producers) publish(p, &p.ctrl->a_count);
     stamp(p, l, 3);
-    if (!grid_sync(p, m)) return;
     stamp(p, l, 4);
 
     // ---------------------------------------------------------------- D phase
-    {
-      const int n_rec = p.n_exp * rec_per_exp * (kACodeBytes / 8);
-      const uint2* srcr = reinterpret_cast<const uint2*>(p.acodes);
-      uint2* dstr = reinterpret_cast<uint2*>(acs);
-      for (int t = tid; t < n_rec; t += kThreads) dstr[t] = __ldcg(srcr + t);
+    // gather every activation record of this layer (CTAs that own rows)
+    if (n_own > 0) {
+      if (!await_count(p, m, &p.ctrl->a_count, (uint32_t)(l + 1) * n_producers)) return;
+      const int n_vec = p.n_exp * rec_per_exp * (kACodeBytes / 16);
+      const uint4* srcr = reinterpret_cast<const uint4*>(p.acodes);
+      uint4* dstr = reinterpret_cast<uint4*>(acs);
+      for (int t = tid; t < n_vec; t += kThreads) dstr[t] = __ldcg(srcr + t);
     }
-    __syncthreads();
+    if (!cta_ok(p, m.flag)) return;
     stamp(p, l, 13);
     for (int k = 0; k < n_own; ++k) {
       const int c = blockIdx.x + k * gridDim.x;
@@ -966,31 +1049,64 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (!mbar_wait(p, &m.bar_d, par_d)) return;
       par_d ^= 1u;
       stamp(p, l, 14);
-      // thread (row r, block column b0): every expert's blocks b0, b0+16, ... of row r
+      // thread (expert i, block column b0): the 16 rows of chunk c against blocks b0,
+      // b0+16, ... of a_i, rows independent; then a 15-shuffle transpose reduction over
+      // the 16 lanes of the expert leaves row b0's sum in lane b0
       {
-        const int r = tid >> 4, b0 = tid & 15;
-        uint32_t off = 0;
-#pragma unroll 3
-        for (int i = 0; i < p.n_exp; ++i) {
-          const int Ii = i < p.K ? p.I : p.Is;
+        const int b0 = tid & 15;
+        // warp-uniform loop: lanes 0-15 take expert base, lanes 16-31 expert base + 1
+        for (int base = 2 * warp; base < p.n_exp; base += 2 * kWarps) {
+          const int i = base + (lane >> 4);
+          const bool act = i < p.n_exp;
+          const int Ii = !act ? 0 : (i < p.K ? p.I : p.Is);
           const int nbd = Ii / 32;
-          const uint8_t* qbase = dch + off;
-          const __half* dbase = reinterpret_cast<const __half*>(dch + off + 8u * Ii);
-          float acc = 0.0f;
-          for (int b = b0; b < nbd; b += 16) {
-            const uint8_t* rec = acs + ((size_t)i * rec_per_exp + b) * kACodeBytes;
-            const int4* ap = reinterpret_cast<const int4*>(rec);
-            const uint4 qv = *reinterpret_cast<const uint4*>(qbase + ((size_t)r * nbd + b) * 16);
-            const float d = __half2float(dbase[(size_t)r * nbd + b]);
-            const float sc = reinterpret_cast<const float*>(rec + 64)[0];
-            const int cs = reinterpret_cast<const int32_t*>(rec + 68)[0];
-            const int v = q4_block_dot16(qv, ap[0], ap[1], ap[2], ap[3]) - 128 * cs;
-            acc = fmaf(d * sc, (float)v, acc);
-          }
+          const uint8_t* qbase = dch + 9u * (i < p.K ? (uint32_t)i * p.I : (uint32_t)p.K * p.I);
+          const __half* dbase = reinterpret_cast<const __half*>(qbase + 8u * Ii);
+          const int4* ap = nullptr;
+          int4 a0 = make_int4(0, 0, 0, 0), a1 = a0, a2 = a0, a3 = a0;
+          float sc = 0.0f;
+          int cs128 = 0;
+#pragma unroll 1
+          for (int rg = 0; rg < kChunk / 4; ++rg) {  // four rows at a time
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int b = b0; b < nbd; b += 16) {
+              if (b != b0 || rg == 0 || nbd > 16) {
+                const uint8_t* rec = acs + ((size_t)i * rec_per_exp + b) * kACodeBytes;
+                ap = reinterpret_cast<const int4*>(rec);
+                a0 = ap[0];
+                a1 = ap[1];
+                a2 = ap[2];
+                a3 = ap[3];
+                sc = reinterpret_cast<const float*>(rec + 64)[0];
+                cs128 = 128 * reinterpret_cast<const int32_t*>(rec + 68)[0];
+              }
 #pragma unroll
-          for (int o2 = 8; o2 >= 1; o2 >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o2);
-          if (b0 == 0) os[i * kChunk + r] = acc;
-          off += 9u * Ii;
+              for (int q = 0; q < 4; ++q) {
+                const int r = 4 * rg + q;
+                const uint4 qv = *reinterpret_cast<const uint4*>(qbase + ((size_t)r * nbd + b) * 16);
+                const float d = __half2float(dbase[(size_t)r * nbd + b]);
+                const int v = q4_block_dot16(qv, a0, a1, a2, a3) - cs128;
+                acc[q] = fmaf(d * sc, (float)v, acc[q]);
+              }
+            }
+            // transpose reduction of 4 rows over the expert's 16 lanes: lane b0 ends with
+            // the sum of row 4 rg + 2 (b0 >> 3 & 1) + (b0 >> 2 & 1)
+            const bool up8 = (b0 & 8) != 0, up4 = (b0 & 4) != 0;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const float send = up8 ? acc[q] : acc[q + 2];
+              const float keep = up8 ? acc[q + 2] : acc[q];
+              acc[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+            }
+            {
+              const float send = up4 ? acc[0] : acc[1];
+              const float keep = up4 ? acc[1] : acc[0];
+              acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+            }
+            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
+            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
+            if (act && (b0 & 3) == 0) os[i * kChunk + 4 * rg + 2 * (up8 ? 1 : 0) + (up4 ? 1 : 0)] = acc[0];
+          }
         }
       }
       __syncthreads();
@@ -1041,14 +1157,33 @@ uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown) {
   return smem_plan(H, E, K, I, Is, nown).total;
 }
 
+// Blocks of one gate/up row each lane covers: 1 below 1024 columns, else H / 1024.
+static int bpl_of(int H) {
+  const int nb = H / 32;
+  return nb <= 32 ? 1 : (nb + 31) / 32;
+}
+
+template <typename F>
+static cudaError_t with_kernel(int H, F f) {
+  switch (bpl_of(H)) {
+    case 1: return f(moe_decode_kernel<1>);
+    case 2: return f(moe_decode_kernel<2>);
+    case 3: return f(moe_decode_kernel<3>);
+    default: return f(moe_decode_kernel<4>);
+  }
+}
+
 cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown) {
   const uint32_t bytes = decode_smem_bytes(H, E, K, I, Is, nown);
-  return cudaFuncSetAttribute(moe_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return with_kernel(H, [&](auto kern) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  });
 }
 
 cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int nown, int* out) {
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, moe_decode_kernel, kThreads,
-                                                       decode_smem_bytes(H, E, K, I, Is, nown));
+  return with_kernel(H, [&](auto kern) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, decode_smem_bytes(H, E, K, I, Is, nown));
+  });
 }
 
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) {
@@ -1062,7 +1197,7 @@ cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_decode_kernel, p);
+  return with_kernel(p.H, [&](auto kern) { return cudaLaunchKernelEx(&cfg, kern, p); });
 }
 
 }  // namespace moe

@@ -214,7 +214,11 @@ static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cud
   CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
   cudaError_t e = cudaSuccess;
   if (host_io) e = cudaMemcpyAsync(c->x_buf, c->x_pin, sizeof(float) * c->H, cudaMemcpyHostToDevice, c->own);
-  if (e == cudaSuccess) e = cudaMemsetAsync(&c->ctrl->bar_count, 0, sizeof(uint32_t), c->own);
+  // the launch's arrival counters (grid barrier, logits, activation codes) start at 0
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(&c->ctrl->bar_count, 0,
+                        reinterpret_cast<char*>(&c->ctrl->a_count + 1) - reinterpret_cast<char*>(&c->ctrl->bar_count),
+                        c->own);
   if (e == cudaSuccess) e = decode_launch(make_params(c, x, y), c->grid, c->own);
   if (e == cudaSuccess && host_io)
     e = cudaMemcpyAsync(c->y_pin, c->y_buf, sizeof(float) * c->H, cudaMemcpyDeviceToHost, c->own);
@@ -604,7 +608,7 @@ int moe_clear_error(moe_ctx* c) {
   const uint32_t last = c->proxy_next.load() - 1;
   ctl.req_seq = last;
   ctl.error = 0;
-  ctl.bar_count = 0;  // (the graphs zero it before every launch as well)
+  ctl.bar_count = ctl.z_count = ctl.a_count = 0;  // (the graphs zero them before every launch too)
   CK(cudaMemcpy(c->ctrl, &ctl, sizeof(Ctrl), cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->done_seq, &last, sizeof(uint32_t), cudaMemcpyHostToDevice));
   const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);

@@ -71,6 +71,10 @@ struct alignas(128) Ctrl {
   uint32_t pad1[31];
   uint32_t bar_count;  // grid barrier arrivals, zeroed before every launch
   uint32_t pad2[31];
+  uint32_t z_count;  // CTAs that have published this launch's logits, per layer (zeroed per launch)
+  uint32_t pad3[31];
+  uint32_t a_count;  // CTAs that have published this launch's activation codes (zeroed per launch)
+  uint32_t pad4[31];
   unsigned long long pin_hits, ring_hits, misses, evictions, staged;
 };
 
@@ -110,7 +114,7 @@ struct DecodeParams {
   float* part;     // [E][nch]
   float* sq;       // [nch]
   float* z;        // [E]
-  uint8_t* acodes; // [n_exp][Imax/32][kACodeBytes]
+  uint8_t* acodes;  // [n_exp][Imax/32][kACodeBytes]
   // stats
   uint32_t* hist;  // [L][E]
   int32_t* log;    // [log_steps][L][K][7]

@@ -168,7 +168,7 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
   p.timeout_ns = (unsigned long long)(cfg->wait_timeout_ms ? cfg->wait_timeout_ms : 2000) * 1000000ull;
   p.phase_trace = nullptr;
 
-  // start from a clean control block (step 0, no error, barrier word 0) every call
+  // start from a clean control block (step 0, no error, arrival counters 0) every call
   if (cudaMemsetAsync(base + cv.ctrl, 0, sizeof(Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
   resident_tables<<<(L * E + 255) / 256, 256, 0, st>>>(reinterpret_cast<int32_t*>(base + cv.pin),
                                                        reinterpret_cast<int32_t*>(base + cv.base),
