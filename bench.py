@@ -243,10 +243,14 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         m.set_residency(1.0)
         t100, per100, st100 = timed()
-        m.set_residency(0.6, hist, moe.MOE_PLACE_CALIBRATED)
-        t60, per60, st60 = timed()
-        m.set_residency(0.6, hist, moe.MOE_PLACE_UNIFORM)
-        t60u, per60u, st60u = timed()
+        if args.phases == "all":
+            m.set_residency(0.6, hist, moe.MOE_PLACE_CALIBRATED)
+            t60, per60, st60 = timed()
+            m.set_residency(0.6, hist, moe.MOE_PLACE_UNIFORM)
+            t60u, per60u, st60u = timed()
+        else:  # full residency only: no miss copies (profilers serialise the proxy's copies)
+            t60, per60, st60 = t100, per100, st100
+            t60u, per60u, st60u = t100, per100, st100
 
     # host-to-device bandwidth for one expert slot from pinned memory (the miss copy)
     src = torch.empty(slot_bytes, dtype=torch.uint8).pin_memory()
@@ -315,7 +319,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": 4 * shape.hidden, "d2h_bytes_per_step": 4 * shape.hidden + 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
-        "setup": {"load_s": load_s},
+        "setup": {"load_s": load_s, "phases": args.phases},
     }
     m.close()
     del m
@@ -340,6 +344,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
+    ap.add_argument("--phases", default="all", choices=["all", "100"],
+                    help="'100' times full residency only (no miss copies), for profiler runs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

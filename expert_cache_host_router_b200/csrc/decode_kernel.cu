@@ -226,7 +226,6 @@ __host__ __device__ inline int pow2_ceil_le32(int n) {
 
 struct Misc {
   uint64_t bar_u[4];  // gate/up unit, four 16-row stages
-  uint64_t bar_d;     // down rows of the owned chunk
   uint64_t bar_r;     // next layer's router columns of the owned chunks
   const uint8_t* src[kMaxK + 1];  // slot base of each active expert (rank order, then shared)
   uint32_t miss_seq[kMaxK + 1];   // copy to wait for (0: resident)
@@ -681,22 +680,35 @@ __device__ bool issue_unit(const DecodeParams& p, Misc& m, uint8_t* unit, int u)
   return true;
 }
 
-// Thread 0: bulk-load the down tile of chunk c of every active expert (one copy each).
-__device__ bool issue_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c) {
-  for (int i = 0; i < p.n_exp; ++i)
-    if (!wait_miss(p, m.miss_seq[i])) return false;
-  uint32_t total = 0;
-  for (int i = 0; i < p.n_exp; ++i) total += 9u * (i < p.K ? p.I : p.Is);
-  mbar_expect_tx(&m.bar_d, total);
-  uint32_t off = 0;
-  for (int i = 0; i < p.n_exp; ++i) {
-    const int Ii = i < p.K ? p.I : p.Is;
+// All threads: copy the down tile of chunk c of every active expert into shared memory
+// with 16-byte cp.async copies (about ten per thread), L2 evict-first.  The caller has
+// made sure the miss copies these tiles depend on have landed.
+__device__ void load_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c) {
+  const uint64_t pol = l2_evict_first_policy();
+  const uint32_t t_r = 9u * p.I, t_s = 9u * p.Is;  // tile bytes of a routed / the shared expert
+  const uint32_t routed_bytes = (uint32_t)p.K * t_r, total = routed_bytes + (p.Is > 0 ? t_s : 0);
+  for (uint32_t off = 16u * threadIdx.x; off < total; off += 16u * kThreads) {
+    const int i = off < routed_bytes ? (int)(off / t_r) : p.K;
+    const uint32_t in_tile = off < routed_bytes ? off - (uint32_t)i * t_r : off - routed_bytes;
     const SlotLayout& L = i < p.K ? p.lay : p.slay;
-    const uint32_t tb = 9u * Ii;
-    bulk_g2s_stream(dch + off, m.src[i] + L.down + (size_t)c * tb, tb, &m.bar_d);
-    off += tb;
+    const uint8_t* src = m.src[i] + L.down + (size_t)c * (i < p.K ? t_r : t_s) + in_tile;
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dch + off)), "l"(src),
+                 "l"(pol)
+                 : "memory");
   }
-  return true;
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Thread 0: bulk-load layer lr's router columns of the owned chunks into rch.
+__device__ void prefetch_router(const DecodeParams& p, Misc& m, uint8_t* rch, int lr, int n_own) {
+  mbar_expect_tx(&m.bar_r, 32u * p.E * n_own);
+  for (int k = 0; k < n_own; ++k) {
+    const int c = blockIdx.x + k * gridDim.x;
+    bulk_g2s_stream(rch + (size_t)k * 32u * p.E, p.router + (((size_t)lr * p.nch + c) * p.E) * kChunk, 32u * p.E,
+                    &m.bar_r);
+  }
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -729,7 +741,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
 
   if (tid == 0) {
     for (int b = 0; b < 4; ++b) mbar_init(&m.bar_u[b], 1);
-    mbar_init(&m.bar_d, 1);
     mbar_init(&m.bar_r, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     m.step = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->step);
@@ -740,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   }
   __syncthreads();
   if (!m.flag) return;
-  uint32_t par_u[4] = {0, 0, 0, 0}, par_d = 0, par_r = 0;  // mbarrier parities (uniform)
+  uint32_t par_u[4] = {0, 0, 0, 0}, par_r = 0;  // mbarrier parities (uniform)
   stamp(p, p.L, 0);
 
   // ---- prologue: h = x on the owned rows, and layer 0's router partials
@@ -757,6 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     prologue_partials(p, m, c, k, has_gain);
     __syncthreads();
   }
+  if (tid == 0 && p.L > 1 && n_own > 0) prefetch_router(p, m, rch, 1, n_own);
   if (!grid_sync(p, m)) return;
   stamp(p, p.L, 1);
 
@@ -764,15 +776,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     stamp(p, l, 0);
     const bool next = l + 1 < p.L;
     // ---------------------------------------------------------------- R phase
-    // prefetch the next layer's router columns of the owned chunks (bulk copies)
-    if (tid == 0 && next && n_own > 0) {
-      mbar_expect_tx(&m.bar_r, 32u * p.E * n_own);
-      for (int k = 0; k < n_own; ++k) {
-        const int c = blockIdx.x + k * gridDim.x;
-        bulk_g2s_stream(rch + (size_t)k * 32u * p.E, p.router + (((size_t)(l + 1) * p.nch + c) * p.E) * kChunk,
-                        32u * p.E, &m.bar_r);
-      }
-    }
     // stage this layer's inputs: every load of the phase is issued before any is used
     float4 hreg[4], greg[4];
     int32_t preg[4];
@@ -840,51 +843,64 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       }
     }
     __syncthreads();
-    // quantised activations x = RMSNorm(h) (or h): one lane per 32-block, int16 codes;
-    // a first pass finds the block's largest |x|, a second writes the codes
-    if (tid < nb) {
-      const int b = tid;
+    // quantised activations x = RMSNorm(h) (or h): four lanes per 32-block, each lane 8
+    // values; the block's largest |x| and code sum combine over the four lanes
+    {
       const float inv = m.inv;
-      const float4* h4 = reinterpret_cast<const float4*>(hbuf + b * 32);
-      const float4* g4 = reinterpret_cast<const float4*>(gbuf + b * 32);
-      auto xval = [&](float4 hv, int q) {
-        if (p.use_norm) {
-          hv.x = __fmul_rn(hv.x, inv);
-          hv.y = __fmul_rn(hv.y, inv);
-          hv.z = __fmul_rn(hv.z, inv);
-          hv.w = __fmul_rn(hv.w, inv);
-          if (has_gain) {
-            const float4 gv = g4[q];
-            hv.x = __fmul_rn(hv.x, gv.x);
-            hv.y = __fmul_rn(hv.y, gv.y);
-            hv.z = __fmul_rn(hv.z, gv.z);
-            hv.w = __fmul_rn(hv.w, gv.w);
+      const int j4 = tid & 3;
+      for (int b0 = tid >> 2; b0 < ((nb + 63) / 64) * 64; b0 += kThreads / 4) {
+        const int b = b0 < nb ? b0 : nb - 1;  // lanes past the end repeat a block, write nothing
+        float v[8];
+        const float4* h4 = reinterpret_cast<const float4*>(hbuf + b * 32 + 8 * j4);
+        const float4* g4 = reinterpret_cast<const float4*>(gbuf + b * 32 + 8 * j4);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float4 hv = h4[q];
+          if (p.use_norm) {
+            hv.x = __fmul_rn(hv.x, inv);
+            hv.y = __fmul_rn(hv.y, inv);
+            hv.z = __fmul_rn(hv.z, inv);
+            hv.w = __fmul_rn(hv.w, inv);
+            if (has_gain) {
+              const float4 gv = g4[q];
+              hv.x = __fmul_rn(hv.x, gv.x);
+              hv.y = __fmul_rn(hv.y, gv.y);
+              hv.z = __fmul_rn(hv.z, gv.z);
+              hv.w = __fmul_rn(hv.w, gv.w);
+            }
+          }
+          v[4 * q] = hv.x;
+          v[4 * q + 1] = hv.y;
+          v[4 * q + 2] = hv.z;
+          v[4 * q + 3] = hv.w;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(v[q]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float mult = amax > 0.0f ? __fdividef(32767.0f, amax) : 0.0f;
+        int c[8];
+        int csum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          c[q] = max(-32767, min(32767, __float2int_rn(v[q] * mult)));
+          csum += c[q];
+        }
+        csum += __shfl_xor_sync(0xffffffffu, csum, 1);
+        csum += __shfl_xor_sync(0xffffffffu, csum, 2);
+        if (b0 < nb) {
+          reinterpret_cast<uint4*>(xcodes + b * 32)[j4] =
+              make_uint4(((uint32_t)c[0] & 0xffffu) | ((uint32_t)c[1] << 16),
+                         ((uint32_t)c[2] & 0xffffu) | ((uint32_t)c[3] << 16),
+                         ((uint32_t)c[4] & 0xffffu) | ((uint32_t)c[5] << 16),
+                         ((uint32_t)c[6] & 0xffffu) | ((uint32_t)c[7] << 16));
+          if (j4 == 0) {
+            xs[b] = amax * (1.0f / (32767.0f * 16.0f));
+            xc[b] = csum;
           }
         }
-        return hv;
-      };
-      float amax = 0.0f;
-#pragma unroll 2
-      for (int q = 0; q < 8; ++q) {
-        const float4 xv = xval(h4[q], q);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(xv.x), fabsf(xv.y)), fmaxf(fabsf(xv.z), fabsf(xv.w))));
       }
-      const float mult = amax > 0.0f ? __fdividef(32767.0f, amax) : 0.0f;
-      int csum = 0;
-      uint2* dst = reinterpret_cast<uint2*>(xcodes + b * 32);
-#pragma unroll 2
-      for (int q = 0; q < 8; ++q) {
-        const float4 xv = xval(h4[q], q);
-        const int c0 = max(-32767, min(32767, __float2int_rn(xv.x * mult)));
-        const int c1 = max(-32767, min(32767, __float2int_rn(xv.y * mult)));
-        const int c2 = max(-32767, min(32767, __float2int_rn(xv.z * mult)));
-        const int c3 = max(-32767, min(32767, __float2int_rn(xv.w * mult)));
-        csum += c0 + c1 + c2 + c3;
-        dst[q] = make_uint2(((uint32_t)c0 & 0xffffu) | ((uint32_t)c1 << 16),
-                            ((uint32_t)c2 & 0xffffu) | ((uint32_t)c3 << 16));
-      }
-      xs[b] = amax * (1.0f / (32767.0f * 16.0f));
-      xc[b] = csum;
     }
     __syncthreads();
     stamp(p, l, 1);
@@ -1020,11 +1036,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     }
     const int n_producers = min((int)gridDim.x, p.n_units);  // CTAs holding gate/up units
     stamp(p, l, 21);
-    // the owned chunk's down tiles (resident experts) load while the other units finish
-    if (tid == 0 && n_own > 0) {
+    // the owned chunk's down tiles (all resident) load while the other units finish
+    if (n_own > 0) {
       bool layer_misses = false;
       for (int i = 0; i < p.n_exp; ++i) layer_misses |= m.miss_seq[i] != 0;
-      if (!layer_misses) m.d_issued = issue_dchunk(p, m, dch, blockIdx.x) ? 1 : 0;
+      if (!layer_misses) {
+        load_dchunk(p, m, dch, blockIdx.x);
+        if (tid == 0) m.d_issued = 1;
+      }
     }
     if ((int)blockIdx.x < n_producers) publish(p, &p.ctrl->a_count);
     stamp(p, l, 3);
@@ -1043,11 +1062,18 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     stamp(p, l, 13);
     for (int k = 0; k < n_own; ++k) {
       const int c = blockIdx.x + k * gridDim.x;
-      if (tid == 0 && !(k == 0 && m.d_issued)) m.flag = issue_dchunk(p, m, dch, c);
+      if (!(k == 0 && m.d_issued)) {  // tiles not loaded yet (misses in the layer, or chunk > 0)
+        if (tid == 0) {
+          m.flag = 1;
+          for (int i = 0; i < p.n_exp; ++i)
+            if (!wait_miss(p, m.miss_seq[i])) m.flag = 0;
+        }
+        __syncthreads();
+        if (!m.flag) return;
+        load_dchunk(p, m, dch, c);
+      }
+      cp_async_wait_all();
       __syncthreads();
-      if (!(k == 0 && m.d_issued) && !m.flag) return;
-      if (!mbar_wait(p, &m.bar_d, par_d)) return;
-      par_d ^= 1u;
       stamp(p, l, 14);
       // thread (expert i, block column b0): the 16 rows of chunk c against blocks b0,
       // b0+16, ... of a_i, rows independent; then a 15-shuffle transpose reduction over
@@ -1131,6 +1157,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       __syncthreads();
     }
     if (next && n_own > 0) par_r ^= 1u;
+    // the router columns for layer l + 2 load during the barrier (rch is free again)
+    if (tid == 0 && l + 2 < p.L && n_own > 0) prefetch_router(p, m, rch, l + 2, n_own);
     stamp(p, l, 5);
     if (!grid_sync(p, m)) return;
     stamp(p, l, 6);
