@@ -31,6 +31,10 @@ import synthetic  # noqa: E402
 
 METRIC = "MoE decode tok/s at 100%/60% expert residency; fraction of HBM/PCIe roofline"
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
+# 4-layer case scaled by 10 (profiles/moe_decode_kernel_4layer_ncu.md), valid only for
+# the kernel source it was taken on; any other source reports null.
+TRAFFIC_REF = {"kernel_sha256_prefix": "2b7e9969101cd83f", "bytes_per_launch": 712.46592e6}
 WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
             "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
             "residency + 8-slot LRU ring (residency_60)")
@@ -48,6 +52,16 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_per_launch(n_layers: int):
+    import hashlib
+    src = os.path.join(ROOT, "expert_cache_host_router_b200", "csrc", "decode_kernel.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if sha != TRAFFIC_REF["kernel_sha256_prefix"] or n_layers != 40:
+        return None
+    return TRAFFIC_REF["bytes_per_launch"]
 
 
 def active_bytes_per_token(s) -> int:
@@ -312,7 +326,7 @@ def run_ours(args):
                          **c60,
                          "uniform_placement": {"value": value60u, **cache_summary(st60u)}},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "frac": achieved / peak, "traffic": traffic_per_launch(shape.n_layers), "peak_kind": peak_kind,
                      "kernel": "moe_decode_kernel", "bytes_per_launch": bytes_tok,
                      "mean_launch_ms": kern_ms},
         "e2e": {"value": e2e_units / (e2e_ms * 1e-3), "unit": "tok/s",
