@@ -73,7 +73,9 @@ class Stats(ctypes.Structure):
                 ("bytes_copied", ctypes.c_uint64), ("staged_misses", ctypes.c_uint64),
                 ("log_dropped", ctypes.c_uint64), ("device_error", ctypes.c_int32),
                 ("n_pinned", ctypes.c_int32), ("residency", ctypes.c_float),
-                ("placement", ctypes.c_int32)]
+                ("placement", ctypes.c_int32), ("repins", ctypes.c_uint64),
+                ("repin_copies", ctypes.c_uint64), ("miss_requests", ctypes.c_uint64),
+                ("miss_served", ctypes.c_uint64), ("proxy_error", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -92,6 +94,8 @@ _SIGS = {
     "moe_stats": (ctypes.c_int, [_P, ctypes.POINTER(Stats), _P, _P, ctypes.c_size_t,
                                  ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
     "moe_set_trace": (ctypes.c_int, [_P, _P, _P]),
+    "moe_recalibrate": (ctypes.c_int, [_P]),
+    "moe_set_router_bias": (ctypes.c_int, [_P, ctypes.c_int32, _P]),
     "moe_set_phase_trace": (ctypes.c_int, [_P, _P]),
     "moe_debug_drop_signals": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(NoAllocWeights),
@@ -197,6 +201,15 @@ def moe_stats(ctx: int, n_layers: int, n_experts: int, log_cap: int = 0, reset: 
     return st.as_dict(), hist, log[: n.value]
 
 
+def moe_recalibrate(ctx: int) -> None:
+    _check(lib().moe_recalibrate(ctx), "moe_recalibrate")
+
+
+def moe_set_router_bias(ctx: int, layer: int, bias) -> None:
+    b = None if bias is None else _arr(bias, np.float32)
+    _check(lib().moe_set_router_bias(ctx, layer, _ptr(b)), "moe_set_router_bias")
+
+
 def moe_set_trace(ctx: int, h_trace_dev: int | None, w_trace_dev: int | None) -> None:
     _check(lib().moe_set_trace(ctx, h_trace_dev, w_trace_dev), "moe_set_trace")
 
@@ -271,6 +284,12 @@ class ExpertCacheMoE:
 
     def sync(self):
         moe_sync(self.ctx)
+
+    def recalibrate(self) -> None:
+        moe_recalibrate(self.ctx)
+
+    def set_router_bias(self, layer: int, bias) -> None:
+        moe_set_router_bias(self.ctx, layer, bias)
 
     def set_phase_trace(self, stamps=None):
         """stamps: torch int64 [(L+1), 8] on the device, or None."""

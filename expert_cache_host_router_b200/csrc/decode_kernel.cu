@@ -512,10 +512,10 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
     const int ps = pinrow[e];
     int kind, slot_log, evicted = -1, pool_idx;
     uint32_t seq = 0;
-    if (ps >= 0) {
+    if (ps >= 0) {  // (logical slot << 16) | physical slot within the layer's pinned region
       kind = MOE_PIN_HIT;
-      slot_log = ps;
-      pool_idx = base + ps;
+      slot_log = ps >> 16;
+      pool_idx = base + (ps & 0xffff);
       ++n_pin;
     } else {
       int r = -1;
@@ -626,7 +626,7 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
   if (!__all_sync(0xffffffffu, ps >= 0)) return false;
   const bool commit = blockIdx.x == 0;
   if (lane < p.K) {
-    m.src[lane] = p.pool + (size_t)(m.base_l + ps) * p.slot_bytes;
+    m.src[lane] = p.pool + (size_t)(m.base_l + (ps & 0xffff)) * p.slot_bytes;
     m.miss_seq[lane] = 0;
     if (commit) {
       int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * p.K + lane) * 7;
@@ -635,7 +635,7 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
       ev[2] = lane;
       ev[3] = my_e;
       ev[4] = MOE_PIN_HIT;
-      ev[5] = ps;
+      ev[5] = ps >> 16;
       ev[6] = -1;
       atomicAdd(p.hist + (size_t)l * p.E + my_e, 1u);
     }

@@ -68,7 +68,12 @@ struct moe_ctx {
   float *x_pin = nullptr, *y_pin = nullptr;
   int32_t* err_pin = nullptr;
   MissReq *mbox_host = nullptr, *mbox_dev = nullptr;
-  // residency
+  // residency and online recalibration
+  std::vector<int32_t> pin_host;   // [L][E] the device table's entries
+  std::vector<int32_t> phys_owner; // [L][P] expert in each physical pinned slot
+  std::vector<uint32_t> score;     // [L][E] decayed routing counts
+  std::vector<uint32_t> hist_snap; // [L][E] device histogram at the last (re)calibration
+  uint64_t repins = 0, repin_copies = 0;
   bool resident = false;
   float residency = 0.0f;
   int placement = 0, P = 0, staging_base = 0;
@@ -264,6 +269,29 @@ static void repack_expert(const uint8_t* src, uint8_t* dst, const SlotLayout& s,
   repack_rows(src, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + (r % 32) / 16) * t_gu; });
   repack_rows(src + gu, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + 2 + (r % 32) / 16) * t_gu; });
   repack_rows(src + 2 * gu, dst, H, I, [&](int64_t r) { return s.down + (r / 16) * t_d; });
+}
+
+// Placement: top-P experts by count (ties -> lower index), or experts 0..P-1.
+static void top_p_mask(const uint32_t* count, int E, int P, int placement, uint8_t* mask) {
+  std::vector<int> order(E);
+  for (int e = 0; e < E; ++e) {
+    order[e] = e;
+    mask[e] = 0;
+  }
+  if (placement == MOE_PLACE_UNIFORM) {
+    for (int e = 0; e < P; ++e) mask[e] = 1;
+    return;
+  }
+  std::stable_sort(order.begin(), order.end(), [count](int a, int b) { return count[a] > count[b]; });
+  for (int p = 0; p < P; ++p) mask[order[p]] = 1;
+}
+
+static int empty_rings(moe_ctx* c, cudaStream_t s) {
+  const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);
+  CK(cudaMemsetAsync(c->ring_owner, 0xff, nr * 4, s));
+  CK(cudaMemsetAsync(c->ring_stamp, 0, nr * 4, s));
+  CK(cudaMemsetAsync(c->ring_clock, 0, (size_t)2 * c->L * 4, s));
+  return MOE_OK;
 }
 
 // ------------------------------------------------------------------ C ABI
@@ -506,28 +534,27 @@ int moe_set_residency(moe_ctx* c, float fraction, const uint32_t* hist, int32_t 
   }
   uint8_t* pool = c->pool.load();
   std::vector<int32_t> pin((size_t)c->L * c->E, -1), base(c->L), npin(c->L, P);
-  std::vector<int> order(c->E);
+  c->phys_owner.assign((size_t)c->L * std::max(P, 1), -1);
+  std::vector<uint8_t> mask(c->E);
   for (int l = 0; l < c->L; ++l) {
     base[l] = l * (P + c->R);
-    std::vector<uint8_t> mask(c->E, 0);
-    if (placement == MOE_PLACE_UNIFORM) {
-      for (int e = 0; e < P; ++e) mask[e] = 1;
-    } else {
-      for (int e = 0; e < c->E; ++e) order[e] = e;
-      const uint32_t* hl = h.data() + (size_t)l * c->E;
-      std::stable_sort(order.begin(), order.end(), [hl](int a, int b) { return hl[a] > hl[b]; });
-      for (int p = 0; p < P; ++p) mask[order[p]] = 1;
-    }
+    top_p_mask(h.data() + (size_t)l * c->E, c->E, P, placement, mask.data());
     int p = 0;
     for (int e = 0; e < c->E; ++e)
-      if (mask[e]) {
-        pin[(size_t)l * c->E + e] = p;
+      if (mask[e]) {  // logical slot == physical slot == rank in ascending expert order
+        pin[(size_t)l * c->E + e] = (p << 16) | p;
+        c->phys_owner[(size_t)l * std::max(P, 1) + p] = e;
         CK(cudaMemcpyAsync(pool + (size_t)(base[l] + p) * c->slot_bytes,
                            c->host_tier + ((size_t)l * c->E + e) * c->slot_bytes, c->slot_bytes,
                            cudaMemcpyHostToDevice, c->own));
         ++p;
       }
   }
+  c->pin_host = pin;
+  c->repins = c->repin_copies = 0;
+  c->score = h;  // the histogram this placement came from seeds the recalibration score
+  c->hist_snap.assign((size_t)c->L * c->E, 0);
+  CK(cudaMemcpyAsync(c->hist_snap.data(), c->hist, c->hist_snap.size() * 4, cudaMemcpyDeviceToHost, c->own));
   c->staging_base = c->L * (P + c->R);
   CK(cudaMemcpyAsync(c->pin_slot, pin.data(), pin.size() * 4, cudaMemcpyHostToDevice, c->own));
   CK(cudaMemcpyAsync(c->layer_base, base.data(), base.size() * 4, cudaMemcpyHostToDevice, c->own));
@@ -641,6 +668,11 @@ int moe_stats(moe_ctx* c, moe_stats_t* out, uint32_t* hist_out, moe_event* log_o
     out->n_pinned = c->P;
     out->residency = c->residency;
     out->placement = c->placement;
+    out->repins = c->repins;
+    out->repin_copies = c->repin_copies;
+    out->miss_requests = ctl.req_seq;
+    out->miss_served = c->proxy_next.load() - 1;
+    out->proxy_error = c->proxy_err.load();
   }
   if (hist_out)
     CK(cudaMemcpy(hist_out, c->hist, sizeof(uint32_t) * c->L * c->E, cudaMemcpyDeviceToHost));
@@ -666,6 +698,75 @@ int moe_stats(moe_ctx* c, moe_stats_t* out, uint32_t* hist_out, moe_event* log_o
     ctl.pin_hits = ctl.ring_hits = ctl.misses = ctl.evictions = ctl.staged = 0;
     CK(cudaMemcpy(&c->ctrl->pin_hits, &ctl.pin_hits, 5 * sizeof(unsigned long long), cudaMemcpyHostToDevice));
     CK(cudaMemset(c->hist, 0, sizeof(uint32_t) * c->L * c->E));
+    std::fill(c->hist_snap.begin(), c->hist_snap.end(), 0u);  // recalibration windows restart at 0
+  }
+  return MOE_OK;
+}
+
+int moe_recalibrate(moe_ctx* c) {
+  if (!c) return MOE_ERR_INVALID;
+  if (!c->resident) return MOE_ERR_STATE;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  const size_t n = (size_t)c->L * c->E;
+  std::vector<uint32_t> h(n);
+  CK(cudaMemcpy(h.data(), c->hist, n * 4, cudaMemcpyDeviceToHost));
+  for (size_t i = 0; i < n; ++i) {
+    const uint32_t window = h[i] >= c->hist_snap[i] ? h[i] - c->hist_snap[i] : h[i];  // a reset restarts it
+    c->score[i] = (c->score[i] >> 1) + window;
+  }
+  c->hist_snap = h;
+  const int P = c->P, Pw = std::max(P, 1);
+  uint8_t* pool = c->pool.load();
+  std::vector<uint8_t> mask(c->E);
+  std::vector<int> freed, entering;
+  for (int l = 0; l < c->L; ++l) {
+    top_p_mask(c->score.data() + (size_t)l * c->E, c->E, P, MOE_PLACE_CALIBRATED, mask.data());
+    int32_t* row = c->pin_host.data() + (size_t)l * c->E;
+    freed.clear();
+    entering.clear();
+    for (int e = 0; e < c->E; ++e) {
+      if (row[e] >= 0 && !mask[e]) {
+        freed.push_back(row[e] & 0xffff);
+        row[e] = -1;
+      } else if (row[e] < 0 && mask[e]) {
+        entering.push_back(e);
+      }
+    }
+    std::sort(freed.begin(), freed.end());
+    for (size_t k = 0; k < entering.size(); ++k) {  // an entering expert takes a freed slot
+      const int e = entering[k], ph = freed[k];
+      row[e] = ph;
+      c->phys_owner[(size_t)l * Pw + ph] = e;
+      CK(cudaMemcpyAsync(pool + (size_t)(l * (P + c->R) + ph) * c->slot_bytes,
+                         c->host_tier + ((size_t)l * c->E + e) * c->slot_bytes, c->slot_bytes,
+                         cudaMemcpyHostToDevice, c->own));
+      ++c->repin_copies;
+    }
+    int rank = 0;  // logical slots: ranks in ascending expert order
+    for (int e = 0; e < c->E; ++e)
+      if (row[e] >= 0) row[e] = (rank++ << 16) | (row[e] & 0xffff);
+  }
+  CK(cudaMemcpyAsync(c->pin_slot, c->pin_host.data(), n * 4, cudaMemcpyHostToDevice, c->own));
+  const int st = empty_rings(c, c->own);
+  if (st != MOE_OK) return st;
+  CK(cudaStreamSynchronize(c->own));
+  ++c->repins;
+  return MOE_OK;
+}
+
+int moe_set_router_bias(moe_ctx* c, int32_t layer, const float* bias) {
+  if (!c || layer < 0 || layer >= c->L) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  if (bias) {
+    CK(cudaMemcpy(c->bias + (size_t)layer * c->E, bias, sizeof(float) * c->E, cudaMemcpyHostToDevice));
+  } else {
+    CK(cudaMemset(c->bias + (size_t)layer * c->E, 0, sizeof(float) * c->E));
+  }
+  if (bias && !c->has_bias) {
+    c->has_bias = true;  // the kernel now reads the bias table: recapture
+    drop_graphs(c);
   }
   return MOE_OK;
 }

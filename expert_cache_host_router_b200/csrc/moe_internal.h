@@ -97,7 +97,7 @@ struct DecodeParams {
   const float* bias;       // [L][E] or null
   const float* gain;       // [L][H] or null
   // cache tables
-  const int32_t* pin_slot;    // [L][E] pinned index or -1
+  const int32_t* pin_slot;    // [L][E] (logical slot << 16) | physical pinned slot, or -1
   const int32_t* layer_base;  // [L] pool index of the layer's pinned slot 0
   const int32_t* n_pinned;    // [L]
   int32_t* ring_owner;        // [2][L][R]

@@ -72,7 +72,7 @@ Carve carve(int L, int H, int E, int K, int I, int Is) {
 __global__ void resident_tables(int32_t* pin, int32_t* base, int32_t* npin, int L, int E) {
   const int n = L * E;
   for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-    pin[t] = t % E;
+    pin[t] = ((t % E) << 16) | (t % E);  // logical slot == physical slot == expert
     if (t % E == 0) {
       base[t / E] = t;
       npin[t / E] = E;

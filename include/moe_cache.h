@@ -113,6 +113,11 @@ typedef struct {
   int32_t n_pinned;      /* P of the current residency */
   float residency;       /* fraction passed to the last moe_set_residency */
   int32_t placement;     /* policy of the last moe_set_residency */
+  uint64_t repins;       /* moe_recalibrate calls since the last moe_set_residency or create */
+  uint64_t repin_copies; /* experts copied host-to-device by those re-pins */
+  uint64_t miss_requests; /* miss requests the kernel has issued since create */
+  uint64_t miss_served;   /* miss requests the proxy has taken from the mailbox since create */
+  int32_t proxy_error;    /* 1 if the proxy met a malformed request (left unsignalled) */
 } moe_stats_t;
 
 #define MOE_DEVERR_BARRIER 1 /* grid barrier wait ran out */
@@ -140,10 +145,30 @@ MOE_API int moe_load_layer(moe_ctx *ctx, int32_t layer, const uint8_t *const *ex
  * device and synchronises the device.  fraction < 1 needs ring_slots >= 1. */
 MOE_API int moe_set_residency(moe_ctx *ctx, float fraction, const uint32_t *hist, int32_t placement);
 
+/* Online recalibration (the write-up's "self-tunes over time"; key components item 1,
+ * routing frequencies accumulated from real requests).  Off the token graph: call it
+ * between steps, e.g. every 64 tokens.  For every layer and expert, the routing counts
+ * since the previous (re)calibration w (from the library's histogram) update the score
+ * score <- floor(score / 2) + w, the score being seeded by the histogram the current
+ * placement came from; the pinned set becomes the top-P experts by score (ties -> lower
+ * index), P unchanged.  Only experts entering the set are copied (host tier -> the slot
+ * an expert leaving the set frees); every ring is emptied.  Synchronises the device. */
+MOE_API int moe_recalibrate(moe_ctx *ctx);
+
+/* Replace one layer's router bias ([E] fp32 host array; NULL = zero), e.g. to follow
+ * traffic whose popularity has drifted.  Synchronises the device. */
+MOE_API int moe_set_router_bias(moe_ctx *ctx, int32_t layer, const float *bias);
+
 /* One decode step (one token through all L layers) as one graph launch on stream:
  * reads x_dev [H] fp32, writes y_dev [H] fp32 (h_L of the stack, or MoE(x) when
  * use_rmsnorm = 0).  Routing, the histogram, the cache and the event log advance.
- * Asynchronous: device-side failures surface at moe_sync / moe_stats. */
+ * Asynchronous: device-side failures surface at moe_sync / moe_stats.
+ * A step that misses waits inside the kernel for the library's proxy thread to issue
+ * the copy; while such a step is in flight, no other host thread should make a CUDA call
+ * that blocks on the device while holding the driver (a synchronous copy to pageable host
+ * memory is one): the proxy's copy would queue behind it and the step would end with
+ * MOE_ERR_TIMEOUT after wait_timeout_ms.  Synchronise (moe_sync, cudaStreamSynchronize)
+ * before such calls. */
 MOE_API int moe_decode_step(moe_ctx *ctx, const float *x_dev, float *y_dev, void *stream);
 
 /* The same step on host buffers, synchronously: x_host [H] fp32 is staged to the

@@ -82,6 +82,7 @@ def lib():
                 "orc_decode_token": (None, [ctypes.POINTER(Dims), ctypes.c_int,
                                             ctypes.POINTER(LayerW), _P, _P, _P, _P]),
                 "orc_select_pinned": (None, [_P, ctypes.c_int, ctypes.c_int, _P]),
+                "orc_recal_score": (None, [_P, _P, ctypes.c_int]),
                 "orc_cache_create": (_P, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
                 "orc_cache_destroy": (None, [_P]),
                 "orc_cache_set_pinned": (None, [_P, ctypes.c_int, _P]),
@@ -179,6 +180,15 @@ def select_pinned(hist, P: int) -> np.ndarray:
     mask = np.empty(hist.size, np.uint8)
     lib().orc_select_pinned(_ptr(hist), hist.size, P, _ptr(mask))
     return mask
+
+
+def recal_score(score, window) -> np.ndarray:
+    """New recalibration scores (uint32) from the old ones and a window of counts."""
+    out = _c(score, np.uint32).copy()
+    window = _c(window, np.uint32)
+    assert out.shape == window.shape
+    lib().orc_recal_score(_ptr(out), _ptr(window), out.size)
+    return out
 
 
 class _LayerRef:

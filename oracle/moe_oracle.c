@@ -38,6 +38,9 @@
  *   y = sum_i w_i o_i + o_shared (shared expert ungated).  Stack: h <- h + y on
  *   RMSNorm(h) input; single layer without norm: y = MoE(x).  All in fp64.
  *
+ *   Recalibration: score <- floor(score / 2) + window count, re-pin top-P by score,
+ *   the ring emptied at every re-pin (orc_cache_set_pinned).
+ *
  *   Cache (key-components item 2): per layer, accesses in the token's rank order;
  *   pinned -> PIN_HIT; resident in the ring -> RING_HIT and refresh recency; else MISS
  *   into the lowest-index empty ring slot, else into the least recently used one.
@@ -312,6 +315,14 @@ void orc_select_pinned(const uint32_t *hist, int E, int P, uint8_t *mask) {
     }
     mask[best] = 1;
   }
+}
+
+/* Online recalibration (reading of the write-up's "self-tunes over time" with routing
+ * frequencies accumulated from real requests): per expert, score <- floor(score / 2) +
+ * the routing count of the window since the previous recalibration; the pinned set is
+ * then orc_select_pinned over the scores. */
+void orc_recal_score(uint32_t *score, const uint32_t *window, int n) {
+  for (int i = 0; i < n; ++i) score[i] = (score[i] >> 1) + window[i];
 }
 
 /* ---------------------------------------------------------------- cache simulator */

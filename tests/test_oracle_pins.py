@@ -459,3 +459,53 @@ def test_calibrated_placement_cuts_cold_hits_vs_uniform():
         cold[name] = np.mean(np.array(kinds) != oracle.PIN_HIT)
     assert cold["cal"] < cold["uni"]
     assert cold["cal"] < 0.15 and cold["uni"] > 0.2
+
+
+# ------------------------------------------------------------------ recalibration
+
+def test_recal_score_closed_forms():
+    # a constant window w = 2^10 from zero: s_n = 2w - w / 2^(n-1), exactly
+    w = np.full(5, 1024, np.uint32)
+    s = np.zeros(5, np.uint32)
+    for n in range(1, 11):
+        s = oracle.recal_score(s, w)
+        assert np.all(s == 2048 - 1024 // 2 ** (n - 1))
+    # fixed points of s = floor(s/2) + w are 2w and 2w - 1
+    for w0 in (1, 7, 1000):
+        for fp in (2 * w0, 2 * w0 - 1):
+            assert oracle.recal_score(np.array([fp]), np.array([w0]))[0] == fp
+    # a one-off burst B then quiet windows: s_n = floor(B / 2^n)
+    s = oracle.recal_score(np.zeros(1, np.uint32), np.array([1000]))
+    for n in range(1, 12):
+        s = oracle.recal_score(s, np.zeros(1, np.uint32))
+        assert s[0] == 1000 >> n
+
+
+def test_recalibration_follows_drifted_popularity():
+    """The write-up's "self-tunes over time": after the popularity permutation changes,
+    re-pinning from decayed routing counts cuts cold hits below a placement frozen at the
+    first calibration."""
+    s = synthetic.Shape(1, 256, 64, 4, 32, 0, ring_slots=4, zipf_s=1.0)
+    layers = [synthetic.layer_weights(0, s)]
+    drifted = [synthetic.layer_weights(0, s, bias_seed=synthetic.SEED_RESHUFFLE)]
+    m_old, m_new = oracle.Model(s, layers), oracle.Model(s, drifted)
+    P = round(0.4 * s.n_experts)
+    calib = np.zeros(s.n_experts, np.uint32)
+    for t in range(64):
+        calib[m_old.layer(0, synthetic.token(t, s.hidden, synthetic.SEED_CALIB))["sel"]] += 1
+    cold = {}
+    for name in ("static", "recal"):
+        c = oracle.Cache(1, s.n_experts, 4)
+        c.set_pinned(0, oracle.select_pinned(calib, P))
+        score, window, kinds = calib.copy(), np.zeros(s.n_experts, np.uint32), []
+        for t in range(256):
+            if name == "recal" and t % 16 == 0 and t:
+                score = oracle.recal_score(score, window)
+                window[:] = 0
+                c.set_pinned(0, oracle.select_pinned(score, P))
+            sel = (m_old if t < 96 else m_new).layer(0, synthetic.token(t, s.hidden))["sel"]
+            window[sel] += 1
+            kinds.append(c.access(t, 0, sel)["kind"])
+        k = np.concatenate(kinds[128:])
+        cold[name] = np.mean(k != oracle.PIN_HIT)
+    assert cold["recal"] < 0.5 * cold["static"]
