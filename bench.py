@@ -141,13 +141,15 @@ def reduce_over_ranks(value_ms: float, units: float, world: int):
 
 # ------------------------------------------------------------------ CPU oracle legs
 
-def oracle_tokens_per_s(shape, n_layers: int, n_tokens: int, warmup: int = 0):
+def oracle_tokens_per_s(shape, n_layers: int, n_tokens: int, warmup: int = 0, layers=None):
     """The oracle, as it stands, on n_tokens tokens through the first n_layers layers;
     returns (tok/s scaled to the full stack, seconds, threads)."""
     import oracle
     sub = synthetic.Shape(n_layers, shape.hidden, shape.n_experts, shape.top_k, shape.inter,
                           shape.shared_inter, shape.ring_slots, shape.use_rmsnorm, shape.zipf_s)
-    layers = [synthetic.layer_weights(l, shape) for l in range(n_layers)]
+    if layers is None:
+        layers = [synthetic.layer_weights(l, shape) for l in range(n_layers)]
+    layers = layers[:n_layers]
     m = oracle.Model(sub, layers)
     for i in range(warmup):
         m.decode(synthetic.token(i, shape.hidden))
@@ -177,6 +179,74 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_drift(args, shape, layers, local, dev, xs_steps=1024, switch=512, every=64,
+              fraction=0.4, ring=4):
+    """Online recalibration under drift: the stack at 40% residency with 4-slot rings;
+    the router bias (traffic popularity) switches to reshuffled Zipf permutations at
+    token 512 of 1024; cold-hit rates before / after the switch for calibrated placement
+    with recalibration every 64 tokens, calibrated placement frozen, and uniform."""
+    import dataclasses
+
+    import torch
+
+    import expert_cache_host_router_b200 as moe
+    s = dataclasses.replace(shape, ring_slots=ring)
+    m = moe.ExpertCacheMoE(s, device=local, log_steps=xs_steps + 256)
+    for l in range(s.n_layers):
+        m.load_layer(l, layers[l])
+    new_bias = [synthetic.zipf_bias(l, s.n_experts, s.zipf_s, synthetic.SEED_RESHUFFLE)
+                for l in range(s.n_layers)]
+    calib = torch.from_numpy(synthetic.tokens(0, args.calib_steps, s.hidden, synthetic.SEED_CALIB)).to(dev)
+    xs = torch.from_numpy(synthetic.tokens(0, xs_steps, s.hidden)).to(dev)
+    y = torch.empty(s.hidden, dtype=torch.float32, device=dev)
+    m.set_residency(1.0)
+    for i in range(args.calib_steps):
+        m.decode(calib[i], y)
+    m.sync()
+    _, hist, _ = m.stats(reset=True, log_cap=args.calib_steps * s.n_layers * s.top_k)
+    out = {"residency": fraction, "ring_slots": ring, "steps": xs_steps, "reshuffle_at": switch,
+           "recalibrate_every": every}
+    stream = torch.cuda.current_stream(dev)
+    for name, place, recal in (("calibrated_recal", moe.MOE_PLACE_CALIBRATED, True),
+                               ("calibrated_static", moe.MOE_PLACE_CALIBRATED, False),
+                               ("uniform", moe.MOE_PLACE_UNIFORM, False)):
+        for l in range(s.n_layers):
+            m.set_router_bias(l, layers[l].bias)
+        m.set_residency(fraction, hist, place)
+        m.stats(reset=True, log_cap=(xs_steps + 256) * s.n_layers * s.top_k)
+        ms = [0.0, 0.0]
+        for half, (a, b) in enumerate(((0, switch), (switch, xs_steps))):
+            if half == 1:
+                for l in range(s.n_layers):
+                    m.set_router_bias(l, new_bias[l])
+            t_dev = 0.0
+            for t0 in range(a, b, every):
+                if recal and t0:
+                    m.recalibrate()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for t in range(t0, min(b, t0 + every)):
+                    m.decode(xs[t], y)
+                e1.record(stream)
+                m.sync()
+                t_dev += e0.elapsed_time(e1)
+            ms[half] = t_dev
+        st, _, log = m.stats(log_cap=xs_steps * s.n_layers * s.top_k)
+        kinds = log["kind"].reshape(xs_steps, -1)
+        res = {}
+        for half, (a, b) in enumerate(((0, switch), (switch, xs_steps))):
+            k = kinds[a:b]
+            res["before" if half == 0 else "after"] = {
+                "cold_hit_rate": float(np.mean(k != moe.MOE_PIN_HIT)),
+                "misses_per_token": float(np.sum(k == moe.MOE_MISS)) / (b - a),
+                "tok_s": (b - a) / (ms[half] * 1e-3)}
+        res["repins"] = st["repins"]
+        res["repin_copies"] = st["repin_copies"]
+        out[name] = res
+    m.close()
+    return out
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_ours(args):
@@ -202,10 +272,13 @@ def run_ours(args):
         shape = dataclasses.replace(shape, n_layers=args.layers)
     dev = torch.device("cuda", local)
     keep_layers = rank == 0 and world == 1 and not args.no_cpu_baseline and args.layers == 40
+    t0 = time.time()
+    layers = [synthetic.layer_weights(l, shape) for l in range(shape.n_layers)]
+    gen_s = time.time() - t0
     m = moe.ExpertCacheMoE(shape, device=local, log_steps=max(4096, args.steps + args.warmup + 16))
     t0 = time.time()
     for l in range(shape.n_layers):
-        m.load_layer(l, synthetic.layer_weights(l, shape))
+        m.load_layer(l, layers[l])
     load_s = time.time() - t0
 
     stream = torch.cuda.current_stream(dev)
@@ -333,12 +406,14 @@ def run_ours(args):
                 "h2d_bytes_per_step": 4 * shape.hidden, "d2h_bytes_per_step": 4 * shape.hidden + 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
-        "setup": {"load_s": load_s, "phases": args.phases},
+        "setup": {"generate_s": gen_s, "load_s": load_s, "phases": args.phases},
     }
     m.close()
     del m
+    if args.phases == "all" and not args.no_drift:
+        line["drift"] = run_drift(args, shape, layers, local, dev, xs_steps=1024)
     if keep_layers:
-        tps, dt, cores = oracle_tokens_per_s(shape, shape.n_layers, args.cpu_tokens)
+        tps, dt, cores = oracle_tokens_per_s(shape, shape.n_layers, args.cpu_tokens, layers=layers)
         line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{args.cpu_tokens} tokens through all 40 layers ({dt:.1f} s)"}
     if rank == 0:
@@ -358,6 +433,7 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
+    ap.add_argument("--no-drift", action="store_true", help="skip the recalibration-under-drift run")
     ap.add_argument("--phases", default="all", choices=["all", "100"],
                     help="'100' times full residency only (no miss copies), for profiler runs")
     args = ap.parse_args()
