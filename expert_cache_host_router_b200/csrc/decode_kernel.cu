@@ -249,7 +249,7 @@ struct Misc {
 };
 
 struct SmemPlan {
-  uint32_t unit, dchunk, rchunk, hbuf, gbuf, pinrow, z, xcodes, xs, xc, acodes, o, misc, total;
+  uint32_t unit, rchunk, hbuf, gbuf, pinrow, z, xcodes, xs, xc, o, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -266,7 +266,6 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
   const int n_exp = K + (Is > 0);
   const int imax = I > Is ? I : Is;
   s.unit = take(36u * H);                        // gate qs|d, up qs|d for 32 rows
-  s.dchunk = take(9u * (uint32_t)(K * I + Is));  // down rows of one chunk, all experts
   s.rchunk = take(32u * E * nown);               // router columns of the owned chunks
   s.hbuf = take(4u * H);
   s.gbuf = take(4u * H);
@@ -275,7 +274,6 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
   s.xcodes = take(2u * H);
   s.xs = take(4u * (H / 32));
   s.xc = take(4u * (H / 32));
-  s.acodes = take((uint32_t)kACodeBytes * n_exp * (imax / 32));
   s.o = take(4u * n_exp * kChunk);
   s.misc = take(sizeof(Misc));
   s.total = align_up(off, 128);
@@ -323,6 +321,12 @@ __device__ bool grid_sync(const DecodeParams& p, Misc& m) {
 
 __device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
   if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = gtimer();
+}
+
+// Per-CTA marks (every CTA, thread 0): after [(L+1)][32] come [L][gridDim][4] stamps.
+__device__ __forceinline__ void cta_stamp(const DecodeParams& p, int l, int k) {
+  if (p.phase_trace && threadIdx.x == 0)
+    p.phase_trace[(size_t)(p.L + 1) * 32 + ((size_t)l * gridDim.x + blockIdx.x) * 4 + k] = gtimer();
 }
 
 // Counted exchange: a producer CTA publishes with one release add after its stores;
@@ -680,26 +684,20 @@ __device__ bool issue_unit(const DecodeParams& p, Misc& m, uint8_t* unit, int u)
   return true;
 }
 
-// All threads: copy the down tile of chunk c of every active expert into shared memory
-// with 16-byte cp.async copies (about ten per thread), L2 evict-first.  The caller has
-// made sure the miss copies these tiles depend on have landed.
-__device__ void load_dchunk(const DecodeParams& p, Misc& m, uint8_t* dch, int c) {
-  const uint64_t pol = l2_evict_first_policy();
-  const uint32_t t_r = 9u * p.I, t_s = 9u * p.Is;  // tile bytes of a routed / the shared expert
+// All threads: pull the down tiles of chunk c of every resident active expert into L2
+// (one prefetch per 128-byte line), so that the down phase reads them from L2.
+__device__ void prefetch_dchunk_l2(const DecodeParams& p, const Misc& m, int c) {
+  const uint32_t t_r = 9u * p.I, t_s = 9u * p.Is;
   const uint32_t routed_bytes = (uint32_t)p.K * t_r, total = routed_bytes + (p.Is > 0 ? t_s : 0);
-  for (uint32_t off = 16u * threadIdx.x; off < total; off += 16u * kThreads) {
+  for (uint32_t off = 128u * threadIdx.x; off < total; off += 128u * kThreads) {
     const int i = off < routed_bytes ? (int)(off / t_r) : p.K;
+    if (m.miss_seq[i] != 0) continue;  // its slot is still being filled
     const uint32_t in_tile = off < routed_bytes ? off - (uint32_t)i * t_r : off - routed_bytes;
     const SlotLayout& L = i < p.K ? p.lay : p.slay;
     const uint8_t* src = m.src[i] + L.down + (size_t)c * (i < p.K ? t_r : t_s) + in_tile;
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dch + off)), "l"(src),
-                 "l"(pol)
-                 : "memory");
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
   }
-  asm volatile("cp.async.commit_group;" ::: "memory");
 }
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Thread 0: bulk-load layer lr's router columns of the owned chunks into rch.
 __device__ void prefetch_router(const DecodeParams& p, Misc& m, uint8_t* rch, int lr, int n_own) {
@@ -725,10 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   int16_t* xcodes = reinterpret_cast<int16_t*>(smem + S.xcodes);
   float* xs = reinterpret_cast<float*>(smem + S.xs);
   int32_t* xc = reinterpret_cast<int32_t*>(smem + S.xc);
-  uint8_t* acs = smem + S.acodes;
   float* os = reinterpret_cast<float*>(smem + S.o);
   uint8_t* unit = smem + S.unit;
-  uint8_t* dch = smem + S.dchunk;
   uint8_t* rch = smem + S.rchunk;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -926,7 +922,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     __syncthreads();
     if (!m.unit_ok) return;
     if (blockIdx.x == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
+    for (int k = 0; k < n_own; ++k) prefetch_dchunk_l2(p, m, blockIdx.x + k * gridDim.x);
     stamp(p, l, 2);
+    cta_stamp(p, l, 0);
 
     // ---------------------------------------------------------------- G phase
     {
@@ -1036,48 +1034,30 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     }
     const int n_producers = min((int)gridDim.x, p.n_units);  // CTAs holding gate/up units
     stamp(p, l, 21);
-    // the owned chunk's down tiles (all resident) load while the other units finish
-    if (n_own > 0) {
-      bool layer_misses = false;
-      for (int i = 0; i < p.n_exp; ++i) layer_misses |= m.miss_seq[i] != 0;
-      if (!layer_misses) {
-        load_dchunk(p, m, dch, blockIdx.x);
-        if (tid == 0) m.d_issued = 1;
-      }
-    }
     if ((int)blockIdx.x < n_producers) publish(p, &p.ctrl->a_count);
     stamp(p, l, 3);
+    cta_stamp(p, l, 1);
     stamp(p, l, 4);
 
     // ---------------------------------------------------------------- D phase
-    // gather every activation record of this layer (CTAs that own rows)
+    // (CTAs that own rows) wait for every activation record of the layer and for the miss
+    // copies the down tiles depend on; tiles and records are then read from L2
     if (n_own > 0) {
+      if (tid == 0) {
+        m.flag = 1;
+        for (int i = 0; i < p.n_exp; ++i)
+          if (!wait_miss(p, m.miss_seq[i])) m.flag = 0;
+      }
       if (!await_count(p, m, &p.ctrl->a_count, (uint32_t)(l + 1) * n_producers)) return;
-      const int n_vec = p.n_exp * rec_per_exp * (kACodeBytes / 16);
-      const uint4* srcr = reinterpret_cast<const uint4*>(p.acodes);
-      uint4* dstr = reinterpret_cast<uint4*>(acs);
-      for (int t = tid; t < n_vec; t += kThreads) dstr[t] = __ldcg(srcr + t);
     }
     if (!cta_ok(p, m.flag)) return;
     stamp(p, l, 13);
     for (int k = 0; k < n_own; ++k) {
       const int c = blockIdx.x + k * gridDim.x;
-      if (!(k == 0 && m.d_issued)) {  // tiles not loaded yet (misses in the layer, or chunk > 0)
-        if (tid == 0) {
-          m.flag = 1;
-          for (int i = 0; i < p.n_exp; ++i)
-            if (!wait_miss(p, m.miss_seq[i])) m.flag = 0;
-        }
-        __syncthreads();
-        if (!m.flag) return;
-        load_dchunk(p, m, dch, c);
-      }
-      cp_async_wait_all();
-      __syncthreads();
       stamp(p, l, 14);
-      // thread (expert i, block column b0): the 16 rows of chunk c against blocks b0,
-      // b0+16, ... of a_i, rows independent; then a 15-shuffle transpose reduction over
-      // the 16 lanes of the expert leaves row b0's sum in lane b0
+      // thread (expert i, block column b0): all 16 rows of chunk c against block b0 (then
+      // b0+16, ...) of a_i, every load of a block issued before any is used; then a
+      // 15-shuffle transpose reduction over the expert's 16 lanes leaves row b0 in lane b0
       {
         const int b0 = tid & 15;
         // warp-uniform loop: lanes 0-15 take expert base, lanes 16-31 expert base + 1
@@ -1086,53 +1066,43 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           const bool act = i < p.n_exp;
           const int Ii = !act ? 0 : (i < p.K ? p.I : p.Is);
           const int nbd = Ii / 32;
-          const uint8_t* qbase = dch + 9u * (i < p.K ? (uint32_t)i * p.I : (uint32_t)p.K * p.I);
-          const __half* dbase = reinterpret_cast<const __half*>(qbase + 8u * Ii);
-          const int4* ap = nullptr;
-          int4 a0 = make_int4(0, 0, 0, 0), a1 = a0, a2 = a0, a3 = a0;
-          float sc = 0.0f;
-          int cs128 = 0;
-#pragma unroll 1
-          for (int rg = 0; rg < kChunk / 4; ++rg) {  // four rows at a time
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            for (int b = b0; b < nbd; b += 16) {
-              if (b != b0 || rg == 0 || nbd > 16) {
-                const uint8_t* rec = acs + ((size_t)i * rec_per_exp + b) * kACodeBytes;
-                ap = reinterpret_cast<const int4*>(rec);
-                a0 = ap[0];
-                a1 = ap[1];
-                a2 = ap[2];
-                a3 = ap[3];
-                sc = reinterpret_cast<const float*>(rec + 64)[0];
-                cs128 = 128 * reinterpret_cast<const int32_t*>(rec + 68)[0];
-              }
+          const uint8_t* tile =
+              act ? m.src[i] + (i < p.K ? p.lay.down : p.slay.down) + (size_t)c * 9u * Ii : nullptr;
+          float acc[kChunk];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int r = 4 * rg + q;
-                const uint4 qv = *reinterpret_cast<const uint4*>(qbase + ((size_t)r * nbd + b) * 16);
-                const float d = __half2float(dbase[(size_t)r * nbd + b]);
-                const int v = q4_block_dot16(qv, a0, a1, a2, a3) - cs128;
-                acc[q] = fmaf(d * sc, (float)v, acc[q]);
-              }
-            }
-            // transpose reduction of 4 rows over the expert's 16 lanes: lane b0 ends with
-            // the sum of row 4 rg + 2 (b0 >> 3 & 1) + (b0 >> 2 & 1)
-            const bool up8 = (b0 & 8) != 0, up4 = (b0 & 4) != 0;
+          for (int r = 0; r < kChunk; ++r) acc[r] = 0.0f;
+          for (int b = b0; b < nbd; b += 16) {
+            const uint4* rec = reinterpret_cast<const uint4*>(p.acodes + ((size_t)i * rec_per_exp + b) * kACodeBytes);
+            const uint4 r0 = __ldcg(rec), r1 = __ldcg(rec + 1), r2 = __ldcg(rec + 2), r3 = __ldcg(rec + 3),
+                        r4 = __ldcg(rec + 4);
+            uint4 qv[kChunk];
+            unsigned short dv[kChunk];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const float send = up8 ? acc[q] : acc[q + 2];
-              const float keep = up8 ? acc[q + 2] : acc[q];
-              acc[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+            for (int r = 0; r < kChunk; ++r) {
+              qv[r] = __ldcg(reinterpret_cast<const uint4*>(tile + ((size_t)r * nbd + b) * 16));
+              dv[r] = __ldcg(reinterpret_cast<const unsigned short*>(tile + 8u * Ii) + (size_t)r * nbd + b);
             }
-            {
-              const float send = up4 ? acc[0] : acc[1];
-              const float keep = up4 ? acc[1] : acc[0];
-              acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+            const int4 a0 = make_int4(r0.x, r0.y, r0.z, r0.w), a1 = make_int4(r1.x, r1.y, r1.z, r1.w),
+                       a2 = make_int4(r2.x, r2.y, r2.z, r2.w), a3 = make_int4(r3.x, r3.y, r3.z, r3.w);
+            const float sc = __uint_as_float(r4.x);
+            const int cs128 = 128 * (int)r4.y;
+#pragma unroll
+            for (int r = 0; r < kChunk; ++r) {
+              const int v = q4_block_dot16(qv[r], a0, a1, a2, a3) - cs128;
+              acc[r] = fmaf(__half2float(__ushort_as_half(dv[r])) * sc, (float)v, acc[r]);
             }
-            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 2);
-            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], 1);
-            if (act && (b0 & 3) == 0) os[i * kChunk + 4 * rg + 2 * (up8 ? 1 : 0) + (up4 ? 1 : 0)] = acc[0];
           }
+#pragma unroll
+          for (int h = 8; h >= 1; h >>= 1) {
+            const bool up = (b0 & h) != 0;
+#pragma unroll
+            for (int r = 0; r < h; ++r) {
+              const float send = up ? acc[r] : acc[r + h];
+              const float keep = up ? acc[r + h] : acc[r];
+              acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, h);
+            }
+          }
+          if (act) os[i * kChunk + b0] = acc[0];
         }
       }
       __syncthreads();
@@ -1160,8 +1130,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     // the router columns for layer l + 2 load during the barrier (rch is free again)
     if (tid == 0 && l + 2 < p.L && n_own > 0) prefetch_router(p, m, rch, l + 2, n_own);
     stamp(p, l, 5);
+    cta_stamp(p, l, 2);
     if (!grid_sync(p, m)) return;
     stamp(p, l, 6);
+    cta_stamp(p, l, 3);
 
     // deferred ring fills (only when a layer misses more often than it has ring slots)
     for (int f = 0; f < m.n_fix; ++f) {

@@ -199,12 +199,13 @@ MOE_API int moe_stats(moe_ctx *ctx, moe_stats_t *out, uint32_t *hist_out, moe_ev
  * the routing weights.  Pass NULLs to stop.  Device pointers owned by the caller. */
 MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
 
-/* Phase timing: when stamps_dev ([(L+1)][32] uint64, device) is non-NULL, every decode
+/* Phase timing: when stamps_dev ([(L+1)][32] + [L][n_sm][4] uint64, device) is non-NULL, every decode
  * step writes the GPU global timer (ns) of CTA 0 at its phase boundaries: per layer l,
  * [l][0] layer start, [1] logits ready, [2] routing and cache decided, [3] gate/up done
  * (this CTA), [4] all gate/up done, [5] down done (this CTA), [6] layer done, [7..31]
  * finer marks inside routing, gate/up and the down phase; [L][0] kernel start, [L][1] prologue
- * done, [L][2] kernel end.  NULL stops it. */
+ * done, [L][2] kernel end.  Then, for every layer and every CTA (one per SM): [0] routing
+ * done, [1] gate/up published, [2] down done, [3] barrier passed.  NULL stops it. */
 MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev);
 
 /* Fault injection for tests: the miss proxy issues the next n copies but never
