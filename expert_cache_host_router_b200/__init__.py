@@ -94,6 +94,7 @@ _SIGS = {
     "moe_stats": (ctypes.c_int, [_P, ctypes.POINTER(Stats), _P, _P, ctypes.c_size_t,
                                  ctypes.POINTER(ctypes.c_size_t), ctypes.c_int32]),
     "moe_set_trace": (ctypes.c_int, [_P, _P, _P]),
+    "moe_set_prefill_trace": (ctypes.c_int, [_P, _P, _P]),
     "moe_recalibrate": (ctypes.c_int, [_P]),
     "moe_set_router_bias": (ctypes.c_int, [_P, ctypes.c_int32, _P]),
     "moe_set_phase_trace": (ctypes.c_int, [_P, _P]),
@@ -214,6 +215,10 @@ def moe_set_trace(ctx: int, h_trace_dev: int | None, w_trace_dev: int | None) ->
     _check(lib().moe_set_trace(ctx, h_trace_dev, w_trace_dev), "moe_set_trace")
 
 
+def moe_set_prefill_trace(ctx: int, h_trace_dev: int | None, sel_trace_dev: int | None) -> None:
+    _check(lib().moe_set_prefill_trace(ctx, h_trace_dev, sel_trace_dev), "moe_set_prefill_trace")
+
+
 def moe_set_phase_trace(ctx: int, stamps_dev: int | None) -> None:
     _check(lib().moe_set_phase_trace(ctx, stamps_dev), "moe_set_phase_trace")
 
@@ -272,6 +277,21 @@ class ExpertCacheMoE:
         s = torch.cuda.current_stream(x.device) if stream is None else stream
         moe_decode_step(self.ctx, x.data_ptr(), y.data_ptr(), s.cuda_stream)
         return y
+
+    def prefill(self, x, y=None, stream=None):
+        """x: torch float32 [T, H] on this device.  Returns y [T, H] (torch, same device)."""
+        import torch
+        assert x.dtype == torch.float32 and x.is_cuda and x.is_contiguous() and x.dim() == 2
+        if y is None:
+            y = torch.empty_like(x)
+        s = torch.cuda.current_stream(x.device) if stream is None else stream
+        moe_prefill(self.ctx, x.data_ptr(), x.shape[0], y.data_ptr(), s.cuda_stream)
+        return y
+
+    def set_prefill_trace(self, h_trace=None, sel_trace=None):
+        """h_trace: torch float32 [L+1, T, H]; sel_trace: torch int32 [L, T, k]; or None."""
+        moe_set_prefill_trace(self.ctx, None if h_trace is None else h_trace.data_ptr(),
+                              None if sel_trace is None else sel_trace.data_ptr())
 
     def decode_host(self, x: np.ndarray) -> np.ndarray:
         x = _arr(x, np.float32)

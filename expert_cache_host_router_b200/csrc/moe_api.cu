@@ -26,6 +26,7 @@
 
 #include "../../include/moe_cache.h"
 #include "moe_internal.h"
+#include "prefill.h"
 
 namespace moe {
 uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown);
@@ -93,6 +94,14 @@ struct moe_ctx {
   float *h_trace = nullptr, *w_trace = nullptr;
   unsigned long long* phase_trace = nullptr;
   uint64_t log_read_step = 0, log_dropped = 0;
+  // batched prefill: scratch for up to prefill_cap tokens (one allocation), tracing
+  uint8_t* prefill_mem = nullptr;
+  int prefill_cap = 0;
+  PrefillScratch pf{};
+  bool prefill_configured = false;
+  void* encode_tiled = nullptr;
+  float* pf_h_trace = nullptr;
+  int32_t* pf_sel_trace = nullptr;
 };
 
 #define CK(call)                                  \
@@ -326,7 +335,7 @@ void moe_destroy(moe_ctx* c) {
   void* dev[] = {c->shared_pool, c->pool.load(), c->router, c->bias, c->gain, c->pin_slot,
                  c->layer_base, c->n_pinned, c->ring_owner, c->ring_stamp, c->ring_clock,
                  c->h, c->part, c->sq, c->z, c->acodes, c->hist, c->log, c->ctrl, c->done_seq,
-                 c->x_buf, c->y_buf};
+                 c->x_buf, c->y_buf, c->prefill_mem};
   for (void* p : dev)
     if (p) cudaFree(p);
   void* hst[] = {c->host_tier, c->x_pin, c->y_pin, c->err_pin, c->mbox_host};
@@ -601,13 +610,107 @@ int moe_decode_step_host(moe_ctx* c, const float* x_host, float* y_host) {
   return deverr_status(*c->err_pin);
 }
 
+// Carve the prefill scratch for T tokens out of one allocation (256-byte aligned parts).
+static int prefill_reserve(moe_ctx* c, int T) {
+  if (T <= c->prefill_cap) return MOE_OK;
+  CK(cudaDeviceSynchronize());
+  if (c->prefill_mem) cudaFree(c->prefill_mem);
+  c->prefill_mem = nullptr;
+  c->prefill_cap = 0;
+  const size_t H = c->H, K = c->K, E = c->E, imax = std::max(c->I, c->Is);
+  const size_t R = (size_t)T * K + (c->Is > 0 ? (size_t)T : 0);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (bytes + 255) / 256 * 256;
+    return at;
+  };
+  const size_t o_h = take((size_t)T * H * 4), o_sel = take((size_t)T * K * 4), o_w = take((size_t)T * K * 4),
+               o_xh = take((size_t)T * H * 2), o_xl = take((size_t)T * H * 2), o_gh = take(R * H * 2),
+               o_gl = take(R * H * 2), o_ah = take(R * imax * 2), o_al = take(R * imax * 2),
+               o_ob = take((size_t)T * (K + 1) * H * 4), o_cnt = take(E * 4), o_cur = take((E + 1) * 4),
+               o_off = take((E + 2) * 4), o_perm = take(R * 4), o_jobs = take((R / 128 + E + 2) * 4),
+               o_nj = take(4);
+  uint8_t* m = nullptr;
+  CK(cudaMalloc((void**)&m, off));
+  c->prefill_mem = m;
+  c->prefill_cap = T;
+  PrefillScratch& s = c->pf;
+  s.h = reinterpret_cast<float*>(m + o_h);
+  s.sel = reinterpret_cast<int32_t*>(m + o_sel);
+  s.w = reinterpret_cast<float*>(m + o_w);
+  s.x_hi = reinterpret_cast<__half*>(m + o_xh);
+  s.x_lo = reinterpret_cast<__half*>(m + o_xl);
+  s.xg_hi = reinterpret_cast<__half*>(m + o_gh);
+  s.xg_lo = reinterpret_cast<__half*>(m + o_gl);
+  s.a_hi = reinterpret_cast<__half*>(m + o_ah);
+  s.a_lo = reinterpret_cast<__half*>(m + o_al);
+  s.obuf = reinterpret_cast<float*>(m + o_ob);
+  s.counts = reinterpret_cast<int32_t*>(m + o_cnt);
+  s.cursor = reinterpret_cast<int32_t*>(m + o_cur);
+  s.offsets = reinterpret_cast<int32_t*>(m + o_off);
+  s.perm = reinterpret_cast<int32_t*>(m + o_perm);
+  s.jobs = reinterpret_cast<int32_t*>(m + o_jobs);
+  s.n_jobs = reinterpret_cast<int32_t*>(m + o_nj);
+  return MOE_OK;
+}
+
 int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, void* stream) {
-  (void)x_dev;
-  (void)n_tokens;
-  (void)y_dev;
-  (void)stream;
+  if (!c || !x_dev || !y_dev || n_tokens < 1 || n_tokens > (1 << 20)) return MOE_ERR_INVALID;
+  if (!c->resident || c->P != c->E) return MOE_ERR_STATE;
+  if (!prefill_supported(c->H, c->E, c->K, c->I, c->Is)) return MOE_ERR_UNSUPPORTED;
+  CK(cudaSetDevice(c->cfg.device));
+  if (!c->prefill_configured) {
+    CK(prefill_configure(c->H, c->E));
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    CK(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return MOE_ERR_UNSUPPORTED;
+    c->encode_tiled = fn;
+    c->prefill_configured = true;
+  }
+  const int st = prefill_reserve(c, n_tokens);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  PrefillScratch sc = c->pf;
+  sc.y = y_dev;
+  sc.h_trace = c->pf_h_trace;
+  sc.sel_trace = c->pf_sel_trace;
+  sc.error = &c->ctrl->error;
+  CK(cudaMemcpyAsync(sc.h, x_dev, sizeof(float) * n_tokens * c->H, cudaMemcpyDeviceToDevice, s));
+  PrefillArgs a{};
+  a.L = c->L;
+  a.H = c->H;
+  a.E = c->E;
+  a.K = c->K;
+  a.I = c->I;
+  a.Is = c->Is;
+  a.use_norm = c->cfg.use_rmsnorm;
+  a.T = n_tokens;
+  a.eps = c->cfg.rms_eps;
+  a.pool = c->pool.load();
+  a.slot_bytes = c->slot_bytes;
+  a.lay = c->lay;
+  a.slay = c->slay;
+  a.shared_pool = c->shared_pool;
+  a.shared_slot_bytes = c->shared_slot_bytes;
+  a.router = c->router;
+  a.bias = c->has_bias ? c->bias : nullptr;
+  a.gain = c->gain;
+  a.pin_slot = c->pin_slot;
+  a.layer_base = c->layer_base;
+  a.hist = c->hist;
+  const int r = prefill_run(a, sc, c->encode_tiled, s);
+  if (r == -1) return MOE_ERR_UNSUPPORTED;
+  if (r != 0) return cuda_fail((cudaError_t)r);
+  return MOE_OK;
+}
+
+int moe_set_prefill_trace(moe_ctx* c, float* h_trace_dev, int32_t* sel_trace_dev) {
   if (!c) return MOE_ERR_INVALID;
-  return MOE_ERR_UNSUPPORTED;
+  c->pf_h_trace = h_trace_dev;
+  c->pf_sel_trace = sel_trace_dev;
+  return MOE_OK;
 }
 
 int moe_sync(moe_ctx* c) {

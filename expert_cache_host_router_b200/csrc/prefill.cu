@@ -1,0 +1,765 @@
+// prefill.cu -- batched prefill of T tokens through the MoE stack (every expert resident)
+// for libmoe: routing for every token in the same canonical fp32 order as decode, tokens
+// grouped by expert, and the expert FFNs as a grouped GEMM on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory, activation tiles brought in by TMA).
+//
+// The write-up serves decode; a prompt's tokens all pass the same layers at once, which
+// turns each expert's GEMVs into GEMMs [n_e x H] x [H x 2I] and [n_e x I] x [I x H]
+// (n_e = tokens routed to expert e): a dense contraction, so it runs on the tensor
+// cores.  Per layer, in stream order:
+//   route    16 (or 8) tokens per CTA: RMSNorm scale, router logits in the canonical
+//            order, top-k, weights, histogram, per-expert counts; x = RMSNorm(h) split
+//            into fp16 hi + lo (x = hi + lo to about 2^-22 relative)
+//   scan     expert offsets and the list of 128-row m-tiles
+//   scatter  one warp per token: its rows of x copied to their place in expert order
+//            (within an expert the order is whatever the atomics give: a GEMM row does
+//            not depend on the other rows of its tile, so results are deterministic)
+//   gemm     one CTA per 128 x 128 output tile: A (activation rows, fp16 hi and lo) by
+//            TMA, B (Q4_0 weights) dequantised to fp16 into 128B-swizzled shared memory,
+//            two tcgen05.mma per 16-wide K step (A_hi B and A_lo B) into one fp32
+//            accumulator in tensor memory; gate/up tiles hold 64 gate and the matching
+//            64 up columns so the epilogue forms a = silu(g) * u (stored as fp16 hi + lo);
+//            down tiles write each row's expert output to its (token, rank) slot
+//   combine  h += sum_rank w * o_rank + o_shared in rank order
+// The activations are split because fp16 operands alone put the element-wise error at
+// the tolerance; the weights are fp16((q - 8) * d), a relative error of at most 2^-12.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_cache.h"
+#include "moe_internal.h"
+#include "prefill.h"
+
+namespace moe {
+
+constexpr int kPT = 256;  // threads per prefill CTA
+constexpr int kTM = 128;  // GEMM tile rows (tokens)
+constexpr int kTN = 128;  // GEMM tile columns
+constexpr int kTK = 64;   // K per pipeline stage: one 128-byte swizzle row of fp16
+constexpr int kStages = 4;
+constexpr uint32_t kTileBytes = kTM * kTK * 2;           // 16 KB per fp16 operand tile
+constexpr uint32_t kRawBytes = kTN * 2 * 16 + kTN * 4;  // nibbles of 2 blocks x 128 rows + their scales
+// Swizzled operand tiles first, each at a multiple of 1024 bytes (the 128-byte swizzle's
+// period: TMA and the MMA take its phase from the address), then the raw weight bytes.
+constexpr uint32_t kTilesBytes = 3 * kTileBytes * kStages;
+static_assert(kTileBytes % 1024 == 0, "operand tiles must keep the swizzle phase");
+
+struct PrefillParams {
+  int L, H, E, K, I, Is, use_norm, T, nch, tpc;
+  float eps;
+  const uint8_t* pool;  // layer l expert e at pool + (base[l] + (pin[l][e] & 0xffff)) * slot_bytes
+  uint64_t slot_bytes;
+  SlotLayout lay, slay;
+  const uint8_t* shared_pool;
+  uint64_t shared_slot_bytes;
+  const uint16_t* router;  // [L][nch][E][16] bf16
+  const float* bias;       // [L][E] or null
+  const float* gain;       // [L][H]
+  const int32_t* pin_slot;
+  const int32_t* layer_base;
+  uint32_t* hist;
+  PrefillScratch s;
+};
+
+__device__ __forceinline__ uint32_t smem_u32p(const void* ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+__device__ __forceinline__ float bf16_lo_p(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_p(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, int l, int e) {
+  if (e >= p.E) return p.shared_pool + (size_t)l * p.shared_slot_bytes;
+  return p.pool + (size_t)(p.layer_base[l] + (p.pin_slot[(size_t)l * p.E + e] & 0xffff)) * p.slot_bytes;
+}
+
+// ------------------------------------------------------------------ route
+
+constexpr int kRTok = 8;  // tokens per warp in the router
+
+// CTA of 8 warps, p.tpc (8 or 16) tokens.  Logit z_e of a token is the canonical fold of
+// its 16-column chunk partials (each an fmaf chain from +0): fold lane q adds chunks
+// q, q + 32, ... from +0, then the lanes combine as the xor butterfly 16, 8, 4, 2, 1
+// does.  That butterfly's result at lane 0 is a fixed binary tree over the 32 lane sums,
+// which this kernel evaluates leaf by leaf in bit-reversed lane order with a 5-deep
+// stack (a binary counter), so one thread forms whole logits for 8 tokens x 2 experts
+// while reusing every weight load 8 times.
+__global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, int l) {
+  extern __shared__ __align__(16) float rsm[];
+  const int H = p.H, E = p.E, nch = p.nch, TPC = p.tpc;
+  float* us = rsm;                       // [TPC][H]  u = g * h (or h)
+  float* zs = us + (size_t)TPC * H;      // [TPC][E]
+  float* invs = zs + (size_t)TPC * E;    // [TPC]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * TPC;
+  const float* g = p.gain + (size_t)l * H;
+
+  // 1. per token: inv (canonical fold of the squares), u into shared memory, x hi/lo out
+  for (int tl = warp; tl < TPC; tl += kPT / 32) {
+    const int t = t0 + tl;
+    float* u = us + (size_t)tl * H;
+    if (t >= p.T) {
+      for (int j = lane; j < H; j += 32) u[j] = 0.0f;
+      if (lane == 0) invs[tl] = 1.0f;
+      continue;
+    }
+    const float* hrow = p.s.h + (size_t)t * H;
+    float inv = 1.0f;
+    if (p.use_norm) {
+      float acc = 0.0f;
+      for (int c = lane; c < nch; c += 32) {
+        const float4* hp = reinterpret_cast<const float4*>(hrow + c * 16);
+        float pc = 0.0f;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 q = hp[v];
+          pc = fmaf(q.x, q.x, pc);
+          pc = fmaf(q.y, q.y, pc);
+          pc = fmaf(q.z, q.z, pc);
+          pc = fmaf(q.w, q.w, pc);
+        }
+        acc = __fadd_rn(acc, pc);
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+      inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(acc, (float)H), p.eps)));
+    }
+    if (lane == 0) invs[tl] = inv;
+    for (int j = lane; j < H; j += 32) {
+      const float hv = hrow[j];
+      float xv = hv;
+      if (p.use_norm) {
+        u[j] = __fmul_rn(g[j], hv);
+        xv = __fmul_rn(__fmul_rn(hv, inv), g[j]);
+      } else {
+        u[j] = hv;
+      }
+      const __half hi = __float2half_rn(xv);
+      p.s.x_hi[(size_t)t * H + j] = hi;
+      p.s.x_lo[(size_t)t * H + j] = __float2half_rn(xv - __half2float(hi));
+    }
+  }
+  __syncthreads();
+
+  // 2. logits: warp job = (token group of 8, block of 64 experts); lane: experts e0, e0 + 32
+  const int neb = (E + 63) / 64, ntg = TPC / kRTok;
+  for (int job = warp; job < ntg * neb; job += kPT / 32) {
+    const int tg = job / neb, eb = job % neb;
+    const int e0 = eb * 64 + lane, e1 = e0 + 32;
+    const bool v0 = e0 < E, v1 = e1 < E;
+    const float* ub = us + (size_t)tg * kRTok * H;
+    float stk[5][kRTok][2];
+    float fin[kRTok][2];
+    for (int i = 0; i < 32; ++i) {
+      const int q = __brev(i) >> 27;  // bit-reversed leaf order
+      float leaf[kRTok][2];
+#pragma unroll
+      for (int t = 0; t < kRTok; ++t) leaf[t][0] = leaf[t][1] = 0.0f;
+      for (int c = q; c < nch; c += 32) {
+        const uint4* w0p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e0) * kChunk);
+        const uint4* w1p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e1) * kChunk);
+        uint4 wa0 = make_uint4(0, 0, 0, 0), wa1 = wa0, wb0 = wa0, wb1 = wa0;
+        if (v0) {
+          wa0 = __ldg(w0p);
+          wa1 = __ldg(w0p + 1);
+        }
+        if (v1) {
+          wb0 = __ldg(w1p);
+          wb1 = __ldg(w1p + 1);
+        }
+        const uint32_t wa[8] = {wa0.x, wa0.y, wa0.z, wa0.w, wa1.x, wa1.y, wa1.z, wa1.w};
+        const uint32_t wb[8] = {wb0.x, wb0.y, wb0.z, wb0.w, wb1.x, wb1.y, wb1.z, wb1.w};
+        float pc[kRTok][2];
+#pragma unroll
+        for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+#pragma unroll
+          for (int t = 0; t < kRTok; ++t) {
+            const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * H + c * kChunk + 4 * j4);
+            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
+            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
+            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
+            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
+            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
+            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
+            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
+            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < kRTok; ++t) {
+          leaf[t][0] = __fadd_rn(leaf[t][0], pc[t][0]);
+          leaf[t][1] = __fadd_rn(leaf[t][1], pc[t][1]);
+        }
+      }
+      // binary counter: level b combines while bit b of i is set
+      bool carry = true;
+#pragma unroll
+      for (int b = 0; b < 5; ++b) {
+        if (carry) {
+          if ((i >> b) & 1) {
+#pragma unroll
+            for (int t = 0; t < kRTok; ++t) {
+              leaf[t][0] = __fadd_rn(stk[b][t][0], leaf[t][0]);
+              leaf[t][1] = __fadd_rn(stk[b][t][1], leaf[t][1]);
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < kRTok; ++t) {
+              stk[b][t][0] = leaf[t][0];
+              stk[b][t][1] = leaf[t][1];
+            }
+            carry = false;
+          }
+        }
+      }
+      if (carry) {
+#pragma unroll
+        for (int t = 0; t < kRTok; ++t) {
+          fin[t][0] = leaf[t][0];
+          fin[t][1] = leaf[t][1];
+        }
+      }
+    }
+    const float b0 = (p.bias && v0) ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
+    const float b1 = (p.bias && v1) ? __ldg(p.bias + (size_t)l * E + e1) : 0.0f;
+#pragma unroll
+    for (int t = 0; t < kRTok; ++t) {
+      const float inv = invs[tg * kRTok + t];
+      if (v0) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(fin[t][0], inv, b0);
+      if (v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(fin[t][1], inv, b1);
+    }
+  }
+  __syncthreads();
+
+  // 3. top-k by (logit desc, index asc; -0 == +0; NaN never preferred), weights, counts
+  for (int tl = warp; tl < TPC; tl += kPT / 32) {
+    const int t = t0 + tl;
+    if (t >= p.T) continue;
+    const float* z = zs + (size_t)tl * E;
+    int my_e = -1;
+    uint32_t taken = 0;
+    for (int i = 0; i < p.K; ++i) {
+      uint64_t best = 0;
+      for (int k = 0; lane + 32 * k < E; ++k) {
+        if ((taken >> k) & 1u) continue;
+        const int e = lane + 32 * k;
+        float v = z[e];
+        if (v == 0.0f) v = 0.0f;
+        const uint32_t uu = __float_as_uint(v);
+        uint32_t o = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
+        if (v != v) o = 0;
+        const uint64_t key = ((uint64_t)o << 32) | (uint32_t)(~(uint32_t)e);
+        best = key > best ? key : best;
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)best, off);
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(best >> 32), off);
+        const uint64_t o = ((uint64_t)hi << 32) | lo;
+        best = o > best ? o : best;
+      }
+      int e = (int)(~(uint32_t)best);
+      if ((best >> 32) == 0ull) {  // only NaN logits left
+        if (lane == 0) atomicCAS(p.s.error, 0, MOE_DEVERR_ROUTE);
+        e = 0;
+      }
+      if ((e & 31) == lane) taken |= 1u << (e >> 5);
+      if (lane == i) my_e = e;
+    }
+    const float zmax = __shfl_sync(0xffffffffu, lane < p.K ? z[my_e] : 0.0f, 0);
+    const float ex = lane < p.K ? expf(z[my_e] - zmax) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < p.K) {
+      p.s.sel[(size_t)t * p.K + lane] = my_e;
+      p.s.w[(size_t)t * p.K + lane] = __fdividef(ex, sum);
+      atomicAdd(p.hist + (size_t)l * E + my_e, 1u);
+      atomicAdd(p.s.counts + my_e, 1);
+      if (p.s.sel_trace) p.s.sel_trace[((size_t)l * p.T + t) * p.K + lane] = my_e;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ grouping
+
+// One CTA of 1024 threads: exclusive offsets over experts 0..E (E = the shared expert,
+// which takes every token), the list of 128-row m-tiles, and the counters zeroed for the
+// next layer.
+__global__ void __launch_bounds__(1024) prefill_scan(const PrefillParams p) {
+  __shared__ int wsum[32], wtil[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_ent = p.E + 1;
+  int n[2] = {0, 0}, m[2] = {0, 0};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = 2 * tid + k;
+    if (e < p.E) n[k] = p.s.counts[e];
+    if (e == p.E) n[k] = p.Is > 0 ? p.T : 0;
+    m[k] = (n[k] + kTM - 1) / kTM;
+  }
+  int a = n[0] + n[1], b = m[0] + m[1];
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {  // inclusive warp scans
+    const int ya = __shfl_up_sync(0xffffffffu, a, off), yb = __shfl_up_sync(0xffffffffu, b, off);
+    if (lane >= off) {
+      a += ya;
+      b += yb;
+    }
+  }
+  if (lane == 31) {
+    wsum[warp] = a;
+    wtil[warp] = b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int x = wsum[lane], y = wtil[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int xa = __shfl_up_sync(0xffffffffu, x, off), yb = __shfl_up_sync(0xffffffffu, y, off);
+      if (lane >= off) {
+        x += xa;
+        y += yb;
+      }
+    }
+    wsum[lane] = x;
+    wtil[lane] = y;
+  }
+  __syncthreads();
+  int off_n = a - n[0] - n[1] + (warp ? wsum[warp - 1] : 0);
+  int off_m = b - m[0] - m[1] + (warp ? wtil[warp - 1] : 0);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = 2 * tid + k;
+    if (e < n_ent) {
+      p.s.offsets[e] = off_n;
+      for (int mt = 0; mt < m[k]; ++mt) p.s.jobs[off_m + mt] = (e << 20) | mt;
+      p.s.cursor[e] = 0;
+      if (e < p.E) p.s.counts[e] = 0;
+    }
+    if (e == n_ent - 1) {
+      p.s.offsets[n_ent] = off_n + n[k];
+      *p.s.n_jobs = off_m + m[k];
+    }
+    off_n += n[k];
+    off_m += m[k];
+  }
+}
+
+// One warp per token: each of its k routed rows (and its shared-expert row) takes a
+// place in its expert's group, and the token's x row (hi and lo) is copied there.
+__global__ void __launch_bounds__(kPT) prefill_scatter(const PrefillParams p) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kPT / 32) + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  const int nr = p.K + (p.Is > 0 ? 1 : 0);
+  const int vec = p.H / 8;
+  const uint4* src_hi = reinterpret_cast<const uint4*>(p.s.x_hi + (size_t)t * p.H);
+  const uint4* src_lo = reinterpret_cast<const uint4*>(p.s.x_lo + (size_t)t * p.H);
+  for (int r = 0; r < nr; ++r) {
+    int pos = 0;
+    if (lane == 0) {
+      if (r < p.K) {
+        const int e = p.s.sel[(size_t)t * p.K + r];
+        pos = p.s.offsets[e] + atomicAdd(p.s.cursor + e, 1);
+      } else {
+        pos = p.s.offsets[p.E] + t;
+      }
+      p.s.perm[pos] = (t << 8) | r;
+    }
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    uint4* dh = reinterpret_cast<uint4*>(p.s.xg_hi + (size_t)pos * p.H);
+    uint4* dl = reinterpret_cast<uint4*>(p.s.xg_lo + (size_t)pos * p.H);
+    for (int c = lane; c < vec; c += 32) {
+      dh[c] = src_hi[c];
+      dl[c] = src_lo[c];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ tcgen05 grouped GEMM
+
+__device__ __forceinline__ void pmbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32p(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool pmbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32p(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (about 2 s); false when it ran out.
+__device__ __forceinline__ bool pmbar_wait(uint64_t* bar, uint32_t parity) {
+  if (pmbar_try(bar, parity)) return true;
+  uint64_t t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (!pmbar_try(bar, parity)) {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > 2000000000ull) return false;
+  }
+  return true;
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (the layout a 64-column fp16 TMA box with 128-byte swizzle writes).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);  // start address / 16
+  d |= (uint64_t)1 << 16;                  // leading byte offset (unused when swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset / 16
+  d |= (uint64_t)1 << 46;                  // descriptor version of sm_100
+  d |= (uint64_t)2 << 61;                  // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: f16 x f16 -> f32, A and B K-major, M = 128, N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem, uint64_t da, uint64_t db, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}" ::"r"(tmem),
+      "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Wait for this thread's tensor-memory loads.  The registers they fill pass through the
+// wait as operands, so no copy of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+
+template <int MODE>  // 0: gate/up + SwiGLU, 1: down
+__global__ void __launch_bounds__(kPT, 1)
+    prefill_gemm(const PrefillParams p, int l, const __grid_constant__ CUtensorMap tm_hi,
+                 const __grid_constant__ CUtensorMap tm_lo) {
+  extern __shared__ __align__(1024) uint8_t psm_raw[];
+  const int imax = p.I > p.Is ? p.I : p.Is;
+  const int n_tiles = MODE == 0 ? (2 * imax) / kTN : p.H / kTN;
+  const int job = blockIdx.x / n_tiles, nt = blockIdx.x % n_tiles;
+  if (job >= *p.s.n_jobs) return;
+  const int je = p.s.jobs[job], e = je >> 20, mt = je & 0xFFFFF;
+  const int Ie = e < p.E ? p.I : p.Is;
+  if (MODE == 0 && nt * (kTN / 2) >= Ie) return;  // past the width of a narrower expert
+  const int g0 = p.s.offsets[e], n_e = p.s.offsets[e + 1] - g0;
+  const int row0 = g0 + mt * kTM;
+  const int K = MODE == 0 ? p.H : Ie;
+  const int nK = K / kTK, nbk = K / 32;
+  const SlotLayout& Ls = e < p.E ? p.lay : p.slay;
+  const uint8_t* slot = expert_slot(p, l, e);
+
+  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, then [raw 4.5K] x S, barriers
+  uint8_t* psm = psm_raw + ((1024u - (smem_u32p(psm_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(psm + kTilesBytes + kStages * kRawBytes);  // a_full[S], mma_done[S], fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  auto a_hi = [&](int s) { return psm + s * 3 * kTileBytes; };
+  auto a_lo = [&](int s) { return psm + s * 3 * kTileBytes + kTileBytes; };
+  auto b_t = [&](int s) { return psm + s * 3 * kTileBytes + 2 * kTileBytes; };
+  auto raw = [&](int s) { return psm + kTilesBytes + s * kRawBytes; };
+
+  if (tid == 0) {
+    for (int s = 0; s < 2 * kStages + 1; ++s) pmbar_init(&bars[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32p(tmem_slot)),
+                 "r"(kTN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  // B row n of this tile -> weight row: gate/up tiles hold 64 gate rows then the same 64 up rows
+  const int brow = tid >> 1, bkb = tid & 1;
+  const int wrow = MODE == 0 ? nt * (kTN / 2) + (brow & 63) : nt * kTN + brow;
+  const uint8_t* rbase;  // the 16-row tile holding that row
+  if (MODE == 0)
+    rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (brow >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
+  else
+    rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * Ie;
+  const int rr = wrow % 16;
+  const uint8_t* qrow = rbase + (size_t)rr * nbk * 16;                          // the row's nibbles
+  const uint8_t* drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;  // the row's scales
+
+  auto load_stage = [&](int ks) {  // A by TMA (thread 0), B's raw Q4_0 bytes by cp.async
+    const int s = ks % kStages;
+    if (tid == 0) {
+      const uint32_t bar = smem_u32p(&bars[s]);
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+              "r"(smem_u32p(a_hi(s))),
+          "l"(&tm_hi), "r"(ks * kTK), "r"(row0), "r"(bar)
+          : "memory");
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+              "r"(smem_u32p(a_lo(s))),
+          "l"(&tm_lo), "r"(ks * kTK), "r"(row0), "r"(bar)
+          : "memory");
+    }
+    uint8_t* rs = raw(s);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + tid * 16)),
+                 "l"(qrow + (size_t)(2 * ks + bkb) * 16)
+                 : "memory");
+    if (bkb == 0)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + kTN * 32 + brow * 4)),
+                   "l"(drow + (size_t)(2 * ks) * 2)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  bool ok = true;
+  for (int ks = 0; ks < kStages - 1 && ks < nK; ++ks) load_stage(ks);
+  for (int ks = 0; ks < nK; ++ks) {
+    const int s = ks % kStages;
+    // this thread's raw bytes of stage ks have landed (groups after it: min(S - 2, nK - 1 - ks))
+    const int later = nK - 1 - ks;
+    if (later >= kStages - 2)
+      asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 2) : "memory");
+    else if (later == 1)
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    // B[s] was last read by the MMAs of stage ks - S, which thread 0 saw complete before
+    // it refilled that stage's buffers at iteration ks - S + 1 (and everyone synced since).
+    {  // dequantise this thread's 32 weights (row brow, block bkb) into the swizzled tile
+      const uint8_t* rs = raw(s);
+      const uint4 q = *reinterpret_cast<const uint4*>(rs + tid * 16);
+      const float d = __half2float(reinterpret_cast<const __half*>(rs + kTN * 32 + brow * 4)[bkb]);
+      const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+      uint8_t* bt = b_t(s) + (brow >> 3) * 1024 + (brow & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // 16-byte chunk c of the block: weights 8c .. 8c + 7
+        const int hi_nib = c >> 1, wsel = (c & 1) * 2;
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {  // weights 8c + 2j, 8c + 2j + 1: bytes 2j, 2j + 1 of the 8
+          const uint32_t word = qw[wsel + (j >> 1)];
+          const int sh = (j & 1) * 16 + hi_nib * 4;
+          const float v0 = (float)((int)((word >> sh) & 15u) - 8) * d;
+          const float v1 = (float)((int)((word >> (sh + 8)) & 15u) - 8) * d;
+          const __half2 hv = __floats2half2_rn(v0, v1);
+          out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        const int chunk = bkb * 4 + c;
+        *reinterpret_cast<uint4*>(bt + ((chunk ^ (brow & 7)) * 16)) = make_uint4(out[0], out[1], out[2], out[3]);
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      if (!pmbar_wait(&bars[s], (uint32_t)(ks / kStages) & 1u)) ok = false;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sh = smem_u32p(a_hi(s)), sl = smem_u32p(a_lo(s)), sb = smem_u32p(b_t(s));
+#pragma unroll
+      for (int kk = 0; kk < kTK / 16; ++kk) {
+        const uint64_t db = umma_desc(sb + kk * 32);
+        umma_f16(tmem, umma_desc(sh + kk * 32), db, (ks > 0 || kk > 0) ? 1u : 0u);
+        umma_f16(tmem, umma_desc(sl + kk * 32), db, 1u);
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32p(&bars[kStages + s]))
+                   : "memory");
+      // stage ks + S - 1 reuses the buffers of stage ks - 1: wait for its MMAs
+      if (ks >= 1 && ks + kStages - 1 < nK &&
+          !pmbar_wait(&bars[kStages + (ks - 1) % kStages], (uint32_t)((ks - 1) / kStages) & 1u))
+        ok = false;
+    }
+    if (ks + kStages - 1 < nK) load_stage(ks + kStages - 1);
+  }
+  if (tid == 0)
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32p(&bars[2 * kStages]))
+                 : "memory");
+  if (!pmbar_wait(&bars[2 * kStages], 0)) ok = false;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (!ok) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
+
+  // epilogue: warp w reads tile rows 32 (w % 4) .. + 31 (its TMEM lane quarter); column half w / 4
+  {
+    const int lane = tid & 31, quarter = warp & 3, colh = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const bool valid = mt * kTM + row < n_e;
+    const int grow = row0 + row;
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (MODE == 0) {  // gate columns 0..63, up columns 64..127
+      for (int c0 = colh * 32; c0 < colh * 32 + 32; c0 += 16) {
+        uint32_t gr[16], ur[16];
+        tmem_ld16(taddr + c0, gr);
+        tmem_ld16(taddr + 64 + c0, ur);
+        tmem_wait16(gr);
+        tmem_wait16(ur);
+        if (valid) {
+          __align__(16) __half hi[16];
+          __align__(16) __half lo[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float gv = __uint_as_float(gr[j]), uv = __uint_as_float(ur[j]);
+            const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+            hi[j] = __float2half_rn(a);
+            lo[j] = __float2half_rn(a - __half2float(hi[j]));
+          }
+          const size_t off = (size_t)grow * imax + nt * (kTN / 2) + c0;
+          uint4* dh = reinterpret_cast<uint4*>(p.s.a_hi + off);
+          uint4* dl = reinterpret_cast<uint4*>(p.s.a_lo + off);
+          dh[0] = reinterpret_cast<const uint4*>(hi)[0];
+          dh[1] = reinterpret_cast<const uint4*>(hi)[1];
+          dl[0] = reinterpret_cast<const uint4*>(lo)[0];
+          dl[1] = reinterpret_cast<const uint4*>(lo)[1];
+        }
+      }
+    } else {
+      const int pr = valid ? p.s.perm[grow] : 0;
+      const int tok = pr >> 8, rank = pr & 0xFF;
+      float* dst = p.s.obuf + ((size_t)tok * (p.K + 1) + rank) * p.H + nt * kTN;
+      for (int c0 = colh * 64; c0 < colh * 64 + 64; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(taddr + c0, o);
+        tmem_wait16(o);
+        if (valid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            d4[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
+                                __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN));
+}
+
+// ------------------------------------------------------------------ combine
+
+// h[t] += sum_rank w * o_rank + o_shared in rank order (without the norm: h = that sum).
+__global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, int l) {
+  const int t = blockIdx.x;
+  const float* w = p.s.w + (size_t)t * p.K;
+  const float* ob = p.s.obuf + (size_t)t * (p.K + 1) * p.H;
+  for (int j = threadIdx.x; j < p.H; j += kPT) {
+    float y = 0.0f;
+    for (int r = 0; r < p.K; ++r) y = fmaf(w[r], ob[(size_t)r * p.H + j], y);
+    if (p.Is > 0) y = __fadd_rn(y, ob[(size_t)p.K * p.H + j]);
+    const size_t o = (size_t)t * p.H + j;
+    const float hn = p.use_norm ? __fadd_rn(p.s.h[o], y) : y;
+    p.s.h[o] = hn;
+    if (p.s.h_trace) p.s.h_trace[((size_t)(l + 1) * p.T + t) * p.H + j] = hn;
+    if (l == p.L - 1) p.s.y[o] = hn;
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+static uint32_t gemm_smem() { return kTilesBytes + kStages * kRawBytes + (2 * kStages + 1) * 8 + 8 + 1024; }
+static int route_tpc(int H, int E) { return ((size_t)16 * (H + E) + 16) * 4 <= 200 * 1024 ? 16 : 8; }
+static uint32_t route_smem(int H, int E) { return (uint32_t)(((size_t)route_tpc(H, E) * (H + E) + 16) * 4); }
+
+int prefill_supported(int H, int E, int K, int I, int Is) {
+  if (H % kTN || H > kMaxH || I % kTK || Is % kTK || E > kMaxE || K > 32) return 0;
+  return route_smem(H, E) <= 227 * 1024;
+}
+
+cudaError_t prefill_configure(int H, int E) {
+  cudaError_t e = cudaFuncSetAttribute(prefill_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_route, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_smem(H, E));
+  return e;
+}
+
+typedef CUresult (*PfnEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// Row-major fp16 [rows x cols] -> tensor map of 64-column x 128-row boxes, 128-byte swizzle.
+static int make_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTK, (cuuint32_t)kTM};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, cudaStream_t st) {
+  PrefillParams p{};
+  p.L = a.L;
+  p.H = a.H;
+  p.E = a.E;
+  p.K = a.K;
+  p.I = a.I;
+  p.Is = a.Is;
+  p.use_norm = a.use_norm;
+  p.T = a.T;
+  p.eps = a.eps;
+  p.nch = a.H / kChunk;
+  p.tpc = route_tpc(a.H, a.E);
+  p.pool = a.pool;
+  p.slot_bytes = a.slot_bytes;
+  p.lay = a.lay;
+  p.slay = a.slay;
+  p.shared_pool = a.shared_pool;
+  p.shared_slot_bytes = a.shared_slot_bytes;
+  p.router = a.router;
+  p.bias = a.bias;
+  p.gain = a.gain;
+  p.pin_slot = a.pin_slot;
+  p.layer_base = a.layer_base;
+  p.hist = a.hist;
+  p.s = s;
+  const int T = a.T, H = a.H, E = a.E;
+  const int imax = a.I > a.Is ? a.I : a.Is;
+  const int R = T * a.K + (a.Is > 0 ? T : 0);
+  PfnEncodeTiled enc = reinterpret_cast<PfnEncodeTiled>(encode_fn);
+  CUtensorMap mx_hi, mx_lo, ma_hi, ma_lo;
+  if (make_map(enc, &mx_hi, s.xg_hi, R, H) || make_map(enc, &mx_lo, s.xg_lo, R, H) ||
+      make_map(enc, &ma_hi, s.a_hi, R, imax) || make_map(enc, &ma_lo, s.a_lo, R, imax))
+    return -1;
+  const int max_jobs = (R + kTM - 1) / kTM + E + 1;
+  cudaError_t e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * E, st);
+  if (e == cudaSuccess && s.h_trace)
+    e = cudaMemcpyAsync(s.h_trace, s.h, sizeof(float) * T * H, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return (int)e;
+  for (int l = 0; l < a.L; ++l) {
+    prefill_route<<<(T + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
+    prefill_scan<<<1, 1024, 0, st>>>(p);
+    prefill_scatter<<<(T + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
+    prefill_gemm<0><<<max_jobs * ((2 * imax) / kTN), kPT, gemm_smem(), st>>>(p, l, mx_hi, mx_lo);
+    prefill_gemm<1><<<max_jobs * (H / kTN), kPT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
+    prefill_combine<<<T, kPT, 0, st>>>(p, l);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+  }
+  return 0;
+}
+
+}  // namespace moe

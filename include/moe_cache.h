@@ -175,9 +175,27 @@ MOE_API int moe_decode_step(moe_ctx *ctx, const float *x_dev, float *y_dev, void
  * device, the step runs, y_host [H] receives the result.  Returns the step's status. */
 MOE_API int moe_decode_step_host(moe_ctx *ctx, const float *x_host, float *y_host);
 
-/* Batched prefill of T tokens (x_dev [T][H] -> y_dev [T][H]).  Not in this build:
- * returns MOE_ERR_UNSUPPORTED. */
+/* Batched prefill: n_tokens tokens through the whole stack at once, x_dev [T][H] ->
+ * y_dev [T][H] (fp32, device, caller-owned, may not overlap), enqueued on stream.
+ * The pages describe decode; this is the same layer computed for a batch: per layer,
+ * each token's routing (logits in the same canonical fp32 order as decode, so the
+ * top-k choices agree with a decode of the same hidden state; the routing histogram
+ * accumulates as in decode), tokens grouped by expert, the expert SwiGLU FFNs as
+ * grouped tensor-core GEMMs (Q4_0 weights dequantised to fp16, activations carried as
+ * fp16 hi + lo pairs, fp32 accumulation), and the weighted combine plus shared expert.
+ * Needs every expert resident (moe_set_residency(1.0)): else MOE_ERR_STATE.  Shapes
+ * need hidden % 128 == 0 and inter, shared_inter % 64 == 0: else MOE_ERR_UNSUPPORTED.
+ * Scratch for the largest n_tokens seen so far is kept by the context (about
+ * T * (k + 1) * hidden * 10 bytes); a larger n_tokens reallocates it, synchronising the
+ * device.  The cache's rings, counters and event log are not touched.  Errors of the
+ * kernels' bounded waits surface at moe_sync as MOE_ERR_TIMEOUT. */
 MOE_API int moe_prefill(moe_ctx *ctx, const float *x_dev, int32_t n_tokens, float *y_dev, void *stream);
+
+/* Prefill tracing: when non-NULL, moe_prefill writes its input and every layer's output
+ * to h_trace_dev ([(L+1)][T][H] fp32) and each layer's top-k choices in rank order to
+ * sel_trace_dev ([L][T][k] int32), T being the call's n_tokens.  Device pointers owned
+ * by the caller; pass NULLs to stop. */
+MOE_API int moe_set_prefill_trace(moe_ctx *ctx, float *h_trace_dev, int32_t *sel_trace_dev);
 
 /* Wait for all work of the context and report a device-side failure as an error code
  * (MOE_ERR_TIMEOUT for a wait that ran out, MOE_ERR_DEVICE otherwise). */
