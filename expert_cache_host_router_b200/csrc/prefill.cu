@@ -40,7 +40,6 @@ constexpr int kTN = 128;  // GEMM tile columns
 constexpr int kTK = 64;   // K per pipeline stage: one 128-byte swizzle row of fp16
 constexpr int kStages = 4;
 constexpr uint32_t kTileBytes = kTM * kTK * 2;           // 16 KB per fp16 operand tile
-constexpr uint32_t kRawBytes = kTN * 2 * 16 + kTN * 4;  // nibbles of 2 blocks x 128 rows + their scales
 // Swizzled operand tiles first, each at a multiple of 1024 bytes (the 128-byte swizzle's
 // period: TMA and the MMA take its phase from the address), then the raw weight bytes.
 constexpr uint32_t kTilesBytes = 3 * kTileBytes * kStages;
@@ -78,19 +77,23 @@ __device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, in
 
 constexpr int kRTok = 8;  // tokens per warp in the router
 
+// Row stride of u in shared memory: 16-column chunks padded to 20 floats, so the 32
+// lanes' 128-bit loads of 32 different chunks fall in 8 different bank groups.
+constexpr int kUChunk = 20;
+
 // CTA of 8 warps, p.tpc (8 or 16) tokens.  Logit z_e of a token is the canonical fold of
 // its 16-column chunk partials (each an fmaf chain from +0): fold lane q adds chunks
-// q, q + 32, ... from +0, then the lanes combine as the xor butterfly 16, 8, 4, 2, 1
-// does.  That butterfly's result at lane 0 is a fixed binary tree over the 32 lane sums,
-// which this kernel evaluates leaf by leaf in bit-reversed lane order with a 5-deep
-// stack (a binary counter), so one thread forms whole logits for 8 tokens x 2 experts
-// while reusing every weight load 8 times.
+// q, q + 32, ... from +0, then the lanes combine as the xor butterfly 16, 8, 4, 2, 1.
+// Here the fold's lanes are the warp's lanes: a warp job is 8 tokens x 2 experts, lane q
+// forms the 16 lane sums of its chunks and the butterfly runs on shuffles, so every
+// router weight a lane loads is used for 8 tokens.
 __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, int l) {
   extern __shared__ __align__(16) float rsm[];
   const int H = p.H, E = p.E, nch = p.nch, TPC = p.tpc;
-  float* us = rsm;                       // [TPC][H]  u = g * h (or h)
-  float* zs = us + (size_t)TPC * H;      // [TPC][E]
-  float* invs = zs + (size_t)TPC * E;    // [TPC]
+  const int ustride = nch * kUChunk;
+  float* us = rsm;                        // [TPC][nch][20]  u = g * h (or h), padded chunks
+  float* zs = us + (size_t)TPC * ustride;  // [TPC][E]
+  float* invs = zs + (size_t)TPC * E;     // [TPC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * TPC;
   const float* g = p.gain + (size_t)l * H;
@@ -98,9 +101,9 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
   // 1. per token: inv (canonical fold of the squares), u into shared memory, x hi/lo out
   for (int tl = warp; tl < TPC; tl += kPT / 32) {
     const int t = t0 + tl;
-    float* u = us + (size_t)tl * H;
+    float* u = us + (size_t)tl * ustride;
     if (t >= p.T) {
-      for (int j = lane; j < H; j += 32) u[j] = 0.0f;
+      for (int j = lane; j < H; j += 32) u[(j >> 4) * kUChunk + (j & 15)] = 0.0f;
       if (lane == 0) invs[tl] = 1.0f;
       continue;
     }
@@ -129,11 +132,12 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
     for (int j = lane; j < H; j += 32) {
       const float hv = hrow[j];
       float xv = hv;
+      float* uj = u + (j >> 4) * kUChunk + (j & 15);
       if (p.use_norm) {
-        u[j] = __fmul_rn(g[j], hv);
+        *uj = __fmul_rn(g[j], hv);
         xv = __fmul_rn(__fmul_rn(hv, inv), g[j]);
       } else {
-        u[j] = hv;
+        *uj = hv;
       }
       const __half hi = __float2half_rn(xv);
       p.s.x_hi[(size_t)t * H + j] = hi;
@@ -142,94 +146,77 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
   }
   __syncthreads();
 
-  // 2. logits: warp job = (token group of 8, block of 64 experts); lane: experts e0, e0 + 32
-  const int neb = (E + 63) / 64, ntg = TPC / kRTok;
-  for (int job = warp; job < ntg * neb; job += kPT / 32) {
-    const int tg = job / neb, eb = job % neb;
-    const int e0 = eb * 64 + lane, e1 = e0 + 32;
-    const bool v0 = e0 < E, v1 = e1 < E;
-    const float* ub = us + (size_t)tg * kRTok * H;
-    float stk[5][kRTok][2];
-    float fin[kRTok][2];
-    for (int i = 0; i < 32; ++i) {
-      const int q = __brev(i) >> 27;  // bit-reversed leaf order
-      float leaf[kRTok][2];
+  // 2. logits: warp job = (token group of 8, expert pair); lane q = fold lane q
+  const int ntg = TPC / kRTok, npair = (E + 1) / 2;
+  for (int job = warp; job < ntg * npair; job += kPT / 32) {
+    const int tg = job % ntg, e0 = 2 * (job / ntg), e1 = e0 + 1;
+    const bool v1 = e1 < E;
+    const float* ub = us + (size_t)tg * kRTok * ustride;
+    auto wload = [&](int c, uint4 (&w)[4]) {
+      const uint4* w0p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e0) * kChunk);
+      w[0] = __ldg(w0p);
+      w[1] = __ldg(w0p + 1);
+      w[2] = w[3] = make_uint4(0, 0, 0, 0);
+      if (v1) {
+        w[2] = __ldg(w0p + 2);  // expert e0 + 1 follows e0 in the same chunk row
+        w[3] = __ldg(w0p + 3);
+      }
+    };
+    float ls[kRTok][2];
 #pragma unroll
-      for (int t = 0; t < kRTok; ++t) leaf[t][0] = leaf[t][1] = 0.0f;
-      for (int c = q; c < nch; c += 32) {
-        const uint4* w0p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e0) * kChunk);
-        const uint4* w1p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e1) * kChunk);
-        uint4 wa0 = make_uint4(0, 0, 0, 0), wa1 = wa0, wb0 = wa0, wb1 = wa0;
-        if (v0) {
-          wa0 = __ldg(w0p);
-          wa1 = __ldg(w0p + 1);
-        }
-        if (v1) {
-          wb0 = __ldg(w1p);
-          wb1 = __ldg(w1p + 1);
-        }
-        const uint32_t wa[8] = {wa0.x, wa0.y, wa0.z, wa0.w, wa1.x, wa1.y, wa1.z, wa1.w};
-        const uint32_t wb[8] = {wb0.x, wb0.y, wb0.z, wb0.w, wb1.x, wb1.y, wb1.z, wb1.w};
-        float pc[kRTok][2];
+    for (int t = 0; t < kRTok; ++t) ls[t][0] = ls[t][1] = 0.0f;
+    uint4 cw[4];
+    if (lane < nch) wload(lane, cw);
+    for (int c = lane; c < nch; c += 32) {
+      uint4 nw[4];
+      const bool more = c + 32 < nch;
+      if (more) wload(c + 32, nw);
+      const uint32_t wa[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w, cw[1].x, cw[1].y, cw[1].z, cw[1].w};
+      const uint32_t wb[8] = {cw[2].x, cw[2].y, cw[2].z, cw[2].w, cw[3].x, cw[3].y, cw[3].z, cw[3].w};
+      float pc[kRTok][2];
 #pragma unroll
-        for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
+      for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
 #pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-#pragma unroll
-          for (int t = 0; t < kRTok; ++t) {
-            const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * H + c * kChunk + 4 * j4);
-            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
-            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
-            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
-            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
-            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
-            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
-            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
-            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
-          }
-        }
+      for (int j4 = 0; j4 < 4; ++j4) {
 #pragma unroll
         for (int t = 0; t < kRTok; ++t) {
-          leaf[t][0] = __fadd_rn(leaf[t][0], pc[t][0]);
-          leaf[t][1] = __fadd_rn(leaf[t][1], pc[t][1]);
+          const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * ustride + c * kUChunk + 4 * j4);
+          pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
+          pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
+          pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
+          pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
+          pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
+          pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
+          pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
+          pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
         }
       }
-      // binary counter: level b combines while bit b of i is set
-      bool carry = true;
 #pragma unroll
-      for (int b = 0; b < 5; ++b) {
-        if (carry) {
-          if ((i >> b) & 1) {
-#pragma unroll
-            for (int t = 0; t < kRTok; ++t) {
-              leaf[t][0] = __fadd_rn(stk[b][t][0], leaf[t][0]);
-              leaf[t][1] = __fadd_rn(stk[b][t][1], leaf[t][1]);
-            }
-          } else {
-#pragma unroll
-            for (int t = 0; t < kRTok; ++t) {
-              stk[b][t][0] = leaf[t][0];
-              stk[b][t][1] = leaf[t][1];
-            }
-            carry = false;
-          }
-        }
+      for (int t = 0; t < kRTok; ++t) {
+        ls[t][0] = __fadd_rn(ls[t][0], pc[t][0]);
+        ls[t][1] = __fadd_rn(ls[t][1], pc[t][1]);
       }
-      if (carry) {
-#pragma unroll
-        for (int t = 0; t < kRTok; ++t) {
-          fin[t][0] = leaf[t][0];
-          fin[t][1] = leaf[t][1];
-        }
+      if (more) {
+        cw[0] = nw[0];
+        cw[1] = nw[1];
+        cw[2] = nw[2];
+        cw[3] = nw[3];
       }
     }
-    const float b0 = (p.bias && v0) ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+#pragma unroll
+      for (int t = 0; t < kRTok; ++t) {
+        ls[t][0] = __fadd_rn(ls[t][0], __shfl_xor_sync(0xffffffffu, ls[t][0], off));
+        ls[t][1] = __fadd_rn(ls[t][1], __shfl_xor_sync(0xffffffffu, ls[t][1], off));
+      }
+    }
+    const float b0 = p.bias ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
     const float b1 = (p.bias && v1) ? __ldg(p.bias + (size_t)l * E + e1) : 0.0f;
 #pragma unroll
     for (int t = 0; t < kRTok; ++t) {
-      const float inv = invs[tg * kRTok + t];
-      if (v0) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(fin[t][0], inv, b0);
-      if (v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(fin[t][1], inv, b1);
+      if (lane == 2 * t) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(ls[t][0], invs[tg * kRTok + t], b0);
+      if (lane == 2 * t + 1 && v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(ls[t][1], invs[tg * kRTok + t], b1);
     }
   }
   __syncthreads();
@@ -394,18 +381,6 @@ __device__ __forceinline__ bool pmbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait (about 2 s); false when it ran out.
-__device__ __forceinline__ bool pmbar_wait(uint64_t* bar, uint32_t parity) {
-  if (pmbar_try(bar, parity)) return true;
-  uint64_t t0, t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-  while (!pmbar_try(bar, parity)) {
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (t - t0 > 2000000000ull) return false;
-  }
-  return true;
-}
-
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (the layout a 64-column fp16 TMA box with 128-byte swizzle writes).
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
@@ -448,6 +423,49 @@ __device__ __forceinline__ void tmem_wait16(uint32_t (&r)[16]) {
                : "memory");
 }
 
+// Bounded wait shared by the CTA's roles: false after about 2 s, or at once when another
+// role already gave up (then the tile's result is garbage, the error word says so, and
+// every role still runs to its end).
+__device__ __forceinline__ bool pmbar_wait_ab(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (pmbar_try(bar, parity)) return true;
+  uint64_t t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (!pmbar_try(bar, parity)) {
+    if (*abort) return false;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > 2000000000ull) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void pmbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32p(bar)) : "memory");
+}
+
+// fp16 pair of Q4_0 weights (q - 8) * d from two nibbles at bits 0..3 and 16..19 of v:
+// 0x6400 | q is the fp16 1024 + q, so subtracting 1032 leaves q - 8 exactly and the
+// product with d is the correctly rounded fp16((q - 8) * d).
+__device__ __forceinline__ uint32_t q4_pair(uint32_t v, __half2 d2) {
+  const uint32_t m = (v & 0x000F000Fu) | 0x64006400u;
+  const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&m), __half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408)));
+  const __half2 w = __hmul2(q, d2);
+  return *reinterpret_cast<const uint32_t*>(&w);
+}
+
+constexpr int kRawStages = 4;     // raw-byte ring depth of each dequant thread
+constexpr uint32_t kRawSlot = 48;  // one thread, one stage: 32 bytes of nibbles, 4 of scales, pad
+constexpr uint32_t kRawRing = kRawStages * kTN * kRawSlot;
+
+// One CTA per 128 x 128 output tile, warp roles joined by mbarriers:
+//   warp 0 lane 0   A producer: TMA of the activation tiles (hi, lo) of each K stage
+//   warp 1 lane 0   MMA issuer: 2 x 4 tcgen05.mma per stage, commit frees the stage
+//   warps 4..7      B producers: thread r owns row r of the weight tile; it streams that
+//                   row's Q4_0 bytes through a private cp.async ring 3 stages ahead and
+//                   dequantises each stage into the 128B-swizzled fp16 tile
+//   all warps       epilogue from tensor memory
 template <int MODE>  // 0: gate/up + SwiGLU, 1: down
 __global__ void __launch_bounds__(kPT, 1)
     prefill_gemm(const PrefillParams p, int l, const __grid_constant__ CUtensorMap tm_hi,
@@ -464,24 +482,32 @@ __global__ void __launch_bounds__(kPT, 1)
   const int row0 = g0 + mt * kTM;
   const int K = MODE == 0 ? p.H : Ie;
   const int nK = K / kTK, nbk = K / 32;
-  const SlotLayout& Ls = e < p.E ? p.lay : p.slay;
-  const uint8_t* slot = expert_slot(p, l, e);
 
-  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, then [raw 4.5K] x S, barriers
+  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, the raw rings, barriers
   uint8_t* psm = psm_raw + ((1024u - (smem_u32p(psm_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(psm + kTilesBytes + kStages * kRawBytes);  // a_full[S], mma_done[S], fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  uint8_t* raw = psm + kTilesBytes;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(raw + kRawRing);
+  uint64_t* full_b = full_a + kStages;
+  uint64_t* empty = full_b + kStages;
+  uint64_t* done = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto a_hi = [&](int s) { return psm + s * 3 * kTileBytes; };
   auto a_lo = [&](int s) { return psm + s * 3 * kTileBytes + kTileBytes; };
   auto b_t = [&](int s) { return psm + s * 3 * kTileBytes + 2 * kTileBytes; };
-  auto raw = [&](int s) { return psm + kTilesBytes + s * kRawBytes; };
 
   if (tid == 0) {
-    for (int s = 0; s < 2 * kStages + 1; ++s) pmbar_init(&bars[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      pmbar_init(&full_a[s], 1);
+      pmbar_init(&full_b[s], 4);
+      pmbar_init(&empty[s], 1);
+    }
+    pmbar_init(done, 1);
+    *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32p(tmem_slot)),
                  "r"(kTN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -491,117 +517,136 @@ __global__ void __launch_bounds__(kPT, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
-  // B row n of this tile -> weight row: gate/up tiles hold 64 gate rows then the same 64 up rows
-  const int brow = tid >> 1, bkb = tid & 1;
-  const int wrow = MODE == 0 ? nt * (kTN / 2) + (brow & 63) : nt * kTN + brow;
-  const uint8_t* rbase;  // the 16-row tile holding that row
-  if (MODE == 0)
-    rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (brow >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
-  else
-    rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * Ie;
-  const int rr = wrow % 16;
-  const uint8_t* qrow = rbase + (size_t)rr * nbk * 16;                          // the row's nibbles
-  const uint8_t* drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;  // the row's scales
-
-  auto load_stage = [&](int ks) {  // A by TMA (thread 0), B's raw Q4_0 bytes by cp.async
-    const int s = ks % kStages;
-    if (tid == 0) {
-      const uint32_t bar = smem_u32p(&bars[s]);
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
-                   : "memory");
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-              "r"(smem_u32p(a_hi(s))),
-          "l"(&tm_hi), "r"(ks * kTK), "r"(row0), "r"(bar)
-          : "memory");
-      asm volatile(
-          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-              "r"(smem_u32p(a_lo(s))),
-          "l"(&tm_lo), "r"(ks * kTK), "r"(row0), "r"(bar)
-          : "memory");
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int ks = 0; ks < nK; ++ks) {
+        const int s = ks % kStages;
+        if (ks >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(ks / kStages - 1) & 1u, abort)) break;
+        const uint32_t bar = smem_u32p(&full_a[s]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+            "[%4];" ::"r"(smem_u32p(a_hi(s))),
+            "l"(&tm_hi), "r"(ks * kTK), "r"(row0), "r"(bar)
+            : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+            "[%4];" ::"r"(smem_u32p(a_lo(s))),
+            "l"(&tm_lo), "r"(ks * kTK), "r"(row0), "r"(bar)
+            : "memory");
+      }
     }
-    uint8_t* rs = raw(s);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + tid * 16)),
-                 "l"(qrow + (size_t)(2 * ks + bkb) * 16)
-                 : "memory");
-    if (bkb == 0)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + kTN * 32 + brow * 4)),
-                   "l"(drow + (size_t)(2 * ks) * 2)
-                   : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-
-  bool ok = true;
-  for (int ks = 0; ks < kStages - 1 && ks < nK; ++ks) load_stage(ks);
-  for (int ks = 0; ks < nK; ++ks) {
-    const int s = ks % kStages;
-    // this thread's raw bytes of stage ks have landed (groups after it: min(S - 2, nK - 1 - ks))
-    const int later = nK - 1 - ks;
-    if (later >= kStages - 2)
-      asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 2) : "memory");
-    else if (later == 1)
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-    // B[s] was last read by the MMAs of stage ks - S, which thread 0 saw complete before
-    // it refilled that stage's buffers at iteration ks - S + 1 (and everyone synced since).
-    {  // dequantise this thread's 32 weights (row brow, block bkb) into the swizzled tile
-      const uint8_t* rs = raw(s);
-      const uint4 q = *reinterpret_cast<const uint4*>(rs + tid * 16);
-      const float d = __half2float(reinterpret_cast<const __half*>(rs + kTN * 32 + brow * 4)[bkb]);
-      const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-      uint8_t* bt = b_t(s) + (brow >> 3) * 1024 + (brow & 7) * 128;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int ks = 0; ks < nK; ++ks) {
+        const int s = ks % kStages;
+        const uint32_t ph = (uint32_t)(ks / kStages) & 1u;
+        if (!pmbar_wait_ab(&full_a[s], ph, abort) || !pmbar_wait_ab(&full_b[s], ph, abort)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t sh = smem_u32p(a_hi(s)), sl = smem_u32p(a_lo(s)), sb = smem_u32p(b_t(s));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {  // 16-byte chunk c of the block: weights 8c .. 8c + 7
-        const int hi_nib = c >> 1, wsel = (c & 1) * 2;
-        uint32_t out[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {  // weights 8c + 2j, 8c + 2j + 1: bytes 2j, 2j + 1 of the 8
-          const uint32_t word = qw[wsel + (j >> 1)];
-          const int sh = (j & 1) * 16 + hi_nib * 4;
-          const float v0 = (float)((int)((word >> sh) & 15u) - 8) * d;
-          const float v1 = (float)((int)((word >> (sh + 8)) & 15u) - 8) * d;
-          const __half2 hv = __floats2half2_rn(v0, v1);
-          out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+        for (int kk = 0; kk < kTK / 16; ++kk) {
+          const uint64_t db = umma_desc(sb + kk * 32);
+          umma_f16(tmem, umma_desc(sh + kk * 32), db, (ks > 0 || kk > 0) ? 1u : 0u);
+          umma_f16(tmem, umma_desc(sl + kk * 32), db, 1u);
         }
-        const int chunk = bkb * 4 + c;
-        *reinterpret_cast<uint4*>(bt + ((chunk ^ (brow & 7)) * 16)) = make_uint4(out[0], out[1], out[2], out[3]);
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32p(&empty[s]))
+                     : "memory");
       }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      if (!pmbar_wait(&bars[s], (uint32_t)(ks / kStages) & 1u)) ok = false;
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sh = smem_u32p(a_hi(s)), sl = smem_u32p(a_lo(s)), sb = smem_u32p(b_t(s));
-#pragma unroll
-      for (int kk = 0; kk < kTK / 16; ++kk) {
-        const uint64_t db = umma_desc(sb + kk * 32);
-        umma_f16(tmem, umma_desc(sh + kk * 32), db, (ks > 0 || kk > 0) ? 1u : 0u);
-        umma_f16(tmem, umma_desc(sl + kk * 32), db, 1u);
-      }
+      // arrives once every MMA issued above has completed (at once if none was)
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       smem_u32p(&bars[kStages + s]))
+                       smem_u32p(done))
                    : "memory");
-      // stage ks + S - 1 reuses the buffers of stage ks - 1: wait for its MMAs
-      if (ks >= 1 && ks + kStages - 1 < nK &&
-          !pmbar_wait(&bars[kStages + (ks - 1) % kStages], (uint32_t)((ks - 1) / kStages) & 1u))
-        ok = false;
     }
-    if (ks + kStages - 1 < nK) load_stage(ks + kStages - 1);
+  } else if (warp >= 4) {
+    // B row r of this tile -> weight row: gate/up tiles hold 64 gate rows then the same 64 up rows
+    const int r = tid - 128;
+    const SlotLayout& Ls = e < p.E ? p.lay : p.slay;
+    const uint8_t* slot = expert_slot(p, l, e);
+    const int wrow = MODE == 0 ? nt * (kTN / 2) + (r & 63) : nt * kTN + r;
+    const uint8_t* rbase;  // the 16-row tile holding that row
+    if (MODE == 0)
+      rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
+    else
+      rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * Ie;
+    const int rr = wrow % 16;
+    const uint8_t* qrow = rbase + (size_t)rr * nbk * 16;                          // the row's nibbles
+    const uint8_t* drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;  // the row's scales
+    auto fetch = [&](int ks) {
+      uint8_t* rs = raw + ((ks % kRawStages) * kTN + r) * kRawSlot;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs)), "l"(qrow + (size_t)ks * 32)
+                   : "memory");
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + 16)),
+                   "l"(qrow + (size_t)ks * 32 + 16)
+                   : "memory");
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + 32)), "l"(drow + (size_t)ks * 4)
+                   : "memory");
+    };
+    for (int ks = 0; ks < kRawStages - 1 && ks < nK; ++ks) {
+      fetch(ks);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    uint8_t* brow_base = nullptr;
+    for (int ks = 0; ks < nK; ++ks) {
+      // refill the ring slot consumed at ks - 1, then wait for stage ks (groups after it:
+      // min(kRawStages - 1, nK - 1 - ks))
+      if (ks + kRawStages - 1 < nK) fetch(ks + kRawStages - 1);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      const int later = nK - 1 - ks;
+      if (later >= kRawStages - 1)
+        asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
+      else if (later == 2)
+        asm volatile("cp.async.wait_group 2;" ::: "memory");
+      else if (later == 1)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      const uint8_t* rs = raw + ((ks % kRawStages) * kTN + r) * kRawSlot;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(rs);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(rs + 16);
+      const uint32_t sc = *reinterpret_cast<const uint32_t*>(rs + 32);
+      const int s = ks % kStages;
+      if (ks >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(ks / kStages - 1) & 1u, abort)) break;
+      brow_base = b_t(s) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        const uint4 q = blk ? q1 : q0;
+        const __half dh = __ushort_as_half((unsigned short)(blk ? (sc >> 16) : (sc & 0xFFFF)));
+        const __half2 d2 = __half2(dh, dh);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        uint32_t lo[8], hi[8];  // half2 pairs of weights (2j, 2j + 1) and (16 + 2j, 17 + 2j)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t r01 = __byte_perm(qw[w], 0, 0x4140), r23 = __byte_perm(qw[w], 0, 0x4342);
+          lo[2 * w] = q4_pair(r01, d2);
+          lo[2 * w + 1] = q4_pair(r23, d2);
+          hi[2 * w] = q4_pair(r01 >> 4, d2);
+          hi[2 * w + 1] = q4_pair(r23 >> 4, d2);
+        }
+        // 16-byte chunks of the block: weights 0-7, 8-15 (low nibbles), 16-23, 24-31 (high)
+        const int c0 = blk * 4;
+        *reinterpret_cast<uint4*>(brow_base + (((c0 + 0) ^ (r & 7)) * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(brow_base + (((c0 + 1) ^ (r & 7)) * 16)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+        *reinterpret_cast<uint4*>(brow_base + (((c0 + 2) ^ (r & 7)) * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(brow_base + (((c0 + 3) ^ (r & 7)) * 16)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) pmbar_arrive(&full_b[s]);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
   }
-  if (tid == 0)
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32p(&bars[2 * kStages]))
-                 : "memory");
-  if (!pmbar_wait(&bars[2 * kStages], 0)) ok = false;
+
+  const bool fin = pmbar_wait_ab(done, 0, abort);
+  __syncwarp();  // the tensor-memory loads below are warp-collective
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (!ok) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
+  if (tid == 0 && (!fin || *abort)) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
 
   // epilogue: warp w reads tile rows 32 (w % 4) .. + 31 (its TMEM lane quarter); column half w / 4
   {
-    const int lane = tid & 31, quarter = warp & 3, colh = warp >> 2;
+    const int quarter = warp & 3, colh = warp >> 2;
     const int row = quarter * 32 + lane;
     const bool valid = mt * kTM + row < n_e;
     const int grow = row0 + row;
@@ -652,7 +697,7 @@ __global__ void __launch_bounds__(kPT, 1)
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN));
 }
 
 // ------------------------------------------------------------------ combine
@@ -676,9 +721,10 @@ __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, in
 
 // ------------------------------------------------------------------ host side
 
-static uint32_t gemm_smem() { return kTilesBytes + kStages * kRawBytes + (2 * kStages + 1) * 8 + 8 + 1024; }
-static int route_tpc(int H, int E) { return ((size_t)16 * (H + E) + 16) * 4 <= 200 * 1024 ? 16 : 8; }
-static uint32_t route_smem(int H, int E) { return (uint32_t)(((size_t)route_tpc(H, E) * (H + E) + 16) * 4); }
+static uint32_t gemm_smem() { return kTilesBytes + kRawRing + (3 * kStages + 1) * 8 + 16 + 1024; }
+static size_t route_floats(int tpc, int H, int E) { return (size_t)tpc * ((size_t)H / kChunk * kUChunk + E) + 16; }
+static int route_tpc(int H, int E) { return route_floats(16, H, E) * 4 <= 200 * 1024 ? 16 : 8; }
+static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
 
 int prefill_supported(int H, int E, int K, int I, int Is) {
   if (H % kTN || H > kMaxH || I % kTK || Is % kTK || E > kMaxE || K > 32) return 0;
