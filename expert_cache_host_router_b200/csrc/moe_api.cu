@@ -687,6 +687,7 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   a.Is = c->Is;
   a.use_norm = c->cfg.use_rmsnorm;
   a.T = n_tokens;
+  a.n_sm = c->nsm;
   a.eps = c->cfg.rms_eps;
   a.pool = c->pool.load();
   a.slot_bytes = c->slot_bytes;

@@ -77,16 +77,20 @@ __device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, in
 
 constexpr int kRTok = 8;  // tokens per warp in the router
 
-// Row stride of u in shared memory: 16-column chunks padded to 20 floats, so the 32
-// lanes' 128-bit loads of 32 different chunks fall in 8 different bank groups.
+// Row stride of u in shared memory: 16-column chunks padded to 20 floats, so the four
+// chunks that a warp's lanes read at once (one per residue, r chunks apart) fall in four
+// different bank groups.
 constexpr int kUChunk = 20;
 
 // CTA of 8 warps, p.tpc (8 or 16) tokens.  Logit z_e of a token is the canonical fold of
 // its 16-column chunk partials (each an fmaf chain from +0): fold lane q adds chunks
-// q, q + 32, ... from +0, then the lanes combine as the xor butterfly 16, 8, 4, 2, 1.
-// Here the fold's lanes are the warp's lanes: a warp job is 8 tokens x 2 experts, lane q
-// forms the 16 lane sums of its chunks and the butterfly runs on shuffles, so every
-// router weight a lane loads is used for 8 tokens.
+// q, q + 32, ... from +0, then the 32 lane sums combine as the xor butterfly 16, 8, 4, 2,
+// 1 does.  In that butterfly's tree the sums of lanes q = r (mod 4) meet first (levels
+// 16, 8, 4) and the four results meet last (levels 2, 1).  So here warp lane
+// 4 * slot + r evaluates residue r's 8-leaf subtree (leaves in bit-reversed order, a
+// 3-deep stack) for 8 tokens x 2 experts, and the last two levels are shuffles.  Lanes of
+// one residue read the same u (one shared-memory wavefront for 8 lanes) and each weight
+// a lane loads serves 8 tokens.
 __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, int l) {
   extern __shared__ __align__(16) float rsm[];
   const int H = p.H, E = p.E, nch = p.nch, TPC = p.tpc;
@@ -146,77 +150,127 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
   }
   __syncthreads();
 
-  // 2. logits: warp job = (token group of 8, expert pair); lane q = fold lane q
-  const int ntg = TPC / kRTok, npair = (E + 1) / 2;
-  for (int job = warp; job < ntg * npair; job += kPT / 32) {
-    const int tg = job % ntg, e0 = 2 * (job / ntg), e1 = e0 + 1;
-    const bool v1 = e1 < E;
+  // 2. logits: warp job = (token group of 8, block of 16 experts); lane = 4 * slot + r
+  const int ntg = TPC / kRTok, nblk = (E + 15) / 16;
+  const int r4 = lane & 3, slot = lane >> 2;
+  for (int job = warp; job < ntg * nblk; job += kPT / 32) {
+    const int tg = job % ntg, e0 = (job / ntg) * 16 + 2 * slot, e1 = e0 + 1;
+    const bool v0 = e0 < E, v1 = e1 < E;
     const float* ub = us + (size_t)tg * kRTok * ustride;
     auto wload = [&](int c, uint4 (&w)[4]) {
       const uint4* w0p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e0) * kChunk);
-      w[0] = __ldg(w0p);
-      w[1] = __ldg(w0p + 1);
-      w[2] = w[3] = make_uint4(0, 0, 0, 0);
+      w[0] = w[1] = w[2] = w[3] = make_uint4(0, 0, 0, 0);
+      if (v0) {
+        w[0] = __ldg(w0p);
+        w[1] = __ldg(w0p + 1);
+      }
       if (v1) {
         w[2] = __ldg(w0p + 2);  // expert e0 + 1 follows e0 in the same chunk row
         w[3] = __ldg(w0p + 3);
       }
     };
-    float ls[kRTok][2];
-#pragma unroll
-    for (int t = 0; t < kRTok; ++t) ls[t][0] = ls[t][1] = 0.0f;
+    // leaf i' of this residue: fold lane r + 4 * brev3(i')
+    auto leaf_q = [&](int i) { return r4 + 4 * (int)(__brev((unsigned)i) >> 29); };
+    float stk[3][kRTok][2];
+    float cr[kRTok][2];
     uint4 cw[4];
-    if (lane < nch) wload(lane, cw);
-    for (int c = lane; c < nch; c += 32) {
-      uint4 nw[4];
-      const bool more = c + 32 < nch;
-      if (more) wload(c + 32, nw);
-      const uint32_t wa[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w, cw[1].x, cw[1].y, cw[1].z, cw[1].w};
-      const uint32_t wb[8] = {cw[2].x, cw[2].y, cw[2].z, cw[2].w, cw[3].x, cw[3].y, cw[3].z, cw[3].w};
-      float pc[kRTok][2];
+    if (leaf_q(0) < nch) wload(leaf_q(0), cw);
+    for (int i = 0; i < 8; ++i) {
+      const int q = leaf_q(i);
+      float ls[kRTok][2];
 #pragma unroll
-      for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
+      for (int t = 0; t < kRTok; ++t) ls[t][0] = ls[t][1] = 0.0f;
+      for (int c = q; c < nch; c += 32) {
+        // the next chunk this lane visits, loaded while this one is summed
+        int cn = c + 32;
+        if (cn >= nch) {
+          cn = -1;
+          for (int i2 = i + 1; i2 < 8; ++i2)
+            if (leaf_q(i2) < nch) {
+              cn = leaf_q(i2);
+              break;
+            }
+        }
+        uint4 nw[4];
+        if (cn >= 0) wload(cn, nw);
+        const uint32_t wa[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w, cw[1].x, cw[1].y, cw[1].z, cw[1].w};
+        const uint32_t wb[8] = {cw[2].x, cw[2].y, cw[2].z, cw[2].w, cw[3].x, cw[3].y, cw[3].z, cw[3].w};
+        float pc[kRTok][2];
 #pragma unroll
-      for (int j4 = 0; j4 < 4; ++j4) {
+        for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+#pragma unroll
+          for (int t = 0; t < kRTok; ++t) {
+            const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * ustride + c * kUChunk + 4 * j4);
+            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
+            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
+            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
+            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
+            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
+            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
+            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
+            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
+          }
+        }
 #pragma unroll
         for (int t = 0; t < kRTok; ++t) {
-          const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * ustride + c * kUChunk + 4 * j4);
-          pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
-          pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
-          pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
-          pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
-          pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
-          pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
-          pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
-          pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
+          ls[t][0] = __fadd_rn(ls[t][0], pc[t][0]);
+          ls[t][1] = __fadd_rn(ls[t][1], pc[t][1]);
+        }
+        if (cn >= 0) {
+          cw[0] = nw[0];
+          cw[1] = nw[1];
+          cw[2] = nw[2];
+          cw[3] = nw[3];
         }
       }
+      // binary counter over the 8 leaves: level b combines while bit b of i is set
+      bool carry = true;
 #pragma unroll
-      for (int t = 0; t < kRTok; ++t) {
-        ls[t][0] = __fadd_rn(ls[t][0], pc[t][0]);
-        ls[t][1] = __fadd_rn(ls[t][1], pc[t][1]);
+      for (int b = 0; b < 3; ++b) {
+        if (carry) {
+          if ((i >> b) & 1) {
+#pragma unroll
+            for (int t = 0; t < kRTok; ++t) {
+              ls[t][0] = __fadd_rn(stk[b][t][0], ls[t][0]);
+              ls[t][1] = __fadd_rn(stk[b][t][1], ls[t][1]);
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < kRTok; ++t) {
+              stk[b][t][0] = ls[t][0];
+              stk[b][t][1] = ls[t][1];
+            }
+            carry = false;
+          }
+        }
       }
-      if (more) {
-        cw[0] = nw[0];
-        cw[1] = nw[1];
-        cw[2] = nw[2];
-        cw[3] = nw[3];
+      if (carry) {
+#pragma unroll
+        for (int t = 0; t < kRTok; ++t) {
+          cr[t][0] = ls[t][0];
+          cr[t][1] = ls[t][1];
+        }
       }
     }
+    // butterfly levels 2 and 1 across the four residues
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
+    for (int off = 2; off >= 1; off >>= 1) {
 #pragma unroll
       for (int t = 0; t < kRTok; ++t) {
-        ls[t][0] = __fadd_rn(ls[t][0], __shfl_xor_sync(0xffffffffu, ls[t][0], off));
-        ls[t][1] = __fadd_rn(ls[t][1], __shfl_xor_sync(0xffffffffu, ls[t][1], off));
+        cr[t][0] = __fadd_rn(cr[t][0], __shfl_xor_sync(0xffffffffu, cr[t][0], off));
+        cr[t][1] = __fadd_rn(cr[t][1], __shfl_xor_sync(0xffffffffu, cr[t][1], off));
       }
     }
-    const float b0 = p.bias ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
+    const float b0 = (p.bias && v0) ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
     const float b1 = (p.bias && v1) ? __ldg(p.bias + (size_t)l * E + e1) : 0.0f;
 #pragma unroll
     for (int t = 0; t < kRTok; ++t) {
-      if (lane == 2 * t) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(ls[t][0], invs[tg * kRTok + t], b0);
-      if (lane == 2 * t + 1 && v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(ls[t][1], invs[tg * kRTok + t], b1);
+      if ((t & 3) != r4) continue;  // the four residue lanes hold the same sums: share the stores
+      const float inv = invs[tg * kRTok + t];
+      if (v0) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(cr[t][0], inv, b0);
+      if (v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(cr[t][1], inv, b1);
     }
   }
   __syncthreads();
@@ -458,30 +512,48 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t v, __half2 d2) {
 constexpr int kRawStages = 4;     // raw-byte ring depth of each dequant thread
 constexpr uint32_t kRawSlot = 48;  // one thread, one stage: 32 bytes of nibbles, 4 of scales, pad
 constexpr uint32_t kRawRing = kRawStages * kTN * kRawSlot;
+constexpr int kGT = 384;           // threads of a GEMM CTA: 12 warps
+constexpr int kAccCols = 2 * kTN;  // two accumulator buffers in tensor memory
 
-// One CTA per 128 x 128 output tile, warp roles joined by mbarriers:
-//   warp 0 lane 0   A producer: TMA of the activation tiles (hi, lo) of each K stage
-//   warp 1 lane 0   MMA issuer: 2 x 4 tcgen05.mma per stage, commit frees the stage
-//   warps 4..7      B producers: thread r owns row r of the weight tile; it streams that
-//                   row's Q4_0 bytes through a private cp.async ring 3 stages ahead and
-//                   dequantises each stage into the 128B-swizzled fp16 tile
-//   all warps       epilogue from tensor memory
+// One output tile: 128 grouped rows of expert e (m-tile mt) x 128 columns (n-tile nt).
+struct GemmTile {
+  int e, mt, nt, row0, n_e, Ie, nK;
+};
+
+// Persistent grouped GEMM.  CTA b takes tiles b, b + grid, ... of the list (m-tile job,
+// n-tile) and runs warp roles joined by mbarriers:
+//   warps 0..3     epilogue: warp w owns tile rows 32 w .. 32 w + 31 (its tensor-memory
+//                  lane quarter); it drains one accumulator buffer while the MMAs fill
+//                  the other
+//   warp 4 lane 0  A producer: TMA of the activation tiles (hi, lo) of each K stage
+//   warp 5 lane 0  MMA issuer: 2 x 4 tcgen05.mma per stage into the tile's buffer;
+//                  commits free the stage and, after the last stage, hand the buffer over
+//   warps 8..11    B producers: thread r owns row r of the weight tile; it streams that
+//                  row's Q4_0 bytes through a private cp.async ring 3 stages ahead (across
+//                  tile boundaries) and dequantises each stage into the swizzled fp16 tile
 template <int MODE>  // 0: gate/up + SwiGLU, 1: down
-__global__ void __launch_bounds__(kPT, 1)
+__global__ void __launch_bounds__(kGT, 1)
     prefill_gemm(const PrefillParams p, int l, const __grid_constant__ CUtensorMap tm_hi,
                  const __grid_constant__ CUtensorMap tm_lo) {
   extern __shared__ __align__(1024) uint8_t psm_raw[];
   const int imax = p.I > p.Is ? p.I : p.Is;
-  const int n_tiles = MODE == 0 ? (2 * imax) / kTN : p.H / kTN;
-  const int job = blockIdx.x / n_tiles, nt = blockIdx.x % n_tiles;
-  if (job >= *p.s.n_jobs) return;
-  const int je = p.s.jobs[job], e = je >> 20, mt = je & 0xFFFFF;
-  const int Ie = e < p.E ? p.I : p.Is;
-  if (MODE == 0 && nt * (kTN / 2) >= Ie) return;  // past the width of a narrower expert
-  const int g0 = p.s.offsets[e], n_e = p.s.offsets[e + 1] - g0;
-  const int row0 = g0 + mt * kTM;
-  const int K = MODE == 0 ? p.H : Ie;
-  const int nK = K / kTK, nbk = K / 32;
+  const int ntn = MODE == 0 ? (2 * imax) / kTN : p.H / kTN;
+  const int total = *p.s.n_jobs * ntn;
+  if ((int)blockIdx.x >= total) return;
+  const int grid = gridDim.x;
+  auto tile_info = [&](int tile, GemmTile& t) {  // false: no work (past a narrower expert's width)
+    const int je = p.s.jobs[tile / ntn];
+    t.nt = tile % ntn;
+    t.e = je >> 20;
+    t.mt = je & 0xFFFFF;
+    t.Ie = t.e < p.E ? p.I : p.Is;
+    if (MODE == 0 && t.nt * (kTN / 2) >= t.Ie) return false;
+    const int g0 = p.s.offsets[t.e];
+    t.n_e = p.s.offsets[t.e + 1] - g0;
+    t.row0 = g0 + t.mt * kTM;
+    t.nK = (MODE == 0 ? p.H : t.Ie) / kTK;
+    return true;
+  };
 
   // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, the raw rings, barriers
   uint8_t* psm = psm_raw + ((1024u - (smem_u32p(psm_raw) & 1023u)) & 1023u);
@@ -489,8 +561,9 @@ __global__ void __launch_bounds__(kPT, 1)
   uint64_t* full_a = reinterpret_cast<uint64_t*>(raw + kRawRing);
   uint64_t* full_b = full_a + kStages;
   uint64_t* empty = full_b + kStages;
-  uint64_t* done = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto a_hi = [&](int s) { return psm + s * 3 * kTileBytes; };
@@ -503,13 +576,16 @@ __global__ void __launch_bounds__(kPT, 1)
       pmbar_init(&full_b[s], 4);
       pmbar_init(&empty[s], 1);
     }
-    pmbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      pmbar_init(&acc_full[b], 1);
+      pmbar_init(&acc_empty[b], 4);
+    }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 5) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32p(tmem_slot)),
-                 "r"(kTN));
+                 "r"(kAccCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -517,187 +593,242 @@ __global__ void __launch_bounds__(kPT, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      for (int ks = 0; ks < nK; ++ks) {
-        const int s = ks % kStages;
-        if (ks >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(ks / kStages - 1) & 1u, abort)) break;
-        const uint32_t bar = smem_u32p(&full_a[s]);
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-            "[%4];" ::"r"(smem_u32p(a_hi(s))),
-            "l"(&tm_hi), "r"(ks * kTK), "r"(row0), "r"(bar)
-            : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-            "[%4];" ::"r"(smem_u32p(a_lo(s))),
-            "l"(&tm_lo), "r"(ks * kTK), "r"(row0), "r"(bar)
-            : "memory");
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      for (int ks = 0; ks < nK; ++ks) {
-        const int s = ks % kStages;
-        const uint32_t ph = (uint32_t)(ks / kStages) & 1u;
-        if (!pmbar_wait_ab(&full_a[s], ph, abort) || !pmbar_wait_ab(&full_b[s], ph, abort)) break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t sh = smem_u32p(a_hi(s)), sl = smem_u32p(a_lo(s)), sb = smem_u32p(b_t(s));
+  if (warp < 4) {
+    // ---------------------------------------------------------------- epilogue
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int tc = 0;
+    for (int tile = blockIdx.x; tile < total; tile += grid) {
+      GemmTile t;
+      if (!tile_info(tile, t)) continue;
+      const int b = tc & 1;
+      // the tensor-memory loads below are warp-collective: the whole warp goes on or stops
+      const bool ok = __all_sync(0xffffffffu, pmbar_wait_ab(&acc_full[b], (uint32_t)(tc >> 1) & 1u, abort));
+      if (!ok) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t taddr = tmem + lane_base + (uint32_t)(b * kTN);
+      const bool valid = t.mt * kTM + row < t.n_e;
+      const int grow = t.row0 + row;
+      if (MODE == 0) {  // gate columns 0..63, up columns 64..127
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTN / 2; c0 += 16) {
+          uint32_t gr[16], ur[16];
+          tmem_ld16(taddr + c0, gr);
+          tmem_ld16(taddr + kTN / 2 + c0, ur);
+          tmem_wait16(gr);
+          tmem_wait16(ur);
+          if (valid) {
+            __align__(16) __half hi[16];
+            __align__(16) __half lo[16];
 #pragma unroll
-        for (int kk = 0; kk < kTK / 16; ++kk) {
-          const uint64_t db = umma_desc(sb + kk * 32);
-          umma_f16(tmem, umma_desc(sh + kk * 32), db, (ks > 0 || kk > 0) ? 1u : 0u);
-          umma_f16(tmem, umma_desc(sl + kk * 32), db, 1u);
+            for (int j = 0; j < 16; ++j) {
+              const float gv = __uint_as_float(gr[j]), uv = __uint_as_float(ur[j]);
+              const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
+              hi[j] = __float2half_rn(a);
+              lo[j] = __float2half_rn(a - __half2float(hi[j]));
+            }
+            const size_t off = (size_t)grow * imax + t.nt * (kTN / 2) + c0;
+            uint4* dh = reinterpret_cast<uint4*>(p.s.a_hi + off);
+            uint4* dl = reinterpret_cast<uint4*>(p.s.a_lo + off);
+            dh[0] = reinterpret_cast<const uint4*>(hi)[0];
+            dh[1] = reinterpret_cast<const uint4*>(hi)[1];
+            dl[0] = reinterpret_cast<const uint4*>(lo)[0];
+            dl[1] = reinterpret_cast<const uint4*>(lo)[1];
+          }
         }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         smem_u32p(&empty[s]))
-                     : "memory");
-      }
-      // arrives once every MMA issued above has completed (at once if none was)
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       smem_u32p(done))
-                   : "memory");
-    }
-  } else if (warp >= 4) {
-    // B row r of this tile -> weight row: gate/up tiles hold 64 gate rows then the same 64 up rows
-    const int r = tid - 128;
-    const SlotLayout& Ls = e < p.E ? p.lay : p.slay;
-    const uint8_t* slot = expert_slot(p, l, e);
-    const int wrow = MODE == 0 ? nt * (kTN / 2) + (r & 63) : nt * kTN + r;
-    const uint8_t* rbase;  // the 16-row tile holding that row
-    if (MODE == 0)
-      rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
-    else
-      rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * Ie;
-    const int rr = wrow % 16;
-    const uint8_t* qrow = rbase + (size_t)rr * nbk * 16;                          // the row's nibbles
-    const uint8_t* drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;  // the row's scales
-    auto fetch = [&](int ks) {
-      uint8_t* rs = raw + ((ks % kRawStages) * kTN + r) * kRawSlot;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs)), "l"(qrow + (size_t)ks * 32)
-                   : "memory");
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + 16)),
-                   "l"(qrow + (size_t)ks * 32 + 16)
-                   : "memory");
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + 32)), "l"(drow + (size_t)ks * 4)
-                   : "memory");
-    };
-    for (int ks = 0; ks < kRawStages - 1 && ks < nK; ++ks) {
-      fetch(ks);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    }
-    uint8_t* brow_base = nullptr;
-    for (int ks = 0; ks < nK; ++ks) {
-      // refill the ring slot consumed at ks - 1, then wait for stage ks (groups after it:
-      // min(kRawStages - 1, nK - 1 - ks))
-      if (ks + kRawStages - 1 < nK) fetch(ks + kRawStages - 1);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      const int later = nK - 1 - ks;
-      if (later >= kRawStages - 1)
-        asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
-      else if (later == 2)
-        asm volatile("cp.async.wait_group 2;" ::: "memory");
-      else if (later == 1)
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      else
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      const uint8_t* rs = raw + ((ks % kRawStages) * kTN + r) * kRawSlot;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(rs);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(rs + 16);
-      const uint32_t sc = *reinterpret_cast<const uint32_t*>(rs + 32);
-      const int s = ks % kStages;
-      if (ks >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(ks / kStages - 1) & 1u, abort)) break;
-      brow_base = b_t(s) + (r >> 3) * 1024 + (r & 7) * 128;
+      } else {
+        const int pr = valid ? p.s.perm[grow] : 0;
+        float* dst = p.s.obuf + ((size_t)(pr >> 8) * (p.K + 1) + (pr & 0xFF)) * p.H + t.nt * kTN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTN; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(taddr + c0, o);
+          tmem_wait16(o);
+          if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        const uint4 q = blk ? q1 : q0;
-        const __half dh = __ushort_as_half((unsigned short)(blk ? (sc >> 16) : (sc & 0xFFFF)));
-        const __half2 d2 = __half2(dh, dh);
-        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
-        uint32_t lo[8], hi[8];  // half2 pairs of weights (2j, 2j + 1) and (16 + 2j, 17 + 2j)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint32_t r01 = __byte_perm(qw[w], 0, 0x4140), r23 = __byte_perm(qw[w], 0, 0x4342);
-          lo[2 * w] = q4_pair(r01, d2);
-          lo[2 * w + 1] = q4_pair(r23, d2);
-          hi[2 * w] = q4_pair(r01 >> 4, d2);
-          hi[2 * w + 1] = q4_pair(r23 >> 4, d2);
+            for (int j = 0; j < 4; ++j)
+              d4[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
+                                  __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
+          }
         }
-        // 16-byte chunks of the block: weights 0-7, 8-15 (low nibbles), 16-23, 24-31 (high)
-        const int c0 = blk * 4;
-        *reinterpret_cast<uint4*>(brow_base + (((c0 + 0) ^ (r & 7)) * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        *reinterpret_cast<uint4*>(brow_base + (((c0 + 1) ^ (r & 7)) * 16)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-        *reinterpret_cast<uint4*>(brow_base + (((c0 + 2) ^ (r & 7)) * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(brow_base + (((c0 + 3) ^ (r & 7)) * 16)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
-      if (lane == 0) pmbar_arrive(&full_b[s]);
+      if (lane == 0) pmbar_arrive(&acc_empty[b]);
+      ++tc;
+    }
+  } else if (warp == 4) {
+    // ---------------------------------------------------------------- A producer
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort; tile += grid) {
+        GemmTile t;
+        if (!tile_info(tile, t)) continue;
+        for (int ks = 0; ks < t.nK; ++ks, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) break;
+          const uint32_t bar = smem_u32p(&full_a[s]);
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
+                       : "memory");
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+              "[%4];" ::"r"(smem_u32p(a_hi(s))),
+              "l"(&tm_hi), "r"(ks * kTK), "r"(t.row0), "r"(bar)
+              : "memory");
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+              "[%4];" ::"r"(smem_u32p(a_lo(s))),
+              "l"(&tm_lo), "r"(ks * kTK), "r"(t.row0), "r"(bar)
+              : "memory");
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int it = 0, tc = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort; tile += grid) {
+        GemmTile t;
+        if (!tile_info(tile, t)) continue;
+        const int b = tc & 1;
+        if (tc >= 2 && !pmbar_wait_ab(&acc_empty[b], (uint32_t)((tc >> 1) - 1) & 1u, abort)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc = tmem + (uint32_t)(b * kTN);
+        bool stop = false;
+        for (int ks = 0; ks < t.nK; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!pmbar_wait_ab(&full_a[s], ph, abort) || !pmbar_wait_ab(&full_b[s], ph, abort)) {
+            stop = true;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+          const uint32_t sh = smem_u32p(a_hi(s)), sl = smem_u32p(a_lo(s)), sb = smem_u32p(b_t(s));
+#pragma unroll
+          for (int kk = 0; kk < kTK / 16; ++kk) {
+            const uint64_t db = umma_desc(sb + kk * 32);
+            umma_f16(acc, umma_desc(sh + kk * 32), db, (ks > 0 || kk > 0) ? 1u : 0u);
+            umma_f16(acc, umma_desc(sl + kk * 32), db, 1u);
+          }
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           smem_u32p(&empty[s]))
+                       : "memory");
+        }
+        if (stop) break;
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32p(&acc_full[b]))
+                     : "memory");
+        ++tc;
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------------- B producers
+    const int r = tid - 256;
+    // weight row r of tile t: gate/up tiles hold 64 gate rows then the same 64 up rows
+    auto row_ptr = [&](const GemmTile& t, const uint8_t*& qrow, const uint8_t*& drow) {
+      const SlotLayout& Ls = t.e < p.E ? p.lay : p.slay;
+      const uint8_t* slot = expert_slot(p, l, t.e);
+      const int wrow = MODE == 0 ? t.nt * (kTN / 2) + (r & 63) : t.nt * kTN + r;
+      const int K = MODE == 0 ? p.H : t.Ie, nbk = K / 32;
+      const uint8_t* rbase;  // the 16-row tile holding that row
+      if (MODE == 0)
+        rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
+      else
+        rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * K;
+      const int rr = wrow % 16;
+      qrow = rbase + (size_t)rr * nbk * 16;
+      drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;
+    };
+    // fetch cursor: the stage kRawStages - 1 items ahead of the one being dequantised
+    int f_tile = blockIdx.x, f_ks = 0, f_nK = 0, f_it = 0;
+    const uint8_t *f_q = nullptr, *f_d = nullptr;
+    auto f_seek = [&]() {  // first valid tile at or after f_tile
+      for (; f_tile < total; f_tile += grid) {
+        GemmTile t;
+        if (tile_info(f_tile, t)) {
+          row_ptr(t, f_q, f_d);
+          f_nK = t.nK;
+          return;
+        }
+      }
+    };
+    auto fetch_next = [&]() {  // issue the next item's copies (if any), one commit group either way
+      if (f_tile < total) {
+        uint8_t* rs = raw + ((f_it % kRawStages) * kTN + r) * kRawSlot;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs)), "l"(f_q + (size_t)f_ks * 32)
+                     : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + 16)),
+                     "l"(f_q + (size_t)f_ks * 32 + 16)
+                     : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + 32)), "l"(f_d + (size_t)f_ks * 4)
+                     : "memory");
+        ++f_it;
+        if (++f_ks == f_nK) {
+          f_ks = 0;
+          f_tile += grid;
+          f_seek();
+        }
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    f_seek();
+    for (int k = 0; k < kRawStages - 1; ++k) fetch_next();
+    int it = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total && !stop; tile += grid) {
+      GemmTile t;
+      if (!tile_info(tile, t)) continue;
+      for (int ks = 0; ks < t.nK; ++ks, ++it) {
+        fetch_next();  // refills the ring slot dequantised one item ago
+        asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
+        const uint8_t* rs = raw + ((it % kRawStages) * kTN + r) * kRawSlot;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(rs);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(rs + 16);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(rs + 32);
+        const int s = it % kStages;
+        if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) {
+          stop = true;
+          break;
+        }
+        uint8_t* brow = b_t(s) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk) {
+          const uint4 q = blk ? q1 : q0;
+          const __half dh = __ushort_as_half((unsigned short)(blk ? (sc >> 16) : (sc & 0xFFFF)));
+          const __half2 d2 = __half2(dh, dh);
+          const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+          uint32_t lo[8], hi[8];  // half2 pairs of weights (2j, 2j + 1) and (16 + 2j, 17 + 2j)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t r01 = __byte_perm(qw[w], 0, 0x4140), r23 = __byte_perm(qw[w], 0, 0x4342);
+            lo[2 * w] = q4_pair(r01, d2);
+            lo[2 * w + 1] = q4_pair(r23, d2);
+            hi[2 * w] = q4_pair(r01 >> 4, d2);
+            hi[2 * w + 1] = q4_pair(r23 >> 4, d2);
+          }
+          // 16-byte chunks of the block: weights 0-7, 8-15 (low nibbles), 16-23, 24-31 (high)
+          const int c0 = blk * 4;
+          *reinterpret_cast<uint4*>(brow + (((c0 + 0) ^ (r & 7)) * 16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(brow + (((c0 + 1) ^ (r & 7)) * 16)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+          *reinterpret_cast<uint4*>(brow + (((c0 + 2) ^ (r & 7)) * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(brow + (((c0 + 3) ^ (r & 7)) * 16)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) pmbar_arrive(&full_b[s]);
+      }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
   }
 
-  const bool fin = pmbar_wait_ab(done, 0, abort);
-  __syncwarp();  // the tensor-memory loads below are warp-collective
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (tid == 0 && (!fin || *abort)) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
-
-  // epilogue: warp w reads tile rows 32 (w % 4) .. + 31 (its TMEM lane quarter); column half w / 4
-  {
-    const int quarter = warp & 3, colh = warp >> 2;
-    const int row = quarter * 32 + lane;
-    const bool valid = mt * kTM + row < n_e;
-    const int grow = row0 + row;
-    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
-    if (MODE == 0) {  // gate columns 0..63, up columns 64..127
-      for (int c0 = colh * 32; c0 < colh * 32 + 32; c0 += 16) {
-        uint32_t gr[16], ur[16];
-        tmem_ld16(taddr + c0, gr);
-        tmem_ld16(taddr + 64 + c0, ur);
-        tmem_wait16(gr);
-        tmem_wait16(ur);
-        if (valid) {
-          __align__(16) __half hi[16];
-          __align__(16) __half lo[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float gv = __uint_as_float(gr[j]), uv = __uint_as_float(ur[j]);
-            const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-            hi[j] = __float2half_rn(a);
-            lo[j] = __float2half_rn(a - __half2float(hi[j]));
-          }
-          const size_t off = (size_t)grow * imax + nt * (kTN / 2) + c0;
-          uint4* dh = reinterpret_cast<uint4*>(p.s.a_hi + off);
-          uint4* dl = reinterpret_cast<uint4*>(p.s.a_lo + off);
-          dh[0] = reinterpret_cast<const uint4*>(hi)[0];
-          dh[1] = reinterpret_cast<const uint4*>(hi)[1];
-          dl[0] = reinterpret_cast<const uint4*>(lo)[0];
-          dl[1] = reinterpret_cast<const uint4*>(lo)[1];
-        }
-      }
-    } else {
-      const int pr = valid ? p.s.perm[grow] : 0;
-      const int tok = pr >> 8, rank = pr & 0xFF;
-      float* dst = p.s.obuf + ((size_t)tok * (p.K + 1) + rank) * p.H + nt * kTN;
-      for (int c0 = colh * 64; c0 < colh * 64 + 64; c0 += 16) {
-        uint32_t o[16];
-        tmem_ld16(taddr + c0, o);
-        tmem_wait16(o);
-        if (valid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            d4[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
-                                __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
-        }
-      }
-    }
-  }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN));
+  if (tid == 0 && *abort) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
+  if (warp == 5) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kAccCols));
+  }
 }
 
 // ------------------------------------------------------------------ combine
@@ -721,7 +852,8 @@ __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, in
 
 // ------------------------------------------------------------------ host side
 
-static uint32_t gemm_smem() { return kTilesBytes + kRawRing + (3 * kStages + 1) * 8 + 16 + 1024; }
+static uint32_t gemm_smem() { return kTilesBytes + kRawRing + (3 * kStages + 4) * 8 + 16 + 1024; }
+static int gemm_grid(int max_tiles, int n_sm) { return max_tiles < n_sm ? max_tiles : n_sm; }
 static size_t route_floats(int tpc, int H, int E) { return (size_t)tpc * ((size_t)H / kChunk * kUChunk + E) + 16; }
 static int route_tpc(int H, int E) { return route_floats(16, H, E) * 4 <= 200 * 1024 ? 16 : 8; }
 static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
@@ -799,8 +931,8 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     prefill_route<<<(T + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
     prefill_scan<<<1, 1024, 0, st>>>(p);
     prefill_scatter<<<(T + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
-    prefill_gemm<0><<<max_jobs * ((2 * imax) / kTN), kPT, gemm_smem(), st>>>(p, l, mx_hi, mx_lo);
-    prefill_gemm<1><<<max_jobs * (H / kTN), kPT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
+    prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, mx_hi, mx_lo);
+    prefill_gemm<1><<<gemm_grid(max_jobs * (H / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
     prefill_combine<<<T, kPT, 0, st>>>(p, l);
     e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;

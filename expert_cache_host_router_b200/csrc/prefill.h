@@ -12,6 +12,7 @@ namespace moe {
 // Model and weights (all resident): what the runtime owns.
 struct PrefillArgs {
   int L, H, E, K, I, Is, use_norm, T;
+  int n_sm;  // the device's SM count: persistent GEMM grids
   float eps;
   const uint8_t* pool;
   uint64_t slot_bytes;
