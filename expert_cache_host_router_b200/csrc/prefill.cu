@@ -7,7 +7,7 @@
 // turns each expert's GEMVs into GEMMs [n_e x H] x [H x 2I] and [n_e x I] x [I x H]
 // (n_e = tokens routed to expert e): a dense contraction, so it runs on the tensor
 // cores.  Per layer, in stream order:
-//   route    16 (or 8) tokens per CTA: RMSNorm scale, router logits in the canonical
+//   route    8 tokens per CTA: RMSNorm scale, router logits in the canonical
 //            order, top-k, weights, histogram, per-expert counts; x = RMSNorm(h) split
 //            into fp16 hi + lo (x = hi + lo to about 2^-22 relative)
 //   scan     expert offsets and the list of 128-row m-tiles
@@ -47,6 +47,7 @@ static_assert(kTileBytes % 1024 == 0, "operand tiles must keep the swizzle phase
 
 struct PrefillParams {
   int L, H, E, K, I, Is, use_norm, T, nch, tpc;
+  int t_base, T_total;  // this chunk's first token and the call's token count (trace rows)
   float eps;
   const uint8_t* pool;  // layer l expert e at pool + (base[l] + (pin[l][e] & 0xffff)) * slot_bytes
   uint64_t slot_bytes;
@@ -75,23 +76,23 @@ __device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, in
 
 // ------------------------------------------------------------------ route
 
-constexpr int kRTok = 8;  // tokens per warp in the router
+constexpr int kRTok = 4;  // tokens per warp in the router
 
 // Row stride of u in shared memory: 16-column chunks padded to 20 floats, so the four
 // chunks that a warp's lanes read at once (one per residue, r chunks apart) fall in four
 // different bank groups.
 constexpr int kUChunk = 20;
 
-// CTA of 8 warps, p.tpc (8 or 16) tokens.  Logit z_e of a token is the canonical fold of
+// CTA of 8 warps, p.tpc (8) tokens.  Logit z_e of a token is the canonical fold of
 // its 16-column chunk partials (each an fmaf chain from +0): fold lane q adds chunks
 // q, q + 32, ... from +0, then the 32 lane sums combine as the xor butterfly 16, 8, 4, 2,
 // 1 does.  In that butterfly's tree the sums of lanes q = r (mod 4) meet first (levels
 // 16, 8, 4) and the four results meet last (levels 2, 1).  So here warp lane
 // 4 * slot + r evaluates residue r's 8-leaf subtree (leaves in bit-reversed order, a
-// 3-deep stack) for 8 tokens x 2 experts, and the last two levels are shuffles.  Lanes of
+// 3-deep stack) for 4 tokens x 2 experts, and the last two levels are shuffles.  Lanes of
 // one residue read the same u (one shared-memory wavefront for 8 lanes) and each weight
-// a lane loads serves 8 tokens.
-__global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, int l) {
+// a lane loads serves 4 tokens.
+__global__ void __launch_bounds__(kPT, 2) prefill_route(const PrefillParams p, int l) {
   extern __shared__ __align__(16) float rsm[];
   const int H = p.H, E = p.E, nch = p.nch, TPC = p.tpc;
   const int ustride = nch * kUChunk;
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
   }
   __syncthreads();
 
-  // 2. logits: warp job = (token group of 8, block of 16 experts); lane = 4 * slot + r
+  // 2. logits: warp job = (token group of 4, block of 16 experts); lane = 4 * slot + r
   const int ntg = TPC / kRTok, nblk = (E + 15) / 16;
   const int r4 = lane & 3, slot = lane >> 2;
   for (int job = warp; job < ntg * nblk; job += kPT / 32) {
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(kPT, 1) prefill_route(const PrefillParams p, i
       p.s.w[(size_t)t * p.K + lane] = __fdividef(ex, sum);
       atomicAdd(p.hist + (size_t)l * E + my_e, 1u);
       atomicAdd(p.s.counts + my_e, 1);
-      if (p.s.sel_trace) p.s.sel_trace[((size_t)l * p.T + t) * p.K + lane] = my_e;
+      if (p.s.sel_trace) p.s.sel_trace[((size_t)l * p.T_total + p.t_base + t) * p.K + lane] = my_e;
     }
   }
 }
@@ -514,20 +515,27 @@ constexpr uint32_t kRawSlot = 48;  // one thread, one stage: 32 bytes of nibbles
 constexpr uint32_t kRawRing = kRawStages * kTN * kRawSlot;
 constexpr int kGT = 384;           // threads of a GEMM CTA: 12 warps
 constexpr int kAccCols = 2 * kTN;  // two accumulator buffers in tensor memory
+constexpr int kTileCap = 224;      // tiles one GEMM CTA may take (its tile table's size)
 
-// One output tile: 128 grouped rows of expert e (m-tile mt) x 128 columns (n-tile nt).
+// One output tile: 128 grouped rows of expert e (m-tile) x 128 columns (n-tile nt); nK == 0
+// marks a tile with no work (past the width of a narrower shared expert).
 struct GemmTile {
-  int e, mt, nt, row0, n_e, Ie, nK;
+  const uint8_t* slot;  // the expert's weights
+  int row0, nvalid, nK, nt, e, Ie;
+  int pad;
 };
+static_assert(sizeof(GemmTile) == 40, "tile table entry");
 
 // Persistent grouped GEMM.  CTA b takes tiles b, b + grid, ... of the list (m-tile job,
-// n-tile) and runs warp roles joined by mbarriers:
+// n-tile); two otherwise idle warps first resolve them into a table in shared memory so
+// that no role waits on global loads at a tile boundary.  Warp roles, joined by mbarriers:
 //   warps 0..3     epilogue: warp w owns tile rows 32 w .. 32 w + 31 (its tensor-memory
 //                  lane quarter); it drains one accumulator buffer while the MMAs fill
 //                  the other
 //   warp 4 lane 0  A producer: TMA of the activation tiles (hi, lo) of each K stage
 //   warp 5 lane 0  MMA issuer: 2 x 4 tcgen05.mma per stage into the tile's buffer;
 //                  commits free the stage and, after the last stage, hand the buffer over
+//   warps 6, 7     the tile table
 //   warps 8..11    B producers: thread r owns row r of the weight tile; it streams that
 //                  row's Q4_0 bytes through a private cp.async ring 3 stages ahead (across
 //                  tile boundaries) and dequantises each stage into the swizzled fp16 tile
@@ -539,26 +547,19 @@ __global__ void __launch_bounds__(kGT, 1)
   const int imax = p.I > p.Is ? p.I : p.Is;
   const int ntn = MODE == 0 ? (2 * imax) / kTN : p.H / kTN;
   const int total = *p.s.n_jobs * ntn;
-  if ((int)blockIdx.x >= total) return;
   const int grid = gridDim.x;
-  auto tile_info = [&](int tile, GemmTile& t) {  // false: no work (past a narrower expert's width)
-    const int je = p.s.jobs[tile / ntn];
-    t.nt = tile % ntn;
-    t.e = je >> 20;
-    t.mt = je & 0xFFFFF;
-    t.Ie = t.e < p.E ? p.I : p.Is;
-    if (MODE == 0 && t.nt * (kTN / 2) >= t.Ie) return false;
-    const int g0 = p.s.offsets[t.e];
-    t.n_e = p.s.offsets[t.e + 1] - g0;
-    t.row0 = g0 + t.mt * kTM;
-    t.nK = (MODE == 0 ? p.H : t.Ie) / kTK;
-    return true;
-  };
+  if ((int)blockIdx.x >= total) return;
+  const int n_my = (total - (int)blockIdx.x + grid - 1) / grid;
+  if (n_my > kTileCap) {  // the host sizes the token chunks so that this cannot happen
+    if (threadIdx.x == 0) atomicCAS(p.s.error, 0, MOE_DEVERR_SLOT);
+    return;
+  }
 
-  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, the raw rings, barriers
+  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, raw rings, tile table, barriers
   uint8_t* psm = psm_raw + ((1024u - (smem_u32p(psm_raw) & 1023u)) & 1023u);
   uint8_t* raw = psm + kTilesBytes;
-  uint64_t* full_a = reinterpret_cast<uint64_t*>(raw + kRawRing);
+  GemmTile* tiles = reinterpret_cast<GemmTile*>(raw + kRawRing);
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(tiles + kTileCap);
   uint64_t* full_b = full_a + kStages;
   uint64_t* empty = full_b + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -588,6 +589,25 @@ __global__ void __launch_bounds__(kGT, 1)
                  "r"(kAccCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  if (warp == 6 || warp == 7) {
+    for (int i = tid - 192; i < n_my; i += 64) {
+      const int tile = (int)blockIdx.x + i * grid;
+      const int je = p.s.jobs[tile / ntn];
+      GemmTile t;
+      t.nt = tile % ntn;
+      t.e = je >> 20;
+      const int mt = je & 0xFFFFF;
+      t.Ie = t.e < p.E ? p.I : p.Is;
+      const int g0 = p.s.offsets[t.e];
+      const int n_e = p.s.offsets[t.e + 1] - g0;
+      t.row0 = g0 + mt * kTM;
+      t.nvalid = n_e - mt * kTM;
+      t.nK = (MODE == 0 && t.nt * (kTN / 2) >= t.Ie) ? 0 : (MODE == 0 ? p.H : t.Ie) / kTK;
+      t.slot = expert_slot(p, l, t.e);
+      t.pad = 0;
+      tiles[i] = t;
+    }
+  }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -598,16 +618,16 @@ __global__ void __launch_bounds__(kGT, 1)
     const int row = warp * 32 + lane;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     int tc = 0;
-    for (int tile = blockIdx.x; tile < total; tile += grid) {
-      GemmTile t;
-      if (!tile_info(tile, t)) continue;
+    for (int i = 0; i < n_my; ++i) {
+      const GemmTile t = tiles[i];
+      if (t.nK == 0) continue;
       const int b = tc & 1;
       // the tensor-memory loads below are warp-collective: the whole warp goes on or stops
       const bool ok = __all_sync(0xffffffffu, pmbar_wait_ab(&acc_full[b], (uint32_t)(tc >> 1) & 1u, abort));
       if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t taddr = tmem + lane_base + (uint32_t)(b * kTN);
-      const bool valid = t.mt * kTM + row < t.n_e;
+      const bool valid = row < t.nvalid;
       const int grow = t.row0 + row;
       if (MODE == 0) {  // gate columns 0..63, up columns 64..127
 #pragma unroll 1
@@ -662,12 +682,15 @@ __global__ void __launch_bounds__(kGT, 1)
     // ---------------------------------------------------------------- A producer
     if (lane == 0) {
       int it = 0;
-      for (int tile = blockIdx.x; tile < total && !*abort; tile += grid) {
-        GemmTile t;
-        if (!tile_info(tile, t)) continue;
+      bool stop = false;
+      for (int i = 0; i < n_my && !stop; ++i) {
+        const GemmTile t = tiles[i];
         for (int ks = 0; ks < t.nK; ++ks, ++it) {
           const int s = it % kStages;
-          if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) break;
+          if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) {
+            stop = true;
+            break;
+          }
           const uint32_t bar = smem_u32p(&full_a[s]);
           asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTileBytes)
                        : "memory");
@@ -688,14 +711,14 @@ __global__ void __launch_bounds__(kGT, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int it = 0, tc = 0;
-      for (int tile = blockIdx.x; tile < total && !*abort; tile += grid) {
-        GemmTile t;
-        if (!tile_info(tile, t)) continue;
+      bool stop = false;
+      for (int i = 0; i < n_my && !stop; ++i) {
+        const GemmTile t = tiles[i];
+        if (t.nK == 0) continue;
         const int b = tc & 1;
         if (tc >= 2 && !pmbar_wait_ab(&acc_empty[b], (uint32_t)((tc >> 1) - 1) & 1u, abort)) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t acc = tmem + (uint32_t)(b * kTN);
-        bool stop = false;
         for (int ks = 0; ks < t.nK; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -728,33 +751,29 @@ __global__ void __launch_bounds__(kGT, 1)
     // weight row r of tile t: gate/up tiles hold 64 gate rows then the same 64 up rows
     auto row_ptr = [&](const GemmTile& t, const uint8_t*& qrow, const uint8_t*& drow) {
       const SlotLayout& Ls = t.e < p.E ? p.lay : p.slay;
-      const uint8_t* slot = expert_slot(p, l, t.e);
       const int wrow = MODE == 0 ? t.nt * (kTN / 2) + (r & 63) : t.nt * kTN + r;
       const int K = MODE == 0 ? p.H : t.Ie, nbk = K / 32;
       const uint8_t* rbase;  // the 16-row tile holding that row
       if (MODE == 0)
-        rbase = slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
+        rbase = t.slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
       else
-        rbase = slot + Ls.down + (size_t)(wrow / 16) * 9u * K;
+        rbase = t.slot + Ls.down + (size_t)(wrow / 16) * 9u * K;
       const int rr = wrow % 16;
       qrow = rbase + (size_t)rr * nbk * 16;
       drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;
     };
     // fetch cursor: the stage kRawStages - 1 items ahead of the one being dequantised
-    int f_tile = blockIdx.x, f_ks = 0, f_nK = 0, f_it = 0;
+    int f_i = 0, f_ks = 0, f_it = 0;
     const uint8_t *f_q = nullptr, *f_d = nullptr;
-    auto f_seek = [&]() {  // first valid tile at or after f_tile
-      for (; f_tile < total; f_tile += grid) {
-        GemmTile t;
-        if (tile_info(f_tile, t)) {
-          row_ptr(t, f_q, f_d);
-          f_nK = t.nK;
+    auto f_seek = [&]() {  // first tile with work at or after f_i
+      for (; f_i < n_my; ++f_i)
+        if (tiles[f_i].nK > 0) {
+          row_ptr(tiles[f_i], f_q, f_d);
           return;
         }
-      }
     };
     auto fetch_next = [&]() {  // issue the next item's copies (if any), one commit group either way
-      if (f_tile < total) {
+      if (f_i < n_my) {
         uint8_t* rs = raw + ((f_it % kRawStages) * kTN + r) * kRawSlot;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs)), "l"(f_q + (size_t)f_ks * 32)
                      : "memory");
@@ -764,9 +783,9 @@ __global__ void __launch_bounds__(kGT, 1)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + 32)), "l"(f_d + (size_t)f_ks * 4)
                      : "memory");
         ++f_it;
-        if (++f_ks == f_nK) {
+        if (++f_ks == tiles[f_i].nK) {
           f_ks = 0;
-          f_tile += grid;
+          ++f_i;
           f_seek();
         }
       }
@@ -776,10 +795,9 @@ __global__ void __launch_bounds__(kGT, 1)
     for (int k = 0; k < kRawStages - 1; ++k) fetch_next();
     int it = 0;
     bool stop = false;
-    for (int tile = blockIdx.x; tile < total && !stop; tile += grid) {
-      GemmTile t;
-      if (!tile_info(tile, t)) continue;
-      for (int ks = 0; ks < t.nK; ++ks, ++it) {
+    for (int i = 0; i < n_my && !stop; ++i) {
+      const int nK = tiles[i].nK;
+      for (int ks = 0; ks < nK; ++ks, ++it) {
         fetch_next();  // refills the ring slot dequantised one item ago
         asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
         const uint8_t* rs = raw + ((it % kRawStages) * kTN + r) * kRawSlot;
@@ -845,17 +863,19 @@ __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, in
     const size_t o = (size_t)t * p.H + j;
     const float hn = p.use_norm ? __fadd_rn(p.s.h[o], y) : y;
     p.s.h[o] = hn;
-    if (p.s.h_trace) p.s.h_trace[((size_t)(l + 1) * p.T + t) * p.H + j] = hn;
+    if (p.s.h_trace) p.s.h_trace[((size_t)(l + 1) * p.T_total + p.t_base + t) * p.H + j] = hn;
     if (l == p.L - 1) p.s.y[o] = hn;
   }
 }
 
 // ------------------------------------------------------------------ host side
 
-static uint32_t gemm_smem() { return kTilesBytes + kRawRing + (3 * kStages + 4) * 8 + 16 + 1024; }
+static uint32_t gemm_smem() {
+  return kTilesBytes + kRawRing + kTileCap * sizeof(GemmTile) + (3 * kStages + 4) * 8 + 16 + 1024;
+}
 static int gemm_grid(int max_tiles, int n_sm) { return max_tiles < n_sm ? max_tiles : n_sm; }
 static size_t route_floats(int tpc, int H, int E) { return (size_t)tpc * ((size_t)H / kChunk * kUChunk + E) + 16; }
-static int route_tpc(int H, int E) { return route_floats(16, H, E) * 4 <= 200 * 1024 ? 16 : 8; }
+static int route_tpc(int, int) { return 2 * kRTok; }  // small enough for two CTAs per SM at hidden 2048
 static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
 
 int prefill_supported(int H, int E, int K, int I, int Is) {
@@ -888,54 +908,82 @@ static int make_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, uint64
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+// Tokens per pass: every GEMM CTA's tiles must fit its tile table.
+static int prefill_chunk(int T, int H, int E, int K, int I, int Is, int grid) {
+  const int imax = I > Is ? I : Is;
+  const int64_t ntn = (2 * imax) / kTN > H / kTN ? (2 * imax) / kTN : H / kTN;
+  int tc = T;
+  while (tc > 1) {
+    const int64_t R = (int64_t)tc * K + (Is > 0 ? tc : 0);
+    const int64_t max_tiles = ((R + kTM - 1) / kTM + E + 1) * ntn;
+    if ((max_tiles + grid - 1) / grid <= kTileCap) break;
+    tc = (tc + 1) / 2;
+  }
+  return tc;
+}
+
 int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, cudaStream_t st) {
-  PrefillParams p{};
-  p.L = a.L;
-  p.H = a.H;
-  p.E = a.E;
-  p.K = a.K;
-  p.I = a.I;
-  p.Is = a.Is;
-  p.use_norm = a.use_norm;
-  p.T = a.T;
-  p.eps = a.eps;
-  p.nch = a.H / kChunk;
-  p.tpc = route_tpc(a.H, a.E);
-  p.pool = a.pool;
-  p.slot_bytes = a.slot_bytes;
-  p.lay = a.lay;
-  p.slay = a.slay;
-  p.shared_pool = a.shared_pool;
-  p.shared_slot_bytes = a.shared_slot_bytes;
-  p.router = a.router;
-  p.bias = a.bias;
-  p.gain = a.gain;
-  p.pin_slot = a.pin_slot;
-  p.layer_base = a.layer_base;
-  p.hist = a.hist;
-  p.s = s;
   const int T = a.T, H = a.H, E = a.E;
   const int imax = a.I > a.Is ? a.I : a.Is;
-  const int R = T * a.K + (a.Is > 0 ? T : 0);
+  const int grid0 = gemm_grid(1 << 30, a.n_sm);
+  const int tcmax = prefill_chunk(T, H, E, a.K, a.I, a.Is, grid0);
+  if ((((int64_t)E + 2) * ((2 * imax) / kTN > H / kTN ? (2 * imax) / kTN : H / kTN) + grid0 - 1) / grid0 > kTileCap)
+    return -1;  // even one token per pass would overflow a tile table
   PfnEncodeTiled enc = reinterpret_cast<PfnEncodeTiled>(encode_fn);
-  CUtensorMap mx_hi, mx_lo, ma_hi, ma_lo;
-  if (make_map(enc, &mx_hi, s.xg_hi, R, H) || make_map(enc, &mx_lo, s.xg_lo, R, H) ||
-      make_map(enc, &ma_hi, s.a_hi, R, imax) || make_map(enc, &ma_lo, s.a_lo, R, imax))
-    return -1;
-  const int max_jobs = (R + kTM - 1) / kTM + E + 1;
-  cudaError_t e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * E, st);
-  if (e == cudaSuccess && s.h_trace)
-    e = cudaMemcpyAsync(s.h_trace, s.h, sizeof(float) * T * H, cudaMemcpyDeviceToDevice, st);
-  if (e != cudaSuccess) return (int)e;
-  for (int l = 0; l < a.L; ++l) {
-    prefill_route<<<(T + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
-    prefill_scan<<<1, 1024, 0, st>>>(p);
-    prefill_scatter<<<(T + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
-    prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, mx_hi, mx_lo);
-    prefill_gemm<1><<<gemm_grid(max_jobs * (H / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
-    prefill_combine<<<T, kPT, 0, st>>>(p, l);
-    e = cudaGetLastError();
+  if (s.h_trace) {
+    cudaError_t e = cudaMemcpyAsync(s.h_trace, s.h, sizeof(float) * T * H, cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return (int)e;
+  }
+  for (int t0 = 0; t0 < T; t0 += tcmax) {
+    const int Tc = T - t0 < tcmax ? T - t0 : tcmax;
+    PrefillParams p{};
+    p.L = a.L;
+    p.H = H;
+    p.E = E;
+    p.K = a.K;
+    p.I = a.I;
+    p.Is = a.Is;
+    p.use_norm = a.use_norm;
+    p.T = Tc;
+    p.t_base = t0;
+    p.T_total = T;
+    p.eps = a.eps;
+    p.nch = H / kChunk;
+    p.tpc = route_tpc(H, E);
+    p.pool = a.pool;
+    p.slot_bytes = a.slot_bytes;
+    p.lay = a.lay;
+    p.slay = a.slay;
+    p.shared_pool = a.shared_pool;
+    p.shared_slot_bytes = a.shared_slot_bytes;
+    p.router = a.router;
+    p.bias = a.bias;
+    p.gain = a.gain;
+    p.pin_slot = a.pin_slot;
+    p.layer_base = a.layer_base;
+    p.hist = a.hist;
+    p.s = s;
+    p.s.h = s.h + (size_t)t0 * H;
+    p.s.y = s.y + (size_t)t0 * H;
+    const int R = Tc * a.K + (a.Is > 0 ? Tc : 0);
+    CUtensorMap mx_hi, mx_lo, ma_hi, ma_lo;
+    if (make_map(enc, &mx_hi, s.xg_hi, R, H) || make_map(enc, &mx_lo, s.xg_lo, R, H) ||
+        make_map(enc, &ma_hi, s.a_hi, R, imax) || make_map(enc, &ma_lo, s.a_lo, R, imax))
+      return -1;
+    const int max_jobs = (R + kTM - 1) / kTM + E + 1;
+    cudaError_t e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * E, st);
+    if (e != cudaSuccess) return (int)e;
+    for (int l = 0; l < a.L; ++l) {
+      prefill_route<<<(Tc + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
+      prefill_scan<<<1, 1024, 0, st>>>(p);
+      prefill_scatter<<<(Tc + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
+      prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, mx_hi,
+                                                                                                   mx_lo);
+      prefill_gemm<1><<<gemm_grid(max_jobs * (H / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
+      prefill_combine<<<Tc, kPT, 0, st>>>(p, l);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return (int)e;
+    }
   }
   return 0;
 }
