@@ -31,6 +31,7 @@ import synthetic  # noqa: E402
 
 METRIC = "MoE decode tok/s at 100%/60% expert residency; fraction of HBM/PCIe roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_TFLOPS = 1400.0  # sustained dense bf16, an earlier measurement on this machine
 # DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
 # 4-layer case scaled by 10 (profiles/moe_decode_kernel_4layer_ncu.md), valid only for
 # the kernel source it was taken on; any other source reports null.
@@ -247,6 +248,51 @@ def run_drift(args, shape, layers, local, dev, xs_steps=1024, switch=512, every=
     return out
 
 
+def run_prefill(m, shape, dev, n_tokens=2048, warmup=2, runs=5):
+    """Batched prefill of n_tokens through the whole stack at full residency (tcgen05
+    grouped GEMM path), timed with CUDA events on the launching stream.  Roofline: per
+    layer and expert, max(its FLOPs at the measured dense tensor peak, its weight bytes
+    at the measured HBM bandwidth), summed; token counts per expert from the routing
+    histogram of the timed runs."""
+    import torch
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    tflops = float(peaks.get("bf16_tflops_sustained", FALLBACK_TFLOPS))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    x = torch.from_numpy(synthetic.tokens(50000, n_tokens, shape.hidden)).to(dev)
+    y = torch.empty_like(x)
+    m.set_residency(1.0)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        m.prefill(x, y)
+    m.sync()
+    m.stats(reset=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(runs):
+        m.prefill(x, y)
+    e1.record(stream)
+    m.sync()
+    ms = e0.elapsed_time(e1) / runs
+    _, hist, _ = m.stats(reset=True)
+    n_e = hist.astype(np.float64) / runs  # [L][E] tokens per expert per pass
+    H, I, Is = shape.hidden, shape.inter, shape.shared_inter
+    fl_tok = 2.0 * 3 * H * I  # one token through one routed expert
+    by_exp = 3 * H * I * 18 / 32
+    t_roof = np.sum(np.maximum(n_e * fl_tok / (tflops * 1e12), np.where(n_e > 0, by_exp, 0.0) / (hbm * 1e9)))
+    t_roof += shape.n_layers * max(n_tokens * 2.0 * 3 * H * Is / (tflops * 1e12), 3 * H * Is * 18 / 32 / (hbm * 1e9))
+    useful = float(np.sum(n_e) * fl_tok + shape.n_layers * n_tokens * 2.0 * 3 * H * Is)
+    tiles = float(np.sum(np.ceil(n_e / 128.0)) + shape.n_layers * np.ceil(n_tokens / 128.0))
+    issued = tiles * 128 * 2.0 * 3 * H * I * 2  # 128-row tiles, activation hi + lo
+    return {"tokens": n_tokens, "value": n_tokens / (ms * 1e-3), "unit": "tok/s", "ms": ms, "runs": runs,
+            "dtype": "q4_0 -> fp16 weights x fp16 hi+lo activations, fp32 accumulate (tcgen05)",
+            "roofline": {"bound": "tensor", "achieved": useful / (ms * 1e-3) / 1e12, "peak": tflops,
+                         "unit": "TFLOP/s", "frac": t_roof / (ms * 1e-3), "roofline_ms": t_roof * 1e3,
+                         "peak_kind": "measured sustained bf16 (fp16 same rate)",
+                         "issued_tflops": issued / (ms * 1e-3) / 1e12,
+                         "note": "frac = per-expert max(flop, weight-byte) time summed / measured time"}}
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_ours(args):
@@ -408,6 +454,8 @@ def run_ours(args):
         "clocks": clk.summary(),
         "setup": {"generate_s": gen_s, "load_s": load_s, "phases": args.phases},
     }
+    if args.phases == "all" and not args.no_prefill:
+        line["prefill"] = run_prefill(m, shape, dev)
     m.close()
     del m
     if args.phases == "all" and not args.no_drift:
@@ -434,6 +482,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
     ap.add_argument("--no-drift", action="store_true", help="skip the recalibration-under-drift run")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the batched-prefill run")
     ap.add_argument("--phases", default="all", choices=["all", "100"],
                     help="'100' times full residency only (no miss copies), for profiler runs")
     args = ap.parse_args()

@@ -852,19 +852,48 @@ __global__ void __launch_bounds__(kGT, 1)
 // ------------------------------------------------------------------ combine
 
 // h[t] += sum_rank w * o_rank + o_shared in rank order (without the norm: h = that sum).
+// Thread: 4 columns; the expert outputs of those columns are loaded 10 ranks at a time
+// (streaming, read once) before they are summed, so the loads overlap.
+constexpr int kCombineGroup = 10;
 __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, int l) {
   const int t = blockIdx.x;
   const float* w = p.s.w + (size_t)t * p.K;
   const float* ob = p.s.obuf + (size_t)t * (p.K + 1) * p.H;
-  for (int j = threadIdx.x; j < p.H; j += kPT) {
-    float y = 0.0f;
-    for (int r = 0; r < p.K; ++r) y = fmaf(w[r], ob[(size_t)r * p.H + j], y);
-    if (p.Is > 0) y = __fadd_rn(y, ob[(size_t)p.K * p.H + j]);
-    const size_t o = (size_t)t * p.H + j;
-    const float hn = p.use_norm ? __fadd_rn(p.s.h[o], y) : y;
-    p.s.h[o] = hn;
-    if (p.s.h_trace) p.s.h_trace[((size_t)(l + 1) * p.T_total + p.t_base + t) * p.H + j] = hn;
-    if (l == p.L - 1) p.s.y[o] = hn;
+  const int nr = p.K + (p.Is > 0 ? 1 : 0);
+  for (int j = threadIdx.x * 4; j < p.H; j += kPT * 4) {
+    float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int r0 = 0; r0 < nr; r0 += kCombineGroup) {
+      float4 o[kCombineGroup];
+#pragma unroll
+      for (int i = 0; i < kCombineGroup; ++i)
+        if (r0 + i < nr) o[i] = __ldcs(reinterpret_cast<const float4*>(ob + (size_t)(r0 + i) * p.H + j));
+#pragma unroll
+      for (int i = 0; i < kCombineGroup; ++i) {
+        const int r = r0 + i;
+        if (r < p.K) {
+          const float wr = w[r];
+          y.x = fmaf(wr, o[i].x, y.x);
+          y.y = fmaf(wr, o[i].y, y.y);
+          y.z = fmaf(wr, o[i].z, y.z);
+          y.w = fmaf(wr, o[i].w, y.w);
+        } else if (r == p.K && p.Is > 0) {  // the shared expert, unweighted, last
+          y.x = __fadd_rn(y.x, o[i].x);
+          y.y = __fadd_rn(y.y, o[i].y);
+          y.z = __fadd_rn(y.z, o[i].z);
+          y.w = __fadd_rn(y.w, o[i].w);
+        }
+      }
+    }
+    const size_t at = (size_t)t * p.H + j;
+    float4 hn = y;
+    if (p.use_norm) {
+      const float4 h = *reinterpret_cast<const float4*>(p.s.h + at);
+      hn = make_float4(__fadd_rn(h.x, y.x), __fadd_rn(h.y, y.y), __fadd_rn(h.z, y.z), __fadd_rn(h.w, y.w));
+    }
+    *reinterpret_cast<float4*>(p.s.h + at) = hn;
+    if (p.s.h_trace)
+      *reinterpret_cast<float4*>(p.s.h_trace + ((size_t)(l + 1) * p.T_total + p.t_base + t) * p.H + j) = hn;
+    if (l == p.L - 1) *reinterpret_cast<float4*>(p.s.y + at) = hn;
   }
 }
 

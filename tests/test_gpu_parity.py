@@ -247,6 +247,9 @@ def test_invalid_calls_on_a_live_context():
     with pytest.raises(moe.MoEError):
         moe.moe_set_residency(m.ctx, 0.5, None, 7)
     with pytest.raises(moe.MoEError) as ei:
-        moe.moe_prefill(m.ctx, x.data_ptr(), 1, x.data_ptr(), 0)
-    assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+        moe.moe_prefill(m.ctx, x.data_ptr(), 1, x.data_ptr(), 0)  # no residency set yet
+    assert ei.value.status == moe.MOE_ERR_STATE
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_prefill(m.ctx, x.data_ptr(), 0, x.data_ptr(), 0)
+    assert ei.value.status == moe.MOE_ERR_INVALID
     m.close()
