@@ -36,14 +36,16 @@ namespace moe {
 
 constexpr int kPT = 256;  // threads per prefill CTA
 constexpr int kTM = 128;  // GEMM tile rows (tokens)
-constexpr int kTN = 128;  // GEMM tile columns
+constexpr int kTN = 256;  // GEMM tile columns (weight rows of the B operand)
 constexpr int kTK = 64;   // K per pipeline stage: one 128-byte swizzle row of fp16
-constexpr int kStages = 4;
-constexpr uint32_t kTileBytes = kTM * kTK * 2;           // 16 KB per fp16 operand tile
+constexpr int kStages = 3;
+constexpr uint32_t kTileBytes = kTM * kTK * 2;   // 16 KB: one activation tile (hi or lo)
+constexpr uint32_t kBTileBytes = kTN * kTK * 2;  // 32 KB: the weight tile
+constexpr uint32_t kStageBytes = 2 * kTileBytes + kBTileBytes;
 // Swizzled operand tiles first, each at a multiple of 1024 bytes (the 128-byte swizzle's
 // period: TMA and the MMA take its phase from the address), then the raw weight bytes.
-constexpr uint32_t kTilesBytes = 3 * kTileBytes * kStages;
-static_assert(kTileBytes % 1024 == 0, "operand tiles must keep the swizzle phase");
+constexpr uint32_t kTilesBytes = kStageBytes * kStages;
+static_assert(kTileBytes % 1024 == 0 && kBTileBytes % 1024 == 0, "operand tiles must keep the swizzle phase");
 
 struct PrefillParams {
   int L, H, E, K, I, Is, use_norm, T, nch, tpc;
@@ -448,7 +450,7 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: f16 x f16 -> f32, A and B K-major, M = 128, N = 128.
+// Instruction descriptor: f16 x f16 -> f32, A and B K-major, M = 128, N = 256.
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kTN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
 
 __device__ __forceinline__ void umma_f16(uint32_t tmem, uint64_t da, uint64_t db, uint32_t accumulate) {
@@ -510,14 +512,14 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t v, __half2 d2) {
   return *reinterpret_cast<const uint32_t*>(&w);
 }
 
-constexpr int kRawStages = 4;     // raw-byte ring depth of each dequant thread
-constexpr uint32_t kRawSlot = 48;  // one thread, one stage: 32 bytes of nibbles, 4 of scales, pad
-constexpr uint32_t kRawRing = kRawStages * kTN * kRawSlot;
-constexpr int kGT = 384;           // threads of a GEMM CTA: 12 warps
-constexpr int kAccCols = 2 * kTN;  // two accumulator buffers in tensor memory
-constexpr int kTileCap = 224;      // tiles one GEMM CTA may take (its tile table's size)
+constexpr int kRawStages = 3;  // raw-byte ring depth of each dequant thread
+// raw rings: [stage][row] 32 bytes of nibbles (two Q4_0 blocks), then [stage][row] 4 bytes of scales
+constexpr uint32_t kRawRing = kRawStages * kTN * (32 + 4);
+constexpr int kGT = 512;           // threads of a GEMM CTA: 16 warps
+constexpr int kAccCols = 2 * kTN;  // two accumulator buffers in tensor memory (all 512 columns)
+constexpr int kTileCap = 128;      // tiles one GEMM CTA may take (its tile table's size)
 
-// One output tile: 128 grouped rows of expert e (m-tile) x 128 columns (n-tile nt); nK == 0
+// One output tile: 128 grouped rows of expert e (m-tile) x 256 columns (n-tile nt); nK == 0
 // marks a tile with no work (past the width of a narrower shared expert).
 struct GemmTile {
   const uint8_t* slot;  // the expert's weights
@@ -533,12 +535,16 @@ static_assert(sizeof(GemmTile) == 40, "tile table entry");
 //                  lane quarter); it drains one accumulator buffer while the MMAs fill
 //                  the other
 //   warp 4 lane 0  A producer: TMA of the activation tiles (hi, lo) of each K stage
-//   warp 5 lane 0  MMA issuer: 2 x 4 tcgen05.mma per stage into the tile's buffer;
-//                  commits free the stage and, after the last stage, hand the buffer over
+//   warp 5 lane 0  MMA issuer: 2 x 4 tcgen05.mma (128 x 256 x 16) per stage into the
+//                  tile's buffer; commits free the stage and, after the last stage, hand
+//                  the buffer over
 //   warps 6, 7     the tile table
-//   warps 8..11    B producers: thread r owns row r of the weight tile; it streams that
-//                  row's Q4_0 bytes through a private cp.async ring 3 stages ahead (across
+//   warps 8..15    B producers: thread r owns row r of the weight tile; it streams that
+//                  row's Q4_0 bytes through a private cp.async ring 2 stages ahead (across
 //                  tile boundaries) and dequantises each stage into the swizzled fp16 tile
+// A 256-wide weight tile halves the activation bytes the MMAs read from shared memory per
+// FLOP against a 128-wide one: with both operands in shared memory, an M = 128, N = 128
+// MMA alone asks for about the whole shared-memory bandwidth.
 template <int MODE>  // 0: gate/up + SwiGLU, 1: down
 __global__ void __launch_bounds__(kGT, 1)
     prefill_gemm(const PrefillParams p, int l, const __grid_constant__ CUtensorMap tm_hi,
@@ -567,14 +573,14 @@ __global__ void __launch_bounds__(kGT, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto a_hi = [&](int s) { return psm + s * 3 * kTileBytes; };
-  auto a_lo = [&](int s) { return psm + s * 3 * kTileBytes + kTileBytes; };
-  auto b_t = [&](int s) { return psm + s * 3 * kTileBytes + 2 * kTileBytes; };
+  auto a_hi = [&](int s) { return psm + s * kStageBytes; };
+  auto a_lo = [&](int s) { return psm + s * kStageBytes + kTileBytes; };
+  auto b_t = [&](int s) { return psm + s * kStageBytes + 2 * kTileBytes; };
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       pmbar_init(&full_a[s], 1);
-      pmbar_init(&full_b[s], 4);
+      pmbar_init(&full_b[s], 8);
       pmbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -629,7 +635,7 @@ __global__ void __launch_bounds__(kGT, 1)
       const uint32_t taddr = tmem + lane_base + (uint32_t)(b * kTN);
       const bool valid = row < t.nvalid;
       const int grow = t.row0 + row;
-      if (MODE == 0) {  // gate columns 0..63, up columns 64..127
+      if (MODE == 0) {  // gate columns 0..127, up columns 128..255
 #pragma unroll 1
         for (int c0 = 0; c0 < kTN / 2; c0 += 16) {
           uint32_t gr[16], ur[16];
@@ -748,14 +754,14 @@ __global__ void __launch_bounds__(kGT, 1)
   } else if (warp >= 8) {
     // ---------------------------------------------------------------- B producers
     const int r = tid - 256;
-    // weight row r of tile t: gate/up tiles hold 64 gate rows then the same 64 up rows
+    // weight row r of tile t: gate/up tiles hold 128 gate rows then the same 128 up rows
     auto row_ptr = [&](const GemmTile& t, const uint8_t*& qrow, const uint8_t*& drow) {
       const SlotLayout& Ls = t.e < p.E ? p.lay : p.slay;
-      const int wrow = MODE == 0 ? t.nt * (kTN / 2) + (r & 63) : t.nt * kTN + r;
+      const int wrow = MODE == 0 ? t.nt * (kTN / 2) + (r & (kTN / 2 - 1)) : t.nt * kTN + r;
       const int K = MODE == 0 ? p.H : t.Ie, nbk = K / 32;
       const uint8_t* rbase;  // the 16-row tile holding that row
       if (MODE == 0)
-        rbase = t.slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= 64 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
+        rbase = t.slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= kTN / 2 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
       else
         rbase = t.slot + Ls.down + (size_t)(wrow / 16) * 9u * K;
       const int rr = wrow % 16;
@@ -774,13 +780,14 @@ __global__ void __launch_bounds__(kGT, 1)
     };
     auto fetch_next = [&]() {  // issue the next item's copies (if any), one commit group either way
       if (f_i < n_my) {
-        uint8_t* rs = raw + ((f_it % kRawStages) * kTN + r) * kRawSlot;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs)), "l"(f_q + (size_t)f_ks * 32)
+        uint8_t* rq = raw + ((f_it % kRawStages) * kTN + r) * 32;
+        uint8_t* rd = raw + kRawStages * kTN * 32 + ((f_it % kRawStages) * kTN + r) * 4;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rq)), "l"(f_q + (size_t)f_ks * 32)
                      : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rs + 16)),
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rq + 16)),
                      "l"(f_q + (size_t)f_ks * 32 + 16)
                      : "memory");
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rs + 32)), "l"(f_d + (size_t)f_ks * 4)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rd)), "l"(f_d + (size_t)f_ks * 4)
                      : "memory");
         ++f_it;
         if (++f_ks == tiles[f_i].nK) {
@@ -800,10 +807,10 @@ __global__ void __launch_bounds__(kGT, 1)
       for (int ks = 0; ks < nK; ++ks, ++it) {
         fetch_next();  // refills the ring slot dequantised one item ago
         asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
-        const uint8_t* rs = raw + ((it % kRawStages) * kTN + r) * kRawSlot;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(rs);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(rs + 16);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(rs + 32);
+        const uint8_t* rq = raw + ((it % kRawStages) * kTN + r) * 32;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(rq);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(rq + 16);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(raw + kRawStages * kTN * 32 + ((it % kRawStages) * kTN + r) * 4);
         const int s = it % kStages;
         if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) {
           stop = true;
@@ -908,7 +915,7 @@ static int route_tpc(int, int) { return 2 * kRTok; }  // small enough for two CT
 static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
 
 int prefill_supported(int H, int E, int K, int I, int Is) {
-  if (H % kTN || H > kMaxH || I % kTK || Is % kTK || E > kMaxE || K > 32) return 0;
+  if (H % kTN || H > kMaxH || I % (kTN / 2) || Is % (kTN / 2) || E > kMaxE || K > 32) return 0;
   return route_smem(H, E) <= 227 * 1024;
 }
 
