@@ -690,6 +690,7 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   a.n_sm = c->nsm;
   a.eps = c->cfg.rms_eps;
   a.pool = c->pool.load();
+  a.pool_slots = c->pool_slots;
   a.slot_bytes = c->slot_bytes;
   a.lay = c->lay;
   a.slay = c->slay;

@@ -512,21 +512,48 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t v, __half2 d2) {
   return *reinterpret_cast<const uint32_t*>(&w);
 }
 
-constexpr int kRawStages = 3;  // raw-byte ring depth of each dequant thread
-// raw rings: [stage][row] 32 bytes of nibbles (two Q4_0 blocks), then [stage][row] 4 bytes of scales
-constexpr uint32_t kRawRing = kRawStages * kTN * (32 + 4);
+constexpr int kRawStages = 2;  // raw weight-byte ring depth (TMA, shared by the dequant warps)
+// raw stage: [256 rows x 32 bytes of nibbles: two Q4_0 blocks of each row]
+//            [256 rows x 16 bytes of scales: eight blocks of each row, i.e. four K stages]
+constexpr uint32_t kRawNib = kTN * 32;
+constexpr uint32_t kRawStage = kRawNib + kTN * 16;
+constexpr uint32_t kRawRing = kRawStages * kRawStage;
 constexpr int kGT = 512;           // threads of a GEMM CTA: 16 warps
 constexpr int kAccCols = 2 * kTN;  // two accumulator buffers in tensor memory (all 512 columns)
-constexpr int kTileCap = 128;      // tiles one GEMM CTA may take (its tile table's size)
+constexpr int kTileCap = 64;       // tiles one GEMM CTA may take (its tile table's size)
 
 // One output tile: 128 grouped rows of expert e (m-tile) x 256 columns (n-tile nt); nK == 0
 // marks a tile with no work (past the width of a narrower shared expert).
 struct GemmTile {
-  const uint8_t* slot;  // the expert's weights
   int row0, nvalid, nK, nt, e, Ie;
+  int slot;  // pool slot of a routed expert, layer of the shared one
   int pad;
 };
-static_assert(sizeof(GemmTile) == 40, "tile table entry");
+static_assert(sizeof(GemmTile) == 32, "tile table entry");
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(dst),
+      "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* m, int c0, int c1, int c2, int c3,
+                                            int c4, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
+      "%6}], [%7];" ::"r"(dst),
+      "l"(m), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+      : "memory");
+}
+
+// Tensor maps of one GEMM launch: the activation tiles and, for routed and shared
+// experts, the weight tile's nibble and scale bytes read straight out of the slot layout.
+struct GemmMaps {
+  CUtensorMap a_hi, a_lo;
+  CUtensorMap nib[2], scl[2];  // [0] routed experts (pool), [1] the shared expert
+};
 
 // Persistent grouped GEMM.  CTA b takes tiles b, b + grid, ... of the list (m-tile job,
 // n-tile); two otherwise idle warps first resolve them into a table in shared memory so
@@ -538,17 +565,18 @@ static_assert(sizeof(GemmTile) == 40, "tile table entry");
 //   warp 5 lane 0  MMA issuer: 2 x 4 tcgen05.mma (128 x 256 x 16) per stage into the
 //                  tile's buffer; commits free the stage and, after the last stage, hand
 //                  the buffer over
-//   warps 6, 7     the tile table
-//   warps 8..15    B producers: thread r owns row r of the weight tile; it streams that
-//                  row's Q4_0 bytes through a private cp.async ring 2 stages ahead (across
-//                  tile boundaries) and dequantises each stage into the swizzled fp16 tile
+//   warps 6, 7     the tile table; then warp 6 lane 0 is the raw producer: TMA of the
+//                  weight tile's Q4_0 nibbles (two blocks of 256 rows) and scales per stage
+//   warps 8..15    B producers: thread r owns row r of the weight tile; it dequantises its
+//                  two blocks of each stage into the 128B-swizzled K-major fp16 tile
 // A 256-wide weight tile halves the activation bytes the MMAs read from shared memory per
 // FLOP against a 128-wide one: with both operands in shared memory, an M = 128, N = 128
-// MMA alone asks for about the whole shared-memory bandwidth.
+// MMA alone asks for about the whole shared-memory bandwidth.  The raw bytes come by TMA
+// because each row's 32 bytes of a stage lie in a different 1 KB-strided row of the slot:
+// per-thread copies cost one cache line per thread.
 template <int MODE>  // 0: gate/up + SwiGLU, 1: down
 __global__ void __launch_bounds__(kGT, 1)
-    prefill_gemm(const PrefillParams p, int l, const __grid_constant__ CUtensorMap tm_hi,
-                 const __grid_constant__ CUtensorMap tm_lo) {
+    prefill_gemm(const PrefillParams p, int l, const __grid_constant__ GemmMaps maps) {
   extern __shared__ __align__(1024) uint8_t psm_raw[];
   const int imax = p.I > p.Is ? p.I : p.Is;
   const int ntn = MODE == 0 ? (2 * imax) / kTN : p.H / kTN;
@@ -561,7 +589,7 @@ __global__ void __launch_bounds__(kGT, 1)
     return;
   }
 
-  // [A_hi 16K | A_lo 16K | B 16K] x S from a 1024-byte boundary, raw rings, tile table, barriers
+  // [A_hi 16K | A_lo 16K | B 32K] x S from a 1024-byte boundary, raw ring, tile table, barriers
   uint8_t* psm = psm_raw + ((1024u - (smem_u32p(psm_raw) & 1023u)) & 1023u);
   uint8_t* raw = psm + kTilesBytes;
   GemmTile* tiles = reinterpret_cast<GemmTile*>(raw + kRawRing);
@@ -570,7 +598,9 @@ __global__ void __launch_bounds__(kGT, 1)
   uint64_t* empty = full_b + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* raw_full = acc_empty + 2;
+  uint64_t* raw_empty = raw_full + kRawStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + kRawStages);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   auto a_hi = [&](int s) { return psm + s * kStageBytes; };
@@ -586,6 +616,10 @@ __global__ void __launch_bounds__(kGT, 1)
     for (int b = 0; b < 2; ++b) {
       pmbar_init(&acc_full[b], 1);
       pmbar_init(&acc_empty[b], 4);
+    }
+    for (int s = 0; s < kRawStages; ++s) {
+      pmbar_init(&raw_full[s], 1);
+      pmbar_init(&raw_empty[s], 8);
     }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -609,7 +643,7 @@ __global__ void __launch_bounds__(kGT, 1)
       t.row0 = g0 + mt * kTM;
       t.nvalid = n_e - mt * kTM;
       t.nK = (MODE == 0 && t.nt * (kTN / 2) >= t.Ie) ? 0 : (MODE == 0 ? p.H : t.Ie) / kTK;
-      t.slot = expert_slot(p, l, t.e);
+      t.slot = t.e < p.E ? p.layer_base[l] + (p.pin_slot[(size_t)l * p.E + t.e] & 0xffff) : l;
       t.pad = 0;
       tiles[i] = t;
     }
@@ -703,12 +737,12 @@ __global__ void __launch_bounds__(kGT, 1)
           asm volatile(
               "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
               "[%4];" ::"r"(smem_u32p(a_hi(s))),
-              "l"(&tm_hi), "r"(ks * kTK), "r"(t.row0), "r"(bar)
+              "l"(&maps.a_hi), "r"(ks * kTK), "r"(t.row0), "r"(bar)
               : "memory");
           asm volatile(
               "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
               "[%4];" ::"r"(smem_u32p(a_lo(s))),
-              "l"(&tm_lo), "r"(ks * kTK), "r"(t.row0), "r"(bar)
+              "l"(&maps.a_lo), "r"(ks * kTK), "r"(t.row0), "r"(bar)
               : "memory");
         }
       }
@@ -751,66 +785,54 @@ __global__ void __launch_bounds__(kGT, 1)
         ++tc;
       }
     }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- raw producer
+    if (lane == 0) {
+      int it = 0;
+      bool stop = false;
+      for (int i = 0; i < n_my && !stop; ++i) {
+        const GemmTile t = tiles[i];
+        const int sh = t.e < p.E ? 0 : 1;
+        for (int ks = 0; ks < t.nK; ++ks, ++it) {
+          const int rs = it % kRawStages;
+          if (it >= kRawStages && !pmbar_wait_ab(&raw_empty[rs], (uint32_t)(it / kRawStages - 1) & 1u, abort)) {
+            stop = true;
+            break;
+          }
+          const uint32_t bar = smem_u32p(&raw_full[rs]);
+          const uint32_t dq = smem_u32p(raw + rs * kRawStage), dd = dq + kRawNib;
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kRawStage)
+                       : "memory");
+          if (MODE == 0) {  // 128 gate rows then the same 128 up rows: row blocks 4 nt .. 4 nt + 3
+            for (int half = 0; half < 2; ++half) {
+              tma_load_5d(dq + half * (kRawNib / 2), &maps.nib[sh], ks * 32, 0, 2 * half, 4 * t.nt, t.slot, bar);
+              tma_load_5d(dd + half * (kTN / 2) * 16, &maps.scl[sh], (ks >> 2) * 16, 0, 2 * half, 4 * t.nt, t.slot,
+                          bar);
+            }
+          } else {  // 256 down rows: 16-row tiles 16 nt .. 16 nt + 15
+            tma_load_4d(dq, &maps.nib[sh], ks * 32, 0, 16 * t.nt, t.slot, bar);
+            tma_load_4d(dd, &maps.scl[sh], (ks >> 2) * 16, 0, 16 * t.nt, t.slot, bar);
+          }
+        }
+      }
+    }
   } else if (warp >= 8) {
     // ---------------------------------------------------------------- B producers
     const int r = tid - 256;
-    // weight row r of tile t: gate/up tiles hold 128 gate rows then the same 128 up rows
-    auto row_ptr = [&](const GemmTile& t, const uint8_t*& qrow, const uint8_t*& drow) {
-      const SlotLayout& Ls = t.e < p.E ? p.lay : p.slay;
-      const int wrow = MODE == 0 ? t.nt * (kTN / 2) + (r & (kTN / 2 - 1)) : t.nt * kTN + r;
-      const int K = MODE == 0 ? p.H : t.Ie, nbk = K / 32;
-      const uint8_t* rbase;  // the 16-row tile holding that row
-      if (MODE == 0)
-        rbase = t.slot + Ls.gu + ((size_t)4 * (wrow / 32) + (r >= kTN / 2 ? 2 : 0) + (wrow % 32) / 16) * 9u * p.H;
-      else
-        rbase = t.slot + Ls.down + (size_t)(wrow / 16) * 9u * K;
-      const int rr = wrow % 16;
-      qrow = rbase + (size_t)rr * nbk * 16;
-      drow = rbase + (size_t)16 * nbk * 16 + (size_t)rr * nbk * 2;
-    };
-    // fetch cursor: the stage kRawStages - 1 items ahead of the one being dequantised
-    int f_i = 0, f_ks = 0, f_it = 0;
-    const uint8_t *f_q = nullptr, *f_d = nullptr;
-    auto f_seek = [&]() {  // first tile with work at or after f_i
-      for (; f_i < n_my; ++f_i)
-        if (tiles[f_i].nK > 0) {
-          row_ptr(tiles[f_i], f_q, f_d);
-          return;
-        }
-    };
-    auto fetch_next = [&]() {  // issue the next item's copies (if any), one commit group either way
-      if (f_i < n_my) {
-        uint8_t* rq = raw + ((f_it % kRawStages) * kTN + r) * 32;
-        uint8_t* rd = raw + kRawStages * kTN * 32 + ((f_it % kRawStages) * kTN + r) * 4;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rq)), "l"(f_q + (size_t)f_ks * 32)
-                     : "memory");
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32p(rq + 16)),
-                     "l"(f_q + (size_t)f_ks * 32 + 16)
-                     : "memory");
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32p(rd)), "l"(f_d + (size_t)f_ks * 4)
-                     : "memory");
-        ++f_it;
-        if (++f_ks == tiles[f_i].nK) {
-          f_ks = 0;
-          ++f_i;
-          f_seek();
-        }
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    f_seek();
-    for (int k = 0; k < kRawStages - 1; ++k) fetch_next();
     int it = 0;
     bool stop = false;
     for (int i = 0; i < n_my && !stop; ++i) {
       const int nK = tiles[i].nK;
       for (int ks = 0; ks < nK; ++ks, ++it) {
-        fetch_next();  // refills the ring slot dequantised one item ago
-        asm volatile("cp.async.wait_group %0;" ::"n"(kRawStages - 1) : "memory");
-        const uint8_t* rq = raw + ((it % kRawStages) * kTN + r) * 32;
+        const int rs = it % kRawStages;
+        if (!pmbar_wait_ab(&raw_full[rs], (uint32_t)(it / kRawStages) & 1u, abort)) {
+          stop = true;
+          break;
+        }
+        const uint8_t* rq = raw + rs * kRawStage + r * 32;
         const uint4 q0 = *reinterpret_cast<const uint4*>(rq);
         const uint4 q1 = *reinterpret_cast<const uint4*>(rq + 16);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(raw + kRawStages * kTN * 32 + ((it % kRawStages) * kTN + r) * 4);
+        const uint32_t sc = *reinterpret_cast<const uint32_t*>(raw + rs * kRawStage + kRawNib + r * 16 + (ks & 3) * 4);
         const int s = it % kStages;
         if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) {
           stop = true;
@@ -839,12 +861,15 @@ __global__ void __launch_bounds__(kGT, 1)
           *reinterpret_cast<uint4*>(brow + (((c0 + 2) ^ (r & 7)) * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(brow + (((c0 + 3) ^ (r & 7)) * 16)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
         }
+        // the fence also orders this warp's reads of the raw slot before the TMA that refills it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) pmbar_arrive(&full_b[s]);
+        if (lane == 0) {
+          pmbar_arrive(&full_b[s]);
+          pmbar_arrive(&raw_empty[rs]);
+        }
       }
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -907,7 +932,7 @@ __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, in
 // ------------------------------------------------------------------ host side
 
 static uint32_t gemm_smem() {
-  return kTilesBytes + kRawRing + kTileCap * sizeof(GemmTile) + (3 * kStages + 4) * 8 + 16 + 1024;
+  return kTilesBytes + kRawRing + kTileCap * sizeof(GemmTile) + (3 * kStages + 4 + 2 * kRawStages) * 8 + 16 + 1024;
 }
 static int gemm_grid(int max_tiles, int n_sm) { return max_tiles < n_sm ? max_tiles : n_sm; }
 static size_t route_floats(int tpc, int H, int E) { return (size_t)tpc * ((size_t)H / kChunk * kUChunk + E) + 16; }
@@ -915,7 +940,8 @@ static int route_tpc(int, int) { return 2 * kRTok; }  // small enough for two CT
 static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
 
 int prefill_supported(int H, int E, int K, int I, int Is) {
-  if (H % kTN || H > kMaxH || I % (kTN / 2) || Is % (kTN / 2) || E > kMaxE || K > 32) return 0;
+  // 256-wide tiles; scale rows (K / 16 bytes) must be TMA strides, multiples of 16 bytes
+  if (H % kTN || H > kMaxH || I % 256 || Is % 256 || E > kMaxE || K > 32) return 0;
   return route_smem(H, E) <= 227 * 1024;
 }
 
@@ -942,6 +968,44 @@ static int make_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, uint64
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+// Byte tensor map over the slot layout (no swizzle): dims[0] is one row's bytes.
+static int make_byte_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                         const cuuint64_t* strides, const cuuint32_t* box) {
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+// Nibble and scale maps of one weight kind.  Gate/up (MODE 0): a slot's tiles are
+// (row block rb of I/32, subtile st of 4) at (4 rb + st) * 9H, each [16 rows x H/32 x 16 B]
+// then [16 rows x H/32 x 2 B]; a box is 16 rows x 2 subtiles x 4 row blocks = 128 rows.
+// Down (MODE 1): 16-row tiles c of H at down + c * 9I; a box is 16 rows x 16 tiles = 256 rows.
+static int make_weight_maps(PfnEncodeTiled enc, int mode, const uint8_t* pool, uint64_t n_slots, uint64_t slot_bytes,
+                            const SlotLayout& lay, int H, int I, CUtensorMap* nib, CUtensorMap* scl) {
+  if (mode == 0) {
+    const uint64_t nbk = H / 32, tile = 9ull * H;
+    const cuuint64_t dq[5] = {nbk * 16, 16, 4, (cuuint64_t)I / 32, n_slots};
+    const cuuint64_t sq[4] = {nbk * 16, tile, 4 * tile, slot_bytes};
+    const cuuint32_t bq[5] = {32, 16, 2, 4, 1};
+    const cuuint64_t dd[5] = {nbk * 2, 16, 4, (cuuint64_t)I / 32, n_slots};
+    const cuuint64_t sd[4] = {nbk * 2, tile, 4 * tile, slot_bytes};
+    const cuuint32_t bd[5] = {16, 16, 2, 4, 1};
+    return make_byte_map(enc, nib, pool + lay.gu, 5, dq, sq, bq) ||
+           make_byte_map(enc, scl, pool + lay.gu + 16 * nbk * 16, 5, dd, sd, bd);
+  }
+  const uint64_t nbk = I / 32, tile = 9ull * I;
+  const cuuint64_t dq[4] = {nbk * 16, 16, (cuuint64_t)H / 16, n_slots};
+  const cuuint64_t sq[3] = {nbk * 16, tile, slot_bytes};
+  const cuuint32_t bq[4] = {32, 16, 16, 1};
+  const cuuint64_t dd[4] = {nbk * 2, 16, (cuuint64_t)H / 16, n_slots};
+  const cuuint64_t sd[3] = {nbk * 2, tile, slot_bytes};
+  const cuuint32_t bd[4] = {16, 16, 16, 1};
+  return make_byte_map(enc, nib, pool + lay.down, 4, dq, sq, bq) ||
+         make_byte_map(enc, scl, pool + lay.down + 16 * nbk * 16, 4, dd, sd, bd);
 }
 
 // Tokens per pass: every GEMM CTA's tiles must fit its tile table.
@@ -1002,10 +1066,24 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.s.h = s.h + (size_t)t0 * H;
     p.s.y = s.y + (size_t)t0 * H;
     const int R = Tc * a.K + (a.Is > 0 ? Tc : 0);
-    CUtensorMap mx_hi, mx_lo, ma_hi, ma_lo;
-    if (make_map(enc, &mx_hi, s.xg_hi, R, H) || make_map(enc, &mx_lo, s.xg_lo, R, H) ||
-        make_map(enc, &ma_hi, s.a_hi, R, imax) || make_map(enc, &ma_lo, s.a_lo, R, imax))
+    GemmMaps m0, m1;  // gate/up, down
+    if (make_map(enc, &m0.a_hi, s.xg_hi, R, H) || make_map(enc, &m0.a_lo, s.xg_lo, R, H) ||
+        make_map(enc, &m1.a_hi, s.a_hi, R, imax) || make_map(enc, &m1.a_lo, s.a_lo, R, imax))
       return -1;
+    for (int mode = 0; mode < 2; ++mode) {
+      GemmMaps& g = mode == 0 ? m0 : m1;
+      if (make_weight_maps(enc, mode, a.pool, (uint64_t)a.pool_slots, a.slot_bytes, a.lay, H, a.I, &g.nib[0],
+                           &g.scl[0]))
+        return -1;
+      if (a.Is > 0) {
+        if (make_weight_maps(enc, mode, a.shared_pool, (uint64_t)a.L, a.shared_slot_bytes, a.slay, H, a.Is, &g.nib[1],
+                             &g.scl[1]))
+          return -1;
+      } else {
+        g.nib[1] = g.nib[0];
+        g.scl[1] = g.scl[0];
+      }
+    }
     const int max_jobs = (R + kTM - 1) / kTM + E + 1;
     cudaError_t e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * E, st);
     if (e != cudaSuccess) return (int)e;
@@ -1013,9 +1091,8 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
       prefill_route<<<(Tc + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
       prefill_scan<<<1, 1024, 0, st>>>(p);
       prefill_scatter<<<(Tc + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
-      prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, mx_hi,
-                                                                                                   mx_lo);
-      prefill_gemm<1><<<gemm_grid(max_jobs * (H / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, ma_hi, ma_lo);
+      prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, m0);
+      prefill_gemm<1><<<gemm_grid(max_jobs * (H / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, m1);
       prefill_combine<<<Tc, kPT, 0, st>>>(p, l);
       e = cudaGetLastError();
       if (e != cudaSuccess) return (int)e;

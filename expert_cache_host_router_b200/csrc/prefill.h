@@ -15,6 +15,7 @@ struct PrefillArgs {
   int n_sm;  // the device's SM count: persistent GEMM grids
   float eps;
   const uint8_t* pool;
+  int64_t pool_slots;  // slots in the pool (the weight tensor maps' extent)
   uint64_t slot_bytes;
   SlotLayout lay, slay;
   const uint8_t* shared_pool;

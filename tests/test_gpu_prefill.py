@@ -75,7 +75,7 @@ def test_prefill_small_layer():
     m.close()
 
 
-STACK = synthetic.Shape(n_layers=3, hidden=512, n_experts=64, top_k=8, inter=256, shared_inter=128,
+STACK = synthetic.Shape(n_layers=3, hidden=512, n_experts=64, top_k=8, inter=512, shared_inter=256,
                         use_rmsnorm=1, zipf_s=1.0)
 
 
