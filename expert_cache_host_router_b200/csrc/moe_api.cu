@@ -628,8 +628,9 @@ static int prefill_reserve(moe_ctx* c, int T) {
   const size_t o_h = take((size_t)T * H * 4), o_sel = take((size_t)T * K * 4), o_w = take((size_t)T * K * 4),
                o_xh = take((size_t)T * H * 2), o_xl = take((size_t)T * H * 2), o_gh = take(R * H * 2),
                o_gl = take(R * H * 2), o_ah = take(R * imax * 2), o_al = take(R * imax * 2),
-               o_ob = take((size_t)T * (K + 1) * H * 4), o_cnt = take(E * 4), o_cur = take((E + 1) * 4),
-               o_off = take((E + 2) * 4), o_perm = take(R * 4), o_jobs = take((R / 128 + E + 2) * 4),
+               o_ob = take(R * H * 4), o_gp = take((size_t)T * (K + 1) * 4), o_cnt = take(E * 4),
+               o_cur = take((E + 1) * 4),
+               o_off = take((E + 2) * 4), o_jobs = take((R / 128 + E + 2) * 4),
                o_nj = take(4);
   uint8_t* m = nullptr;
   CK(cudaMalloc((void**)&m, off));
@@ -646,10 +647,10 @@ static int prefill_reserve(moe_ctx* c, int T) {
   s.a_hi = reinterpret_cast<__half*>(m + o_ah);
   s.a_lo = reinterpret_cast<__half*>(m + o_al);
   s.obuf = reinterpret_cast<float*>(m + o_ob);
+  s.gpos = reinterpret_cast<int32_t*>(m + o_gp);
   s.counts = reinterpret_cast<int32_t*>(m + o_cnt);
   s.cursor = reinterpret_cast<int32_t*>(m + o_cur);
   s.offsets = reinterpret_cast<int32_t*>(m + o_off);
-  s.perm = reinterpret_cast<int32_t*>(m + o_perm);
   s.jobs = reinterpret_cast<int32_t*>(m + o_jobs);
   s.n_jobs = reinterpret_cast<int32_t*>(m + o_nj);
   return MOE_OK;

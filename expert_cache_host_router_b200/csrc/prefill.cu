@@ -50,6 +50,7 @@ static_assert(kTileBytes % 1024 == 0 && kBTileBytes % 1024 == 0, "operand tiles 
 struct PrefillParams {
   int L, H, E, K, I, Is, use_norm, T, nch, tpc;
   int t_base, T_total;  // this chunk's first token and the call's token count (trace rows)
+  int R;                // grouped rows of this chunk: T * k (+ T with a shared expert)
   float eps;
   const uint8_t* pool;  // layer l expert e at pool + (base[l] + (pin[l][e] & 0xffff)) * slot_bytes
   uint64_t slot_bytes;
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(kPT) prefill_scatter(const PrefillParams p) {
       } else {
         pos = p.s.offsets[p.E] + t;
       }
-      p.s.perm[pos] = (t << 8) | r;
+      p.s.gpos[(size_t)t * (p.K + 1) + r] = pos;
     }
     pos = __shfl_sync(0xffffffffu, pos, 0);
     uint4* dh = reinterpret_cast<uint4*>(p.s.xg_hi + (size_t)pos * p.H);
@@ -696,16 +697,14 @@ __global__ void __launch_bounds__(kGT, 1)
             dl[1] = reinterpret_cast<const uint4*>(lo)[1];
           }
         }
-      } else {
-        const int pr = valid ? p.s.perm[grow] : 0;
-        float* dst = p.s.obuf + ((size_t)(pr >> 8) * (p.K + 1) + (pr & 0xFF)) * p.H + t.nt * kTN;
+      } else {  // expert outputs as [H / 16][R][16]: a warp's 32 rows x 16 columns are 2 KB in a row
 #pragma unroll 1
         for (int c0 = 0; c0 < kTN; c0 += 16) {
           uint32_t o[16];
           tmem_ld16(taddr + c0, o);
           tmem_wait16(o);
           if (valid) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c0);
+            float4* d4 = reinterpret_cast<float4*>(p.s.obuf + (((size_t)(t.nt * kTN + c0) / 16) * p.R + grow) * 16);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               d4[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
@@ -884,21 +883,23 @@ __global__ void __launch_bounds__(kGT, 1)
 // ------------------------------------------------------------------ combine
 
 // h[t] += sum_rank w * o_rank + o_shared in rank order (without the norm: h = that sum).
-// Thread: 4 columns; the expert outputs of those columns are loaded 10 ranks at a time
-// (streaming, read once) before they are summed, so the loads overlap.
+// Expert outputs are column-block-major over grouped rows ([H / 16][R][16]); the token's
+// grouped positions come from the scatter.  Thread: 4 columns; the outputs of those
+// columns are loaded 10 ranks at a time (streaming, read once) before they are summed.
 constexpr int kCombineGroup = 10;
 __global__ void __launch_bounds__(kPT) prefill_combine(const PrefillParams p, int l) {
   const int t = blockIdx.x;
   const float* w = p.s.w + (size_t)t * p.K;
-  const float* ob = p.s.obuf + (size_t)t * (p.K + 1) * p.H;
+  const int* gp = p.s.gpos + (size_t)t * (p.K + 1);
   const int nr = p.K + (p.Is > 0 ? 1 : 0);
   for (int j = threadIdx.x * 4; j < p.H; j += kPT * 4) {
+    const float* col = p.s.obuf + (size_t)(j / 16) * p.R * 16 + (j & 15);
     float4 y = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     for (int r0 = 0; r0 < nr; r0 += kCombineGroup) {
       float4 o[kCombineGroup];
 #pragma unroll
       for (int i = 0; i < kCombineGroup; ++i)
-        if (r0 + i < nr) o[i] = __ldcs(reinterpret_cast<const float4*>(ob + (size_t)(r0 + i) * p.H + j));
+        if (r0 + i < nr) o[i] = __ldcs(reinterpret_cast<const float4*>(col + (size_t)gp[r0 + i] * 16));
 #pragma unroll
       for (int i = 0; i < kCombineGroup; ++i) {
         const int r = r0 + i;
@@ -1066,6 +1067,7 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.s.h = s.h + (size_t)t0 * H;
     p.s.y = s.y + (size_t)t0 * H;
     const int R = Tc * a.K + (a.Is > 0 ? Tc : 0);
+    p.R = R;
     GemmMaps m0, m1;  // gate/up, down
     if (make_map(enc, &m0.a_hi, s.xg_hi, R, H) || make_map(enc, &m0.a_lo, s.xg_lo, R, H) ||
         make_map(enc, &m1.a_hi, s.a_hi, R, imax) || make_map(enc, &m1.a_lo, s.a_lo, R, imax))

@@ -40,11 +40,11 @@ struct PrefillScratch {
   __half *x_hi, *x_lo;    // [T][H]
   __half *xg_hi, *xg_lo;  // [R][H]
   __half *a_hi, *a_lo;    // [R][max(I, Is)]
-  float* obuf;       // [T][K + 1][H]
+  float* obuf;       // [H / 16][R][16] expert outputs over grouped rows
+  int32_t* gpos;     // [T][K + 1] grouped row of each (token, rank)
   int32_t* counts;   // [E]
   int32_t* cursor;   // [E + 1]
   int32_t* offsets;  // [E + 2]
-  int32_t* perm;     // [R]
   int32_t* jobs;     // [R / 128 + E + 1]
   int32_t* n_jobs;   // [1]
   int32_t* error;    // device error word (MOE_DEVERR_*)
