@@ -53,6 +53,8 @@ struct moe_ctx {
   std::atomic<uint8_t*> pool{nullptr};
   int64_t pool_slots = 0;
   uint16_t* router = nullptr;
+  uint16_t* router_rows = nullptr;  // [L][E][H] bf16 (prefill's router GEMM)
+  float* wnorm = nullptr;           // [L] max_e ||w_e||_2 rounded up (prefill's routing bound)
   float* bias = nullptr;
   float* gain = nullptr;
   bool has_bias = false, has_gain = false;
@@ -335,7 +337,7 @@ void moe_destroy(moe_ctx* c) {
   void* dev[] = {c->shared_pool, c->pool.load(), c->router, c->bias, c->gain, c->pin_slot,
                  c->layer_base, c->n_pinned, c->ring_owner, c->ring_stamp, c->ring_clock,
                  c->h, c->part, c->sq, c->z, c->acodes, c->hist, c->log, c->ctrl, c->done_seq,
-                 c->x_buf, c->y_buf, c->prefill_mem};
+                 c->x_buf, c->y_buf, c->prefill_mem, c->router_rows, c->wnorm};
   for (void* p : dev)
     if (p) cudaFree(p);
   void* hst[] = {c->host_tier, c->x_pin, c->y_pin, c->err_pin, c->mbox_host};
@@ -377,6 +379,21 @@ int moe_load_layer(moe_ctx* c, int32_t l, const uint8_t* const* experts, const u
         memcpy(&tmp[((size_t)ch * c->E + e) * kChunk], router_bf16 + (size_t)e * c->H + ch * kChunk,
                kChunk * sizeof(uint16_t));
     CK(cudaMemcpy(c->router + (size_t)l * c->E * c->H, tmp.data(), tmp.size() * 2, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(c->router_rows + (size_t)l * c->E * c->H, router_bf16, (size_t)c->E * c->H * 2,
+                  cudaMemcpyHostToDevice));
+    double wmax = 0.0;  // the largest router row norm, for the prefill routing error bound
+    for (int e = 0; e < c->E; ++e) {
+      double ss = 0.0;
+      for (int j = 0; j < c->H; ++j) {
+        uint32_t bits = (uint32_t)router_bf16[(size_t)e * c->H + j] << 16;
+        float w;
+        memcpy(&w, &bits, 4);
+        ss += (double)w * w;
+      }
+      wmax = std::max(wmax, std::sqrt(ss));
+    }
+    const float wn = std::nextafter((float)(wmax * (1.0 + 1e-9)), INFINITY);
+    CK(cudaMemcpy(c->wnorm + l, &wn, sizeof(float), cudaMemcpyHostToDevice));
   }
   if (bias) {
     CK(cudaMemcpy(c->bias + (size_t)l * c->E, bias, sizeof(float) * c->E, cudaMemcpyHostToDevice));
@@ -458,6 +475,8 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   const int n_exp = c->K + (c->Is > 0);
   const int imax = std::max(c->I, c->Is);
   CKC(dalloc(&c->router, (size_t)c->L * c->E * c->H));
+  CKC(dalloc(&c->router_rows, (size_t)c->L * c->E * c->H));
+  CKC(dalloc(&c->wnorm, c->L));
   CKC(dalloc(&c->bias, (size_t)c->L * c->E));
   CKC(dalloc(&c->gain, (size_t)c->L * c->H));
   if (c->Is > 0) CKC(dalloc(&c->shared_pool, (size_t)c->L * c->shared_slot_bytes));
@@ -627,6 +646,8 @@ static int prefill_reserve(moe_ctx* c, int T) {
   };
   const size_t o_h = take((size_t)T * H * 4), o_sel = take((size_t)T * K * 4), o_w = take((size_t)T * K * 4),
                o_xh = take((size_t)T * H * 2), o_xl = take((size_t)T * H * 2), o_gh = take(R * H * 2),
+               o_u = take((size_t)T * H * 4), o_ua = take((size_t)T * 3 * H * 2), o_inv = take((size_t)T * 4),
+               o_un = take((size_t)T * 4), o_part = take((size_t)8 * T * E * 4),
                o_gl = take(R * H * 2), o_ah = take(R * imax * 2), o_al = take(R * imax * 2),
                o_ob = take(R * H * 4), o_gp = take((size_t)T * (K + 1) * 4), o_cnt = take(E * 4),
                o_cur = take((E + 1) * 4),
@@ -640,6 +661,11 @@ static int prefill_reserve(moe_ctx* c, int T) {
   s.h = reinterpret_cast<float*>(m + o_h);
   s.sel = reinterpret_cast<int32_t*>(m + o_sel);
   s.w = reinterpret_cast<float*>(m + o_w);
+  s.u = reinterpret_cast<float*>(m + o_u);
+  s.ua = reinterpret_cast<__nv_bfloat16*>(m + o_ua);
+  s.inv = reinterpret_cast<float*>(m + o_inv);
+  s.unorm = reinterpret_cast<float*>(m + o_un);
+  s.part = reinterpret_cast<float*>(m + o_part);
   s.x_hi = reinterpret_cast<__half*>(m + o_xh);
   s.x_lo = reinterpret_cast<__half*>(m + o_xl);
   s.xg_hi = reinterpret_cast<__half*>(m + o_gh);
@@ -703,6 +729,8 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   a.pin_slot = c->pin_slot;
   a.layer_base = c->layer_base;
   a.hist = c->hist;
+  a.router_rows = c->router_rows;
+  a.wnorm = c->wnorm;
   const int r = prefill_run(a, sc, c->encode_tiled, s);
   if (r == -1) return MOE_ERR_UNSUPPORTED;
   if (r != 0) return cuda_fail((cudaError_t)r);

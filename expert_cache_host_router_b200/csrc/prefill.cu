@@ -7,9 +7,10 @@
 // turns each expert's GEMVs into GEMMs [n_e x H] x [H x 2I] and [n_e x I] x [I x H]
 // (n_e = tokens routed to expert e): a dense contraction, so it runs on the tensor
 // cores.  Per layer, in stream order:
-//   route    8 tokens per CTA: RMSNorm scale, router logits in the canonical
-//            order, top-k, weights, histogram, per-expert counts; x = RMSNorm(h) split
-//            into fp16 hi + lo (x = hi + lo to about 2^-22 relative)
+//   route    RMSNorm scale and x = RMSNorm(h) split into fp16 hi + lo (x = hi + lo to
+//            about 2^-22 relative); router logits approximated on the tensor cores, the
+//            top-k certified with exact canonical-order logits of the candidates (below);
+//            weights, histogram, per-expert counts
 //   scan     expert offsets and the list of 128-row m-tiles
 //   scatter  one warp per token: its rows of x copied to their place in expert order
 //            (within an expert the order is whatever the atomics give: a GEMM row does
@@ -48,7 +49,7 @@ constexpr uint32_t kTilesBytes = kStageBytes * kStages;
 static_assert(kTileBytes % 1024 == 0 && kBTileBytes % 1024 == 0, "operand tiles must keep the swizzle phase");
 
 struct PrefillParams {
-  int L, H, E, K, I, Is, use_norm, T, nch, tpc;
+  int L, H, E, K, I, Is, use_norm, T, nch;
   int t_base, T_total;  // this chunk's first token and the call's token count (trace rows)
   int R;                // grouped rows of this chunk: T * k (+ T with a shared expert)
   float eps;
@@ -63,6 +64,7 @@ struct PrefillParams {
   const int32_t* pin_slot;
   const int32_t* layer_base;
   uint32_t* hist;
+  const float* wnorm;  // [L] max_e ||w_e||_2 of the router rows, rounded up
   PrefillScratch s;
 };
 
@@ -75,258 +77,6 @@ __device__ __forceinline__ float bf16_hi_p(uint32_t w) { return __uint_as_float(
 __device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, int l, int e) {
   if (e >= p.E) return p.shared_pool + (size_t)l * p.shared_slot_bytes;
   return p.pool + (size_t)(p.layer_base[l] + (p.pin_slot[(size_t)l * p.E + e] & 0xffff)) * p.slot_bytes;
-}
-
-// ------------------------------------------------------------------ route
-
-constexpr int kRTok = 4;  // tokens per warp in the router
-
-// Row stride of u in shared memory: 16-column chunks padded to 20 floats, so the four
-// chunks that a warp's lanes read at once (one per residue, r chunks apart) fall in four
-// different bank groups.
-constexpr int kUChunk = 20;
-
-// CTA of 8 warps, p.tpc (8) tokens.  Logit z_e of a token is the canonical fold of
-// its 16-column chunk partials (each an fmaf chain from +0): fold lane q adds chunks
-// q, q + 32, ... from +0, then the 32 lane sums combine as the xor butterfly 16, 8, 4, 2,
-// 1 does.  In that butterfly's tree the sums of lanes q = r (mod 4) meet first (levels
-// 16, 8, 4) and the four results meet last (levels 2, 1).  So here warp lane
-// 4 * slot + r evaluates residue r's 8-leaf subtree (leaves in bit-reversed order, a
-// 3-deep stack) for 4 tokens x 2 experts, and the last two levels are shuffles.  Lanes of
-// one residue read the same u (one shared-memory wavefront for 8 lanes) and each weight
-// a lane loads serves 4 tokens.
-__global__ void __launch_bounds__(kPT, 2) prefill_route(const PrefillParams p, int l) {
-  extern __shared__ __align__(16) float rsm[];
-  const int H = p.H, E = p.E, nch = p.nch, TPC = p.tpc;
-  const int ustride = nch * kUChunk;
-  float* us = rsm;                        // [TPC][nch][20]  u = g * h (or h), padded chunks
-  float* zs = us + (size_t)TPC * ustride;  // [TPC][E]
-  float* invs = zs + (size_t)TPC * E;     // [TPC]
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * TPC;
-  const float* g = p.gain + (size_t)l * H;
-
-  // 1. per token: inv (canonical fold of the squares), u into shared memory, x hi/lo out
-  for (int tl = warp; tl < TPC; tl += kPT / 32) {
-    const int t = t0 + tl;
-    float* u = us + (size_t)tl * ustride;
-    if (t >= p.T) {
-      for (int j = lane; j < H; j += 32) u[(j >> 4) * kUChunk + (j & 15)] = 0.0f;
-      if (lane == 0) invs[tl] = 1.0f;
-      continue;
-    }
-    const float* hrow = p.s.h + (size_t)t * H;
-    float inv = 1.0f;
-    if (p.use_norm) {
-      float acc = 0.0f;
-      for (int c = lane; c < nch; c += 32) {
-        const float4* hp = reinterpret_cast<const float4*>(hrow + c * 16);
-        float pc = 0.0f;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 q = hp[v];
-          pc = fmaf(q.x, q.x, pc);
-          pc = fmaf(q.y, q.y, pc);
-          pc = fmaf(q.z, q.z, pc);
-          pc = fmaf(q.w, q.w, pc);
-        }
-        acc = __fadd_rn(acc, pc);
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
-      inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(acc, (float)H), p.eps)));
-    }
-    if (lane == 0) invs[tl] = inv;
-    for (int j = lane; j < H; j += 32) {
-      const float hv = hrow[j];
-      float xv = hv;
-      float* uj = u + (j >> 4) * kUChunk + (j & 15);
-      if (p.use_norm) {
-        *uj = __fmul_rn(g[j], hv);
-        xv = __fmul_rn(__fmul_rn(hv, inv), g[j]);
-      } else {
-        *uj = hv;
-      }
-      const __half hi = __float2half_rn(xv);
-      p.s.x_hi[(size_t)t * H + j] = hi;
-      p.s.x_lo[(size_t)t * H + j] = __float2half_rn(xv - __half2float(hi));
-    }
-  }
-  __syncthreads();
-
-  // 2. logits: warp job = (token group of 4, block of 16 experts); lane = 4 * slot + r
-  const int ntg = TPC / kRTok, nblk = (E + 15) / 16;
-  const int r4 = lane & 3, slot = lane >> 2;
-  for (int job = warp; job < ntg * nblk; job += kPT / 32) {
-    const int tg = job % ntg, e0 = (job / ntg) * 16 + 2 * slot, e1 = e0 + 1;
-    const bool v0 = e0 < E, v1 = e1 < E;
-    const float* ub = us + (size_t)tg * kRTok * ustride;
-    auto wload = [&](int c, uint4 (&w)[4]) {
-      const uint4* w0p = reinterpret_cast<const uint4*>(p.router + (((size_t)l * nch + c) * E + e0) * kChunk);
-      w[0] = w[1] = w[2] = w[3] = make_uint4(0, 0, 0, 0);
-      if (v0) {
-        w[0] = __ldg(w0p);
-        w[1] = __ldg(w0p + 1);
-      }
-      if (v1) {
-        w[2] = __ldg(w0p + 2);  // expert e0 + 1 follows e0 in the same chunk row
-        w[3] = __ldg(w0p + 3);
-      }
-    };
-    // leaf i' of this residue: fold lane r + 4 * brev3(i')
-    auto leaf_q = [&](int i) { return r4 + 4 * (int)(__brev((unsigned)i) >> 29); };
-    float stk[3][kRTok][2];
-    float cr[kRTok][2];
-    uint4 cw[4];
-    if (leaf_q(0) < nch) wload(leaf_q(0), cw);
-    for (int i = 0; i < 8; ++i) {
-      const int q = leaf_q(i);
-      float ls[kRTok][2];
-#pragma unroll
-      for (int t = 0; t < kRTok; ++t) ls[t][0] = ls[t][1] = 0.0f;
-      for (int c = q; c < nch; c += 32) {
-        // the next chunk this lane visits, loaded while this one is summed
-        int cn = c + 32;
-        if (cn >= nch) {
-          cn = -1;
-          for (int i2 = i + 1; i2 < 8; ++i2)
-            if (leaf_q(i2) < nch) {
-              cn = leaf_q(i2);
-              break;
-            }
-        }
-        uint4 nw[4];
-        if (cn >= 0) wload(cn, nw);
-        const uint32_t wa[8] = {cw[0].x, cw[0].y, cw[0].z, cw[0].w, cw[1].x, cw[1].y, cw[1].z, cw[1].w};
-        const uint32_t wb[8] = {cw[2].x, cw[2].y, cw[2].z, cw[2].w, cw[3].x, cw[3].y, cw[3].z, cw[3].w};
-        float pc[kRTok][2];
-#pragma unroll
-        for (int t = 0; t < kRTok; ++t) pc[t][0] = pc[t][1] = 0.0f;
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-#pragma unroll
-          for (int t = 0; t < kRTok; ++t) {
-            const float4 uv = *reinterpret_cast<const float4*>(ub + (size_t)t * ustride + c * kUChunk + 4 * j4);
-            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4]), uv.x, pc[t][0]);
-            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4]), uv.x, pc[t][1]);
-            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4]), uv.y, pc[t][0]);
-            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4]), uv.y, pc[t][1]);
-            pc[t][0] = fmaf(bf16_lo_p(wa[2 * j4 + 1]), uv.z, pc[t][0]);
-            pc[t][1] = fmaf(bf16_lo_p(wb[2 * j4 + 1]), uv.z, pc[t][1]);
-            pc[t][0] = fmaf(bf16_hi_p(wa[2 * j4 + 1]), uv.w, pc[t][0]);
-            pc[t][1] = fmaf(bf16_hi_p(wb[2 * j4 + 1]), uv.w, pc[t][1]);
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < kRTok; ++t) {
-          ls[t][0] = __fadd_rn(ls[t][0], pc[t][0]);
-          ls[t][1] = __fadd_rn(ls[t][1], pc[t][1]);
-        }
-        if (cn >= 0) {
-          cw[0] = nw[0];
-          cw[1] = nw[1];
-          cw[2] = nw[2];
-          cw[3] = nw[3];
-        }
-      }
-      // binary counter over the 8 leaves: level b combines while bit b of i is set
-      bool carry = true;
-#pragma unroll
-      for (int b = 0; b < 3; ++b) {
-        if (carry) {
-          if ((i >> b) & 1) {
-#pragma unroll
-            for (int t = 0; t < kRTok; ++t) {
-              ls[t][0] = __fadd_rn(stk[b][t][0], ls[t][0]);
-              ls[t][1] = __fadd_rn(stk[b][t][1], ls[t][1]);
-            }
-          } else {
-#pragma unroll
-            for (int t = 0; t < kRTok; ++t) {
-              stk[b][t][0] = ls[t][0];
-              stk[b][t][1] = ls[t][1];
-            }
-            carry = false;
-          }
-        }
-      }
-      if (carry) {
-#pragma unroll
-        for (int t = 0; t < kRTok; ++t) {
-          cr[t][0] = ls[t][0];
-          cr[t][1] = ls[t][1];
-        }
-      }
-    }
-    // butterfly levels 2 and 1 across the four residues
-#pragma unroll
-    for (int off = 2; off >= 1; off >>= 1) {
-#pragma unroll
-      for (int t = 0; t < kRTok; ++t) {
-        cr[t][0] = __fadd_rn(cr[t][0], __shfl_xor_sync(0xffffffffu, cr[t][0], off));
-        cr[t][1] = __fadd_rn(cr[t][1], __shfl_xor_sync(0xffffffffu, cr[t][1], off));
-      }
-    }
-    const float b0 = (p.bias && v0) ? __ldg(p.bias + (size_t)l * E + e0) : 0.0f;
-    const float b1 = (p.bias && v1) ? __ldg(p.bias + (size_t)l * E + e1) : 0.0f;
-#pragma unroll
-    for (int t = 0; t < kRTok; ++t) {
-      if ((t & 3) != r4) continue;  // the four residue lanes hold the same sums: share the stores
-      const float inv = invs[tg * kRTok + t];
-      if (v0) zs[(size_t)(tg * kRTok + t) * E + e0] = fmaf(cr[t][0], inv, b0);
-      if (v1) zs[(size_t)(tg * kRTok + t) * E + e1] = fmaf(cr[t][1], inv, b1);
-    }
-  }
-  __syncthreads();
-
-  // 3. top-k by (logit desc, index asc; -0 == +0; NaN never preferred), weights, counts
-  for (int tl = warp; tl < TPC; tl += kPT / 32) {
-    const int t = t0 + tl;
-    if (t >= p.T) continue;
-    const float* z = zs + (size_t)tl * E;
-    int my_e = -1;
-    uint32_t taken = 0;
-    for (int i = 0; i < p.K; ++i) {
-      uint64_t best = 0;
-      for (int k = 0; lane + 32 * k < E; ++k) {
-        if ((taken >> k) & 1u) continue;
-        const int e = lane + 32 * k;
-        float v = z[e];
-        if (v == 0.0f) v = 0.0f;
-        const uint32_t uu = __float_as_uint(v);
-        uint32_t o = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
-        if (v != v) o = 0;
-        const uint64_t key = ((uint64_t)o << 32) | (uint32_t)(~(uint32_t)e);
-        best = key > best ? key : best;
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)best, off);
-        const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(best >> 32), off);
-        const uint64_t o = ((uint64_t)hi << 32) | lo;
-        best = o > best ? o : best;
-      }
-      int e = (int)(~(uint32_t)best);
-      if ((best >> 32) == 0ull) {  // only NaN logits left
-        if (lane == 0) atomicCAS(p.s.error, 0, MOE_DEVERR_ROUTE);
-        e = 0;
-      }
-      if ((e & 31) == lane) taken |= 1u << (e >> 5);
-      if (lane == i) my_e = e;
-    }
-    const float zmax = __shfl_sync(0xffffffffu, lane < p.K ? z[my_e] : 0.0f, 0);
-    const float ex = lane < p.K ? expf(z[my_e] - zmax) : 0.0f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane < p.K) {
-      p.s.sel[(size_t)t * p.K + lane] = my_e;
-      p.s.w[(size_t)t * p.K + lane] = __fdividef(ex, sum);
-      atomicAdd(p.hist + (size_t)l * E + my_e, 1u);
-      atomicAdd(p.s.counts + my_e, 1);
-      if (p.s.sel_trace) p.s.sel_trace[((size_t)l * p.T_total + p.t_base + t) * p.K + lane] = my_e;
-    }
-  }
 }
 
 // ------------------------------------------------------------------ grouping
@@ -880,6 +630,373 @@ __global__ void __launch_bounds__(kGT, 1)
   }
 }
 
+// ------------------------------------------------------------------ certified router
+//
+// The canonical-order logits above cost H x E fp32 FMAs per token on CUDA cores.  The
+// routing decision only needs them for the experts that can make the top-k, so:
+//   prep    u = g * h (fp32) split exactly into three bf16 parts (u = u0 + u1 + u2), plus
+//           inv, ||u||_2 and x hi/lo
+//   gemm    approximate S~ = sum_p u_p . w_e on the tensor cores (bf16 x bf16, products exact
+//           in fp32, fp32 accumulation), split over K, partials summed in a fixed order
+//   select  per token: the kCand best approximate logits are evaluated exactly in the
+//           canonical order; the top-k among them is final once the k-th exact logit beats
+//           the best approximate logit left out by more than twice the error bound
+//           delta = 2^-9 * ||u|| * max_e ||w_e|| * inv  (the accumulation error of S~ is at
+//           most 2^-10 * sum_j |w_j u_j| <= 2^-10 ||u|| ||w_e||, Cauchy-Schwarz); otherwise
+//           the candidate set widens (64, then every expert).
+// Every selection is therefore the canonical one, bit for bit.
+constexpr int kRParts = 3;   // bf16 parts of u
+constexpr int kRSplit = 8;   // K splits of the router GEMM
+constexpr int kCand = 16;    // candidates evaluated exactly first
+constexpr int kRGT = 192;    // router GEMM threads: 6 warps
+constexpr int kRStages = 4;
+
+// Warp per token: inv (canonical fold of the squares), u and its three bf16 parts, ||u||,
+// and x = RMSNorm(h) as fp16 hi + lo; four consecutive columns per lane.
+__global__ void __launch_bounds__(kPT) prefill_route_prep(const PrefillParams p, int l) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kPT / 32) + (threadIdx.x >> 5);
+  if (t >= p.T) return;
+  const int H = p.H, nch = p.nch;
+  const float* hrow = p.s.h + (size_t)t * H;
+  const float* g = p.gain + (size_t)l * H;
+  float inv = 1.0f;
+  if (p.use_norm) {
+    float acc = 0.0f;
+    for (int c = lane; c < nch; c += 32) {
+      const float4* hp = reinterpret_cast<const float4*>(hrow + c * 16);
+      float pc = 0.0f;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 q = hp[v];
+        pc = fmaf(q.x, q.x, pc);
+        pc = fmaf(q.y, q.y, pc);
+        pc = fmaf(q.z, q.z, pc);
+        pc = fmaf(q.w, q.w, pc);
+      }
+      acc = __fadd_rn(acc, pc);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(acc, (float)H), p.eps)));
+  }
+  float uu = 0.0f;
+  float* urow = p.s.u + (size_t)t * H;
+  __nv_bfloat16* ua = p.s.ua + (size_t)t * kRParts * H;
+  for (int j = lane * 4; j < H; j += 128) {
+    const float4 h4 = *reinterpret_cast<const float4*>(hrow + j);
+    const float hv[4] = {h4.x, h4.y, h4.z, h4.w};
+    float4 g4 = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+    if (p.use_norm) g4 = *reinterpret_cast<const float4*>(g + j);
+    const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+    float u[4];
+    __nv_bfloat16 b0[4], b1[4], b2[4];
+    __half xh[4], xl[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      u[i] = p.use_norm ? __fmul_rn(gv[i], hv[i]) : hv[i];
+      const float xv = p.use_norm ? __fmul_rn(__fmul_rn(hv[i], inv), gv[i]) : hv[i];
+      b0[i] = __float2bfloat16_rn(u[i]);
+      const float r1 = u[i] - __bfloat162float(b0[i]);
+      b1[i] = __float2bfloat16_rn(r1);
+      b2[i] = __float2bfloat16_rn(r1 - __bfloat162float(b1[i]));
+      uu = fmaf(u[i], u[i], uu);
+      xh[i] = __float2half_rn(xv);
+      xl[i] = __float2half_rn(xv - __half2float(xh[i]));
+    }
+    *reinterpret_cast<float4*>(urow + j) = make_float4(u[0], u[1], u[2], u[3]);
+    *reinterpret_cast<uint2*>(ua + j) = *reinterpret_cast<const uint2*>(b0);
+    *reinterpret_cast<uint2*>(ua + H + j) = *reinterpret_cast<const uint2*>(b1);
+    *reinterpret_cast<uint2*>(ua + 2 * H + j) = *reinterpret_cast<const uint2*>(b2);
+    *reinterpret_cast<uint2*>(p.s.x_hi + (size_t)t * H + j) = *reinterpret_cast<const uint2*>(xh);
+    *reinterpret_cast<uint2*>(p.s.x_lo + (size_t)t * H + j) = *reinterpret_cast<const uint2*>(xl);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, off);
+  if (lane == 0) {
+    p.s.inv[t] = inv;
+    // fp32 sum of H squares: relative error below H * 2^-23; 1e-3 covers it for H <= 4096
+    p.s.unorm[t] = __fsqrt_ru(uu * 1.001f);
+  }
+}
+
+// Approximate router logits before the norm scale: part[split][t][e] = sum over the
+// split's K range of [u0|u1|u2] . [w|w|w].  CTA = 128 tokens x N experts x one K split;
+// warp 0 lane 0 TMA, warp 1 lane 0 MMA (tensor memory allocated by warp 1), warps 2..5
+// the epilogue (one tensor-memory lane quarter each).
+__global__ void __launch_bounds__(kRGT, 1)
+    prefill_router_gemm(const PrefillParams p, const __grid_constant__ CUtensorMap ma,
+                        const __grid_constant__ CUtensorMap mb, int N, int kst_per_split) {
+  extern __shared__ __align__(1024) uint8_t rsm_raw[];
+  const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * N, split = blockIdx.z;
+  const int total_k = kRParts * p.H / kTK;
+  const int k0 = split * kst_per_split;
+  const int nK = (k0 + kst_per_split < total_k ? k0 + kst_per_split : total_k) - k0;
+  if (nK <= 0) return;
+  const uint32_t a_bytes = kTM * kTK * 2, b_bytes = (uint32_t)N * kTK * 2;
+  const uint32_t stage = a_bytes + ((b_bytes + 1023) & ~1023u);
+  uint8_t* sm = rsm_raw + ((1024u - (smem_u32p(rsm_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kRStages * stage);
+  uint64_t* empty = full + kRStages;
+  uint64_t* done = empty + kRStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t ncols = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  if (tid == 0) {
+    for (int s = 0; s < kRStages; ++s) {
+      pmbar_init(&full[s], 1);
+      pmbar_init(&empty[s], 1);
+    }
+    pmbar_init(done, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32p(tmem_slot)),
+                 "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  // bf16 x bf16 -> f32, K-major A and B, M = 128, N
+  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < nK; ++i) {
+      const int s = i % kRStages, ks = k0 + i;
+      if (i >= kRStages && !pmbar_wait_ab(&empty[s], (uint32_t)(i / kRStages - 1) & 1u, abort)) break;
+      const uint32_t bar = smem_u32p(&full[s]);
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(a_bytes + b_bytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+          "[%4];" ::"r"(smem_u32p(sm + s * stage)),
+          "l"(&ma), "r"(ks * kTK), "r"(m0), "r"(bar)
+          : "memory");
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+          "[%4];" ::"r"(smem_u32p(sm + s * stage + a_bytes)),
+          "l"(&mb), "r"((ks * kTK) % p.H), "r"(n0), "r"(bar)
+          : "memory");
+    }
+  } else if (warp == 1 && lane == 0) {
+    for (int i = 0; i < nK; ++i) {
+      const int s = i % kRStages;
+      if (!pmbar_wait_ab(&full[s], (uint32_t)(i / kRStages) & 1u, abort)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t sa = smem_u32p(sm + s * stage), sb = sa + a_bytes;
+#pragma unroll
+      for (int kk = 0; kk < kTK / 16; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}" ::"r"(tmem),
+            "l"(umma_desc(sa + kk * 32)), "l"(umma_desc(sb + kk * 32)), "r"(idesc), "r"(acc)
+            : "memory");
+      }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32p(&empty[s]))
+                   : "memory");
+    }
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32p(done))
+                 : "memory");
+  } else if (warp >= 2) {
+    const int q = warp & 3;  // tensor-memory lane quarter of this warp
+    const bool ok = __all_sync(0xffffffffu, pmbar_wait_ab(done, 0, abort));
+    if (ok) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const int t = m0 + q * 32 + lane;
+      float* dst = p.s.part + ((size_t)split * p.T + t) * p.E + n0;
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c0, o);
+        tmem_wait16(o);
+        if (t < p.T) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n0 + c0 + j < p.E) dst[c0 + j] = __uint_as_float(o[j]);
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (tid == 0 && *abort) atomicCAS(p.s.error, 0, MOE_DEVERR_TMA);
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols));
+  }
+}
+
+// Canonical logits of nc experts (cand[0..nc)) for the token whose u the lanes read; lane
+// = fold lane: each lane sums its chunks of every candidate (all loads in flight at once),
+// then one butterfly per candidate.  zx[cand[i]] receives the logit.
+constexpr int kCandBatch = 16;
+__device__ __forceinline__ void canonical_logits(const PrefillParams& p, int l, const float* urow,
+                                                 const uint32_t* cand, int nc, float inv, float* zx, int lane) {
+  for (int i0 = 0; i0 < nc; i0 += kCandBatch) {
+    float acc[kCandBatch];
+#pragma unroll
+    for (int i = 0; i < kCandBatch; ++i) acc[i] = 0.0f;
+    for (int c = lane; c < p.nch; c += 32) {
+      const float4* up = reinterpret_cast<const float4*>(urow + c * kChunk);
+      const float4 ua = up[0], ub = up[1], uc = up[2], ud = up[3];
+#pragma unroll
+      for (int i = 0; i < kCandBatch; ++i) {
+        if (i0 + i < nc) {
+          const int e = (int)cand[i0 + i];
+          const uint4* wp = reinterpret_cast<const uint4*>(p.router + (((size_t)l * p.nch + c) * p.E + e) * kChunk);
+          const uint4 w0 = __ldg(wp), w1 = __ldg(wp + 1);
+          float pc = 0.0f;
+          pc = fmaf(bf16_lo_p(w0.x), ua.x, pc);
+          pc = fmaf(bf16_hi_p(w0.x), ua.y, pc);
+          pc = fmaf(bf16_lo_p(w0.y), ua.z, pc);
+          pc = fmaf(bf16_hi_p(w0.y), ua.w, pc);
+          pc = fmaf(bf16_lo_p(w0.z), ub.x, pc);
+          pc = fmaf(bf16_hi_p(w0.z), ub.y, pc);
+          pc = fmaf(bf16_lo_p(w0.w), ub.z, pc);
+          pc = fmaf(bf16_hi_p(w0.w), ub.w, pc);
+          pc = fmaf(bf16_lo_p(w1.x), uc.x, pc);
+          pc = fmaf(bf16_hi_p(w1.x), uc.y, pc);
+          pc = fmaf(bf16_lo_p(w1.y), uc.z, pc);
+          pc = fmaf(bf16_hi_p(w1.y), uc.w, pc);
+          pc = fmaf(bf16_lo_p(w1.z), ud.x, pc);
+          pc = fmaf(bf16_hi_p(w1.z), ud.y, pc);
+          pc = fmaf(bf16_lo_p(w1.w), ud.z, pc);
+          pc = fmaf(bf16_hi_p(w1.w), ud.w, pc);
+          acc[i] = __fadd_rn(acc[i], pc);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kCandBatch; ++i) {
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) acc[i] = __fadd_rn(acc[i], __shfl_xor_sync(0xffffffffu, acc[i], off));
+    }
+#pragma unroll
+    for (int i = 0; i < kCandBatch; ++i)
+      if (lane == i && i0 + i < nc) {
+        const int e = (int)cand[i0 + i];
+        zx[e] = fmaf(acc[i], inv, p.bias ? __ldg(p.bias + (size_t)l * p.E + e) : 0.0f);
+      }
+  }
+}
+
+// Order key of a logit: larger first, equal -> lower expert index, -0 == +0, NaN last.
+__device__ __forceinline__ uint64_t logit_key(float v, int e) {
+  if (v == 0.0f) v = 0.0f;
+  const uint32_t uu = __float_as_uint(v);
+  uint32_t o = (uu & 0x80000000u) ? ~uu : (uu | 0x80000000u);
+  if (v != v) o = 0;
+  return ((uint64_t)o << 32) | (uint32_t)(~(uint32_t)e);
+}
+__device__ __forceinline__ uint64_t warp_max_key(uint64_t k) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)k, off);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(k >> 32), off);
+    const uint64_t o = ((uint64_t)hi << 32) | lo;
+    k = o > k ? o : k;
+  }
+  return k;
+}
+
+// Warp per token: approximate logits, exact candidates, certified top-k, weights, counts.
+// Shared memory per warp: approximate logits [E], exact logits [E], candidate list [E],
+// flags [E] (1 = candidate, 2 = selected).
+__global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams p, int l, int nsplit) {
+  extern __shared__ __align__(16) float ssm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * (kPT / 32) + warp;
+  if (t >= p.T) return;
+  const int E = p.E, K = p.K;
+  float* za = ssm + (size_t)warp * 3 * E;
+  float* zx = za + E;
+  uint32_t* cand = reinterpret_cast<uint32_t*>(zx + E);
+  uint8_t* flag = reinterpret_cast<uint8_t*>(ssm + (size_t)(kPT / 32) * 3 * E) + (size_t)warp * E;
+  const float inv = p.s.inv[t];
+  const float* urow = p.s.u + (size_t)t * p.H;
+  for (int e = lane; e < E; e += 32) {
+    float S = 0.0f;
+    for (int sp = 0; sp < nsplit; ++sp) S += p.s.part[((size_t)sp * p.T + t) * E + e];
+    za[e] = fmaf(S, inv, p.bias ? __ldg(p.bias + (size_t)l * E + e) : 0.0f);
+    flag[e] = 0;
+  }
+  __syncwarp();
+  const float delta = 0x1p-9f * p.s.unorm[t] * p.wnorm[l] * inv * 1.001f + 1e-30f;
+  // best approximate logit among experts that are not candidates yet
+  auto best_left = [&]() {
+    uint64_t best = 0;
+    for (int e = lane; e < E; e += 32)
+      if (flag[e] == 0) {
+        const uint64_t k = logit_key(za[e], e);
+        best = k > best ? k : best;
+      }
+    return warp_max_key(best);
+  };
+  int have = 0;
+  int sel_e = -1;
+  float sel_z = 0.0f;
+  const int want0 = kCand > K ? kCand : K;
+  for (int want = want0 < E ? want0 : E;; want = want * 4 < E ? want * 4 : E) {
+    const int first = have;
+    for (; have < want; ++have) {  // the next best approximate logits become candidates
+      const int e = (int)(~(uint32_t)best_left());
+      if (lane == 0) {
+        flag[e] = 1;
+        cand[have] = (uint32_t)e;
+      }
+      __syncwarp();
+    }
+    canonical_logits(p, l, urow, cand + first, have - first, inv, zx, lane);
+    __syncwarp();
+    const float thr = want < E ? za[(int)(~(uint32_t)best_left())] : -INFINITY;
+    // top-k of the candidates by exact logit; lane r keeps rank r
+    float zk = 0.0f;
+    for (int r = 0; r < K; ++r) {
+      uint64_t best = 0;
+      for (int i = lane; i < have; i += 32) {
+        const int e = (int)cand[i];
+        if (flag[e] == 1) {
+          const uint64_t k = logit_key(zx[e], e);
+          best = k > best ? k : best;
+        }
+      }
+      best = warp_max_key(best);
+      const int e = (int)(~(uint32_t)best);
+      if (lane == r) {
+        sel_e = e;
+        sel_z = zx[e];
+      }
+      zk = zx[e];
+      __syncwarp();
+      if (lane == 0) flag[e] = 2;
+      __syncwarp();
+    }
+    if (want >= E || (zk == zk && zk > thr + delta)) break;
+    for (int i = lane; i < have; i += 32)  // not certified: widen, ranks open again
+      if (flag[cand[i]] == 2) flag[cand[i]] = 1;
+    __syncwarp();
+  }
+  if ((logit_key(__shfl_sync(0xffffffffu, sel_z, 0), 0) >> 32) == 0 && lane == 0)
+    atomicCAS(p.s.error, 0, MOE_DEVERR_ROUTE);  // a NaN logit won
+  const float zmax = __shfl_sync(0xffffffffu, sel_z, 0);
+  const float ex = lane < K ? expf(sel_z - zmax) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < K) {
+    p.s.sel[(size_t)t * K + lane] = sel_e;
+    p.s.w[(size_t)t * K + lane] = __fdividef(ex, sum);
+    atomicAdd(p.hist + (size_t)l * E + sel_e, 1u);
+    atomicAdd(p.s.counts + sel_e, 1);
+    if (p.s.sel_trace) p.s.sel_trace[((size_t)l * p.T_total + p.t_base + t) * K + lane] = sel_e;
+  }
+}
+
 // ------------------------------------------------------------------ combine
 
 // h[t] += sum_rank w * o_rank + o_shared in rank order (without the norm: h = that sum).
@@ -936,22 +1053,31 @@ static uint32_t gemm_smem() {
   return kTilesBytes + kRawRing + kTileCap * sizeof(GemmTile) + (3 * kStages + 4 + 2 * kRawStages) * 8 + 16 + 1024;
 }
 static int gemm_grid(int max_tiles, int n_sm) { return max_tiles < n_sm ? max_tiles : n_sm; }
-static size_t route_floats(int tpc, int H, int E) { return (size_t)tpc * ((size_t)H / kChunk * kUChunk + E) + 16; }
-static int route_tpc(int, int) { return 2 * kRTok; }  // small enough for two CTAs per SM at hidden 2048
-static uint32_t route_smem(int H, int E) { return (uint32_t)(route_floats(route_tpc(H, E), H, E) * 4); }
+
+static int router_n(int E) { return E <= 256 ? E : 256; }
+static uint32_t router_gemm_smem(int E) {
+  const uint32_t b = ((uint32_t)router_n(E) * kTK * 2 + 1023) & ~1023u;
+  return kRStages * (kTM * kTK * 2 + b) + (2 * kRStages + 1) * 8 + 16 + 1024;
+}
+static uint32_t route_select_smem(int E) { return (uint32_t)(kPT / 32) * 13u * E; }
 
 int prefill_supported(int H, int E, int K, int I, int Is) {
+  if (E % 16) return 0;  // router GEMM: N = E (or 256) is a multiple of 16
   // 256-wide tiles; scale rows (K / 16 bytes) must be TMA strides, multiples of 16 bytes
   if (H % kTN || H > kMaxH || I % 256 || Is % 256 || E > kMaxE || K > 32) return 0;
-  return route_smem(H, E) <= 227 * 1024;
+  return route_select_smem(E) <= 227 * 1024 && router_gemm_smem(E) <= 227 * 1024;
 }
 
-cudaError_t prefill_configure(int H, int E) {
+cudaError_t prefill_configure(int, int E) {
   cudaError_t e = cudaFuncSetAttribute(prefill_gemm<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(prefill_gemm<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem());
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_route, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_smem(H, E));
+    e = cudaFuncSetAttribute(prefill_router_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)router_gemm_smem(E));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_route_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)route_select_smem(E));
   return e;
 }
 
@@ -959,14 +1085,15 @@ typedef CUresult (*PfnEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// Row-major fp16 [rows x cols] -> tensor map of 64-column x 128-row boxes, 128-byte swizzle.
-static int make_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+// Row-major 16-bit [rows x cols] -> tensor map of 64-column x box_rows boxes, 128-byte swizzle.
+static int make_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_FLOAT16, uint32_t box_rows = kTM) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kTK, (cuuint32_t)kTM};
+  const cuuint32_t box[2] = {(cuuint32_t)kTK, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  const CUresult r = enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -1;
 }
@@ -1050,7 +1177,6 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.T_total = T;
     p.eps = a.eps;
     p.nch = H / kChunk;
-    p.tpc = route_tpc(H, E);
     p.pool = a.pool;
     p.slot_bytes = a.slot_bytes;
     p.lay = a.lay;
@@ -1063,6 +1189,7 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.pin_slot = a.pin_slot;
     p.layer_base = a.layer_base;
     p.hist = a.hist;
+    p.wnorm = a.wnorm;
     p.s = s;
     p.s.h = s.h + (size_t)t0 * H;
     p.s.y = s.y + (size_t)t0 * H;
@@ -1089,8 +1216,18 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     const int max_jobs = (R + kTM - 1) / kTM + E + 1;
     cudaError_t e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * E, st);
     if (e != cudaSuccess) return (int)e;
+    CUtensorMap mua;
+    if (make_map(enc, &mua, s.ua, Tc, (uint64_t)kRParts * H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) return -1;
+    const int rn = router_n(E), total_k = kRParts * H / kTK;
+    const int nsplit = kRSplit < total_k ? kRSplit : total_k;
+    const int kps = (total_k + nsplit - 1) / nsplit;
+    const dim3 rgrid((Tc + kTM - 1) / kTM, (E + rn - 1) / rn, nsplit);
     for (int l = 0; l < a.L; ++l) {
-      prefill_route<<<(Tc + p.tpc - 1) / p.tpc, kPT, route_smem(H, E), st>>>(p, l);
+      CUtensorMap mw;
+      if (make_map(enc, &mw, a.router_rows + (size_t)l * E * H, E, H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rn)) return -1;
+      prefill_route_prep<<<(Tc + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p, l);
+      prefill_router_gemm<<<rgrid, kRGT, router_gemm_smem(E), st>>>(p, mua, mw, rn, kps);
+      prefill_route_select<<<(Tc + kPT / 32 - 1) / (kPT / 32), kPT, route_select_smem(E), st>>>(p, l, nsplit);
       prefill_scan<<<1, 1024, 0, st>>>(p);
       prefill_scatter<<<(Tc + kPT / 32 - 1) / (kPT / 32), kPT, 0, st>>>(p);
       prefill_gemm<0><<<gemm_grid(max_jobs * ((2 * imax) / kTN), a.n_sm), kGT, gemm_smem(), st>>>(p, l, m0);

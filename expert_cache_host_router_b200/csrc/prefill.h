@@ -1,6 +1,7 @@
 // prefill.h -- host-side interface of the batched prefill kernels (prefill.cu) for the
 // runtime (moe_api.cu).  Plain structs of device pointers and sizes.
 #pragma once
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -26,6 +27,8 @@ struct PrefillArgs {
   const int32_t* pin_slot;    // [L][E], every entry valid
   const int32_t* layer_base;  // [L]
   uint32_t* hist;             // [L][E] routing histogram, accumulated
+  const uint16_t* router_rows;  // [L][E][H] bf16, the router in plain row order
+  const float* wnorm;           // [L] max_e ||w_e||_2, rounded up
 };
 
 // Per-call device buffers for T tokens (R = T * K + T rows when there is a shared
@@ -36,6 +39,11 @@ struct PrefillScratch {
   float* h_trace;    // [(L+1)][T][H] or null
   int32_t* sel_trace;  // [L][T][K] or null
   int32_t* sel;      // [T][K]
+  float* u;          // [T][H] router input u = g * h (or h)
+  __nv_bfloat16* ua; // [T][3H] u split into three bf16 parts
+  float* inv;        // [T] RMSNorm scale
+  float* unorm;      // [T] ||u||_2, rounded up
+  float* part;       // [8][T][E] router partial sums per K split
   float* w;          // [T][K]
   __half *x_hi, *x_lo;    // [T][H]
   __half *xg_hi, *xg_lo;  // [R][H]
