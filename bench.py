@@ -327,6 +327,13 @@ def run_ours(args):
         m.load_layer(l, layers[l])
     load_s = time.time() - t0
 
+    if args.only_prefill:  # the batched-prefill measurement alone (profiling runs)
+        line = {"metric": "prefill tok/s", "config": {"workload": f"batched prefill, {shape.n_layers}-layer stack"},
+                "prefill": run_prefill(m, shape, dev, runs=args.prefill_runs)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        m.close()
+        return
     stream = torch.cuda.current_stream(dev)
     n_tok = args.warmup + args.steps
     xs = torch.from_numpy(synthetic.tokens(0, n_tok, shape.hidden)).to(dev)
@@ -455,7 +462,7 @@ def run_ours(args):
         "setup": {"generate_s": gen_s, "load_s": load_s, "phases": args.phases},
     }
     if args.phases == "all" and not args.no_prefill:
-        line["prefill"] = run_prefill(m, shape, dev)
+        line["prefill"] = run_prefill(m, shape, dev, runs=args.prefill_runs)
     m.close()
     del m
     if args.phases == "all" and not args.no_drift:
@@ -483,6 +490,8 @@ def main():
     ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
     ap.add_argument("--no-drift", action="store_true", help="skip the recalibration-under-drift run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the batched-prefill run")
+    ap.add_argument("--only-prefill", action="store_true", help="run only the batched-prefill measurement")
+    ap.add_argument("--prefill-runs", type=int, default=5, help="timed prefill passes")
     ap.add_argument("--phases", default="all", choices=["all", "100"],
                     help="'100' times full residency only (no miss copies), for profiler runs")
     args = ap.parse_args()
