@@ -145,32 +145,50 @@ __global__ void __launch_bounds__(1024) prefill_scan(const PrefillParams p) {
 }
 
 // One warp per token: each of its k routed rows (and its shared-expert row) takes a
-// place in its expert's group, and the token's x row (hi and lo) is copied there.
+// place in its expert's group, and the token's x row (hi and lo) is copied there; each
+// 2048-column piece of the row is read once and stored k + 1 times.
+constexpr int kScatterRegs = 8;  // 16-byte pieces per lane and array: 2048 columns per pass
 __global__ void __launch_bounds__(kPT) prefill_scatter(const PrefillParams p) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (kPT / 32) + (threadIdx.x >> 5);
   if (t >= p.T) return;
   const int nr = p.K + (p.Is > 0 ? 1 : 0);
-  const int vec = p.H / 8;
-  const uint4* src_hi = reinterpret_cast<const uint4*>(p.s.x_hi + (size_t)t * p.H);
-  const uint4* src_lo = reinterpret_cast<const uint4*>(p.s.x_lo + (size_t)t * p.H);
-  for (int r = 0; r < nr; ++r) {
-    int pos = 0;
-    if (lane == 0) {
+  int32_t* gp = p.s.gpos + (size_t)t * (p.K + 1);
+  if (lane == 0)
+    for (int r = 0; r < nr; ++r) {
       if (r < p.K) {
         const int e = p.s.sel[(size_t)t * p.K + r];
-        pos = p.s.offsets[e] + atomicAdd(p.s.cursor + e, 1);
+        gp[r] = p.s.offsets[e] + atomicAdd(p.s.cursor + e, 1);
       } else {
-        pos = p.s.offsets[p.E] + t;
+        gp[r] = p.s.offsets[p.E] + t;
       }
-      p.s.gpos[(size_t)t * (p.K + 1) + r] = pos;
     }
-    pos = __shfl_sync(0xffffffffu, pos, 0);
-    uint4* dh = reinterpret_cast<uint4*>(p.s.xg_hi + (size_t)pos * p.H);
-    uint4* dl = reinterpret_cast<uint4*>(p.s.xg_lo + (size_t)pos * p.H);
-    for (int c = lane; c < vec; c += 32) {
-      dh[c] = src_hi[c];
-      dl[c] = src_lo[c];
+  __syncwarp();
+  const int vec = p.H / 8;  // 16-byte pieces per row
+  const uint4* src_hi = reinterpret_cast<const uint4*>(p.s.x_hi + (size_t)t * p.H);
+  const uint4* src_lo = reinterpret_cast<const uint4*>(p.s.x_lo + (size_t)t * p.H);
+  for (int base = 0; base < vec; base += 32 * kScatterRegs) {
+    uint4 rh[kScatterRegs], rl[kScatterRegs];
+#pragma unroll
+    for (int i = 0; i < kScatterRegs; ++i) {
+      const int c = base + lane + 32 * i;
+      if (c < vec) {
+        rh[i] = src_hi[c];
+        rl[i] = src_lo[c];
+      }
+    }
+    for (int r = 0; r < nr; ++r) {
+      const size_t pos = (size_t)gp[r];
+      uint4* dh = reinterpret_cast<uint4*>(p.s.xg_hi + pos * p.H);
+      uint4* dl = reinterpret_cast<uint4*>(p.s.xg_lo + pos * p.H);
+#pragma unroll
+      for (int i = 0; i < kScatterRegs; ++i) {
+        const int c = base + lane + 32 * i;
+        if (c < vec) {
+          dh[c] = rh[i];
+          dl[c] = rl[i];
+        }
+      }
     }
   }
 }
@@ -815,9 +833,17 @@ __global__ void __launch_bounds__(kRGT, 1)
         tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c0, o);
         tmem_wait16(o);
         if (t < p.T) {
+          if (n0 + c0 + 16 <= p.E) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (n0 + c0 + j < p.E) dst[c0 + j] = __uint_as_float(o[j]);
+            for (int j = 0; j < 4; ++j)
+              d4[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
+                                  __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (n0 + c0 + j < p.E) dst[c0 + j] = __uint_as_float(o[j]);
+          }
         }
       }
     }
@@ -920,8 +946,12 @@ __global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams 
   const float inv = p.s.inv[t];
   const float* urow = p.s.u + (size_t)t * p.H;
   for (int e = lane; e < E; e += 32) {
+    float v[kRSplit];  // the split partials are independent loads, summed in split order
+#pragma unroll
+    for (int sp = 0; sp < kRSplit; ++sp) v[sp] = sp < nsplit ? p.s.part[((size_t)sp * p.T + t) * E + e] : 0.0f;
     float S = 0.0f;
-    for (int sp = 0; sp < nsplit; ++sp) S += p.s.part[((size_t)sp * p.T + t) * E + e];
+#pragma unroll
+    for (int sp = 0; sp < kRSplit; ++sp) S += v[sp];
     za[e] = fmaf(S, inv, p.bias ? __ldg(p.bias + (size_t)l * E + e) : 0.0f);
     flag[e] = 0;
   }
