@@ -33,9 +33,9 @@ METRIC = "MoE decode tok/s at 100%/60% expert residency; fraction of HBM/PCIe ro
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_TFLOPS = 1400.0  # sustained dense bf16, an earlier measurement on this machine
 # DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
-# 4-layer case scaled by 10 (profiles/moe_decode_kernel_4layer_ncu.md), valid only for
-# the kernel source it was taken on; any other source reports null.
-TRAFFIC_REF = {"kernel_sha256_prefix": "2b7e9969101cd83f", "bytes_per_launch": 712.46592e6}
+# 4-layer case scaled by 10, valid only for the kernel source it was taken on; any other
+# source reports null.
+TRAFFIC_REF = {"kernel_sha256_prefix": "710db75c13ec8306", "bytes_per_launch": 714.08128e6}
 WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
             "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
             "residency + 8-slot LRU ring (residency_60)")
