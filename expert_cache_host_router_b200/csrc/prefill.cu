@@ -65,6 +65,7 @@ struct PrefillParams {
   const int32_t* layer_base;
   uint32_t* hist;
   const float* wnorm;  // [L] max_e ||w_e||_2 of the router rows, rounded up
+  const uint16_t* router_rows;  // [L][E][H] bf16
   PrefillScratch s;
 };
 
@@ -874,7 +875,8 @@ __device__ __forceinline__ void canonical_logits(const PrefillParams& p, int l, 
       for (int i = 0; i < kCandBatch; ++i) {
         if (i0 + i < nc) {
           const int e = (int)cand[i0 + i];
-          const uint4* wp = reinterpret_cast<const uint4*>(p.router + (((size_t)l * p.nch + c) * p.E + e) * kChunk);
+          // plain-row copy: a warp's 32 chunks of one expert are 1 KB in a row
+          const uint4* wp = reinterpret_cast<const uint4*>(p.router_rows + ((size_t)l * p.E + e) * p.H + c * kChunk);
           const uint4 w0 = __ldg(wp), w1 = __ldg(wp + 1);
           float pc = 0.0f;
           pc = fmaf(bf16_lo_p(w0.x), ua.x, pc);
@@ -1220,6 +1222,7 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.layer_base = a.layer_base;
     p.hist = a.hist;
     p.wnorm = a.wnorm;
+    p.router_rows = a.router_rows;
     p.s = s;
     p.s.h = s.h + (size_t)t0 * H;
     p.s.y = s.y + (size_t)t0 * H;
