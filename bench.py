@@ -248,6 +248,75 @@ def run_drift(args, shape, layers, local, dev, xs_steps=1024, switch=512, every=
     return out
 
 
+def decode_point(m, shape, xs, y, stream, steps):
+    """Decode `steps` tokens of xs on m as placed now: tok/s (CUDA events), cold-hit rate
+    and miss copies per token from the run's own log."""
+    import torch
+    m.stats(reset=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        m.decode(xs[i], y)
+    e1.record(stream)
+    m.sync()
+    st, _, _ = m.stats(reset=True)
+    acc = max(st["accesses"], 1)
+    return {"tok_s": steps / (e0.elapsed_time(e1) * 1e-3),
+            "cold_hit_rate": (st["ring_hits"] + st["misses"]) / acc,
+            "misses_per_token": st["misses"] / steps}
+
+
+def run_residency_curve(m, shape, hist, xs, y, stream, steps=128):
+    """tok/s and cold-hit rate over residency 1.0, 0.8, 0.6, 0.4 for calibrated placement
+    (pinned = top-P of the calibration histogram) and uniform placement (experts 0..P-1):
+    the offload comparison the write-up makes at one point, as a curve."""
+    import expert_cache_host_router_b200 as moe
+    out = []
+    for rho in (1.0, 0.8, 0.6, 0.4):
+        for name, place in (("calibrated", moe.MOE_PLACE_CALIBRATED), ("uniform", moe.MOE_PLACE_UNIFORM)):
+            if rho == 1.0 and place == moe.MOE_PLACE_UNIFORM:
+                continue  # every expert pinned: the same placement
+            m.set_residency(rho, hist, place)
+            out.append({"residency": rho, "placement": name, **decode_point(m, shape, xs, y, stream, steps)})
+    return out
+
+
+def run_small_stack(dev, local, calib_steps, steps=256, warmup=8):
+    """The 40-layer stack at the small layer shape (hidden 512, 64 experts, top-4, SwiGLU
+    256, no shared expert) at 100% and at 60% residency (calibrated and uniform), 8-slot
+    rings."""
+    import dataclasses
+
+    import torch
+
+    import expert_cache_host_router_b200 as moe
+    s = dataclasses.replace(synthetic.SMALL, n_layers=40, use_rmsnorm=1, ring_slots=8, zipf_s=1.0)
+    m = moe.ExpertCacheMoE(s, device=local, log_steps=max(4096, steps + warmup + 16))
+    for l in range(s.n_layers):
+        m.load_layer(l, synthetic.layer_weights(l, s))
+    y = torch.empty(s.hidden, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    m.set_residency(1.0)
+    calib = torch.from_numpy(synthetic.tokens(0, calib_steps, s.hidden, synthetic.SEED_CALIB)).to(dev)
+    for i in range(calib_steps):
+        m.decode(calib[i], y)
+    m.sync()
+    _, hist, _ = m.stats(reset=True)
+    xs = torch.from_numpy(synthetic.tokens(0, warmup + steps, s.hidden)).to(dev)
+    out = {"shape": {"layers": 40, "hidden": 512, "experts": 64, "top_k": 4, "inter": 256, "shared_inter": 0,
+                     "ring_slots": 8},
+           "active_bytes_per_token": active_bytes_per_token(s)}
+    for name, rho, place in (("100", 1.0, moe.MOE_PLACE_CALIBRATED), ("60_calibrated", 0.6, moe.MOE_PLACE_CALIBRATED),
+                             ("60_uniform", 0.6, moe.MOE_PLACE_UNIFORM)):
+        m.set_residency(rho, hist, place)
+        for i in range(warmup):
+            m.decode(xs[i], y)
+        m.sync()
+        out[name] = decode_point(m, s, xs[warmup:], y, stream, steps)
+    m.close()
+    return out
+
+
 def run_prefill(m, shape, dev, n_tokens=2048, warmup=2, runs=5):
     """Batched prefill of n_tokens through the whole stack at full residency (tcgen05
     grouped GEMM path), timed with CUDA events on the launching stream.  Roofline: per
@@ -461,12 +530,16 @@ def run_ours(args):
         "clocks": clk.summary(),
         "setup": {"generate_s": gen_s, "load_s": load_s, "phases": args.phases},
     }
+    if args.phases == "all" and not args.no_curve:
+        line["residency_curve"] = run_residency_curve(m, shape, hist, xs, y, stream, steps=min(128, len(xs)))
     if args.phases == "all" and not args.no_prefill:
         line["prefill"] = run_prefill(m, shape, dev, runs=args.prefill_runs)
     m.close()
     del m
     if args.phases == "all" and not args.no_drift:
         line["drift"] = run_drift(args, shape, layers, local, dev, xs_steps=1024)
+    if args.phases == "all" and not args.no_curve:
+        line["small_stack"] = run_small_stack(dev, local, args.calib_steps)
     if keep_layers:
         tps, dt, cores = oracle_tokens_per_s(shape, shape.n_layers, args.cpu_tokens, layers=layers)
         line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": cores, "kind": "oracle",
@@ -491,6 +564,8 @@ def main():
     ap.add_argument("--no-drift", action="store_true", help="skip the recalibration-under-drift run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the batched-prefill run")
     ap.add_argument("--only-prefill", action="store_true", help="run only the batched-prefill measurement")
+    ap.add_argument("--no-curve", action="store_true",
+                    help="skip the residency curve and the small-shape stack")
     ap.add_argument("--prefill-runs", type=int, default=5, help="timed prefill passes")
     ap.add_argument("--phases", default="all", choices=["all", "100"],
                     help="'100' times full residency only (no miss copies), for profiler runs")
