@@ -1,7 +1,7 @@
 // prefill.cu -- batched prefill of T tokens through the MoE stack (every expert resident)
-// for libmoe: routing for every token in the same canonical fp32 order as decode, tokens
+// for libmoe: each token's top-k in the same canonical fp32 order as decode, tokens
 // grouped by expert, and the expert FFNs as a grouped GEMM on the 5th-generation tensor
-// cores (tcgen05, accumulators in tensor memory, activation tiles brought in by TMA).
+// cores (tcgen05, accumulators in tensor memory, operands brought in by TMA).
 //
 // The write-up serves decode; a prompt's tokens all pass the same layers at once, which
 // turns each expert's GEMVs into GEMMs [n_e x H] x [H x 2I] and [n_e x I] x [I x H]
@@ -9,18 +9,19 @@
 // cores.  Per layer, in stream order:
 //   route    RMSNorm scale and x = RMSNorm(h) split into fp16 hi + lo (x = hi + lo to
 //            about 2^-22 relative); router logits approximated on the tensor cores, the
-//            top-k certified with exact canonical-order logits of the candidates (below);
-//            weights, histogram, per-expert counts
+//            top-k certified with exact canonical-order logits of the candidates (see the
+//            certified-router section); weights, histogram, per-expert counts
 //   scan     expert offsets and the list of 128-row m-tiles
 //   scatter  one warp per token: its rows of x copied to their place in expert order
 //            (within an expert the order is whatever the atomics give: a GEMM row does
 //            not depend on the other rows of its tile, so results are deterministic)
-//   gemm     one CTA per 128 x 128 output tile: A (activation rows, fp16 hi and lo) by
-//            TMA, B (Q4_0 weights) dequantised to fp16 into 128B-swizzled shared memory,
-//            two tcgen05.mma per 16-wide K step (A_hi B and A_lo B) into one fp32
-//            accumulator in tensor memory; gate/up tiles hold 64 gate and the matching
-//            64 up columns so the epilogue forms a = silu(g) * u (stored as fp16 hi + lo);
-//            down tiles write each row's expert output to its (token, rank) slot
+//   gemm     persistent, one CTA per SM, 128 x 256 output tiles: A (activation rows, fp16
+//            hi and lo) and the raw Q4_0 weight bytes by TMA, the weights dequantised to
+//            fp16 into 128B-swizzled shared memory, two tcgen05.mma per 16-wide K step
+//            (A_hi B and A_lo B) into one fp32 accumulator in tensor memory; gate/up tiles
+//            hold 128 gate and the matching 128 up columns so the epilogue forms
+//            a = silu(g) * u (stored as fp16 hi + lo); down tiles write fp32 outputs
+//            column-block-major over grouped rows
 //   combine  h += sum_rank w * o_rank + o_shared in rank order
 // The activations are split because fp16 operands alone put the element-wise error at
 // the tolerance; the weights are fp16((q - 8) * d), a relative error of at most 2^-12.

@@ -178,17 +178,20 @@ MOE_API int moe_decode_step_host(moe_ctx *ctx, const float *x_host, float *y_hos
 /* Batched prefill: n_tokens tokens through the whole stack at once, x_dev [T][H] ->
  * y_dev [T][H] (fp32, device, caller-owned, may not overlap), enqueued on stream.
  * The pages describe decode; this is the same layer computed for a batch: per layer,
- * each token's routing (logits in the same canonical fp32 order as decode, so the
- * top-k choices agree with a decode of the same hidden state; the routing histogram
- * accumulates as in decode), tokens grouped by expert, the expert SwiGLU FFNs as
- * grouped tensor-core GEMMs (Q4_0 weights dequantised to fp16, activations carried as
- * fp16 hi + lo pairs, fp32 accumulation), and the weighted combine plus shared expert.
- * Needs every expert resident (moe_set_residency(1.0)): else MOE_ERR_STATE.  Shapes
- * need hidden % 128 == 0 and inter, shared_inter % 64 == 0: else MOE_ERR_UNSUPPORTED.
- * Scratch for the largest n_tokens seen so far is kept by the context (about
- * T * (k + 1) * hidden * 10 bytes); a larger n_tokens reallocates it, synchronising the
- * device.  The cache's rings, counters and event log are not touched.  Errors of the
- * kernels' bounded waits surface at moe_sync as MOE_ERR_TIMEOUT. */
+ * each token's top-k is the one the canonical fp32 logits give, as in decode (found
+ * from tensor-core approximate logits, certified against exact canonical logits of the
+ * candidates), so it agrees with a decode of the same hidden state; the routing
+ * histogram accumulates as in decode), tokens grouped by expert, the expert SwiGLU FFNs
+ * as grouped tensor-core GEMMs (Q4_0 weights dequantised to fp16, activations carried
+ * as fp16 hi + lo pairs, fp32 accumulation), and the weighted combine plus shared
+ * expert.  Needs every expert resident (moe_set_residency(1.0)): else MOE_ERR_STATE.
+ * Shapes need experts % 16 == 0, hidden % 256 == 0 and inter, shared_inter % 256 == 0:
+ * else MOE_ERR_UNSUPPORTED.  Scratch for the largest n_tokens seen so far is kept by
+ * the context (about T * ((k + 1) * (8 * hidden + 4 * max(inter, shared_inter)) +
+ * 18 * hidden + 32 * experts) bytes: 430 MB for 2048 tokens of the 2048-hidden,
+ * 256-expert, top-8 shape); a larger n_tokens reallocates it, synchronising the device.
+ * The cache's rings, counters and event log are not touched.  Errors of the kernels'
+ * bounded waits surface at moe_sync as MOE_ERR_TIMEOUT. */
 MOE_API int moe_prefill(moe_ctx *ctx, const float *x_dev, int32_t n_tokens, float *y_dev, void *stream);
 
 /* Prefill tracing: when non-NULL, moe_prefill writes its input and every layer's output

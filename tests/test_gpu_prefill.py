@@ -161,3 +161,22 @@ def test_prefill_needs_full_residency_and_supported_shape():
         m2.prefill(torch.zeros((2, s2.hidden), dtype=torch.float32, device=DEV))
     assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
     m2.close()
+
+
+@pytest.mark.parametrize("shape", [
+    # two router tiles of 256 experts; shared expert as wide as the routed ones
+    synthetic.Shape(n_layers=1, hidden=512, n_experts=512, top_k=8, inter=256, shared_inter=256,
+                    use_rmsnorm=1, zipf_s=1.0),
+    # hidden 256: fold lanes 16..31 hold no chunk; top-1 routing; 32 experts (N = 32 router tile)
+    synthetic.Shape(n_layers=2, hidden=256, n_experts=32, top_k=1, inter=256, shared_inter=0,
+                    use_rmsnorm=1, zipf_s=0.5),
+])
+def test_prefill_other_shapes(shape):
+    layers = make_layers(shape, gain_kind="random")
+    m = build_gpu(shape, layers)
+    m.set_residency(1.0)
+    xs = synthetic.tokens(3, 200, shape.hidden)
+    y, hs, sels = _prefill(m, xs, trace=True)
+    assert np.array_equal(y, hs[-1])
+    _check_layers(shape, layers, xs, hs, sels, sample=[0, 1, 99, 130, 199])
+    m.close()
