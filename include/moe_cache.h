@@ -191,7 +191,9 @@ MOE_API int moe_decode_step_host(moe_ctx *ctx, const float *x_host, float *y_hos
  * 18 * hidden + 32 * experts) bytes: 430 MB for 2048 tokens of the 2048-hidden,
  * 256-expert, top-8 shape); a larger n_tokens reallocates it, synchronising the device.
  * The cache's rings, counters and event log are not touched.  Errors of the kernels'
- * bounded waits surface at moe_sync as MOE_ERR_TIMEOUT. */
+ * bounded waits surface at moe_sync as MOE_ERR_TIMEOUT.  Prefill calls on one context
+ * share its scratch: calls that overlap on the GPU (different streams, no ordering)
+ * race on it. */
 MOE_API int moe_prefill(moe_ctx *ctx, const float *x_dev, int32_t n_tokens, float *y_dev, void *stream);
 
 /* Prefill tracing: when non-NULL, moe_prefill writes its input and every layer's output
