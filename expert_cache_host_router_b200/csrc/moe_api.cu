@@ -104,6 +104,15 @@ struct moe_ctx {
   void* encode_tiled = nullptr;
   float* pf_h_trace = nullptr;
   int32_t* pf_sel_trace = nullptr;
+  // the captured prefill pass and what it was captured for
+  cudaGraphExec_t g_pf = nullptr;
+  const float* gpf_x = nullptr;
+  float* gpf_y = nullptr;
+  int gpf_T = 0;
+  float* gpf_ht = nullptr;
+  int32_t* gpf_st = nullptr;
+  const uint8_t* gpf_pool = nullptr;
+  const uint8_t* gpf_mem = nullptr;
 };
 
 #define CK(call)                                  \
@@ -219,7 +228,8 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
 static void drop_graphs(moe_ctx* c) {
   if (c->g_dev) cudaGraphExecDestroy(c->g_dev);
   if (c->g_host) cudaGraphExecDestroy(c->g_host);
-  c->g_dev = c->g_host = nullptr;
+  if (c->g_pf) cudaGraphExecDestroy(c->g_pf);
+  c->g_dev = c->g_host = c->g_pf = nullptr;
   c->g_x = nullptr;
   c->g_y = nullptr;
 }
@@ -699,12 +709,20 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   const int st = prefill_reserve(c, n_tokens);
   if (st != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
+  // one captured graph per pass (x copy-in, then every layer's launches), replayed while
+  // the tokens, buffers, trace and slot pool stay the same
+  if (c->g_pf && c->gpf_x == x_dev && c->gpf_y == y_dev && c->gpf_T == n_tokens && c->gpf_ht == c->pf_h_trace &&
+      c->gpf_st == c->pf_sel_trace && c->gpf_pool == c->pool.load() && c->gpf_mem == c->prefill_mem) {
+    CK(cudaGraphLaunch(c->g_pf, s));
+    return MOE_OK;
+  }
+  if (c->g_pf) cudaGraphExecDestroy(c->g_pf);
+  c->g_pf = nullptr;
   PrefillScratch sc = c->pf;
   sc.y = y_dev;
   sc.h_trace = c->pf_h_trace;
   sc.sel_trace = c->pf_sel_trace;
   sc.error = &c->ctrl->error;
-  CK(cudaMemcpyAsync(sc.h, x_dev, sizeof(float) * n_tokens * c->H, cudaMemcpyDeviceToDevice, s));
   PrefillArgs a{};
   a.L = c->L;
   a.H = c->H;
@@ -731,9 +749,30 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   a.hist = c->hist;
   a.router_rows = c->router_rows;
   a.wnorm = c->wnorm;
-  const int r = prefill_run(a, sc, c->encode_tiled, s);
-  if (r == -1) return MOE_ERR_UNSUPPORTED;
-  if (r != 0) return cuda_fail((cudaError_t)r);
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = cudaMemcpyAsync(sc.h, x_dev, sizeof(float) * n_tokens * c->H, cudaMemcpyDeviceToDevice, c->own);
+  const int r = e == cudaSuccess ? prefill_run(a, sc, c->encode_tiled, c->own) : (int)e;
+  const cudaError_t e2 = cudaStreamEndCapture(c->own, &graph);
+  if (r != 0 || e2 != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    if (r == -1) return MOE_ERR_UNSUPPORTED;
+    return cuda_fail(r != 0 ? (cudaError_t)r : e2);
+  }
+  e = cudaGraphInstantiate(&c->g_pf, graph, 0);
+  cudaGraphDestroy(graph);
+  if (e != cudaSuccess) {
+    c->g_pf = nullptr;
+    return cuda_fail(e);
+  }
+  c->gpf_x = x_dev;
+  c->gpf_y = y_dev;
+  c->gpf_T = n_tokens;
+  c->gpf_ht = c->pf_h_trace;
+  c->gpf_st = c->pf_sel_trace;
+  c->gpf_pool = c->pool.load();
+  c->gpf_mem = c->prefill_mem;
+  CK(cudaGraphLaunch(c->g_pf, s));
   return MOE_OK;
 }
 
