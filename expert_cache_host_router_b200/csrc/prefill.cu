@@ -658,16 +658,15 @@ __global__ void __launch_bounds__(kGT, 1)
 //           inv, ||u||_2 and x hi/lo
 //   gemm    approximate S~ = sum_p u_p . w_e on the tensor cores (bf16 x bf16, products exact
 //           in fp32, fp32 accumulation), split over K, partials summed in a fixed order
-//   select  per token: the kCand best approximate logits are evaluated exactly in the
-//           canonical order; the top-k among them is final once the k-th exact logit beats
-//           the best approximate logit left out by more than twice the error bound
-//           delta = 2^-9 * ||u|| * max_e ||w_e|| * inv  (the accumulation error of S~ is at
-//           most 2^-10 * sum_j |w_j u_j| <= 2^-10 ||u|| ||w_e||, Cauchy-Schwarz); otherwise
-//           the candidate set widens (64, then every expert).
+//   select  per token: with delta = 2^-9 * ||u|| * max_e ||w_e|| * inv, twice a bound on
+//           |z~ - z| (the accumulation error of S~ is at most 2^-10 * sum_j |w_j u_j| <=
+//           2^-10 ||u|| ||w_e||, Cauchy-Schwarz), every expert whose approximate logit is
+//           within 2 delta of the k-th largest (or above it) is a candidate; the rest have
+//           exact logits strictly below the k-th exact one.  The candidates are evaluated
+//           exactly in the canonical order and the top-k among them is the answer.
 // Every selection is therefore the canonical one, bit for bit.
 constexpr int kRParts = 3;   // bf16 parts of u
 constexpr int kRSplit = 8;   // K splits of the router GEMM
-constexpr int kCand = 16;    // candidates evaluated exactly first
 constexpr int kRGT = 192;    // router GEMM threads: 6 warps
 constexpr int kRStages = 4;
 
@@ -970,48 +969,52 @@ __global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams 
       }
     return warp_max_key(best);
   };
-  int have = 0;
+  // 1. the k-th largest approximate logit
+  float zk_approx = 0.0f;
+  for (int r = 0; r < K; ++r) {
+    const int e = (int)(~(uint32_t)best_left());
+    zk_approx = za[e];
+    if (lane == 0) flag[e] = 1;
+    __syncwarp();
+  }
+  // 2. candidates: the k best approximate logits and every expert within 2 delta below
+  //    the k-th.  An expert outside has z~ < z~(k) - 2 delta, so its exact logit is below
+  //    z~(k) - delta, which the k-th exact logit is not: the exact top-k is inside.
+  const float thr = zk_approx - 2.0f * delta;
+  int nc = 0;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const bool in = e < E && (flag[e] == 1 || za[e] >= thr);
+    const unsigned b = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      cand[nc + __popc(b & ((1u << lane) - 1u))] = (uint32_t)e;
+      flag[e] = 1;
+    }
+    nc += __popc(b);
+  }
+  __syncwarp();
+  canonical_logits(p, l, urow, cand, nc, inv, zx, lane);
+  __syncwarp();
+  // 3. top-k of the candidates by exact logit; lane r keeps rank r
   int sel_e = -1;
   float sel_z = 0.0f;
-  const int want0 = kCand > K ? kCand : K;
-  for (int want = want0 < E ? want0 : E;; want = want * 4 < E ? want * 4 : E) {
-    const int first = have;
-    for (; have < want; ++have) {  // the next best approximate logits become candidates
-      const int e = (int)(~(uint32_t)best_left());
-      if (lane == 0) {
-        flag[e] = 1;
-        cand[have] = (uint32_t)e;
+  for (int r = 0; r < K; ++r) {
+    uint64_t best = 0;
+    for (int i = lane; i < nc; i += 32) {
+      const int e = (int)cand[i];
+      if (flag[e] == 1) {
+        const uint64_t k = logit_key(zx[e], e);
+        best = k > best ? k : best;
       }
-      __syncwarp();
     }
-    canonical_logits(p, l, urow, cand + first, have - first, inv, zx, lane);
+    best = warp_max_key(best);
+    const int e = (int)(~(uint32_t)best);
+    if (lane == r) {
+      sel_e = e;
+      sel_z = zx[e];
+    }
     __syncwarp();
-    const float thr = want < E ? za[(int)(~(uint32_t)best_left())] : -INFINITY;
-    // top-k of the candidates by exact logit; lane r keeps rank r
-    float zk = 0.0f;
-    for (int r = 0; r < K; ++r) {
-      uint64_t best = 0;
-      for (int i = lane; i < have; i += 32) {
-        const int e = (int)cand[i];
-        if (flag[e] == 1) {
-          const uint64_t k = logit_key(zx[e], e);
-          best = k > best ? k : best;
-        }
-      }
-      best = warp_max_key(best);
-      const int e = (int)(~(uint32_t)best);
-      if (lane == r) {
-        sel_e = e;
-        sel_z = zx[e];
-      }
-      zk = zx[e];
-      __syncwarp();
-      if (lane == 0) flag[e] = 2;
-      __syncwarp();
-    }
-    if (want >= E || (zk == zk && zk > thr + delta)) break;
-    for (int i = lane; i < have; i += 32)  // not certified: widen, ranks open again
-      if (flag[cand[i]] == 2) flag[cand[i]] = 1;
+    if (lane == 0) flag[e] = 2;
     __syncwarp();
   }
   if ((logit_key(__shfl_sync(0xffffffffu, sel_z, 0), 0) >> 32) == 0 && lane == 0)
