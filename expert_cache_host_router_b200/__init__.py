@@ -7,9 +7,11 @@ the binding's functions raises.
 """
 from __future__ import annotations
 
+import atexit
 import ctypes
 import os
 import re
+import weakref
 
 import numpy as np
 
@@ -239,6 +241,15 @@ def moe_destroy(ctx: int) -> None:
 
 # ------------------------------------------------------------------ convenience wrapper
 
+_live = weakref.WeakSet()  # contexts still open, closed at interpreter exit
+
+
+@atexit.register
+def _close_live_contexts() -> None:
+    for m in list(_live):
+        m.close()
+
+
 class ExpertCacheMoE:
     """One libmoe context plus the torch plumbing (device buffers, current stream).
 
@@ -253,14 +264,21 @@ class ExpertCacheMoE:
                           device, log_steps, wait_timeout_ms)
         self.device = device
         self.ctx = moe_create(self.cfg)
+        _live.add(self)
 
     def close(self):
-        if getattr(self, "ctx", None):
-            moe_destroy(self.ctx)
+        ctx = getattr(self, "ctx", None)
+        if ctx:
             self.ctx = None
+            moe_destroy(ctx)
 
     def __del__(self):
-        self.close()
+        # contexts left open at exit are closed by the atexit hook while the module is
+        # intact; a finaliser that runs during interpreter teardown has nothing to do
+        try:
+            self.close()
+        except Exception:
+            pass
 
     def load_layer(self, layer: int, lw) -> None:
         moe_load_layer(self.ctx, layer, lw.experts, lw.shared, lw.router, lw.bias, lw.gain)
