@@ -345,21 +345,35 @@ def run_prefill(m, shape, dev, n_tokens=2048, warmup=2, runs=5):
     ms = e0.elapsed_time(e1) / runs
     _, hist, _ = m.stats(reset=True)
     n_e = hist.astype(np.float64) / runs  # [L][E] tokens per expert per pass
+    roof = prefill_roofline(n_e, n_tokens, shape, tflops, hbm)
+    sec = ms * 1e-3
+    return {"tokens": n_tokens, "value": n_tokens / sec, "unit": "tok/s", "ms": ms, "runs": runs,
+            "dtype": "q4_0 -> fp16 weights x fp16 hi+lo activations, fp32 accumulate (tcgen05)",
+            "roofline": {"bound": "tensor", "achieved": roof["useful_flops"] / sec / 1e12, "peak": tflops,
+                         "unit": "TFLOP/s", "frac": roof["time_s"] / sec, "roofline_ms": roof["time_s"] * 1e3,
+                         "peak_kind": "measured sustained bf16 (fp16 same rate)",
+                         "issued_tflops": roof["issued_flops"] / sec / 1e12,
+                         "note": "frac = per-expert max(flop, weight-byte) time summed / measured time"}}
+
+
+def prefill_roofline(n_e, n_tokens, shape, tflops, hbm_gbs):
+    """Roofline of a prefill pass: per layer and routed expert, the larger of its FLOPs at
+    the tensor peak and its Q4_0 weight bytes at HBM bandwidth (experts no token chose
+    cost nothing), plus the shared expert (every token) per layer.  n_e: [L][E] tokens per
+    expert.  Also the useful FLOPs and the FLOPs the kernels issue (128-row tiles, each
+    K step twice: activation hi and lo)."""
+    n_e = np.asarray(n_e, np.float64)
     H, I, Is = shape.hidden, shape.inter, shape.shared_inter
     fl_tok = 2.0 * 3 * H * I  # one token through one routed expert
     by_exp = 3 * H * I * 18 / 32
-    t_roof = np.sum(np.maximum(n_e * fl_tok / (tflops * 1e12), np.where(n_e > 0, by_exp, 0.0) / (hbm * 1e9)))
-    t_roof += shape.n_layers * max(n_tokens * 2.0 * 3 * H * Is / (tflops * 1e12), 3 * H * Is * 18 / 32 / (hbm * 1e9))
+    t = float(np.sum(np.maximum(n_e * fl_tok / (tflops * 1e12), np.where(n_e > 0, by_exp, 0.0) / (hbm_gbs * 1e9))))
+    if Is > 0:
+        t += shape.n_layers * max(n_tokens * 2.0 * 3 * H * Is / (tflops * 1e12), 3 * H * Is * 18 / 32 / (hbm_gbs * 1e9))
     useful = float(np.sum(n_e) * fl_tok + shape.n_layers * n_tokens * 2.0 * 3 * H * Is)
-    tiles = float(np.sum(np.ceil(n_e / 128.0)) + shape.n_layers * np.ceil(n_tokens / 128.0))
-    issued = tiles * 128 * 2.0 * 3 * H * I * 2  # 128-row tiles, activation hi + lo
-    return {"tokens": n_tokens, "value": n_tokens / (ms * 1e-3), "unit": "tok/s", "ms": ms, "runs": runs,
-            "dtype": "q4_0 -> fp16 weights x fp16 hi+lo activations, fp32 accumulate (tcgen05)",
-            "roofline": {"bound": "tensor", "achieved": useful / (ms * 1e-3) / 1e12, "peak": tflops,
-                         "unit": "TFLOP/s", "frac": t_roof / (ms * 1e-3), "roofline_ms": t_roof * 1e3,
-                         "peak_kind": "measured sustained bf16 (fp16 same rate)",
-                         "issued_tflops": issued / (ms * 1e-3) / 1e12,
-                         "note": "frac = per-expert max(flop, weight-byte) time summed / measured time"}}
+    issued = float(np.sum(np.ceil(n_e / 128.0))) * 128 * 2.0 * 3 * H * I * 2
+    if Is > 0:
+        issued += shape.n_layers * np.ceil(n_tokens / 128.0) * 128 * 2.0 * 3 * H * Is * 2
+    return {"time_s": t, "useful_flops": useful, "issued_flops": float(issued)}
 
 
 # ------------------------------------------------------------------ GPU arm
