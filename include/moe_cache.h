@@ -51,7 +51,7 @@ extern "C" {
 #define MOE_ERR_CUDA (-3)        /* a CUDA runtime/driver call failed */
 #define MOE_ERR_TIMEOUT (-4)     /* a bounded device-side wait ran out (see moe_sync) */
 #define MOE_ERR_STATE (-5)       /* call out of order (e.g. decode before residency) */
-#define MOE_ERR_UNSUPPORTED (-6) /* shape or feature outside this build's limits */
+#define MOE_ERR_UNSUPPORTED (-6) /* shape or feature outside the library's limits */
 #define MOE_ERR_DEVICE (-7)      /* the kernel flagged a bad route or slot (see moe_sync) */
 
 /* Cache event kinds (key-components item 2 of the Luce Spark write-up). */
