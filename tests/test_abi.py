@@ -75,3 +75,44 @@ def test_null_arguments_are_rejected(lib):
     assert lib.moe_load_layer(None, 0, None, None, None, None, None) == moe.MOE_ERR_INVALID
     assert lib.moe_decode_step_noalloc(None, None, None, None, None) == moe.MOE_ERR_INVALID
     lib.moe_destroy(None)  # no-op
+
+
+_STRUCTS = {
+    "moe_config": ("Config", ["n_layers", "hidden", "n_experts", "top_k", "inter", "shared_inter", "ring_slots",
+                              "use_rmsnorm", "rms_eps", "device", "log_steps", "wait_timeout_ms"]),
+    "moe_weights": ("Weights", ["expert_q4_0", "shared_q4_0", "router_bf16", "router_bias", "rms_gain"]),
+    "moe_noalloc_weights": ("NoAllocWeights", ["experts_dev", "shared_dev", "router_dev", "bias_dev", "gain_dev"]),
+    "moe_event": ("Event", ["step", "layer", "rank", "expert", "kind", "slot", "evicted"]),
+    "moe_stats_t": ("Stats", ["steps", "accesses", "pin_hits", "ring_hits", "misses", "evictions", "bytes_copied",
+                              "staged_misses", "log_dropped", "device_error", "n_pinned", "residency", "placement",
+                              "repins", "repin_copies", "miss_requests", "miss_served", "proxy_error"]),
+}
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The binding's ctypes structures have the header's sizes and field offsets (a C
+    program compiled against include/moe_cache.h prints them)."""
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "moe_cache.h"', "int main(void) {"]
+    for c, (_, fields) in _STRUCTS.items():
+        lines.append(f'  printf("{c} size %zu\\n", sizeof({c}));')
+        for f in fields:
+            lines.append(f'  printf("{c} {f} %zu\\n", offsetof({c}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", f"-I{os.path.join(root, 'include')}", str(src), "-o", str(exe)])
+    out = subprocess.check_output([str(exe)], text=True).split("\n")
+    got = {}
+    for ln in out:
+        if ln:
+            c, f, v = ln.split()
+            got[(c, f)] = int(v)
+    for c, (py, fields) in _STRUCTS.items():
+        cls = getattr(moe, py)
+        assert ctypes.sizeof(cls) == got[(c, "size")], c
+        assert [n for n, _ in cls._fields_] == fields, c
+        for f in fields:
+            assert getattr(cls, f).offset == got[(c, f)], (c, f)
