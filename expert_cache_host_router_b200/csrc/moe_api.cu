@@ -741,7 +741,6 @@ int moe_prefill(moe_ctx* c, const float* x_dev, int32_t n_tokens, float* y_dev, 
   a.slay = c->slay;
   a.shared_pool = c->shared_pool;
   a.shared_slot_bytes = c->shared_slot_bytes;
-  a.router = c->router;
   a.bias = c->has_bias ? c->bias : nullptr;
   a.gain = c->gain;
   a.pin_slot = c->pin_slot;

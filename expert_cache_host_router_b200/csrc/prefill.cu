@@ -54,16 +54,10 @@ struct PrefillParams {
   int t_base, T_total;  // this chunk's first token and the call's token count (trace rows)
   int R;                // grouped rows of this chunk: T * k (+ T with a shared expert)
   float eps;
-  const uint8_t* pool;  // layer l expert e at pool + (base[l] + (pin[l][e] & 0xffff)) * slot_bytes
-  uint64_t slot_bytes;
-  SlotLayout lay, slay;
-  const uint8_t* shared_pool;
-  uint64_t shared_slot_bytes;
-  const uint16_t* router;  // [L][nch][E][16] bf16
-  const float* bias;       // [L][E] or null
-  const float* gain;       // [L][H]
-  const int32_t* pin_slot;
-  const int32_t* layer_base;
+  const float* bias;          // [L][E] or null
+  const float* gain;          // [L][H]
+  const int32_t* pin_slot;    // [L][E]: pool slot of expert e at layer l is base[l] + (entry & 0xffff)
+  const int32_t* layer_base;  // [L]
   uint32_t* hist;
   const float* wnorm;  // [L] max_e ||w_e||_2 of the router rows, rounded up
   const uint16_t* router_rows;  // [L][E][H] bf16
@@ -76,10 +70,6 @@ __device__ __forceinline__ uint32_t smem_u32p(const void* ptr) {
 __device__ __forceinline__ float bf16_lo_p(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_p(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ const uint8_t* expert_slot(const PrefillParams& p, int l, int e) {
-  if (e >= p.E) return p.shared_pool + (size_t)l * p.shared_slot_bytes;
-  return p.pool + (size_t)(p.layer_base[l] + (p.pin_slot[(size_t)l * p.E + e] & 0xffff)) * p.slot_bytes;
-}
 
 // ------------------------------------------------------------------ grouping
 
@@ -1213,13 +1203,6 @@ int prefill_run(const PrefillArgs& a, const PrefillScratch& s, void* encode_fn, 
     p.T_total = T;
     p.eps = a.eps;
     p.nch = H / kChunk;
-    p.pool = a.pool;
-    p.slot_bytes = a.slot_bytes;
-    p.lay = a.lay;
-    p.slay = a.slay;
-    p.shared_pool = a.shared_pool;
-    p.shared_slot_bytes = a.shared_slot_bytes;
-    p.router = a.router;
     p.bias = a.bias;
     p.gain = a.gain;
     p.pin_slot = a.pin_slot;

@@ -21,7 +21,6 @@ struct PrefillArgs {
   SlotLayout lay, slay;
   const uint8_t* shared_pool;
   uint64_t shared_slot_bytes;
-  const uint16_t* router;  // [L][H/16][E][16] bf16
   const float* bias;       // [L][E] or null
   const float* gain;       // [L][H]
   const int32_t* pin_slot;    // [L][E], every entry valid
