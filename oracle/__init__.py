@@ -26,14 +26,25 @@ PIN_HIT, RING_HIT, MISS = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
-    """Compile moe_oracle.c with gcc (single-threaded, no FP contraction)."""
+    """Compile moe_oracle.c with gcc (single-threaded, no FP contraction).
+
+    ``ORACLE_LIB`` in the environment names an already built copy to load instead; the
+    mutation check of the pins uses it to run them against deliberately broken copies."""
+    override = os.environ.get("ORACLE_LIB")
+    if override:
+        return override
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".{os.getpid()}.tmp"
-        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
-                               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        compile_c(_SRC, tmp)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
+
+
+def compile_c(src: str, out: str) -> None:
+    """gcc flags of the oracle: -O2, no FP contraction, no fast-math, C11."""
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
+                           "-shared", "-fPIC", "-o", out, src, "-lm"])
 
 
 class Dims(ctypes.Structure):

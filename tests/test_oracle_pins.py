@@ -111,6 +111,12 @@ def test_canonical_sum_order_hand_computed():
     p = np.zeros(64, np.float32)
     p[1], p[33], p[17], p[0] = 2.0 ** 24 + 2, 2.0, 1.0, 1.0
     assert oracle.canonical_sum(p) == 2.0 ** 24 + 4
+    # Offset 16 comes first: lanes 1 and 17 meet (1 + 1 = 2) before lane 1 joins lane 0
+    # at offset 1, giving 2^24 + 2 exactly; offsets taken from 1 upwards would add each
+    # 1.0 to 2^24 on its own and lose both (2^24).
+    p = np.zeros(32, np.float32)
+    p[0], p[1], p[17] = 2.0 ** 24, 1.0, 1.0
+    assert oracle.canonical_sum(p) == 2.0 ** 24 + 2
 
 
 def test_canonical_sum_within_error_bound():
@@ -134,6 +140,25 @@ def test_rms_inv_closed_forms(H):
     h = np.ones(H, np.float32)
     h[::2] = -1
     assert oracle.rms_inv(h, 3.0) == 0.5
+
+
+def test_rms_inv_sum_of_squares_is_one_fused_chain():
+    # One 16-element chunk, h = (a, b, 0, ...) with a = 2051/1024 and b = 1 + 2^-23.
+    # a^2 = 4206601 * 2^-20 is exact in fp32; b^2 = 1 + 2^-22 + 2^-46.  The fused step
+    # fmaf(b, b, a^2) rounds a^2 + 1 + 2^-22 + 2^-46 once, where a^2 + 1 = 10510354 * 2^-21
+    # and fp32 steps by 2^-21 here: just above halfway, so ss = 10510355 * 2^-21.
+    # Rounding b^2 first (to 1 + 2^-22) would leave an exact tie, resolved to the even
+    # 10510354 * 2^-21, and a different 1/sqrt(ss/16).
+    h = np.zeros(16, np.float32)
+    h[0], h[1] = 2051 / 1024, 1 + 2.0 ** -23
+    ss_fused = np.float32(10510355 * 2.0 ** -21)
+    ss_split = np.float32(10510354 * 2.0 ** -21)
+
+    def inv_of(ss):
+        return np.float32(1) / np.sqrt(ss / np.float32(16))
+
+    assert inv_of(ss_fused) != inv_of(ss_split)
+    assert oracle.rms_inv(h, 0.0) == inv_of(ss_fused)
 
 
 def test_rms_inv_matches_fp64_within_bound():
@@ -172,6 +197,36 @@ def test_router_gain_and_scale_closed_form():
     b = np.full(E, -1.0, np.float32)
     z = oracle.router_logits(w, h, g, 0.25, b)
     assert np.all(z == H * 0.5 * 0.25 - 1.0)
+
+
+def test_router_rounding_hand_computed():
+    one = _bf16(1.0)
+    # Each product joins its chunk's chain in one rounding (fmaf): w = (-1, 1 + 2^-7),
+    # u = (1 + 2^-7 + 2^-23, 1 + 2^-23).  The chain is -(1 + 2^-7 + 2^-23), then
+    # (1 + 2^-7)(1 + 2^-23) - (1 + 2^-7 + 2^-23) = 2^-30 exactly; rounding the product
+    # first would drop its 2^-30 and give 0.
+    w = np.zeros((1, 16), np.uint16)
+    w[0, 0], w[0, 1] = _bf16(-1.0), _bf16(1 + 2.0 ** -7)
+    h = np.zeros(16, np.float32)
+    h[0], h[1] = 1 + 2.0 ** -7 + 2.0 ** -23, 1 + 2.0 ** -23
+    assert oracle.router_logits(w, h, None, 1.0, None)[0] == 2.0 ** -30
+    # Chunks of 16 columns: u = (2^24, 1, ..., 1) over 32 columns of ones.  The first
+    # chunk's fifteen ones each round away against 2^24 (ties to even); the second chunk
+    # sums its sixteen ones to 16 on its own; the fold gives 2^24 + 16.  One chain over
+    # all 32 columns would give 2^24, chunks of 8 would give 2^24 + 24.
+    w = np.full((1, 32), one, np.uint16)
+    h = np.ones(32, np.float32)
+    h[0] = 2.0 ** 24
+    assert oracle.router_logits(w, h, None, 1.0, None)[0] == 2.0 ** 24 + 16
+    # The norm scale and the bias join the folded sum in one rounding:
+    # S = 1 + 2^-23, inv = 1 + 2^-23, b = -(1 + 2^-22): S * inv + b = 2^-46 exactly;
+    # rounding S * inv first gives 1 + 2^-22 and then 0.
+    w = np.zeros((1, 16), np.uint16)
+    w[0, 0] = one
+    h = np.zeros(16, np.float32)
+    h[0] = 1 + 2.0 ** -23
+    b = np.array([-(1 + 2.0 ** -22)], np.float32)
+    assert oracle.router_logits(w, h, None, np.float32(1 + 2.0 ** -23), b)[0] == 2.0 ** -46
 
 
 def test_router_matches_fp64_within_bound():
@@ -322,6 +377,14 @@ def test_norm_layer_special_cases():
     assert np.array_equal(out_g["z"], plain_g["z"])
     assert np.array_equal(out_g["sel"], plain_g["sel"])
     assert np.allclose(out_g["h_out"] - h, plain_g["y"], rtol=1e-12, atol=1e-12)
+    # eps = 3 on the same unit-RMS h: mean(h^2) + eps = 4, so the norm is x = g * h / 2
+    # exactly, routing included (a power-of-two scale passes through every fmaf)
+    s3 = synthetic.Shape(1, 256, 16, 4, 64, 64, use_rmsnorm=1, zipf_s=1.0, rms_eps=3.0)
+    out_e = oracle.Model(s3, lw_g).layer(0, h)
+    plain_e = oracle.Model(synthetic.Shape(1, 256, 16, 4, 64, 64, zipf_s=1.0), lw_g).layer(0, g * h / 2)
+    assert np.array_equal(out_e["z"], plain_e["z"])
+    assert np.array_equal(out_e["sel"], plain_e["sel"])
+    assert np.allclose(out_e["h_out"] - h, plain_e["y"], rtol=1e-12, atol=1e-12)
     # scale invariance of RMSNorm (eps = 0): y(4h) == y(h) and routing is unchanged
     h = rng.standard_normal(s.hidden).astype(np.float32)
     a, b = m.layer(0, h), m.layer(0, 4 * h)
@@ -435,6 +498,22 @@ def test_ring_reused_within_one_token_when_misses_exceed_ring():
     assert ev["slot"].tolist() == [0, 1, 0, 1]
     assert ev["evicted"].tolist() == [-1, -1, 3, 5]
     assert c.ring(0).tolist() == [7, 9]
+
+
+def test_repin_empties_the_ring():
+    """A new pinned set starts with an empty ring: an expert the ring held before misses
+    again, into the first ring slot, with nothing evicted."""
+    c = oracle.Cache(1, 8, 2)
+    c.set_pinned(0, np.zeros(8, np.uint8))
+    c.access(0, 0, np.array([1, 2], np.int32))
+    assert c.ring(0).tolist() == [1, 2]
+    mask = np.zeros(8, np.uint8)
+    mask[5] = 1
+    c.set_pinned(0, mask)
+    assert c.ring(0).tolist() == [-1, -1]
+    ev = c.access(1, 0, np.array([1, 5], np.int32))
+    assert ev["kind"].tolist() == [oracle.MISS, oracle.PIN_HIT]
+    assert ev["slot"].tolist() == [1, 0] and ev["evicted"].tolist() == [-1, -1]
 
 
 def test_calibrated_placement_cuts_cold_hits_vs_uniform():
