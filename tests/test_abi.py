@@ -74,6 +74,10 @@ def test_null_arguments_are_rejected(lib):
     assert lib.moe_debug_drop_signals(None, 1) == moe.MOE_ERR_INVALID
     assert lib.moe_load_layer(None, 0, None, None, None, None, None) == moe.MOE_ERR_INVALID
     assert lib.moe_decode_step_noalloc(None, None, None, None, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_recalibrate(None) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_router_bias(None, 0, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_prefill_trace(None, None, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_phase_trace(None, None) == moe.MOE_ERR_INVALID
     lib.moe_destroy(None)  # no-op
 
 
