@@ -106,7 +106,7 @@ def test_every_planted_slip_fails_a_pin(tmp_path):
         so_path = str(tmp_path / f"mutant{i}.so")
         oracle.compile_c(str(c_path), so_path)
         libs.append(so_path)
-    workers = max(1, min(8, (os.cpu_count() or 2)))
+    workers = max(1, min(4, (os.cpu_count() or 2)))
     with ThreadPoolExecutor(workers) as ex:
         results = list(ex.map(_run_pins, libs))
     survivors = [name for (name, _, _), r in zip(MUTANTS, results) if r.returncode == 0]
