@@ -41,6 +41,17 @@ WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 5
             "residency + 8-slot LRU ring (residency_60)")
 
 
+def compact(obj, digits=5):
+    """Floats rounded to `digits` significant digits, recursively (keeps the JSON line short)."""
+    if isinstance(obj, float):
+        return float(f"{obj:.{digits}g}")
+    if isinstance(obj, dict):
+        return {k: compact(v, digits) for k, v in obj.items()}
+    if isinstance(obj, (list, tuple)):
+        return [compact(v, digits) for v in obj]
+    return obj
+
+
 def env_rank():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
             int(os.environ.get("LOCAL_RANK", 0)))
@@ -376,6 +387,83 @@ def prefill_roofline(n_e, n_tokens, shape, tflops, hbm_gbs):
     return {"time_s": t, "useful_flops": useful, "issued_flops": float(issued)}
 
 
+def decode_precision(m, shape, layers, dev):
+    """Largest per-layer error of one traced decode token (full residency) against the
+    oracle run on the GPU's own layer input, as a fraction of the 2e-3 x RMS bar."""
+    import torch
+
+    import oracle
+    orc = oracle.Model(shape, layers)
+    ht = torch.zeros((shape.n_layers + 1, shape.hidden), dtype=torch.float32, device=dev)
+    m.set_trace(ht, None)
+    m.decode(torch.from_numpy(synthetic.token(900, shape.hidden)).to(dev))
+    m.sync()
+    m.set_trace(None, None)
+    h = ht.cpu().numpy()
+    worst = 0.0
+    for l in range(shape.n_layers):
+        ref = orc.layer(l, h[l])
+        rms = float(np.sqrt(np.mean(ref["y"] ** 2)))
+        err = float(np.max(np.abs(h[l + 1].astype(np.float64) - ref["h_out"])))
+        worst = max(worst, err / (2e-3 * rms))
+    # prefill: 16 tokens through the whole stack, two of them checked at every layer
+    T = 16
+    hp = torch.zeros((shape.n_layers + 1, T, shape.hidden), dtype=torch.float32, device=dev)
+    sp = torch.zeros((shape.n_layers, T, shape.top_k), dtype=torch.int32, device=dev)
+    m.set_prefill_trace(hp, sp)
+    m.prefill(torch.from_numpy(synthetic.tokens(901, T, shape.hidden)).to(dev))
+    m.sync()
+    m.set_prefill_trace(None, None)
+    hpn = hp.cpu().numpy()
+    worst_p = 0.0
+    for t in (0, T - 1):
+        for l in range(shape.n_layers):
+            ref = orc.layer(l, hpn[l, t])
+            rms = float(np.sqrt(np.mean(ref["y"] ** 2)))
+            err = float(np.max(np.abs(hpn[l + 1, t].astype(np.float64) - ref["h_out"])))
+            worst_p = max(worst_p, err / (2e-3 * rms))
+    return {"decode_max_layer_err_over_bar": round(worst, 4),
+            "prefill_max_layer_err_over_bar": round(worst_p, 4), "bar": "2e-3 x RMS(y) per element",
+            "sample": "decode: one token, prefill: two of 16 tokens; every layer, teacher-forced"}
+
+
+def write_phase_table(m, shape, xs, y, path, n_tokens=8):
+    """Per-layer phase times of CTA 0 (median over n_tokens full-residency tokens) from
+    the kernel's global-timer stamps, written as JSON to path."""
+    import torch
+
+    import expert_cache_host_router_b200 as moe
+    n_sm = torch.cuda.get_device_properties(y.device).multi_processor_count
+    words = moe.phase_trace_words(shape.n_layers, n_sm)
+    st = torch.zeros(words, dtype=torch.int64, device=y.device)
+    m.set_residency(1.0)
+    m.set_phase_trace(st)
+    runs = []
+    for i in range(n_tokens):
+        m.decode(xs[i % len(xs)], y)
+        m.sync()
+        runs.append(st.cpu().numpy().copy())
+    m.set_phase_trace(None)
+    L = shape.n_layers
+    marks = np.stack([r[: (L + 1) * 32].reshape(L + 1, 32) for r in runs]).astype(np.float64)
+    names = {1: "prev_layer_output", 2: "h_updated", 10: "norm_u", 11: "own_logit", 12: "x_quantised",
+             3: "logits_published", 4: "logits_read", 13: "topk", 14: "cache", 5: "routed", 15: "loads_issued_t0",
+             6: "loads_issued", 7: "gateup_done", 16: "swiglu", 17: "down_landed", 18: "down_adds", 19: "fence",
+             8: "units_done", 9: "arrived"}
+    table = []
+    for l in range(L):
+        row = {"layer": l}
+        for k, n in names.items():
+            row[n] = float(np.median(marks[:, l, k] - marks[:, l, 0])) / 1e3
+        nxt = marks[:, l + 1, 0] if l + 1 < L else marks[:, L, 2]
+        row["layer_us"] = float(np.median(nxt - marks[:, l, 0])) / 1e3
+        table.append(row)
+    total = float(np.median(marks[:, L, 2] - marks[:, L, 0])) / 1e3
+    with open(path, "w") as f:
+        json.dump({"unit": "us since layer start (CTA 0), median over tokens", "tokens": n_tokens,
+                   "kernel_us": total, "layers": table}, f, indent=1)
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def run_ours(args):
@@ -405,6 +493,8 @@ def run_ours(args):
     layers = [synthetic.layer_weights(l, shape) for l in range(shape.n_layers)]
     gen_s = time.time() - t0
     m = moe.ExpertCacheMoE(shape, device=local, log_steps=max(4096, args.steps + args.warmup + 16))
+    if args.prefetch:
+        m.set_prefetch(args.prefetch)
     t0 = time.time()
     for l in range(shape.n_layers):
         m.load_layer(l, layers[l])
@@ -469,26 +559,28 @@ def run_ours(args):
         if args.phases == "all":
             m.set_residency(0.6, hist, moe.MOE_PLACE_CALIBRATED)
             t60, per60, st60 = timed()
+            m.set_miss_path(moe.MOE_MISS_SM_PULL)
+            m.set_residency(0.6, hist, moe.MOE_PLACE_CALIBRATED)
+            t60p, per60p, st60p = timed()
+            m.set_miss_path(moe.MOE_MISS_COPY_ENGINE)
             m.set_residency(0.6, hist, moe.MOE_PLACE_UNIFORM)
             t60u, per60u, st60u = timed()
         else:  # full residency only: no miss copies (profilers serialise the proxy's copies)
             t60, per60, st60 = t100, per100, st100
+            t60p, per60p, st60p = t100, per100, st100
             t60u, per60u, st60u = t100, per100, st100
 
-    # host-to-device bandwidth for one expert slot from pinned memory (the miss copy)
-    src = torch.empty(slot_bytes, dtype=torch.uint8).pin_memory()
-    dst = torch.empty(slot_bytes, dtype=torch.uint8, device=dev)
-    side = torch.cuda.Stream(dev)
-    with torch.cuda.stream(side):
-        for _ in range(5):
-            dst.copy_(src, non_blocking=True)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(side)
-        for _ in range(100):
-            dst.copy_(src, non_blocking=True)
-        b.record(side)
-    side.synchronize()
-    h2d_gbs = 100 * slot_bytes / (a.elapsed_time(b) * 1e-3) / 1e9
+    # host-to-device rate of the miss path: the library's own copy (pinned host tier ->
+    # device slot, cudaMemcpyAsync on the proxy's side stream), back to back
+    m.set_residency(1.0)
+    h2d_gbs = m.measure_h2d(64)
+    # and the copies the proxy made during the 60% run, each timed on the device
+    h2d_run = (st60["copies_timed"] * slot_bytes / (st60["copy_ns_timed"] * 1e-9) / 1e9
+               if st60.get("copies_timed") else None)
+
+    precision = None
+    if args.phases == "all" and keep_layers:
+        precision = decode_precision(m, shape, layers, dev)
 
     # end to end through the host-buffer entry point at full residency
     m.set_residency(1.0)
@@ -504,21 +596,27 @@ def run_ours(args):
 
     t100_max, units100 = reduce_over_ranks(t100, args.steps, world)
     t60_max, units60 = reduce_over_ranks(t60, args.steps, world)
+    t60p_max, units60p = reduce_over_ranks(t60p, args.steps, world)
     value100 = units100 / (t100_max * 1e-3)
     value60 = units60 / (t60_max * 1e-3)
+    value60p = units60p / (t60p_max * 1e-3)
     value60u = args.steps * world / (max(t60u, 1e-9) * 1e-3)
     kern_ms = statistics.mean(per100)
     achieved = bytes_tok / (kern_ms * 1e-3) / 1e9
 
     def cache_summary(st):
         acc = max(st["accesses"], 1)
-        return {"cold_hit_rate": (st["ring_hits"] + st["misses"]) / acc, "miss_rate": st["misses"] / acc,
-                "misses_per_token": st["misses"] / args.steps,
+        return {"cold_hit_rate": round((st["ring_hits"] + st["misses"]) / acc, 5),
+                "miss_rate": round(st["misses"] / acc, 5),
+                "misses_per_token": round(st["misses"] / args.steps, 4),
                 "staged_misses": st["staged_misses"]}
 
+    def roof60(st, t_ms, link_gbs):
+        miss_bytes = st["misses"] / args.steps * slot_bytes
+        r = max(bytes_tok / (peak * 1e9), miss_bytes / (link_gbs * 1e9))
+        return {"roofline_frac": round(r / (t_ms * 1e-3 / args.steps), 4), "roofline_us_per_token": round(r * 1e6, 2)}
+
     c60 = cache_summary(st60)
-    miss_bytes = c60["misses_per_token"] * slot_bytes
-    roof60_s = max(bytes_tok / (peak * 1e9), miss_bytes / (h2d_gbs * 1e9))
     line = {
         "metric": METRIC, "value": value100, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t100_max / args.steps, "higher_is_better": True,
@@ -529,10 +627,13 @@ def run_ours(args):
                    "shared_inter": shape.shared_inter, "ring_slots": shape.ring_slots,
                    "calibration_tokens": args.calib_steps, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: 637 MB of expert weights streamed per token"},
-        "residency_60": {"value": value60, "unit": "tok/s", "ratio_to_100": value60 / value100,
-                         "roofline_frac": roof60_s / (t60_max * 1e-3 / args.steps),
-                         "roofline_us_per_token": roof60_s * 1e6, "h2d_gbs": h2d_gbs,
+        "residency_60": {"value": value60, "unit": "tok/s", "ratio_to_100": round(value60 / value100, 4),
+                         "miss_path": "copy engine (proxy thread)",
+                         **roof60(st60, t60_max, h2d_gbs), "h2d_gbs": round(h2d_gbs, 2),
+                         "h2d_gbs_miss_copies": None if h2d_run is None else round(h2d_run, 2),
                          **c60,
+                         "sm_pull": {"value": value60p, "ratio_to_100": round(value60p / value100, 4),
+                                     **roof60(st60p, t60p_max, h2d_gbs), **cache_summary(st60p)},
                          "uniform_placement": {"value": value60u, **cache_summary(st60u)}},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic_per_launch(shape.n_layers), "peak_kind": peak_kind,
@@ -542,8 +643,23 @@ def run_ours(args):
                 "h2d_bytes_per_step": 4 * shape.hidden, "d2h_bytes_per_step": 4 * shape.hidden + 4},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
-        "setup": {"generate_s": gen_s, "load_s": load_s, "phases": args.phases},
+        "setup": {"generate_s": round(gen_s, 1), "load_s": round(load_s, 1), "phases": args.phases},
     }
+    if precision is not None:
+        line["precision"] = precision
+    if args.phase_trace:
+        write_phase_table(m, shape, xs, y, args.phase_trace)
+    if args.prefetch_sweep:
+        sweep = []
+        m.set_residency(1.0)
+        for n in (0, 4, 8, 12, 16):
+            m.set_prefetch(n)
+            for i in range(args.warmup):
+                m.decode(xs[i], y)
+            sweep.append({"prefetch_experts": n, **decode_point(m, shape, xs[args.warmup:], y, stream,
+                                                                min(64, args.steps))})
+        m.set_prefetch(args.prefetch)
+        line["prefetch_sweep"] = sweep
     if args.phases == "all" and not args.no_curve:
         line["residency_curve"] = run_residency_curve(m, shape, hist, xs, y, stream, steps=min(128, len(xs)))
     if args.phases == "all" and not args.no_prefill:
@@ -559,7 +675,7 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": tps, "unit": "tok/s", "cores": cores, "kind": "oracle",
                                 "sample": f"{args.cpu_tokens} tokens through all 40 layers ({dt:.1f} s)"}
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(compact(line, 6)), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -581,6 +697,9 @@ def main():
     ap.add_argument("--no-curve", action="store_true",
                     help="skip the residency curve and the small-shape stack")
     ap.add_argument("--prefill-runs", type=int, default=5, help="timed prefill passes")
+    ap.add_argument("--prefetch", type=int, default=0, help="likely experts prefetched into L2 per layer")
+    ap.add_argument("--prefetch-sweep", action="store_true", help="decode tok/s at 100%% over prefetch depths")
+    ap.add_argument("--phase-trace", default=None, help="write a per-layer phase table (JSON) to this path")
     ap.add_argument("--phases", default="all", choices=["all", "100"],
                     help="'100' times full residency only (no miss copies), for profiler runs")
     args = ap.parse_args()

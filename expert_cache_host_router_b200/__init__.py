@@ -29,6 +29,7 @@ MOE_ERR_UNSUPPORTED = -6
 MOE_ERR_DEVICE = -7
 MOE_PIN_HIT, MOE_RING_HIT, MOE_MISS = 0, 1, 2
 MOE_PLACE_CALIBRATED, MOE_PLACE_UNIFORM = 0, 1
+MOE_MISS_COPY_ENGINE, MOE_MISS_SM_PULL = 0, 1
 
 
 class MoEError(RuntimeError):
@@ -77,7 +78,9 @@ class Stats(ctypes.Structure):
                 ("n_pinned", ctypes.c_int32), ("residency", ctypes.c_float),
                 ("placement", ctypes.c_int32), ("repins", ctypes.c_uint64),
                 ("repin_copies", ctypes.c_uint64), ("miss_requests", ctypes.c_uint64),
-                ("miss_served", ctypes.c_uint64), ("proxy_error", ctypes.c_int32)]
+                ("miss_served", ctypes.c_uint64), ("proxy_error", ctypes.c_int32),
+                ("miss_path", ctypes.c_int32), ("pulled_misses", ctypes.c_uint64),
+                ("copies_timed", ctypes.c_uint64), ("copy_ns_timed", ctypes.c_uint64)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -99,7 +102,10 @@ _SIGS = {
     "moe_set_prefill_trace": (ctypes.c_int, [_P, _P, _P]),
     "moe_recalibrate": (ctypes.c_int, [_P]),
     "moe_set_router_bias": (ctypes.c_int, [_P, ctypes.c_int32, _P]),
-    "moe_set_phase_trace": (ctypes.c_int, [_P, _P]),
+    "moe_set_phase_trace": (ctypes.c_int, [_P, _P, ctypes.c_size_t]),
+    "moe_set_miss_path": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "moe_measure_h2d": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]),
+    "moe_set_prefetch": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_debug_drop_signals": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(NoAllocWeights),
                                                 _P, _P, _P]),
@@ -221,8 +227,27 @@ def moe_set_prefill_trace(ctx: int, h_trace_dev: int | None, sel_trace_dev: int 
     _check(lib().moe_set_prefill_trace(ctx, h_trace_dev, sel_trace_dev), "moe_set_prefill_trace")
 
 
-def moe_set_phase_trace(ctx: int, stamps_dev: int | None) -> None:
-    _check(lib().moe_set_phase_trace(ctx, stamps_dev), "moe_set_phase_trace")
+def moe_set_phase_trace(ctx: int, stamps_dev: int | None, n_words: int = 0) -> None:
+    _check(lib().moe_set_phase_trace(ctx, stamps_dev, n_words), "moe_set_phase_trace")
+
+
+def moe_set_miss_path(ctx: int, mode: int) -> None:
+    _check(lib().moe_set_miss_path(ctx, mode), "moe_set_miss_path")
+
+
+def moe_set_prefetch(ctx: int, n_experts: int) -> None:
+    _check(lib().moe_set_prefetch(ctx, n_experts), "moe_set_prefetch")
+
+
+def moe_measure_h2d(ctx: int, n_copies: int) -> float:
+    g = ctypes.c_double(0.0)
+    _check(lib().moe_measure_h2d(ctx, n_copies, ctypes.byref(g)), "moe_measure_h2d")
+    return g.value
+
+
+def phase_trace_words(n_layers: int, n_sm: int) -> int:
+    """Length (uint64 words) moe_set_phase_trace needs: [(L+1)][32] + [L][n_sm][4]."""
+    return (n_layers + 1) * 32 + n_layers * n_sm * 4
 
 
 def moe_debug_drop_signals(ctx: int, n: int) -> None:
@@ -330,8 +355,22 @@ class ExpertCacheMoE:
         moe_set_router_bias(self.ctx, layer, bias)
 
     def set_phase_trace(self, stamps=None):
-        """stamps: torch int64 [(L+1), 8] on the device, or None."""
-        moe_set_phase_trace(self.ctx, None if stamps is None else stamps.data_ptr())
+        """stamps: contiguous torch int64 tensor on the device with at least
+        phase_trace_words(L, n_sm) elements (n_sm = the device's SM count), or None."""
+        if stamps is None:
+            moe_set_phase_trace(self.ctx, None, 0)
+        else:
+            assert stamps.is_contiguous() and stamps.element_size() == 8
+            moe_set_phase_trace(self.ctx, stamps.data_ptr(), stamps.numel())
+
+    def set_miss_path(self, mode: int) -> None:
+        moe_set_miss_path(self.ctx, mode)
+
+    def set_prefetch(self, n_experts: int) -> None:
+        moe_set_prefetch(self.ctx, n_experts)
+
+    def measure_h2d(self, n_copies: int = 64) -> float:
+        return moe_measure_h2d(self.ctx, n_copies)
 
     def set_trace(self, h_trace=None, w_trace=None):
         moe_set_trace(self.ctx, None if h_trace is None else h_trace.data_ptr(),

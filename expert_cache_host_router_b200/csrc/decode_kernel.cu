@@ -3,29 +3,31 @@
 //
 // Luce Spark (theneuralfeed.com write-up, key-components paragraph) runs the whole
 // token as one graph instead of one per layer; here the token is one cooperative
-// kernel launch, captured in a CUDA graph by the runtime.  Per layer:
+// kernel launch, captured in a CUDA graph by the runtime.  Every CTA keeps the whole
+// residual stream h in shared memory.  Per layer:
 //
-//   R  router logits z_e = fmaf(S_e, inv, b_e) for this CTA's experts, where S_e folds
-//      the per-chunk partials that the previous layer's D phase produced (canonical
-//      order: lane l adds chunks l, l+32, ... from +0, then xor-butterfly 16..1)
-//   -- grid barrier --
-//      every CTA: warp-shuffle top-k (value desc, index asc), routing weights (softmax
-//      over the kept logits), the cache decision (pinned / ring hit / miss into the LRU
-//      ring slot, key-components item 2), and the quantised activations x
-//      (int16 per 32-block) for the integer expert GEMVs; CTA 0 alone commits the ring
-//      state, the event log, the atomic routing histogram and the miss requests that
-//      the host proxy turns into copy-engine copies from pinned host memory
-//   G  gate/up GEMV + SwiGLU: work unit = 32 rows of gate and up of one expert,
-//      streamed into shared memory by bulk (TMA) copies; a = silu(g) * u is quantised
-//      per 32-block and published
-//   -- grid barrier --
-//   D  down GEMV + weighted combine + shared expert + residual for 16 rows of h per
-//      chunk, then the next layer's router partials and RMSNorm partial sums over the
-//      same 16 columns
-//   -- grid barrier --
+//   1. h += y of the previous layer, read from a 64-bit fixed-point accumulator that
+//      the previous layer's units added into (the layer's one grid-wide exchange)
+//   2. RMSNorm scale and the canonical-order router logits of this CTA's experts
+//      (router rows staged in shared memory one layer ahead), published as 8-byte
+//      words that carry the layer as an epoch, so readers need no separate flag
+//   3. every CTA reads all logits: warp-shuffle top-k (value desc, index asc), routing
+//      weights (softmax over the kept logits), the cache decision (pinned / ring hit /
+//      miss into the LRU ring slot, key-components item 2); CTA 0 commits the ring
+//      state, the event log, the atomic routing histogram and the miss requests
+//   4. units: unit (expert, rb) = gate/up rows 32rb..32rb+31 and down column block rb
+//      of one expert, one contiguous run of the slot streamed into shared memory by
+//      bulk (TMA) copies; Q4_0 x int16 dot products (dp2a) give g and u,
+//      a = silu(g) * u is quantised per block, and the unit's share of the layer output
+//      w_i * D_i[:, rb] a_rb is added into the accumulator (fixed point: the sum does
+//      not depend on the order in which units finish, so outputs are bit-identical
+//      across residency levels and runs)
+//   5. one release add per CTA on the arrival counter
 //
-// Every wait is bounded by a globaltimer deadline; a wait that runs out sets the error
-// word and the CTA returns, so a lost miss signal ends the launch instead of hanging.
+// Shared-expert units do not depend on routing: a CTA whose first unit is a shared one
+// loads the next layer's unit as soon as its buffer is free.  Every wait is bounded by a
+// globaltimer deadline; a wait that runs out sets the error word and the CTA returns, so
+// a lost miss signal ends the launch instead of hanging.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -51,6 +53,20 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* ptr) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
   return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* ptr) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* ptr, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_u64(unsigned long long* ptr, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(ptr), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ int32_t ld_volatile(const int32_t* ptr) {
@@ -82,26 +98,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bulk (non-tensor TMA) copy global -> shared; completion counted on bar in bytes.
-// dst, src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Same copy with an L2 cache policy: streamed expert and router weights are read once
-// per token, so they are marked evict-first and do not push the kernel's code and the
-// small exchange buffers out of L2.
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+// Bulk (non-tensor TMA) copy global -> shared with an L2 evict-first policy: streamed
+// expert and router weights are read once per token, so they do not push the kernel's
+// code and the small exchange buffers out of L2.  dst, src 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  const uint64_t pol = l2_evict_first_policy();
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
           "r"(smem_u32(dst)),
@@ -109,17 +112,13 @@ __device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint
       : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
+// Bulk prefetch of [src, src + bytes) into L2 (bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* ptr) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(uint32_t* ptr, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Two-way dot products: a holds two int16 (signed), b four uint8; .lo uses bytes 0-1,
@@ -136,8 +135,8 @@ __device__ __forceinline__ int dp2a_hi(int a, uint32_t b, int c) {
 }
 
 // 16 * sum_e q_e * c_e over one Q4_0 block: q from the 16 nibble bytes, c the block's 32
-// int16 codes packed in pairs (xw[m] = {c[2m], c[2m+1]}).  Low nibbles are weights 0-15,
-// high nibbles (kept in place, i.e. times 16) weights 16-31.
+// int16 codes packed in pairs (x0..x3 = codes 0-7, 8-15, 16-23, 24-31).  Low nibbles
+// are weights 0-15, high nibbles (kept in place, i.e. times 16) weights 16-31.
 __device__ __forceinline__ int q4_block_dot16(const uint4 q, const int4 x0, const int4 x1,
                                               const int4 x2, const int4 x3) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -169,17 +168,9 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-// Canonical fold of n partials (n <= 256, stride 1) by one warp; every lane returns
-// the total.  Lane l adds parts l, l+32, ... from +0 in that order, then the lanes
-// combine by xor-butterfly offsets 16, 8, 4, 2, 1.
-__device__ __forceinline__ float canonical_fold(const float* parts, int n, int lane) {
-  float v[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v[k] = lane + 32 * k < n ? __ldcg(parts + lane + 32 * k) : 0.0f;
-  float acc = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    if (lane + 32 * k < n) acc = __fadd_rn(acc, v[k]);
+// The canonical fold's last step: xor-butterfly offsets 16, 8, 4, 2, 1; every lane ends
+// with the total.
+__device__ __forceinline__ float butterfly_sum(float acc) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
   return acc;
@@ -225,10 +216,12 @@ __host__ __device__ inline int pow2_ceil_le32(int n) {
 // ------------------------------------------------------------------ shared memory plan
 
 struct Misc {
-  uint64_t bar_u[4];  // gate/up unit, four 16-row stages
-  uint64_t bar_r;     // next layer's router columns of the owned chunks
+  uint64_t bar_u[4];  // the four gate/up tiles of the unit in flight
+  uint64_t bar_d;     // its down part
+  uint64_t bar_r;     // this CTA's router rows of the current layer
   const uint8_t* src[kMaxK + 1];  // slot base of each active expert (rank order, then shared)
-  uint32_t miss_seq[kMaxK + 1];   // copy to wait for (0: resident)
+  uint32_t miss_seq[kMaxK + 1];   // proxy copy to wait for (0: none)
+  long long pull[kMaxK + 1];      // pull mode: the expert's byte offset in the host tier, or -1
   int32_t sel[kMaxK];
   float w[kMaxK];
   int32_t fix_dst[kMaxR], fix_src[kMaxR];  // deferred ring fills (pool indices)
@@ -236,25 +229,25 @@ struct Misc {
   int32_t ring_owner[kMaxR];
   uint32_t ring_stamp[kMaxR];
   uint32_t ring_clock;
-  float hown[kMaxOwn][kChunk];   // this CTA's rows of the residual stream
-  float gnext[kMaxOwn][kChunk];  // next layer's RMSNorm gain on those rows
-  float u[kChunk];
   float gu[2 * kUnitRows];
+  int4 acodes[4];  // the unit's activation block: 32 int16 codes in pairs
+  float asc;
+  int32_t acs;
   float inv;
-  uint32_t step, seq_base, n_miss, gen;
+  float bias[kWarps];  // router bias of this CTA's experts, current layer
+  uint32_t step, seq_base, n_miss;
   int32_t flag;
-  int32_t P_l, base_l;  // pinned count and pool base of the current layer
-  int32_t unit_ok;   // first gate/up unit issued
-  int32_t d_issued;  // down rows of the first owned chunk issued during routing
+  int32_t P_l, base_l;
+  int32_t pre;  // the first unit of the next layer was issued ahead (shared expert)
 };
 
 struct SmemPlan {
-  uint32_t unit, rchunk, hbuf, gbuf, pinrow, z, xcodes, xs, xc, o, misc, total;
+  uint32_t unit, rrows, h, g, up, xcodes, xs, xc, z, pinrow, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is, int nown) {
+__host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_late) {
   SmemPlan s;
   uint32_t off = 0;
   auto take = [&](uint32_t bytes) {
@@ -263,35 +256,33 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int K, int I, int Is
     off += bytes;
     return r;
   };
-  const int n_exp = K + (Is > 0);
-  const int imax = I > Is ? I : Is;
-  s.unit = take(36u * H);                        // gate qs|d, up qs|d for 32 rows
-  s.rchunk = take(32u * E * nown);               // router columns of the owned chunks
-  s.hbuf = take(4u * H);
-  s.gbuf = take(4u * H);
-  s.pinrow = take(4u * E);
-  s.z = take(4u * E);
+  const uint32_t nch = (uint32_t)H / kChunk;
+  s.unit = take((down_late ? 36u : 54u) * H);
+  s.rrows = take(2u * H * (uint32_t)rx);
+  s.h = take(4u * H);
+  s.g = take(4u * H);
+  s.up = take(4u * kChunk * 32u * ((nch + 31) / 32));
   s.xcodes = take(2u * H);
   s.xs = take(4u * (H / 32));
   s.xc = take(4u * (H / 32));
-  s.o = take(4u * n_exp * kChunk);
+  s.z = take(4u * E);
+  s.pinrow = take(4u * E);
   s.misc = take(sizeof(Misc));
   s.total = align_up(off, 128);
   return s;
 }
 
-// ------------------------------------------------------------------ barriers and waits
+// ------------------------------------------------------------------ waits
 
 // Out-of-line slow paths of the bounded waits: the common case (already there) stays
-// inline and short; the spin loops live in separate functions so that the code each
-// layer runs through stays small enough for the SM instruction cache.
+// inline; the spin loops live in separate functions so the per-layer code stays small
+// enough for the SM instruction cache.
 
 // Spin until *count >= target (acquire), with back-off; false on timeout / error.
 __device__ __noinline__ bool spin_count(const DecodeParams& p, const uint32_t* count, uint32_t target) {
   const uint64_t t0 = gtimer();
   for (uint32_t polls = 1; ld_acquire(count) < target; ++polls) {
-    __nanosleep(32);
-    if ((polls & 31u) == 0) {
+    if ((polls & 15u) == 0) {
       if (has_error(p.ctrl)) return false;
       if (gtimer() - t0 > p.timeout_ns) {
         set_error(p.ctrl, MOE_DEVERR_BARRIER);
@@ -302,48 +293,28 @@ __device__ __noinline__ bool spin_count(const DecodeParams& p, const uint32_t* c
   return true;
 }
 
-// Grid barrier over all CTAs (co-resident by cooperative launch).  The arrival counter
-// only grows during a launch (the graph zeroes it before the kernel), so barrier b of
-// the launch completes when it reaches (b + 1) * gridDim.x.  Returns false when the
-// wait ran out or another CTA flagged an error.
-__device__ bool grid_sync(const DecodeParams& p, Misc& m) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t target = (m.gen + 1) * gridDim.x;
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
-    int ok = ld_acquire(&p.ctrl->bar_count) >= target || spin_count(p, &p.ctrl->bar_count, target);
-    m.gen += 1;
-    m.flag = ok;
+__device__ __forceinline__ bool wait_count(const DecodeParams& p, const uint32_t* count, uint32_t target) {
+  return ld_acquire(count) >= target || spin_count(p, count, target);
+}
+
+// Spin until the published logit word carries epoch; false on timeout / error.
+__device__ __noinline__ bool spin_logit(const DecodeParams& p, const unsigned long long* w, uint32_t epoch,
+                                        unsigned long long* out) {
+  const uint64_t t0 = gtimer();
+  for (uint32_t polls = 1;; ++polls) {
+    const unsigned long long v = ld_relaxed_u64(w);
+    if ((uint32_t)(v >> 32) == epoch) {
+      *out = v;
+      return true;
+    }
+    if ((polls & 15u) == 0) {
+      if (has_error(p.ctrl)) return false;
+      if (gtimer() - t0 > p.timeout_ns) {
+        set_error(p.ctrl, MOE_DEVERR_BARRIER);
+        return false;
+      }
+    }
   }
-  __syncthreads();
-  return m.flag != 0;
-}
-
-__device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = gtimer();
-}
-
-// Per-CTA marks (every CTA, thread 0): after [(L+1)][32] come [L][gridDim][4] stamps.
-__device__ __forceinline__ void cta_stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && threadIdx.x == 0)
-    p.phase_trace[(size_t)(p.L + 1) * 32 + ((size_t)l * gridDim.x + blockIdx.x) * 4 + k] = gtimer();
-}
-
-// Counted exchange: a producer CTA publishes with one release add after its stores;
-// a consumer CTA's thread 0 waits (with back-off) until the count reaches target, then
-// the CTA reads the data.  Only producers arrive and only consumers wait.
-__device__ __forceinline__ void publish(const DecodeParams& p, uint32_t* count) {
-  __syncthreads();
-  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
-}
-
-__device__ bool await_count(const DecodeParams& p, Misc& m, const uint32_t* count, uint32_t target) {
-  if (threadIdx.x == 0) {
-    const int ok = ld_acquire(count) >= target || spin_count(p, count, target);
-    m.flag = ok && !has_error(p.ctrl);
-  }
-  __syncthreads();
-  return m.flag != 0;
 }
 
 // Thread 0: wait until the proxy has signalled miss copy seq (0: nothing to wait for).
@@ -362,7 +333,7 @@ __device__ __noinline__ bool spin_miss(const DecodeParams& p, uint32_t seq) {
 __device__ __forceinline__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
   if (seq == 0) return true;
   if ((int32_t)(ld_acquire(p.done_seq) - seq) < 0 && !spin_miss(p, seq)) return false;
-  fence_proxy_async();
+  fence_proxy_async();  // the copy engine's writes, then bulk-copy reads of the same slot
   return true;
 }
 
@@ -382,46 +353,23 @@ __device__ __forceinline__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, 
   return mbar_try_wait(bar, parity) || spin_mbar(p, bar, parity);
 }
 
-// CTA-uniform check of the error word: one thread reads it, everyone acts on that read
-// (threads reading it themselves could disagree and split at the next barrier).
-__device__ __forceinline__ bool cta_ok(const DecodeParams& p, int32_t& flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) flag = !has_error(p.ctrl);
-  __syncthreads();
-  return flag != 0;
+// Barrier + agreement: true when every thread of the CTA passed ok, so that the CTA
+// leaves as a whole.  A failure elsewhere in the grid reaches this CTA through its own
+// bounded waits (every spin loop also watches the error word), so the common path reads
+// no global memory here.
+__device__ __forceinline__ bool cta_ok(const DecodeParams&, bool ok) { return __syncthreads_and(ok) != 0; }
+
+__device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
+  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = gtimer();
 }
 
-// ------------------------------------------------------------------ phases
-
-// Router partials of layer l over chunk c (16 columns): every thread e folds
-// w[e][t] * u_t, u_t = g_t * h_t (g = 1 without a gain; u = h without the norm), from
-// +0 in ascending column order; plus the chunk's sum of squares of h.  wrow(e) points
-// at the 16 bf16 weights of expert e for this chunk (global or shared memory).
-template <typename WRow>
-__device__ void router_partials(const DecodeParams& p, Misc& m, int c, const float* hv, const float* gv,
-                                WRow wrow) {
-  const int tid = threadIdx.x;
-  if (tid < kChunk) m.u[tid] = (p.use_norm && gv) ? __fmul_rn(gv[tid], hv[tid]) : hv[tid];
-  __syncthreads();
-  for (int e = tid; e < p.E; e += kThreads) {
-    const uint4* wp = wrow(e);
-    const uint4 w0 = wp[0], w1 = wp[1];
-    const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    float acc = 0.0f;
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      acc = fmaf(bf16_lo(ws[t]), m.u[2 * t], acc);
-      acc = fmaf(bf16_hi(ws[t]), m.u[2 * t + 1], acc);
-    }
-    __stcg(p.part + (size_t)e * p.nch + c, acc);
-  }
-  if (tid == 0 && p.use_norm) {
-    float s = 0.0f;
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) s = fmaf(hv[t], hv[t], s);
-    __stcg(p.sq + c, s);
-  }
+// Per-CTA marks (every CTA, thread 0): after [(L+1)][32] come [L][gridDim][4] stamps.
+__device__ __forceinline__ void cta_stamp(const DecodeParams& p, int l, int k) {
+  if (p.phase_trace && threadIdx.x == 0)
+    p.phase_trace[(size_t)(p.L + 1) * 32 + ((size_t)l * gridDim.x + blockIdx.x) * 4 + k] = gtimer();
 }
+
+// ------------------------------------------------------------------ routing
 
 // Top-k for more than 256 experts: keys re-read from shared memory every round.
 __device__ __noinline__ int topk_large(const DecodeParams& p, const float* zs) {
@@ -449,7 +397,7 @@ __device__ __noinline__ int topk_large(const DecodeParams& p, const float* zs) {
 
 // Warp 0: top-k of z (value desc, index asc) and the renormalised softmax weights.
 // Keys live in registers (E <= 256: 8 per lane); each round is a lane-local max and a
-// 64-bit butterfly max.  Lane i returns the expert of rank i (and m.sel / m.w are set).
+// redux max / min.  Lane i returns the expert of rank i (and m.sel / m.w are set).
 __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
   const int lane = threadIdx.x & 31;
   const int E = p.E;
@@ -496,7 +444,8 @@ __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
 
 // Thread 0 of every CTA: the cache decision for layer l (identical in all CTAs), from
 // the layer's pinned-slot row and ring state staged in shared memory.  CTA 0 also
-// commits the next ring state, the event log, histogram, counters and miss requests.
+// commits the next ring state, the event log, histogram, counters and (proxy mode) the
+// miss requests.
 __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow) {
   const int R = p.R, K = p.K;
   const int par = m.step & 1;
@@ -516,6 +465,7 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
     const int ps = pinrow[e];
     int kind, slot_log, evicted = -1, pool_idx;
     uint32_t seq = 0;
+    long long pull = -1;
     if (ps >= 0) {  // (logical slot << 16) | physical slot within the layer's pinned region
       kind = MOE_PIN_HIT;
       slot_log = ps >> 16;
@@ -551,7 +501,6 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
         m.ring_stamp[v] = ++clock;
         kind = MOE_MISS;
         slot_log = P + v;
-        seq = m.seq_base + 1 + m.n_miss++;
         if (busy[v]) {  // slot still read by an earlier rank of this layer: stage
           pool_idx = p.staging_base + i;
           fix[v] = pool_idx;
@@ -563,20 +512,26 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
         }
         ++n_miss;
         if (evicted >= 0) ++n_evict;
-        if (commit) {
-          MissReq* q = p.mbox + (seq % kMboxCap);
-          volatile uint32_t* qv = reinterpret_cast<volatile uint32_t*>(q);
-          qv[1] = (uint32_t)l;
-          qv[2] = (uint32_t)e;
-          qv[3] = (uint32_t)pool_idx;
-          __threadfence_system();
-          qv[0] = seq;
-          __threadfence_system();
+        if (p.miss_mode == kMissPull) {
+          pull = (long long)(((size_t)l * p.E + e) * p.slot_bytes);
+        } else {
+          seq = m.seq_base + 1 + m.n_miss++;
+          if (commit) {
+            MissReq* q = p.mbox + (seq % kMboxCap);
+            volatile uint32_t* qv = reinterpret_cast<volatile uint32_t*>(q);
+            qv[1] = (uint32_t)l;
+            qv[2] = (uint32_t)e;
+            qv[3] = (uint32_t)pool_idx;
+            __threadfence_system();
+            qv[0] = seq;
+            __threadfence_system();
+          }
         }
       }
     }
     m.src[i] = p.pool + (size_t)pool_idx * p.slot_bytes;
     m.miss_seq[i] = seq;
+    m.pull[i] = pull;
     if (commit) {
       int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * K + i) * 7;
       ev[0] = (int32_t)m.step;
@@ -588,10 +543,6 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
       ev[6] = evicted;
       atomicAdd(p.hist + (size_t)l * p.E + e, 1u);
     }
-  }
-  if (p.Is > 0) {
-    m.src[K] = p.shared_pool + (size_t)l * p.shared_slot_bytes;
-    m.miss_seq[K] = 0;
   }
   m.n_fix = 0;
   for (int r = 0; r < R; ++r)
@@ -612,14 +563,8 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
     atomicAdd(&p.ctrl->misses, n_miss);
     atomicAdd(&p.ctrl->evictions, n_evict);
     atomicAdd(&p.ctrl->staged, n_staged);
+    if (p.miss_mode == kMissPull) atomicAdd(&p.ctrl->pulled, n_miss);
   }
-}
-
-// Layer 0's router partials over chunk c from global router weights (once per launch).
-__device__ __noinline__ void prologue_partials(const DecodeParams& p, Misc& m, int c, int k, bool has_gain) {
-  router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
-    return reinterpret_cast<const uint4*>(p.router + ((size_t)c * p.E + e) * kChunk);
-  });
 }
 
 // Warp 0: the common case where every selected expert is pinned; lane i handles rank
@@ -632,6 +577,7 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
   if (lane < p.K) {
     m.src[lane] = p.pool + (size_t)(m.base_l + (ps & 0xffff)) * p.slot_bytes;
     m.miss_seq[lane] = 0;
+    m.pull[lane] = -1;
     if (commit) {
       int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * p.K + lane) * 7;
       ev[0] = (int32_t)m.step;
@@ -651,10 +597,6 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
     p.ring_stamp[ws + lane] = m.ring_stamp[lane];
   }
   if (lane == 0) {
-    if (p.Is > 0) {
-      m.src[p.K] = p.shared_pool + (size_t)l * p.shared_slot_bytes;
-      m.miss_seq[p.K] = 0;
-    }
     m.n_fix = 0;
     if (commit) {
       p.ring_clock[(size_t)((m.step & 1) ^ 1) * p.L + l] = m.ring_clock;
@@ -665,47 +607,88 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
   return true;
 }
 
-// Thread 0: bulk-load gate/up unit u (32 rows of gate and of up of one expert) into
-// shared memory as four 16-row tiles, one bulk copy each, after its miss copy (if any)
-// has landed.
-__device__ bool issue_unit(const DecodeParams& p, Misc& m, uint8_t* unit, int u) {
-  const int per = p.I / 32, routed = p.K * per;
-  const int i = u < routed ? u / per : p.K;
-  const int rb = u < routed ? u % per : u - routed;
-  const SlotLayout& L = i < p.K ? p.lay : p.slay;
-  if (!wait_miss(p, m.miss_seq[i])) return false;
+// ------------------------------------------------------------------ units
+
+// Thread 0: bulk-load a unit (src = its first byte in a slot) into the unit buffer:
+// four gate/up tiles on bar_u[0..3] and, unless the down part comes later, the down
+// nibbles and scales (one run of 18H bytes) on bar_d.
+__device__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src) {
   const uint32_t tb = 9u * p.H;
-  const uint8_t* src = m.src[i] + L.gu + (size_t)rb * 4 * tb;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
     mbar_expect_tx(&m.bar_u[st], tb);
-    bulk_g2s_stream(unit + st * tb, src + st * tb, tb, &m.bar_u[st]);
+    bulk_g2s_stream(ubuf + st * tb, src + st * tb, tb, &m.bar_u[st]);
   }
-  return true;
-}
-
-// All threads: pull the down tiles of chunk c of every resident active expert into L2
-// (one prefetch per 128-byte line), so that the down phase reads them from L2.
-__device__ void prefetch_dchunk_l2(const DecodeParams& p, const Misc& m, int c) {
-  const uint32_t t_r = 9u * p.I, t_s = 9u * p.Is;
-  const uint32_t routed_bytes = (uint32_t)p.K * t_r, total = routed_bytes + (p.Is > 0 ? t_s : 0);
-  for (uint32_t off = 128u * threadIdx.x; off < total; off += 128u * kThreads) {
-    const int i = off < routed_bytes ? (int)(off / t_r) : p.K;
-    if (m.miss_seq[i] != 0) continue;  // its slot is still being filled
-    const uint32_t in_tile = off < routed_bytes ? off - (uint32_t)i * t_r : off - routed_bytes;
-    const SlotLayout& L = i < p.K ? p.lay : p.slay;
-    const uint8_t* src = m.src[i] + L.down + (size_t)c * (i < p.K ? t_r : t_s) + in_tile;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+  if (!p.down_late) {
+    mbar_expect_tx(&m.bar_d, 18u * p.H);
+    bulk_g2s_stream(ubuf + 36u * p.H, src + 36u * p.H, 18u * p.H, &m.bar_d);
   }
 }
 
-// Thread 0: bulk-load layer lr's router columns of the owned chunks into rch.
-__device__ void prefetch_router(const DecodeParams& p, Misc& m, uint8_t* rch, int lr, int n_own) {
-  mbar_expect_tx(&m.bar_r, 32u * p.E * n_own);
-  for (int k = 0; k < n_own; ++k) {
-    const int c = blockIdx.x + k * gridDim.x;
-    bulk_g2s_stream(rch + (size_t)k * 32u * p.E, p.router + (((size_t)lr * p.nch + c) * p.E) * kChunk, 32u * p.E,
-                    &m.bar_r);
+// All threads: copy a unit from the mapped pinned host tier into its slot (pull mode),
+// then order those writes before the bulk copies that read the slot back.
+__device__ void pull_unit(const DecodeParams& p, const uint8_t* host, uint8_t* dst) {
+  const uint4* s = reinterpret_cast<const uint4*>(host);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  const uint32_t n16 = (uint32_t)(p.unit_bytes / 16);
+  constexpr int kBatch = 8;
+  for (uint32_t base = threadIdx.x; base < n16; base += kThreads * kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const uint32_t t = base + k * kThreads;
+      if (t < n16) v[k] = __ldcv(s + t);
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const uint32_t t = base + k * kThreads;
+      if (t < n16) __stcg(d + t, v[k]);
+    }
+  }
+  fence_proxy_async();
+}
+
+// One thread: this CTA's share of a layer's speculative prefetch: the slots of the
+// layer's most frequently routed pinned experts (slots, loaded beforehand), as one byte
+// range split evenly over the grid.
+__device__ void prefetch_likely(const DecodeParams& p, const int32_t (&slots)[kMaxLikely]) {
+  const uint64_t sb = p.slot_bytes, total = (uint64_t)p.n_likely * sb;
+  const uint64_t per = ((total + gridDim.x - 1) / gridDim.x + 255) / 256 * 256;
+  uint64_t lo = (uint64_t)blockIdx.x * per;
+  const uint64_t hi = lo + per < total ? lo + per : total;
+  while (lo < hi) {
+    const int m = (int)(lo / sb);
+    const uint64_t in = lo - (uint64_t)m * sb, end = (uint64_t)(m + 1) * sb < hi ? (uint64_t)(m + 1) * sb : hi;
+    int32_t slot = -1;
+#pragma unroll
+    for (int q = 0; q < kMaxLikely; ++q)
+      if (q == m) slot = slots[q];
+    if (slot >= 0) bulk_prefetch_l2(p.pool + (size_t)slot * sb + in, (uint32_t)(end - lo));
+    lo = end;
+  }
+}
+
+// All threads: h += y (or h = y without the residual) from a layer's accumulator; all of
+// a thread's loads are issued before any of them is used (one L2 round trip, not one
+// per element).  trace: where to write the new h, or null.
+__device__ __forceinline__ void add_layer_output(const DecodeParams& p, const unsigned long long* acc, float* hs,
+                                                 float* trace) {
+  constexpr int kPer = kMaxH / kThreads;  // 16
+  long long v[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int j = threadIdx.x + k * kThreads;
+    v[k] = j < p.H ? (long long)__ldcg(acc + j) : 0;
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int j = threadIdx.x + k * kThreads;
+    if (j < p.H) {
+      const float y = __ll2float_rn(v[k]) * kAccInvScale;
+      const float hn = p.use_norm ? __fadd_rn(hs[j], y) : y;
+      hs[j] = hn;
+      if (trace) trace[j] = hn;
+    }
   }
 }
 
@@ -714,83 +697,86 @@ __device__ void prefetch_router(const DecodeParams& p, Misc& m, uint8_t* rch, in
 template <int BPL>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const SmemPlan S = smem_plan(p.H, p.E, p.K, p.I, p.Is, p.nown);
+  const SmemPlan S = smem_plan(p.H, p.E, p.rx_per_cta, p.down_late);
   Misc& m = *reinterpret_cast<Misc*>(smem + S.misc);
-  float* zs = reinterpret_cast<float*>(smem + S.z);
-  float* hbuf = reinterpret_cast<float*>(smem + S.hbuf);
-  float* gbuf = reinterpret_cast<float*>(smem + S.gbuf);
-  int32_t* pinrow = reinterpret_cast<int32_t*>(smem + S.pinrow);
+  uint8_t* ubuf = smem + S.unit;
+  const uint16_t* rrows = reinterpret_cast<const uint16_t*>(smem + S.rrows);
+  float* hs = reinterpret_cast<float*>(smem + S.h);
+  float* gs = reinterpret_cast<float*>(smem + S.g);
+  float* up = reinterpret_cast<float*>(smem + S.up);
   int16_t* xcodes = reinterpret_cast<int16_t*>(smem + S.xcodes);
   float* xs = reinterpret_cast<float*>(smem + S.xs);
   int32_t* xc = reinterpret_cast<int32_t*>(smem + S.xc);
-  float* os = reinterpret_cast<float*>(smem + S.o);
-  uint8_t* unit = smem + S.unit;
-  uint8_t* rch = smem + S.rchunk;
+  float* zs = reinterpret_cast<float*>(smem + S.z);
+  int32_t* pinrow = reinterpret_cast<int32_t*>(smem + S.pinrow);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, nb = H / 32;
-  const int imax = p.I > p.Is ? p.I : p.Is;
-  const int rec_per_exp = imax / 32;
+  const int G = gridDim.x, b = blockIdx.x;
+  const int H = p.H, nb = H / 32, nch = H / kChunk;
+  const int routed = p.K * (p.I / 32);
   const bool has_gain = p.use_norm && p.gain;
-  int n_own = 0;  // chunks of h owned by this CTA
-  while (n_own < p.nown && (int)blockIdx.x + n_own * (int)gridDim.x < p.nch) ++n_own;
+  const int nrx = b < p.E ? min(p.rx_per_cta, (p.E - b + G - 1) / G) : 0;  // my router experts b, b+G, ...
+  const bool first_shared = b < p.n_units && b >= routed;  // my first unit does not depend on routing
+  const uint32_t gbase = 0;  // arrival counter starts at 0 every launch
+  uint32_t par_u[4] = {0, 0, 0, 0}, par_d = 0, par_r = 0;  // mbarrier parities (uniform)
+  bool ok = true;
 
   if (tid == 0) {
-    for (int b = 0; b < 4; ++b) mbar_init(&m.bar_u[b], 1);
+    for (int k = 0; k < 4; ++k) mbar_init(&m.bar_u[k], 1);
+    mbar_init(&m.bar_d, 1);
     mbar_init(&m.bar_r, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     m.step = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->step);
     m.seq_base = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->req_seq);
-    m.gen = 0;
     m.n_miss = 0;
-    m.flag = !has_error(p.ctrl);
+    m.n_fix = 0;
+    m.pre = 0;
   }
-  __syncthreads();
-  if (!m.flag) return;
-  uint32_t par_u[4] = {0, 0, 0, 0}, par_r = 0;  // mbarrier parities (uniform)
   stamp(p, p.L, 0);
+  if (!cta_ok(p, true)) goto fail;
 
-  // ---- prologue: h = x on the owned rows, and layer 0's router partials
-  for (int k = 0; k < n_own; ++k) {
-    const int c = blockIdx.x + k * gridDim.x;
-    if (tid < kChunk) {
-      const float v = p.x[c * kChunk + tid];
-      m.hown[k][tid] = v;
-      m.gnext[k][tid] = has_gain ? p.gain[c * kChunk + tid] : 1.0f;
-      __stcg(p.h + c * kChunk + tid, v);
-      if (p.h_trace) p.h_trace[c * kChunk + tid] = v;
+  // ---- prologue: accumulators 0 and 1 and the logit words zeroed, h = x, first loads
+  for (int j = b * kThreads + tid; j < 2 * H; j += G * kThreads) p.acc[j] = 0ull;
+  for (int e = b * kThreads + tid; e < p.E; e += G * kThreads) p.zll[e] = 0ull;
+  for (int j = tid; j < H; j += kThreads) hs[j] = __ldg(p.x + j);
+  if (tid == 0) {
+    if (nrx > 0) {
+      mbar_expect_tx(&m.bar_r, 2u * H * nrx);
+      for (int k = 0; k < nrx; ++k)
+        bulk_g2s_stream(const_cast<uint16_t*>(rrows) + (size_t)k * H, p.router + (size_t)(b + k * G) * H, 2u * H,
+                        &m.bar_r);
     }
-    __syncthreads();
-    prologue_partials(p, m, c, k, has_gain);
-    __syncthreads();
+    if (first_shared) {
+      issue_unit(p, m, ubuf, p.shared_pool + (size_t)(b - routed) * p.unit_bytes);
+      m.pre = 1;
+    }
   }
-  if (tid == 0 && p.L > 1 && n_own > 0) prefetch_router(p, m, rch, 1, n_own);
-  if (!grid_sync(p, m)) return;
+  int32_t lk[kMaxLikely];  // thread 32: the likely experts' slots of the current layer
+  if (tid == 32 && p.n_likely > 0) {
+#pragma unroll
+    for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely + q);
+    prefetch_likely(p, lk);
+  }
+  if (b == 0 && p.h_trace)
+    for (int j = tid; j < H; j += kThreads) p.h_trace[j] = hs[j];
+  __syncthreads();
+  if (tid == 0) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
+    ok = wait_count(p, &p.ctrl->bar_count, gbase + G);
+  }
+  if (!cta_ok(p, ok)) goto fail;
   stamp(p, p.L, 1);
 
   for (int l = 0; l < p.L; ++l) {
     stamp(p, l, 0);
     const bool next = l + 1 < p.L;
-    // ---------------------------------------------------------------- R phase
-    // stage this layer's inputs: every load of the phase is issued before any is used
-    float4 hreg[4], greg[4];
-    int32_t preg[4];
+    // ---------------------------------------------------------------- layer inputs
+    // loads that do not depend on the previous layer go out first
     {
-      const float4* h4 = reinterpret_cast<const float4*>(p.h);
       const float4* g4 = has_gain ? reinterpret_cast<const float4*>(p.gain + (size_t)l * H) : nullptr;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = tid + q * kThreads;
-        if (t < H / 4) {
-          hreg[q] = __ldcg(h4 + t);
-          if (has_gain) greg[q] = __ldg(g4 + t);
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = tid + q * kThreads;
-        if (e < p.E) preg[q] = __ldg(p.pin_slot + (size_t)l * p.E + e);
-      }
+      for (int t = tid; t < H / 4; t += kThreads)
+        reinterpret_cast<float4*>(gs)[t] = has_gain ? __ldg(g4 + t) : make_float4(1.f, 1.f, 1.f, 1.f);
+      for (int e = tid; e < p.E; e += kThreads) pinrow[e] = __ldg(p.pin_slot + (size_t)l * p.E + e);
       const int par = m.step & 1;
       const size_t rs = ((size_t)par * p.L + l) * p.R;
       if (tid < p.R) {
@@ -800,70 +786,136 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (tid == kThreads - 1) m.ring_clock = __ldcg(p.ring_clock + (size_t)par * p.L + l);
       if (tid == kThreads - 2) m.P_l = __ldg(p.n_pinned + l);
       if (tid == kThreads - 3) m.base_l = __ldg(p.layer_base + l);
-      if (next && tid < n_own * kChunk) {
-        const int k = tid / kChunk, t = tid % kChunk;
-        const int c = blockIdx.x + k * gridDim.x;
-        m.gnext[k][t] = has_gain ? __ldg(p.gain + (size_t)(l + 1) * H + c * kChunk + t) : 1.0f;
+      if (tid < nrx) m.bias[tid] = p.bias ? __ldg(p.bias + (size_t)l * p.E + b + tid * G) : 0.0f;
+      if (tid == 32 && p.n_likely > 0 && l > 0) {
+#pragma unroll
+        for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely + (size_t)l * kMaxLikely + q);
       }
     }
-    // logits of this CTA's experts (and the norm scale, in every CTA)
-    {
-      float inv = 1.0f;
-      if (p.use_norm) {
-        const float ss = canonical_fold(p.sq, p.nch, lane);
-        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), p.eps)));
+    if (l > 0) {
+      // ---------------------------------------------------------------- h += y(l - 1)
+      if (tid == 0) ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G);
+      // the HBM is idle until this layer's routing is known: fetch its likely experts
+      // (a thread off the critical path, after the wait)
+      if (tid == 32 && p.n_likely > 0) {
+        if (wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G)) prefetch_likely(p, lk);
       }
-      if (warp == 0 && lane == 0) m.inv = inv;
-      for (int e = blockIdx.x * kWarps + warp; e < p.E; e += gridDim.x * kWarps) {
-        const float sum = canonical_fold(p.part + (size_t)e * p.nch, p.nch, lane);
-        if (lane == 0) __stcg(p.z + e, fmaf(sum, inv, p.bias ? __ldg(p.bias + (size_t)l * p.E + e) : 0.0f));
+      if (!cta_ok(p, ok)) goto fail;
+      stamp(p, l, 1);
+      add_layer_output(p, p.acc + (size_t)((l - 1) % kAccBufs) * H, hs,
+                       (b == 0 && p.h_trace) ? p.h_trace + (size_t)l * H : nullptr);
+      // deferred ring fills of layer l - 1 (a layer that missed more often than it has
+      // ring slots): its readers are done
+      for (int f = 0; f < m.n_fix; ++f) {
+        const uint4* s = reinterpret_cast<const uint4*>(p.pool + (size_t)m.fix_src[f] * p.slot_bytes);
+        uint4* d = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) + (size_t)m.fix_dst[f] * p.slot_bytes);
+        const size_t n16 = p.slot_bytes / 16;
+        for (size_t t = (size_t)b * kThreads + tid; t < n16; t += (size_t)G * kThreads) d[t] = __ldcg(s + t);
       }
-    }
-    const int n_folders = min((int)gridDim.x, (p.E + kWarps - 1) / kWarps);  // CTAs holding logits
-    if ((int)blockIdx.x < n_folders) publish(p, &p.ctrl->z_count);
-    {
-      float4* hb4 = reinterpret_cast<float4*>(hbuf);
-      float4* gb4 = reinterpret_cast<float4*>(gbuf);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = tid + q * kThreads;
-        if (t < H / 4) {
-          hb4[t] = hreg[q];
-          if (has_gain) gb4[t] = greg[q];
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = tid + q * kThreads;
-        if (e < p.E) pinrow[e] = preg[q];
+      // the accumulator of layer l + 1 was last read at the start of layer l - 1, by CTAs
+      // that have all published layer l - 1's logits since
+      if (next) {
+        unsigned long long* z = p.acc + (size_t)((l + 1) % kAccBufs) * H;
+        for (int j = b * kThreads + tid; j < H; j += G * kThreads) z[j] = 0ull;
       }
     }
     __syncthreads();
-    // quantised activations x = RMSNorm(h) (or h): four lanes per 32-block, each lane 8
+    stamp(p, l, 2);
+
+    // ---------------------------------------------------------------- norm and router
+    // inv = 1 / sqrt(ss / H + eps), ss folded canonically from 16-column fmaf chunks
+    if (warp == 0) {
+      float inv = 1.0f;
+      if (p.use_norm) {
+        float acc = 0.0f;
+        for (int c = lane; c < nch; c += 32) {
+          const float4* h4 = reinterpret_cast<const float4*>(hs + c * kChunk);
+          float pc = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 v = h4[q];
+            pc = fmaf(v.x, v.x, pc);
+            pc = fmaf(v.y, v.y, pc);
+            pc = fmaf(v.z, v.z, pc);
+            pc = fmaf(v.w, v.w, pc);
+          }
+          acc = __fadd_rn(acc, pc);
+        }
+        const float ss = butterfly_sum(acc);
+        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), p.eps)));
+      }
+      if (lane == 0) m.inv = inv;
+    }
+    // router input u = g * h in the lane-major order the canonical fold reads: column
+    // 16 c + 4 q + r, c = lane + 32 m, at float4 (4 m + q) * 32 + lane, component r
+    for (int j = tid; j < H; j += kThreads) {
+      const int c = j >> 4, t = j & 15;
+      const float u = p.use_norm ? __fmul_rn(gs[j], hs[j]) : hs[j];
+      up[((((c >> 5) * 4 + (t >> 2)) * 32 + (c & 31)) << 2) + (t & 3)] = u;
+    }
+    __syncthreads();
+    stamp(p, l, 10);
+    // logits of my experts: warp k folds expert b + k G in the canonical order
+    if (warp < nrx) {
+      if (!__all_sync(0xffffffffu, ok && mbar_wait(p, &m.bar_r, par_r))) ok = false;
+      if (ok) {
+        const uint16_t* wr = rrows + (size_t)warp * H;
+        float acc = 0.0f;
+        for (int mm = 0; mm * 32 < nch; ++mm) {
+          const int c = lane + 32 * mm;
+          if (c < nch) {
+            const uint4 w0 = *reinterpret_cast<const uint4*>(wr + c * kChunk);
+            const uint4 w1 = *reinterpret_cast<const uint4*>(wr + c * kChunk + 8);
+            const float4* u4 = reinterpret_cast<const float4*>(up) + (mm * 4) * 32 + lane;
+            const float4 u0 = u4[0], u1 = u4[32], u2 = u4[64], u3 = u4[96];
+            float pc = 0.0f;
+            pc = fmaf(bf16_lo(w0.x), u0.x, pc);
+            pc = fmaf(bf16_hi(w0.x), u0.y, pc);
+            pc = fmaf(bf16_lo(w0.y), u0.z, pc);
+            pc = fmaf(bf16_hi(w0.y), u0.w, pc);
+            pc = fmaf(bf16_lo(w0.z), u1.x, pc);
+            pc = fmaf(bf16_hi(w0.z), u1.y, pc);
+            pc = fmaf(bf16_lo(w0.w), u1.z, pc);
+            pc = fmaf(bf16_hi(w0.w), u1.w, pc);
+            pc = fmaf(bf16_lo(w1.x), u2.x, pc);
+            pc = fmaf(bf16_hi(w1.x), u2.y, pc);
+            pc = fmaf(bf16_lo(w1.y), u2.z, pc);
+            pc = fmaf(bf16_hi(w1.y), u2.w, pc);
+            pc = fmaf(bf16_lo(w1.z), u3.x, pc);
+            pc = fmaf(bf16_hi(w1.z), u3.y, pc);
+            pc = fmaf(bf16_lo(w1.w), u3.z, pc);
+            pc = fmaf(bf16_hi(w1.w), u3.w, pc);
+            acc = __fadd_rn(acc, pc);
+          }
+        }
+        const float S_e = butterfly_sum(acc);
+        if (lane == 0) {
+          const int e = b + warp * G;
+          const float z = fmaf(S_e, m.inv, m.bias[warp]);
+          st_relaxed_u64(p.zll + e, ((unsigned long long)(uint32_t)(l + 1) << 32) | __float_as_uint(z));
+          if (warp == 0) stamp(p, l, 11);
+        }
+      }
+    }
+    // quantised expert input x = RMSNorm(h) (or h): four lanes per 32-block, each lane 8
     // values; the block's largest |x| and code sum combine over the four lanes
     {
       const float inv = m.inv;
       const int j4 = tid & 3;
       for (int b0 = tid >> 2; b0 < ((nb + 63) / 64) * 64; b0 += kThreads / 4) {
-        const int b = b0 < nb ? b0 : nb - 1;  // lanes past the end repeat a block, write nothing
+        const int bb = b0 < nb ? b0 : nb - 1;  // lanes past the end repeat a block, write nothing
         float v[8];
-        const float4* h4 = reinterpret_cast<const float4*>(hbuf + b * 32 + 8 * j4);
-        const float4* g4 = reinterpret_cast<const float4*>(gbuf + b * 32 + 8 * j4);
+        const float4* h4 = reinterpret_cast<const float4*>(hs + bb * 32 + 8 * j4);
+        const float4* g4 = reinterpret_cast<const float4*>(gs + bb * 32 + 8 * j4);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           float4 hv = h4[q];
           if (p.use_norm) {
-            hv.x = __fmul_rn(hv.x, inv);
-            hv.y = __fmul_rn(hv.y, inv);
-            hv.z = __fmul_rn(hv.z, inv);
-            hv.w = __fmul_rn(hv.w, inv);
-            if (has_gain) {
-              const float4 gv = g4[q];
-              hv.x = __fmul_rn(hv.x, gv.x);
-              hv.y = __fmul_rn(hv.y, gv.y);
-              hv.z = __fmul_rn(hv.z, gv.z);
-              hv.w = __fmul_rn(hv.w, gv.w);
-            }
+            const float4 gv = g4[q];
+            hv.x = __fmul_rn(__fmul_rn(hv.x, inv), gv.x);
+            hv.y = __fmul_rn(__fmul_rn(hv.y, inv), gv.y);
+            hv.z = __fmul_rn(__fmul_rn(hv.z, inv), gv.z);
+            hv.w = __fmul_rn(__fmul_rn(hv.w, inv), gv.w);
           }
           v[4 * q] = hv.x;
           v[4 * q + 1] = hv.y;
@@ -886,276 +938,245 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         csum += __shfl_xor_sync(0xffffffffu, csum, 1);
         csum += __shfl_xor_sync(0xffffffffu, csum, 2);
         if (b0 < nb) {
-          reinterpret_cast<uint4*>(xcodes + b * 32)[j4] =
+          reinterpret_cast<uint4*>(xcodes + bb * 32)[j4] =
               make_uint4(((uint32_t)c[0] & 0xffffu) | ((uint32_t)c[1] << 16),
                          ((uint32_t)c[2] & 0xffffu) | ((uint32_t)c[3] << 16),
                          ((uint32_t)c[4] & 0xffffu) | ((uint32_t)c[5] << 16),
                          ((uint32_t)c[6] & 0xffffu) | ((uint32_t)c[7] << 16));
           if (j4 == 0) {
-            xs[b] = amax * (1.0f / (32767.0f * 16.0f));
-            xc[b] = csum;
+            xs[bb] = amax * (1.0f / (32767.0f * 16.0f));
+            xc[bb] = csum;
           }
         }
       }
     }
-    __syncthreads();
-    stamp(p, l, 1);
+    stamp(p, l, 12);
+    if (!cta_ok(p, ok)) goto fail;
+    stamp(p, l, 3);
+    // this layer's router rows are read: the buffer takes the next layer's
+    if (nrx > 0) {
+      if (tid == 0 && next) {
+        mbar_expect_tx(&m.bar_r, 2u * H * nrx);
+        for (int k = 0; k < nrx; ++k)
+          bulk_g2s_stream(const_cast<uint16_t*>(rrows) + (size_t)k * H,
+                          p.router + ((size_t)(l + 1) * p.E + b + k * G) * H, 2u * H, &m.bar_r);
+      }
+      par_r ^= 1u;
+    }
 
     // ---------------------------------------------------------------- routing
-    if (!await_count(p, m, &p.ctrl->z_count, (uint32_t)(l + 1) * n_folders)) return;
-    for (int e = tid; e < p.E; e += kThreads) zs[e] = __ldcg(p.z + e);
-    if (!cta_ok(p, m.flag)) return;
-    stamp(p, l, 8);
-    if (warp == 0) {
-      const int my_e = topk_weights(p, m, zs);
-      stamp(p, l, 9);
-      const bool fast = cache_all_pinned(p, m, l, pinrow, my_e);
-      if (lane == 0) {
-        if (!fast) cache_decide(p, m, l, pinrow);
-        stamp(p, l, 10);
-        m.unit_ok = (int)blockIdx.x < p.n_units ? issue_unit(p, m, unit, blockIdx.x) : 1;
-        stamp(p, l, 11);
-        m.d_issued = 0;
-        stamp(p, l, 12);
+    {
+      const uint32_t epoch = (uint32_t)(l + 1);
+      for (int e = tid; e < p.E; e += kThreads) {
+        unsigned long long v = ld_relaxed_u64(p.zll + e);
+        if ((uint32_t)(v >> 32) != epoch && !spin_logit(p, p.zll + e, epoch, &v)) {
+          ok = false;
+          break;
+        }
+        zs[e] = __uint_as_float((uint32_t)v);
       }
     }
+    if (!cta_ok(p, ok)) goto fail;
+    stamp(p, l, 4);
+    if (warp == 0) {
+      const int my_e = topk_weights(p, m, zs);
+      stamp(p, l, 13);
+      const bool fast = cache_all_pinned(p, m, l, pinrow, my_e);
+      if (lane == 0 && !fast) cache_decide(p, m, l, pinrow);
+      stamp(p, l, 14);
+    }
     __syncthreads();
-    if (!m.unit_ok) return;
-    if (blockIdx.x == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
-    for (int k = 0; k < n_own; ++k) prefetch_dchunk_l2(p, m, blockIdx.x + k * gridDim.x);
-    stamp(p, l, 2);
+    if (b == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
+    stamp(p, l, 5);
     cta_stamp(p, l, 0);
 
-    // ---------------------------------------------------------------- G phase
+    // ---------------------------------------------------------------- units
     {
-      // lane groups of GS lanes per row; each lane covers BPL blocks of the row
+      // this lane's blocks of the quantised input: lane groups of GS lanes per row,
+      // each lane BPL blocks of the row
       const int GS = pow2_ceil_le32(nb), RPW = 32 / GS, g = lane % GS, sub = lane / GS;
-      const int rows_per_lane = (2 * kUnitRows + kWarps * RPW - 1) / (kWarps * RPW);
+      const int rstep = kWarps * RPW;
       int4 xq[BPL][4];
       float xsc[BPL];
       int xsum[BPL];
 #pragma unroll
       for (int mb = 0; mb < BPL; ++mb) {
-        const int b = g + GS * mb;
-        if (b < nb) {
-          const int4* src = reinterpret_cast<const int4*>(xcodes + b * 32);
+        const int bb = g + GS * mb;
+        if (bb < nb) {
+          const int4* src = reinterpret_cast<const int4*>(xcodes + bb * 32);
           xq[mb][0] = src[0];
           xq[mb][1] = src[1];
           xq[mb][2] = src[2];
           xq[mb][3] = src[3];
-          xsc[mb] = xs[b];
-          xsum[mb] = xc[b];
+          xsc[mb] = xs[bb];
+          xsum[mb] = xc[bb];
         } else {
           xq[mb][0] = xq[mb][1] = xq[mb][2] = xq[mb][3] = make_int4(0, 0, 0, 0);
           xsc[mb] = 0.0f;
           xsum[mb] = 0;
         }
       }
-      const int routed = p.K * (p.I / 32);
-      for (int u = blockIdx.x, k = 0; u < p.n_units; u += gridDim.x, ++k) {
-        const int i = u < routed ? u / (p.I / 32) : p.K;
-        const int rb = u < routed ? u % (p.I / 32) : u - routed;
-        if (k > 0) {
-          __syncthreads();  // the previous unit's buffer is free
-          if (tid == 0) m.flag = issue_unit(p, m, unit, u);
-          __syncthreads();
-          if (!m.flag) return;
+      unsigned long long* acc_l = p.acc + (size_t)(l % kAccBufs) * H;
+      for (int u = b, k = 0; u < p.n_units; u += G, ++k) {
+        const bool shared = u >= routed;
+        const int i = shared ? p.K : u / (p.I / 32);
+        const int rb = shared ? u - routed : u % (p.I / 32);
+        const float wi = shared ? 1.0f : m.w[i];
+        const uint8_t* usrc = (shared ? p.shared_pool + (size_t)l * p.shared_slot_bytes : m.src[i]) +
+                              (size_t)rb * p.unit_bytes;
+        if (!(k == 0 && m.pre)) {
+          if (!shared && m.pull[i] >= 0) {  // pull mode miss: this CTA fills its unit of the slot
+            pull_unit(p, p.host_tier + m.pull[i] + (size_t)rb * p.unit_bytes, const_cast<uint8_t*>(usrc));
+            __syncthreads();
+          }
+          if (tid == 0) {
+            ok = shared || wait_miss(p, m.miss_seq[i]);
+            if (ok) issue_unit(p, m, ubuf, usrc);
+            stamp(p, l, 15);
+          }
+          if (!cta_ok(p, ok)) goto fail;
         }
-        uint32_t done = 0;
-        // four rows at a time per lane group, their dot products and reductions
-        // interleaved; row r of the unit: gate rows 0-31, then up rows 0-31
-        for (int k0 = 0; k0 < rows_per_lane; k0 += 4) {
-          int rows[4];
-          float acc[4];
-          bool live[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            rows[q] = warp * RPW + sub + (k0 + q) * kWarps * RPW;
-            live[q] = k0 + q < rows_per_lane && rows[q] < 2 * kUnitRows;
-            acc[q] = 0.0f;
+        stamp(p, l, 6);
+        // gate/up: rows r = gate 0..31, up 0..31 of the unit, tile r / 16; two rows at a
+        // time per lane group, in tile order
+        for (int rw = warp * RPW; rw < 2 * kUnitRows; rw += 2 * rstep) {  // warp-uniform
+          const int rows[2] = {rw + sub, rw + sub + rstep};
+          const bool live0 = rows[0] < 2 * kUnitRows, live1 = rows[1] < 2 * kUnitRows;
+          bool w_ok = ok;
+          if (w_ok && live0) w_ok = mbar_wait(p, &m.bar_u[rows[0] / 16], par_u[rows[0] / 16]);
+          if (w_ok && live1) w_ok = mbar_wait(p, &m.bar_u[rows[1] / 16], par_u[rows[1] / 16]);
+          if (!__all_sync(0xffffffffu, w_ok)) {
+            ok = false;
+            break;
           }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (!live[q]) continue;
-            const int st = rows[q] / 16;
-            if (!((done >> st) & 1u)) {
-              if (!mbar_wait(p, &m.bar_u[st], par_u[st])) return;
-              done |= 1u << st;
-            }
-          }
-          stamp(p, l, 7);
+          float acc[2] = {0.0f, 0.0f};
 #pragma unroll
           for (int mb = 0; mb < BPL; ++mb) {
-            const int b = g + GS * mb;
-            if (b >= nb) continue;
+            const int bb = g + GS * mb;
+            if (bb >= nb) continue;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (!live[q]) continue;
+            for (int q = 0; q < 2; ++q) {
+              if ((q == 0 && !live0) || (q == 1 && !live1)) continue;
               const int r = rows[q];
-              const uint8_t* tile = unit + (r / 16) * 9u * H;
-              const uint4 qv = *reinterpret_cast<const uint4*>(tile + ((size_t)(r % 16) * nb + b) * 16);
-              const float d = __half2float(reinterpret_cast<const __half*>(tile + 8u * H)[(r % 16) * nb + b]);
+              const uint8_t* tile = ubuf + (r / 16) * 9u * H;
+              const uint4 qv = *reinterpret_cast<const uint4*>(tile + ((size_t)(r % 16) * nb + bb) * 16);
+              const float d = __half2float(reinterpret_cast<const __half*>(tile + 8u * H)[(r % 16) * nb + bb]);
               const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
               acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
             }
           }
           for (int off = GS / 2; off >= 1; off >>= 1) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
+            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+            acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], off);
           }
           if (g == 0) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (live[q]) m.gu[rows[q]] = acc[q];
+            if (live0) m.gu[rows[0]] = acc[0];
+            if (live1) m.gu[rows[1]] = acc[1];
           }
         }
-#pragma unroll
-        for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
-        stamp(p, l, 16);
-        __syncthreads();
-        stamp(p, l, 17);
+        if (!cta_ok(p, ok)) goto fail;
+        stamp(p, l, 7);
+        // a = silu(g) * u, quantised as one int16 block
         if (warp == 0) {
           const float gv = m.gu[lane], uv = m.gu[kUnitRows + lane];
           const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-          stamp(p, l, 18);
           float sc;
           int csum;
           const int code = quant_block(a, sc, csum);
-          stamp(p, l, 19);
-          uint8_t* rec = p.acodes + ((size_t)i * rec_per_exp + rb) * kACodeBytes;
-          __stcg(reinterpret_cast<int16_t*>(rec) + lane, (int16_t)code);
+          reinterpret_cast<int16_t*>(m.acodes)[lane] = (int16_t)code;
           if (lane == 0) {
-            __stcg(reinterpret_cast<float*>(rec + 64), sc);
-            __stcg(reinterpret_cast<int32_t*>(rec + 68), csum);
+            m.asc = sc;
+            m.acs = csum;
+            stamp(p, l, 16);
           }
-          stamp(p, l, 20);
         }
+        __syncthreads();  // codes ready; the gate/up tiles are no longer read
+        const uint8_t* dn = ubuf + (p.down_late ? 0u : 36u * H);
+        if (p.down_late && tid == 0) {
+          mbar_expect_tx(&m.bar_d, 18u * H);
+          bulk_g2s_stream(ubuf, usrc + 36u * H, 18u * H, &m.bar_d);
+        }
+        if (!mbar_wait(p, &m.bar_d, par_d)) ok = false;
+        stamp(p, l, 17);
+        if (ok) {
+          // down: output row j against the unit's activation block; the weighted share
+          // w_i * d_j * scale * dot goes into the accumulator as round(v * 2^28)
+          const int4 a0 = m.acodes[0], a1 = m.acodes[1], a2 = m.acodes[2], a3 = m.acodes[3];
+          const float asc = m.asc;
+          const int cs128 = 128 * m.acs;
+          const __half* dsc = reinterpret_cast<const __half*>(dn + 16u * H);
+          bool range_ok = true;
+#pragma unroll 4
+          for (int j = tid; j < H; j += kThreads) {
+            const uint4 qv = *reinterpret_cast<const uint4*>(dn + 16 * j);
+            const int v = q4_block_dot16(qv, a0, a1, a2, a3) - cs128;
+            float c = (__half2float(dsc[j]) * asc) * (float)v;
+            if (!shared) c *= wi;
+            long long qf = 0;
+            if (fabsf(c) < kAccLimit) {
+              qf = __float2ll_rn(c * kAccScale);
+            } else {
+              range_ok = false;
+            }
+            red_add_u64(acc_l + j, (unsigned long long)qf);
+          }
+          if (!range_ok) set_error(p.ctrl, MOE_DEVERR_RANGE);
+          stamp(p, l, 18);
+          __threadfence();  // this thread's adds, before the CTA's arrival below
+          stamp(p, l, 19);
+        }
+        if (!cta_ok(p, ok)) goto fail;
+#pragma unroll
+        for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
+        par_d ^= 1u;
+        if (tid == 0) m.pre = 0;
       }
     }
-    const int n_producers = min((int)gridDim.x, p.n_units);  // CTAs holding gate/up units
-    stamp(p, l, 21);
-    if ((int)blockIdx.x < n_producers) publish(p, &p.ctrl->a_count);
-    stamp(p, l, 3);
+    stamp(p, l, 8);
     cta_stamp(p, l, 1);
-    stamp(p, l, 4);
-
-    // ---------------------------------------------------------------- D phase
-    // (CTAs that own rows) wait for every activation record of the layer and for the miss
-    // copies the down tiles depend on; tiles and records are then read from L2
-    if (n_own > 0) {
-      if (tid == 0) {
-        m.flag = 1;
-        for (int i = 0; i < p.n_exp; ++i)
-          if (!wait_miss(p, m.miss_seq[i])) m.flag = 0;
-      }
-      if (!await_count(p, m, &p.ctrl->a_count, (uint32_t)(l + 1) * n_producers)) return;
+    // the next layer's shared-expert unit does not depend on routing: load it now
+    if (first_shared && next && tid == 0) {
+      issue_unit(p, m, ubuf, p.shared_pool + (size_t)(l + 1) * p.shared_slot_bytes + (size_t)(b - routed) * p.unit_bytes);
+      m.pre = 1;
     }
-    if (!cta_ok(p, m.flag)) return;
-    stamp(p, l, 13);
-    for (int k = 0; k < n_own; ++k) {
-      const int c = blockIdx.x + k * gridDim.x;
-      stamp(p, l, 14);
-      // thread (expert i, block column b0): all 16 rows of chunk c against block b0 (then
-      // b0+16, ...) of a_i, every load of a block issued before any is used; then a
-      // 15-shuffle transpose reduction over the expert's 16 lanes leaves row b0 in lane b0
-      {
-        const int b0 = tid & 15;
-        // warp-uniform loop: lanes 0-15 take expert base, lanes 16-31 expert base + 1
-        for (int base = 2 * warp; base < p.n_exp; base += 2 * kWarps) {
-          const int i = base + (lane >> 4);
-          const bool act = i < p.n_exp;
-          const int Ii = !act ? 0 : (i < p.K ? p.I : p.Is);
-          const int nbd = Ii / 32;
-          const uint8_t* tile =
-              act ? m.src[i] + (i < p.K ? p.lay.down : p.slay.down) + (size_t)c * 9u * Ii : nullptr;
-          float acc[kChunk];
-#pragma unroll
-          for (int r = 0; r < kChunk; ++r) acc[r] = 0.0f;
-          for (int b = b0; b < nbd; b += 16) {
-            const uint4* rec = reinterpret_cast<const uint4*>(p.acodes + ((size_t)i * rec_per_exp + b) * kACodeBytes);
-            const uint4 r0 = __ldcg(rec), r1 = __ldcg(rec + 1), r2 = __ldcg(rec + 2), r3 = __ldcg(rec + 3),
-                        r4 = __ldcg(rec + 4);
-            uint4 qv[kChunk];
-            unsigned short dv[kChunk];
-#pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-              qv[r] = __ldcg(reinterpret_cast<const uint4*>(tile + ((size_t)r * nbd + b) * 16));
-              dv[r] = __ldcg(reinterpret_cast<const unsigned short*>(tile + 8u * Ii) + (size_t)r * nbd + b);
-            }
-            const int4 a0 = make_int4(r0.x, r0.y, r0.z, r0.w), a1 = make_int4(r1.x, r1.y, r1.z, r1.w),
-                       a2 = make_int4(r2.x, r2.y, r2.z, r2.w), a3 = make_int4(r3.x, r3.y, r3.z, r3.w);
-            const float sc = __uint_as_float(r4.x);
-            const int cs128 = 128 * (int)r4.y;
-#pragma unroll
-            for (int r = 0; r < kChunk; ++r) {
-              const int v = q4_block_dot16(qv[r], a0, a1, a2, a3) - cs128;
-              acc[r] = fmaf(__half2float(__ushort_as_half(dv[r])) * sc, (float)v, acc[r]);
-            }
-          }
-#pragma unroll
-          for (int h = 8; h >= 1; h >>= 1) {
-            const bool up = (b0 & h) != 0;
-#pragma unroll
-            for (int r = 0; r < h; ++r) {
-              const float send = up ? acc[r] : acc[r + h];
-              const float keep = up ? acc[r + h] : acc[r];
-              acc[r] = keep + __shfl_xor_sync(0xffffffffu, send, h);
-            }
-          }
-          if (act) os[i * kChunk + b0] = acc[0];
-        }
-      }
-      __syncthreads();
-      stamp(p, l, 15);
-      if (tid < kChunk) {
-        const int j = c * kChunk + tid;
-        float y = 0.0f;
-        for (int i = 0; i < p.K; ++i) y = fmaf(m.w[i], os[i * kChunk + tid], y);
-        if (p.Is > 0) y = __fadd_rn(y, os[p.K * kChunk + tid]);
-        const float hn = p.use_norm ? __fadd_rn(m.hown[k][tid], y) : y;
-        m.hown[k][tid] = hn;
-        __stcg(p.h + j, hn);
-        if (p.h_trace) p.h_trace[(size_t)(l + 1) * H + j] = hn;
-        if (l == p.L - 1) p.y[j] = hn;
-      }
-      if (next) {
-        if (k == 0 && !mbar_wait(p, &m.bar_r, par_r)) return;
-        router_partials(p, m, c, m.hown[k], has_gain ? m.gnext[k] : nullptr, [&](int e) {
-          return reinterpret_cast<const uint4*>(rch + (size_t)k * 32u * p.E + (size_t)e * 32u);
-        });
-      }
-      __syncthreads();
-    }
-    if (next && n_own > 0) par_r ^= 1u;
-    // the router columns for layer l + 2 load during the barrier (rch is free again)
-    if (tid == 0 && l + 2 < p.L && n_own > 0) prefetch_router(p, m, rch, l + 2, n_own);
-    stamp(p, l, 5);
+    __syncthreads();
+    if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
+    stamp(p, l, 9);
     cta_stamp(p, l, 2);
-    if (!grid_sync(p, m)) return;
-    stamp(p, l, 6);
-    cta_stamp(p, l, 3);
+  }
 
-    // deferred ring fills (only when a layer misses more often than it has ring slots)
+  // ---- the last layer's output
+  if (tid == 0) ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(p.L + 1) * G);
+  if (!cta_ok(p, ok)) goto fail;
+  {
+    add_layer_output(p, p.acc + (size_t)((p.L - 1) % kAccBufs) * H, hs, nullptr);
+    for (int j0 = b * kThreads; j0 < H; j0 += G * kThreads)
+      if (j0 + tid < H) p.y[j0 + tid] = hs[j0 + tid];
+    if (b == 0 && p.h_trace)
+      for (int j = tid; j < H; j += kThreads) p.h_trace[(size_t)p.L * H + j] = hs[j];
     for (int f = 0; f < m.n_fix; ++f) {
       const uint4* s = reinterpret_cast<const uint4*>(p.pool + (size_t)m.fix_src[f] * p.slot_bytes);
       uint4* d = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) + (size_t)m.fix_dst[f] * p.slot_bytes);
       const size_t n16 = p.slot_bytes / 16;
-      for (size_t t = (size_t)blockIdx.x * kThreads + tid; t < n16; t += (size_t)gridDim.x * kThreads)
-        d[t] = __ldcg(s + t);
+      for (size_t t = (size_t)b * kThreads + tid; t < n16; t += (size_t)G * kThreads) d[t] = __ldcg(s + t);
     }
   }
   stamp(p, p.L, 2);
-  if (blockIdx.x == 0 && tid == 0) {
+  if (b == 0 && tid == 0) {
     p.ctrl->step = m.step + 1;
     p.ctrl->req_seq = m.seq_base + m.n_miss;
   }
+  return;
+
+fail:
+  // a failed launch: the error word says why (moe_sync); callers that cannot read it
+  // see NaN outputs
+  if (p.nan_on_error)
+    for (int j0 = b * kThreads; j0 < H; j0 += G * kThreads)
+      if (j0 + tid < H) p.y[j0 + tid] = __int_as_float(0x7fc00000);
 }
 
 // ------------------------------------------------------------------ host-side launch
-
-uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown) {
-  return smem_plan(H, E, K, I, Is, nown).total;
-}
 
 // Blocks of one gate/up row each lane covers: 1 below 1024 columns, else H / 1024.
 static int bpl_of(int H) {
@@ -1173,24 +1194,46 @@ static cudaError_t with_kernel(int H, F f) {
   }
 }
 
-cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown) {
-  const uint32_t bytes = decode_smem_bytes(H, E, K, I, Is, nown);
-  return with_kernel(H, [&](auto kern) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  });
+uint32_t decode_smem_bytes(int H, int E, int rx, int down_late) { return smem_plan(H, E, rx, down_late).total; }
+
+// Shape-dependent launch settings: router experts per CTA and whether a unit's down part
+// must reuse its gate/up buffer; false when no setting fits in smem_optin.
+bool decode_plan(int H, int E, int grid, int smem_optin, int* rx, int* down_late, uint32_t* smem) {
+  *rx = (E + grid - 1) / grid;
+  if (*rx > kWarps) return false;
+  for (int late = 0; late < 2; ++late) {
+    const uint32_t bytes = decode_smem_bytes(H, E, *rx, late);
+    if (bytes <= (uint32_t)smem_optin) {
+      *down_late = late;
+      *smem = bytes;
+      return true;
+    }
+  }
+  return false;
 }
 
-cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int nown, int* out) {
-  return with_kernel(H, [&](auto kern) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, decode_smem_bytes(H, E, K, I, Is, nown));
-  });
+// Every instance of the kernel may use up to limit bytes of dynamic shared memory; set
+// for all of them at once, so that contexts or calls of different shapes never leave
+// one instance below what another call needs.
+cudaError_t decode_configure(int limit) {
+  cudaError_t e = cudaSuccess;
+  auto set = [&](auto kern) { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, limit); };
+  if (e == cudaSuccess) e = set(moe_decode_kernel<1>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<2>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<3>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<4>);
+  return e;
+}
+
+cudaError_t decode_max_blocks_per_sm(int H, uint32_t smem, int* out) {
+  return with_kernel(H, [&](auto kern) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, smem); });
 }
 
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, p.E, p.K, p.I, p.Is, p.nown);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, p.E, p.rx_per_cta, p.down_late);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

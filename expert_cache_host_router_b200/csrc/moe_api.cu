@@ -20,6 +20,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <thread>
 #include <vector>
@@ -29,9 +30,9 @@
 #include "prefill.h"
 
 namespace moe {
-uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown);
-cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown);
-cudaError_t decode_max_blocks_per_sm(int H, int E, int K, int I, int Is, int nown, int* out);
+bool decode_plan(int H, int E, int grid, int smem_optin, int* rx, int* down_late, uint32_t* smem);
+cudaError_t decode_configure(int limit);
+cudaError_t decode_max_blocks_per_sm(int H, uint32_t smem, int* out);
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream);
 }  // namespace moe
 
@@ -42,26 +43,30 @@ typedef CUresult (*PfnWriteValue32)(CUstream, CUdeviceptr, cuuint32_t, unsigned 
 struct moe_ctx {
   moe_config cfg{};
   int L = 0, H = 0, E = 0, K = 0, I = 0, Is = 0, R = 0;
-  int nsm = 0, grid = 0, nown = 1;
+  int nsm = 0, grid = 0, rx = 1, down_late = 0;
+  uint32_t smem = 0;
+  int miss_mode = kMissProxy;
   SlotLayout lay{}, slay{};
   uint64_t slot_bytes = 0, shared_slot_bytes = 0;
-  // host tier
+  // host tier (mapped: the kernel reads it directly in the SM-pull miss path)
   uint8_t* host_tier = nullptr;
+  const uint8_t* host_tier_dev = nullptr;
   std::vector<uint8_t> loaded;
   // device
   uint8_t* shared_pool = nullptr;
   std::atomic<uint8_t*> pool{nullptr};
   int64_t pool_slots = 0;
-  uint16_t* router = nullptr;
-  uint16_t* router_rows = nullptr;  // [L][E][H] bf16 (prefill's router GEMM)
+  uint16_t* router_rows = nullptr;  // [L][E][H] bf16 (decode router rows; prefill's router GEMM)
   float* wnorm = nullptr;           // [L] max_e ||w_e||_2 rounded up (prefill's routing bound)
   float* bias = nullptr;
   float* gain = nullptr;
   bool has_bias = false, has_gain = false;
   int32_t *pin_slot = nullptr, *layer_base = nullptr, *n_pinned = nullptr, *ring_owner = nullptr;
   uint32_t *ring_stamp = nullptr, *ring_clock = nullptr;
-  float *h = nullptr, *part = nullptr, *sq = nullptr, *z = nullptr;
-  uint8_t* acodes = nullptr;
+  unsigned long long* acc = nullptr;  // [kAccBufs][H] fixed-point layer outputs
+  unsigned long long* zll = nullptr;  // [E] published logits
+  int32_t* likely = nullptr;          // [L][kMaxLikely] pool slots of the likeliest pinned experts
+  int n_likely = 0;
   uint32_t* hist = nullptr;
   int32_t* log = nullptr;
   int log_steps = 0;
@@ -91,10 +96,18 @@ struct moe_ctx {
   std::atomic<uint32_t> proxy_next{1};
   std::atomic<int> drop{0};
   std::atomic<int> proxy_err{0};
+  // timing of the proxy's copies: event pairs recorded around each cudaMemcpyAsync on
+  // the side stream, harvested by moe_stats (a copy finds no free pair: untimed)
+  static constexpr int kCopyTimers = 64;
+  cudaEvent_t ev_start[kCopyTimers] = {}, ev_end[kCopyTimers] = {};
+  std::mutex timer_mu;
+  std::vector<int> timer_free, timer_pending;
+  uint64_t copy_ns = 0, copies_timed = 0;
   PfnWriteValue32 write_value32 = nullptr;
   // tracing and log reading
   float *h_trace = nullptr, *w_trace = nullptr;
   unsigned long long* phase_trace = nullptr;
+  size_t phase_trace_words = 0;
   uint64_t log_read_step = 0, log_dropped = 0;
   // batched prefill: scratch for up to prefill_cap tokens (one allocation), tracing
   uint8_t* prefill_mem = nullptr;
@@ -158,13 +171,31 @@ static void proxy_main(moe_ctx* c) {
     if (layer >= (uint32_t)c->L || expert >= (uint32_t)c->E || (int64_t)dst >= c->pool_slots || !pool) {
       c->proxy_err.store(1);  // leave it unsignalled: the kernel's bounded wait reports it
     } else {
-      cudaMemcpyAsync(pool + (size_t)dst * c->slot_bytes,
-                      c->host_tier + ((size_t)layer * c->E + expert) * c->slot_bytes, c->slot_bytes,
-                      cudaMemcpyHostToDevice, c->side);
-      if (c->drop.load() > 0) {
+      int timer = -1;
+      {
+        std::lock_guard<std::mutex> lk(c->timer_mu);
+        if (!c->timer_free.empty()) {
+          timer = c->timer_free.back();
+          c->timer_free.pop_back();
+        }
+      }
+      if (timer >= 0) cudaEventRecord(c->ev_start[timer], c->side);
+      const cudaError_t ce = cudaMemcpyAsync(pool + (size_t)dst * c->slot_bytes,
+                                             c->host_tier + ((size_t)layer * c->E + expert) * c->slot_bytes,
+                                             c->slot_bytes, cudaMemcpyHostToDevice, c->side);
+      if (timer >= 0) {
+        cudaEventRecord(c->ev_end[timer], c->side);
+        std::lock_guard<std::mutex> lk(c->timer_mu);
+        c->timer_pending.push_back(timer);
+      }
+      if (ce != cudaSuccess) {
+        // a copy that was not enqueued must not be signalled: the slot would be read
+        // stale; the kernel's bounded wait turns the missing signal into MOE_ERR_TIMEOUT
+        c->proxy_err.store(2);
+      } else if (c->drop.load() > 0) {
         c->drop.fetch_sub(1);
-      } else {
-        c->write_value32((CUstream)c->side, (CUdeviceptr)c->done_seq, next, 0);
+      } else if (c->write_value32((CUstream)c->side, (CUdeviceptr)c->done_seq, next, 0) != CUDA_SUCCESS) {
+        c->proxy_err.store(3);
       }
     }
     c->proxy_next.store(next + 1, std::memory_order_release);
@@ -185,17 +216,17 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
   p.R = c->R;
   p.use_norm = c->cfg.use_rmsnorm;
   p.eps = c->cfg.rms_eps;
-  p.nch = c->H / kChunk;
   p.n_units = c->K * (c->I / 32) + c->Is / 32;
-  p.n_exp = c->K + (c->Is > 0 ? 1 : 0);
-  p.nown = c->nown;
+  p.rx_per_cta = c->rx;
+  p.down_late = c->down_late;
+  p.miss_mode = c->miss_mode;
+  p.nan_on_error = 0;
   p.pool = c->pool.load();
   p.slot_bytes = c->slot_bytes;
-  p.lay = c->lay;
+  p.unit_bytes = c->lay.unit;
   p.shared_pool = c->shared_pool;
   p.shared_slot_bytes = c->shared_slot_bytes;
-  p.slay = c->slay;
-  p.router = c->router;
+  p.router = c->router_rows;
   p.bias = c->has_bias ? c->bias : nullptr;
   p.gain = c->has_gain ? c->gain : nullptr;
   p.pin_slot = c->pin_slot;
@@ -209,19 +240,19 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
   p.y = y;
   p.h_trace = c->h_trace;
   p.w_trace = c->w_trace;
-  p.h = c->h;
-  p.part = c->part;
-  p.sq = c->sq;
-  p.z = c->z;
-  p.acodes = c->acodes;
+  p.acc = c->acc;
+  p.zll = c->zll;
   p.hist = c->hist;
   p.log = c->log;
   p.log_steps = c->log_steps;
   p.ctrl = c->ctrl;
   p.mbox = c->mbox_dev;
   p.done_seq = c->done_seq;
+  p.host_tier = c->host_tier_dev;
   p.timeout_ns = (unsigned long long)c->cfg.wait_timeout_ms * 1000000ull;
   p.phase_trace = c->phase_trace;
+  p.likely = c->likely;
+  p.n_likely = c->n_likely;
   return p;
 }
 
@@ -240,11 +271,8 @@ static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cud
   CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
   cudaError_t e = cudaSuccess;
   if (host_io) e = cudaMemcpyAsync(c->x_buf, c->x_pin, sizeof(float) * c->H, cudaMemcpyHostToDevice, c->own);
-  // the launch's arrival counters (grid barrier, logits, activation codes) start at 0
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(&c->ctrl->bar_count, 0,
-                        reinterpret_cast<char*>(&c->ctrl->a_count + 1) - reinterpret_cast<char*>(&c->ctrl->bar_count),
-                        c->own);
+  // the launch's arrival counter starts at 0
+  if (e == cudaSuccess) e = cudaMemsetAsync(&c->ctrl->bar_count, 0, sizeof(uint32_t), c->own);
   if (e == cudaSuccess) e = decode_launch(make_params(c, x, y), c->grid, c->own);
   if (e == cudaSuccess && host_io)
     e = cudaMemcpyAsync(c->y_pin, c->y_buf, sizeof(float) * c->H, cudaMemcpyDeviceToHost, c->own);
@@ -284,12 +312,25 @@ static void repack_rows(const uint8_t* src, uint8_t* dst, int64_t rows, int64_t 
   }
 }
 
+// Canonical gate | up | down of one expert (width I) -> the unit layout of moe_internal.h.
 static void repack_expert(const uint8_t* src, uint8_t* dst, const SlotLayout& s, int H, int I) {
   const uint64_t gu = q4_bytes(I, H);
-  const uint64_t t_gu = 9ull * H, t_d = 9ull * I;
-  repack_rows(src, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + (r % 32) / 16) * t_gu; });
-  repack_rows(src + gu, dst, I, H, [&](int64_t r) { return s.gu + (4 * (r / 32) + 2 + (r % 32) / 16) * t_gu; });
-  repack_rows(src + 2 * gu, dst, H, I, [&](int64_t r) { return s.down + (r / 16) * t_d; });
+  const uint64_t t_gu = 9ull * H;
+  repack_rows(src, dst, I, H,
+              [&](int64_t r) { return (r / 32) * s.unit + unit_gu_tile(H, (int)((r % 32) / 16)); });
+  repack_rows(src + gu, dst, I, H,
+              [&](int64_t r) { return (r / 32) * s.unit + unit_gu_tile(H, 2 + (int)((r % 32) / 16)); });
+  (void)t_gu;
+  // down [H x I]: block rb of row j -> unit rb, nibbles at j * 16, scale at j * 2
+  const uint8_t* D = src + 2 * gu;
+  const int nbd = I / 32;
+  for (int64_t j = 0; j < H; ++j)
+    for (int rb = 0; rb < nbd; ++rb) {
+      const uint8_t* blk = D + (j * nbd + rb) * 18;
+      uint8_t* u = dst + rb * s.unit;
+      memcpy(u + unit_down_nib(H) + j * 16, blk + 2, 16);
+      memcpy(u + unit_down_scl(H) + j * 2, blk, 2);
+    }
 }
 
 // Placement: top-P experts by count (ties -> lower index), or experts 0..P-1.
@@ -313,6 +354,39 @@ static int empty_rings(moe_ctx* c, cudaStream_t s) {
   CK(cudaMemsetAsync(c->ring_stamp, 0, nr * 4, s));
   CK(cudaMemsetAsync(c->ring_clock, 0, (size_t)2 * c->L * 4, s));
   return MOE_OK;
+}
+
+// Speculative-prefetch table from the recalibration score (the placement histogram,
+// decayed): per layer, the pool slots of the n_likely pinned experts with the highest
+// counts (ties -> lower index).
+static int upload_likely(moe_ctx* c, cudaStream_t s) {
+  std::vector<int32_t> t((size_t)c->L * kMaxLikely, -1);
+  std::vector<int> order(c->E);
+  for (int l = 0; l < c->L && c->n_likely > 0; ++l) {
+    const uint32_t* cnt = c->score.data() + (size_t)l * c->E;
+    const int32_t* row = c->pin_host.data() + (size_t)l * c->E;
+    for (int e = 0; e < c->E; ++e) order[e] = e;
+    std::stable_sort(order.begin(), order.end(), [cnt](int a, int b) { return cnt[a] > cnt[b]; });
+    int n = 0;
+    for (int k = 0; k < c->E && n < c->n_likely; ++k)
+      if (row[order[k]] >= 0) t[(size_t)l * kMaxLikely + n++] = l * (c->P + c->R) + (row[order[k]] & 0xffff);
+  }
+  CK(cudaMemcpyAsync(c->likely, t.data(), t.size() * 4, cudaMemcpyHostToDevice, s));
+  return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Add the durations of the proxy's timed copies that have completed (device idle).
+static void harvest_copy_timers(moe_ctx* c) {
+  std::lock_guard<std::mutex> lk(c->timer_mu);
+  for (int t : c->timer_pending) {
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, c->ev_start[t], c->ev_end[t]) == cudaSuccess) {
+      c->copy_ns += (uint64_t)((double)ms * 1e6);
+      ++c->copies_timed;
+    }
+    c->timer_free.push_back(t);
+  }
+  c->timer_pending.clear();
 }
 
 // ------------------------------------------------------------------ C ABI
@@ -342,11 +416,15 @@ void moe_destroy(moe_ctx* c) {
   cudaSetDevice(c->cfg.device);
   cudaDeviceSynchronize();
   drop_graphs(c);
+  for (int t = 0; t < moe_ctx::kCopyTimers; ++t) {
+    if (c->ev_start[t]) cudaEventDestroy(c->ev_start[t]);
+    if (c->ev_end[t]) cudaEventDestroy(c->ev_end[t]);
+  }
   if (c->side) cudaStreamDestroy(c->side);
   if (c->own) cudaStreamDestroy(c->own);
-  void* dev[] = {c->shared_pool, c->pool.load(), c->router, c->bias, c->gain, c->pin_slot,
+  void* dev[] = {c->shared_pool, c->pool.load(), c->bias, c->gain, c->pin_slot,
                  c->layer_base, c->n_pinned, c->ring_owner, c->ring_stamp, c->ring_clock,
-                 c->h, c->part, c->sq, c->z, c->acodes, c->hist, c->log, c->ctrl, c->done_seq,
+                 c->acc, c->zll, c->likely, c->hist, c->log, c->ctrl, c->done_seq,
                  c->x_buf, c->y_buf, c->prefill_mem, c->router_rows, c->wnorm};
   for (void* p : dev)
     if (p) cudaFree(p);
@@ -381,14 +459,7 @@ int moe_load_layer(moe_ctx* c, int32_t l, const uint8_t* const* experts, const u
     CK(cudaMemcpy(c->shared_pool + (size_t)l * c->shared_slot_bytes, tmp.data(), c->shared_slot_bytes,
                   cudaMemcpyHostToDevice));
   }
-  {  // router [E][H] -> [H/16][E][16]
-    const int nch = c->H / kChunk;
-    std::vector<uint16_t> tmp((size_t)c->E * c->H);
-    for (int ch = 0; ch < nch; ++ch)
-      for (int e = 0; e < c->E; ++e)
-        memcpy(&tmp[((size_t)ch * c->E + e) * kChunk], router_bf16 + (size_t)e * c->H + ch * kChunk,
-               kChunk * sizeof(uint16_t));
-    CK(cudaMemcpy(c->router + (size_t)l * c->E * c->H, tmp.data(), tmp.size() * 2, cudaMemcpyHostToDevice));
+  {  // router rows [E][H] as given
     CK(cudaMemcpy(c->router_rows + (size_t)l * c->E * c->H, router_bf16, (size_t)c->E * c->H * 2,
                   cudaMemcpyHostToDevice));
     double wmax = 0.0;  // the largest router row norm, for the prefill routing error bound
@@ -472,19 +543,13 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   CKC(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, cfg.device));
   CKC(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, cfg.device));
   c->grid = c->nsm;  // one persistent CTA per SM
-  c->nown = (c->H / kChunk + c->grid - 1) / c->grid;
-  if (!coop || c->nown > kMaxOwn ||
-      decode_smem_bytes(c->H, c->E, c->K, c->I, c->Is, c->nown) > (uint32_t)smem_optin)
+  if (!coop || !decode_plan(c->H, c->E, c->grid, smem_optin, &c->rx, &c->down_late, &c->smem))
     return fail(MOE_ERR_UNSUPPORTED);
-  CKC(decode_configure(c->H, c->E, c->K, c->I, c->Is, c->nown));
+  CKC(decode_configure(smem_optin));
   int per_sm = 0;
-  CKC(decode_max_blocks_per_sm(c->H, c->E, c->K, c->I, c->Is, c->nown, &per_sm));
+  CKC(decode_max_blocks_per_sm(c->H, c->smem, &per_sm));
   if (per_sm < 1) return fail(MOE_ERR_UNSUPPORTED);
 
-  const size_t nch = c->H / kChunk;
-  const int n_exp = c->K + (c->Is > 0);
-  const int imax = std::max(c->I, c->Is);
-  CKC(dalloc(&c->router, (size_t)c->L * c->E * c->H));
   CKC(dalloc(&c->router_rows, (size_t)c->L * c->E * c->H));
   CKC(dalloc(&c->wnorm, c->L));
   CKC(dalloc(&c->bias, (size_t)c->L * c->E));
@@ -496,11 +561,9 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   CKC(dalloc(&c->ring_owner, (size_t)2 * c->L * std::max(c->R, 1)));
   CKC(dalloc(&c->ring_stamp, (size_t)2 * c->L * std::max(c->R, 1)));
   CKC(dalloc(&c->ring_clock, (size_t)2 * c->L));
-  CKC(dalloc(&c->h, c->H));
-  CKC(dalloc(&c->part, (size_t)c->E * nch));
-  CKC(dalloc(&c->sq, nch));
-  CKC(dalloc(&c->z, c->E));
-  CKC(dalloc(&c->acodes, (size_t)n_exp * (imax / 32) * kACodeBytes));
+  CKC(dalloc(&c->acc, (size_t)kAccBufs * c->H));
+  CKC(dalloc(&c->zll, c->E));
+  CKC(dalloc(&c->likely, (size_t)c->L * kMaxLikely));
   CKC(dalloc(&c->hist, (size_t)c->L * c->E));
   CKC(dalloc(&c->log, (size_t)c->log_steps * c->L * c->K * 7));
   CKC(dalloc(&c->ctrl, 1));
@@ -510,8 +573,15 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   CKC(cudaMemset(c->hist, 0, sizeof(uint32_t) * c->L * c->E));
   CKC(cudaMemset(c->ctrl, 0, sizeof(Ctrl)));
   CKC(cudaMemset(c->done_seq, 0, sizeof(uint32_t)));
-  CKC(cudaMemset(c->acodes, 0, (size_t)n_exp * (imax / 32) * kACodeBytes));
-  CKC(cudaHostAlloc((void**)&c->host_tier, (size_t)c->L * c->E * c->slot_bytes, cudaHostAllocPortable));
+  CKC(cudaMemset(c->acc, 0, sizeof(unsigned long long) * kAccBufs * c->H));
+  CKC(cudaMemset(c->zll, 0, sizeof(unsigned long long) * c->E));
+  CKC(cudaHostAlloc((void**)&c->host_tier, (size_t)c->L * c->E * c->slot_bytes,
+                    cudaHostAllocPortable | cudaHostAllocMapped));
+  {
+    void* dp = nullptr;
+    CKC(cudaHostGetDevicePointer(&dp, c->host_tier, 0));
+    c->host_tier_dev = static_cast<const uint8_t*>(dp);
+  }
   CKC(cudaHostAlloc((void**)&c->x_pin, sizeof(float) * c->H, cudaHostAllocPortable));
   CKC(cudaHostAlloc((void**)&c->y_pin, sizeof(float) * c->H, cudaHostAllocPortable));
   CKC(cudaHostAlloc((void**)&c->err_pin, sizeof(int32_t), cudaHostAllocPortable));
@@ -526,6 +596,11 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
     CKC(cudaGetDriverEntryPointByVersion("cuStreamWriteValue32", &fn, 12000, cudaEnableDefault, &q));
     if (q != cudaDriverEntryPointSuccess || !fn) return fail(MOE_ERR_UNSUPPORTED);
     c->write_value32 = (PfnWriteValue32)fn;
+  }
+  for (int t = 0; t < moe_ctx::kCopyTimers; ++t) {
+    CKC(cudaEventCreate(&c->ev_start[t]));
+    CKC(cudaEventCreate(&c->ev_end[t]));
+    c->timer_free.push_back(t);
   }
   c->proxy = std::thread(proxy_main, c);
   if (w) {
@@ -607,7 +682,7 @@ int moe_set_residency(moe_ctx* c, float fraction, const uint32_t* hist, int32_t 
   c->placement = placement;
   c->resident = true;
   drop_graphs(c);
-  return MOE_OK;
+  return upload_likely(c, c->own);
 }
 
 int moe_decode_step(moe_ctx* c, const float* x_dev, float* y_dev, void* stream) {
@@ -807,9 +882,11 @@ int moe_clear_error(moe_ctx* c) {
   const uint32_t last = c->proxy_next.load() - 1;
   ctl.req_seq = last;
   ctl.error = 0;
-  ctl.bar_count = ctl.z_count = ctl.a_count = 0;  // (the graphs zero them before every launch too)
+  ctl.bar_count = 0;  // (the graphs zero it before every launch too)
   CK(cudaMemcpy(c->ctrl, &ctl, sizeof(Ctrl), cudaMemcpyHostToDevice));
   CK(cudaMemcpy(c->done_seq, &last, sizeof(uint32_t), cudaMemcpyHostToDevice));
+  // published logits carry a per-launch epoch: a failed launch may leave some behind
+  CK(cudaMemset(c->zll, 0, sizeof(unsigned long long) * c->E));
   const size_t nr = (size_t)2 * c->L * std::max(c->R, 1);
   CK(cudaMemset(c->ring_owner, 0xff, nr * 4));
   CK(cudaMemset(c->ring_stamp, 0, nr * 4));
@@ -845,6 +922,13 @@ int moe_stats(moe_ctx* c, moe_stats_t* out, uint32_t* hist_out, moe_event* log_o
     out->miss_requests = ctl.req_seq;
     out->miss_served = c->proxy_next.load() - 1;
     out->proxy_error = c->proxy_err.load();
+    out->miss_path = c->miss_mode == kMissPull ? MOE_MISS_SM_PULL : MOE_MISS_COPY_ENGINE;
+    out->pulled_misses = ctl.pulled;
+  }
+  harvest_copy_timers(c);
+  if (out) {
+    out->copies_timed = c->copies_timed;
+    out->copy_ns_timed = c->copy_ns;
   }
   if (hist_out)
     CK(cudaMemcpy(hist_out, c->hist, sizeof(uint32_t) * c->L * c->E, cudaMemcpyDeviceToHost));
@@ -867,10 +951,11 @@ int moe_stats(moe_ctx* c, moe_stats_t* out, uint32_t* hist_out, moe_event* log_o
   if (log_n) *log_n = n;
   if (out) out->log_dropped = c->log_dropped;
   if (reset) {
-    ctl.pin_hits = ctl.ring_hits = ctl.misses = ctl.evictions = ctl.staged = 0;
-    CK(cudaMemcpy(&c->ctrl->pin_hits, &ctl.pin_hits, 5 * sizeof(unsigned long long), cudaMemcpyHostToDevice));
+    ctl.pin_hits = ctl.ring_hits = ctl.misses = ctl.evictions = ctl.staged = ctl.pulled = 0;
+    CK(cudaMemcpy(&c->ctrl->pin_hits, &ctl.pin_hits, 6 * sizeof(unsigned long long), cudaMemcpyHostToDevice));
     CK(cudaMemset(c->hist, 0, sizeof(uint32_t) * c->L * c->E));
     std::fill(c->hist_snap.begin(), c->hist_snap.end(), 0u);  // recalibration windows restart at 0
+    c->copy_ns = c->copies_timed = 0;
   }
   return MOE_OK;
 }
@@ -924,7 +1009,16 @@ int moe_recalibrate(moe_ctx* c) {
   if (st != MOE_OK) return st;
   CK(cudaStreamSynchronize(c->own));
   ++c->repins;
-  return MOE_OK;
+  return upload_likely(c, c->own);
+}
+
+int moe_set_prefetch(moe_ctx* c, int32_t n_experts) {
+  if (!c || n_experts < 0 || n_experts > kMaxLikely) return MOE_ERR_INVALID;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  c->n_likely = n_experts;
+  drop_graphs(c);
+  return c->resident ? upload_likely(c, c->own) : MOE_OK;
 }
 
 int moe_set_router_bias(moe_ctx* c, int32_t layer, const float* bias) {
@@ -951,10 +1045,53 @@ int moe_set_trace(moe_ctx* c, float* h_trace_dev, float* w_trace_dev) {
   return MOE_OK;
 }
 
-int moe_set_phase_trace(moe_ctx* c, uint64_t* stamps_dev) {
+int moe_set_phase_trace(moe_ctx* c, uint64_t* stamps_dev, size_t n_words) {
   if (!c) return MOE_ERR_INVALID;
+  if (stamps_dev && n_words < phase_trace_words(c->L, c->grid)) return MOE_ERR_INVALID;
   c->phase_trace = reinterpret_cast<unsigned long long*>(stamps_dev);
+  c->phase_trace_words = stamps_dev ? n_words : 0;
   drop_graphs(c);
+  return MOE_OK;
+}
+
+int moe_set_miss_path(moe_ctx* c, int32_t mode) {
+  if (!c || (mode != MOE_MISS_COPY_ENGINE && mode != MOE_MISS_SM_PULL)) return MOE_ERR_INVALID;
+  const int m = mode == MOE_MISS_SM_PULL ? kMissPull : kMissProxy;
+  if (m != c->miss_mode) {
+    CK(cudaSetDevice(c->cfg.device));
+    CK(cudaDeviceSynchronize());
+    c->miss_mode = m;
+    drop_graphs(c);
+  }
+  return MOE_OK;
+}
+
+int moe_measure_h2d(moe_ctx* c, int32_t n_copies, double* gbs) {
+  if (!c || n_copies < 1 || !gbs) return MOE_ERR_INVALID;
+  if (!c->resident) return MOE_ERR_STATE;
+  CK(cudaSetDevice(c->cfg.device));
+  CK(cudaDeviceSynchronize());
+  uint8_t* pool = c->pool.load();
+  cudaEvent_t a = nullptr, b = nullptr;
+  CK(cudaEventCreate(&a));
+  cudaError_t e = cudaEventCreate(&b);
+  const size_t n_src = (size_t)c->L * c->E;
+  for (int pass = 0; pass < 2 && e == cudaSuccess; ++pass) {  // pass 0 warms the path up
+    if (pass == 1) e = cudaEventRecord(a, c->side);
+    for (int i = 0; i < n_copies && e == cudaSuccess; ++i) {
+      const size_t src = ((size_t)i * 7919) % n_src;  // spread over the tier
+      e = cudaMemcpyAsync(pool + (size_t)(c->staging_base + i % c->K) * c->slot_bytes,
+                          c->host_tier + src * c->slot_bytes, c->slot_bytes, cudaMemcpyHostToDevice, c->side);
+    }
+    if (pass == 1 && e == cudaSuccess) e = cudaEventRecord(b, c->side);
+  }
+  float ms = 0.0f;
+  if (e == cudaSuccess) e = cudaEventSynchronize(b);
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, a, b);
+  cudaEventDestroy(a);
+  cudaEventDestroy(b);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *gbs = (double)n_copies * (double)c->slot_bytes / ((double)ms * 1e-3) / 1e9;
   return MOE_OK;
 }
 

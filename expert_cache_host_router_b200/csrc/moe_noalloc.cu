@@ -1,11 +1,10 @@
 // moe_noalloc.cu -- moe_decode_step_noalloc: the decode kernel with its scratch in a
 // static device array, for callers that cannot allocate device memory.
 //
-// Everything the kernel writes besides y lives in g_scratch: the control block (grid
-// barrier word, error word, counters), the exchange buffers (h, router partials, norm
-// partials, logits, quantised activations), the slot tables of a fully resident model,
-// the routing histogram and one step of event log.  The array is carved per call from
-// the shape; nothing is allocated.
+// Everything the kernel writes besides y lives in g_scratch: the control block (arrival
+// counter, error word, counters), the output accumulators, the published logit words,
+// the slot tables of a fully resident model, the routing histogram and one step of event
+// log.  The array is carved per call from the shape; nothing is allocated.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -14,14 +13,14 @@
 #include "moe_internal.h"
 
 namespace moe {
-uint32_t decode_smem_bytes(int H, int E, int K, int I, int Is, int nown);
-cudaError_t decode_configure(int H, int E, int K, int I, int Is, int nown);
+bool decode_plan(int H, int E, int grid, int smem_optin, int* rx, int* down_late, uint32_t* smem);
+cudaError_t decode_configure(int limit);
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream);
 }  // namespace moe
 
 using namespace moe;
 
-constexpr size_t kScratchBytes = 512u << 10;  // 512 KiB per device
+constexpr size_t kScratchBytes = 2u << 20;  // 2 MiB per device
 
 // The scratch array.  In host code this name is only a stand-in for the symbol, not a
 // device address: the address comes from cudaGetSymbolAddress, once per device.
@@ -32,14 +31,16 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 std::mutex g_mu;
-uint8_t* g_addr[kMaxDevices];     // device address of g_scratch, per device
-uint32_t g_smem_set[kMaxDevices];  // largest shared-memory limit set so far, per device
+uint8_t* g_addr[kMaxDevices];  // device address of g_scratch, per device
+bool g_configured[kMaxDevices];  // kernel shared-memory limit raised to the device maximum
 
 struct Carve {
-  size_t ctrl, h, part, sq, z, acodes, pin, base, npin, rown, rstamp, rclock, hist, log, done, total;
+  size_t ctrl, acc, zll, pin, base, npin, rown, rstamp, rclock, done, reset_end, hist, log, total;
 };
 
-Carve carve(int L, int H, int E, int K, int I, int Is) {
+// Everything a step depends on comes first and is reset by every call (one memset);
+// the histogram and log after it are only written by the kernel.
+Carve carve(int L, int H, int E, int K) {
   Carve c{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -48,22 +49,19 @@ Carve carve(int L, int H, int E, int K, int I, int Is) {
     off += bytes;
     return r;
   };
-  const int nch = H / kChunk, n_exp = K + (Is > 0), imax = I > Is ? I : Is;
   c.ctrl = take(sizeof(Ctrl));
-  c.h = take(4u * H);
-  c.part = take(4u * (size_t)E * nch);
-  c.sq = take(4u * nch);
-  c.z = take(4u * E);
-  c.acodes = take((size_t)kACodeBytes * n_exp * (imax / 32));
+  c.acc = take(8u * kAccBufs * (size_t)H);
+  c.zll = take(8u * (size_t)E);
   c.pin = take(4u * (size_t)L * E);
   c.base = take(4u * L);
   c.npin = take(4u * L);
   c.rown = take(4u * 2 * L);
   c.rstamp = take(4u * 2 * L);
   c.rclock = take(4u * 2 * L);
+  c.done = take(4u);
+  c.reset_end = off;
   c.hist = take(4u * (size_t)L * E);
   c.log = take(4u * 7 * (size_t)L * K);
-  c.done = take(4u);
   c.total = off;
   return c;
 }
@@ -90,16 +88,18 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
   if (L < 1 || H < 32 || H % 32 || H > kMaxH || K < 1 || K > kMaxK || E < K || E > kMaxE) return MOE_ERR_INVALID;
   if (I < 32 || I % 32 || Is < 0 || Is % 32 || (Is > 0 && !w->shared_dev)) return MOE_ERR_INVALID;
   if ((cfg->use_rmsnorm != 0 && cfg->use_rmsnorm != 1) || !(cfg->rms_eps >= 0.0f)) return MOE_ERR_INVALID;
+  const Carve cv = carve(L, H, E, K);
+  if (cv.total > kScratchBytes) return MOE_ERR_UNSUPPORTED;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev != cfg->device || dev < 0 || dev >= kMaxDevices)
     return MOE_ERR_INVALID;
-  const Carve cv = carve(L, H, E, K, I, Is);
-  if (cv.total > kScratchBytes) return MOE_ERR_UNSUPPORTED;
-  int nsm = 0;
-  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
-  const int nch = H / kChunk, nown = (nch + nsm - 1) / nsm;
-  if (nown > kMaxOwn) return MOE_ERR_UNSUPPORTED;
-  const uint32_t smem = decode_smem_bytes(H, E, K, I, Is, nown);
+  int nsm = 0, optin = 0;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int rx = 0, down_late = 0;
+  uint32_t smem = 0;
+  if (!decode_plan(H, E, nsm, optin, &rx, &down_late, &smem)) return MOE_ERR_UNSUPPORTED;
   uint8_t* base = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -108,13 +108,9 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
       if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
       g_addr[dev] = static_cast<uint8_t*>(ptr);
     }
-    if (smem > g_smem_set[dev]) {
-      int optin = 0;
-      if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-        return MOE_ERR_CUDA;
-      if (smem > (uint32_t)optin) return MOE_ERR_UNSUPPORTED;
-      if (decode_configure(H, E, K, I, Is, nown) != cudaSuccess) return MOE_ERR_CUDA;
-      g_smem_set[dev] = smem;
+    if (!g_configured[dev]) {  // every kernel instance, up to the device's limit
+      if (decode_configure(optin) != cudaSuccess) return MOE_ERR_CUDA;
+      g_configured[dev] = true;
     }
     base = g_addr[dev];
   }
@@ -130,16 +126,16 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
   p.R = 0;
   p.use_norm = cfg->use_rmsnorm;
   p.eps = cfg->rms_eps;
-  p.nch = nch;
   p.n_units = K * (I / 32) + Is / 32;
-  p.n_exp = K + (Is > 0 ? 1 : 0);
-  p.nown = nown;
+  p.rx_per_cta = rx;
+  p.down_late = down_late;
+  p.miss_mode = kMissProxy;  // never used: every expert is resident
+  p.nan_on_error = 1;        // no moe_sync here: a failed step shows as NaN outputs
   p.pool = w->experts_dev;
-  p.lay = slot_layout(H, I);
-  p.slot_bytes = p.lay.bytes;
-  p.slay = slot_layout(H, Is > 0 ? Is : 32);
+  p.slot_bytes = slot_layout(H, I).bytes;
+  p.unit_bytes = slot_layout(H, I).unit;
   p.shared_pool = w->shared_dev;
-  p.shared_slot_bytes = Is > 0 ? p.slay.bytes : 0;
+  p.shared_slot_bytes = Is > 0 ? slot_layout(H, Is).bytes : 0;
   p.router = w->router_dev;
   p.bias = w->bias_dev;
   p.gain = w->gain_dev;
@@ -154,22 +150,23 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
   p.y = y_dev;
   p.h_trace = nullptr;
   p.w_trace = nullptr;
-  p.h = reinterpret_cast<float*>(base + cv.h);
-  p.part = reinterpret_cast<float*>(base + cv.part);
-  p.sq = reinterpret_cast<float*>(base + cv.sq);
-  p.z = reinterpret_cast<float*>(base + cv.z);
-  p.acodes = base + cv.acodes;
+  p.acc = reinterpret_cast<unsigned long long*>(base + cv.acc);
+  p.zll = reinterpret_cast<unsigned long long*>(base + cv.zll);
   p.hist = reinterpret_cast<uint32_t*>(base + cv.hist);
   p.log = reinterpret_cast<int32_t*>(base + cv.log);
   p.log_steps = 1;
   p.ctrl = reinterpret_cast<Ctrl*>(base + cv.ctrl);
-  p.mbox = nullptr;  // no misses: every expert is resident
+  p.mbox = nullptr;
   p.done_seq = reinterpret_cast<const uint32_t*>(base + cv.done);
+  p.host_tier = nullptr;
   p.timeout_ns = (unsigned long long)(cfg->wait_timeout_ms ? cfg->wait_timeout_ms : 2000) * 1000000ull;
   p.phase_trace = nullptr;
+  p.likely = nullptr;
+  p.n_likely = 0;
 
-  // start from a clean control block (step 0, no error, arrival counters 0) every call
-  if (cudaMemsetAsync(base + cv.ctrl, 0, sizeof(Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
+  // a clean start every call: control block (step 0, no error, counter 0), accumulators,
+  // logit words and tables
+  if (cudaMemsetAsync(base, 0, cv.reset_end, st) != cudaSuccess) return MOE_ERR_CUDA;
   resident_tables<<<(L * E + 255) / 256, 256, 0, st>>>(reinterpret_cast<int32_t*>(base + cv.pin),
                                                        reinterpret_cast<int32_t*>(base + cv.base),
                                                        reinterpret_cast<int32_t*>(base + cv.npin), L, E);

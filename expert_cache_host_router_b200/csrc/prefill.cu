@@ -568,9 +568,9 @@ __global__ void __launch_bounds__(kGT, 1)
               tma_load_5d(dd + half * (kTN / 2) * 16, &maps.scl[sh], (ks >> 2) * 16, 0, 2 * half, 4 * t.nt, t.slot,
                           bar);
             }
-          } else {  // 256 down rows: 16-row tiles 16 nt .. 16 nt + 15
-            tma_load_4d(dq, &maps.nib[sh], ks * 32, 0, 16 * t.nt, t.slot, bar);
-            tma_load_4d(dd, &maps.scl[sh], (ks >> 2) * 16, 0, 16 * t.nt, t.slot, bar);
+          } else {  // 256 down rows 256 nt..: blocks 2 ks, 2 ks + 1 (units), scales of 8 units
+            tma_load_4d(dq, &maps.nib[sh], 0, 16 * t.nt, 2 * ks, t.slot, bar);
+            tma_load_4d(dd, &maps.scl[sh], 0, 2 * t.nt, 8 * (ks >> 2), t.slot, bar);
           }
         }
       }
@@ -588,10 +588,22 @@ __global__ void __launch_bounds__(kGT, 1)
           stop = true;
           break;
         }
-        const uint8_t* rq = raw + rs * kRawStage + r * 32;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(rq);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(rq + 16);
-        const uint32_t sc = *reinterpret_cast<const uint32_t*>(raw + rs * kRawStage + kRawNib + r * 16 + (ks & 3) * 4);
+        // row r's two Q4_0 blocks of this K stage and their fp16 scales (low, high half)
+        uint4 q0, q1;
+        uint32_t sc;
+        if (MODE == 0) {  // [row][2 blocks x 16 B]; scales [row][8 blocks x 2 B]
+          const uint8_t* rq = raw + rs * kRawStage + r * 32;
+          q0 = *reinterpret_cast<const uint4*>(rq);
+          q1 = *reinterpret_cast<const uint4*>(rq + 16);
+          sc = *reinterpret_cast<const uint32_t*>(raw + rs * kRawStage + kRawNib + r * 16 + (ks & 3) * 4);
+        } else {  // [2 blocks][row][16 B]; scales [8 blocks][row][2 B]
+          const uint8_t* rq = raw + rs * kRawStage + r * 16;
+          q0 = *reinterpret_cast<const uint4*>(rq);
+          q1 = *reinterpret_cast<const uint4*>(rq + kTN * 16);
+          const uint8_t* rd = raw + rs * kRawStage + kRawNib + (ks & 3) * 2 * (kTN * 2) + r * 2;
+          sc = (uint32_t)*reinterpret_cast<const uint16_t*>(rd) |
+               ((uint32_t)*reinterpret_cast<const uint16_t*>(rd + kTN * 2) << 16);
+        }
         const int s = it % kStages;
         if (it >= kStages && !pmbar_wait_ab(&empty[s], (uint32_t)(it / kStages - 1) & 1u, abort)) {
           stop = true;
@@ -1134,32 +1146,32 @@ static int make_byte_map(PfnEncodeTiled enc, CUtensorMap* m, const void* base, i
   return r == CUDA_SUCCESS ? 0 : -1;
 }
 
-// Nibble and scale maps of one weight kind.  Gate/up (MODE 0): a slot's tiles are
-// (row block rb of I/32, subtile st of 4) at (4 rb + st) * 9H, each [16 rows x H/32 x 16 B]
-// then [16 rows x H/32 x 2 B]; a box is 16 rows x 2 subtiles x 4 row blocks = 128 rows.
-// Down (MODE 1): 16-row tiles c of H at down + c * 9I; a box is 16 rows x 16 tiles = 256 rows.
+// Nibble and scale maps of one weight kind over the unit layout of moe_internal.h (unit
+// rb of a slot at rb * unit).  Gate/up (MODE 0): tiles (rb, subtile st of 4) at
+// rb * unit + st * 9H, each [16 rows x H/32 x 16 B] then [16 rows x H/32 x 2 B]; a box
+// is 16 rows x 2 subtiles x 4 units = 128 rows, 2 blocks (nibbles) or 8 blocks (scales)
+// wide.  Down (MODE 1): unit rb holds block rb of every row j, nibbles at 36H + 16 j and
+// scales at 52H + 2 j; a nibble box is 256 rows x 2 units, a scale box 256 rows x 8 units.
 static int make_weight_maps(PfnEncodeTiled enc, int mode, const uint8_t* pool, uint64_t n_slots, uint64_t slot_bytes,
                             const SlotLayout& lay, int H, int I, CUtensorMap* nib, CUtensorMap* scl) {
   if (mode == 0) {
     const uint64_t nbk = H / 32, tile = 9ull * H;
     const cuuint64_t dq[5] = {nbk * 16, 16, 4, (cuuint64_t)I / 32, n_slots};
-    const cuuint64_t sq[4] = {nbk * 16, tile, 4 * tile, slot_bytes};
+    const cuuint64_t sq[4] = {nbk * 16, tile, lay.unit, slot_bytes};
     const cuuint32_t bq[5] = {32, 16, 2, 4, 1};
     const cuuint64_t dd[5] = {nbk * 2, 16, 4, (cuuint64_t)I / 32, n_slots};
-    const cuuint64_t sd[4] = {nbk * 2, tile, 4 * tile, slot_bytes};
+    const cuuint64_t sd[4] = {nbk * 2, tile, lay.unit, slot_bytes};
     const cuuint32_t bd[5] = {16, 16, 2, 4, 1};
-    return make_byte_map(enc, nib, pool + lay.gu, 5, dq, sq, bq) ||
-           make_byte_map(enc, scl, pool + lay.gu + 16 * nbk * 16, 5, dd, sd, bd);
+    return make_byte_map(enc, nib, pool, 5, dq, sq, bq) || make_byte_map(enc, scl, pool + 16 * nbk * 16, 5, dd, sd, bd);
   }
-  const uint64_t nbk = I / 32, tile = 9ull * I;
-  const cuuint64_t dq[4] = {nbk * 16, 16, (cuuint64_t)H / 16, n_slots};
-  const cuuint64_t sq[3] = {nbk * 16, tile, slot_bytes};
-  const cuuint32_t bq[4] = {32, 16, 16, 1};
-  const cuuint64_t dd[4] = {nbk * 2, 16, (cuuint64_t)H / 16, n_slots};
-  const cuuint64_t sd[3] = {nbk * 2, tile, slot_bytes};
-  const cuuint32_t bd[4] = {16, 16, 16, 1};
-  return make_byte_map(enc, nib, pool + lay.down, 4, dq, sq, bq) ||
-         make_byte_map(enc, scl, pool + lay.down + 16 * nbk * 16, 4, dd, sd, bd);
+  const cuuint64_t dq[4] = {256, (cuuint64_t)H / 16, (cuuint64_t)I / 32, n_slots};
+  const cuuint64_t sq[3] = {256, lay.unit, slot_bytes};
+  const cuuint32_t bq[4] = {256, 16, 2, 1};
+  const cuuint64_t dd[4] = {256, (cuuint64_t)H / 128, (cuuint64_t)I / 32, n_slots};
+  const cuuint64_t sd[3] = {256, lay.unit, slot_bytes};
+  const cuuint32_t bd[4] = {256, 2, 8, 1};
+  return make_byte_map(enc, nib, pool + unit_down_nib(H), 4, dq, sq, bq) ||
+         make_byte_map(enc, scl, pool + unit_down_scl(H), 4, dd, sd, bd);
 }
 
 // Tokens per pass: every GEMM CTA's tiles must fit its tile table.

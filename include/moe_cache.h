@@ -117,7 +117,15 @@ typedef struct {
   uint64_t repin_copies; /* experts copied host-to-device by those re-pins */
   uint64_t miss_requests; /* miss requests the kernel has issued since create */
   uint64_t miss_served;   /* miss requests the proxy has taken from the mailbox since create */
-  int32_t proxy_error;    /* 1 if the proxy met a malformed request (left unsignalled) */
+  int32_t proxy_error;    /* 0; 1 the proxy met a malformed request, 2 a copy could not be
+                             enqueued, 3 its completion signal could not be enqueued (each
+                             left unsignalled: the step ends with MOE_ERR_TIMEOUT) */
+  int32_t miss_path;      /* MOE_MISS_COPY_ENGINE or MOE_MISS_SM_PULL */
+  uint64_t pulled_misses; /* misses served by the kernel's own reads of host memory since the last reset */
+  uint64_t copies_timed;  /* proxy copies whose duration was measured (CUDA events on the side
+                             stream around each copy) since the last reset */
+  uint64_t copy_ns_timed; /* their summed device durations, ns: copies_timed * slot bytes /
+                             copy_ns_timed is the host-to-device rate of the miss path itself */
 } moe_stats_t;
 
 #define MOE_DEVERR_BARRIER 1 /* grid barrier wait ran out */
@@ -125,10 +133,18 @@ typedef struct {
 #define MOE_DEVERR_TMA 3     /* wait for a bulk shared-memory load ran out */
 #define MOE_DEVERR_ROUTE 4   /* a logit was NaN: no valid top-k */
 #define MOE_DEVERR_SLOT 5    /* an expert had no slot (cold with an empty ring) */
+#define MOE_DEVERR_RANGE 6   /* a unit's share of a layer output was not finite or |v| >= 2^26 */
 
-/* Create a context on cfg->device: allocates the pinned host tier (all experts), the
- * device tables and the proxy thread that serves miss copies.  weights may be NULL
- * (then load layers with moe_load_layer).  *out is set only on MOE_OK. */
+/* Miss-path variants for moe_set_miss_path. */
+#define MOE_MISS_COPY_ENGINE 0 /* host proxy thread + cudaMemcpyAsync on a side stream (default) */
+#define MOE_MISS_SM_PULL 1     /* the kernel's CTAs read the expert from mapped pinned host memory */
+
+/* Create a context on cfg->device: allocates the pinned host tier that holds every
+ * expert (the write-up's long tail "in system RAM", baguaai.com event core; "pinned host
+ * memory", theneuralfeed.com key components item 2), the device tables, and the proxy
+ * thread that serves miss copies.  weights may be NULL (then load layers with
+ * moe_load_layer).  *out is set only on MOE_OK.  MOE_ERR_UNSUPPORTED when the decode
+ * kernel's shared-memory plan for the shape does not fit the device. */
 MOE_API int moe_create(const moe_config *cfg, const moe_weights *weights, moe_ctx **out);
 
 /* Load (or replace) one layer's weights.  Experts go to the pinned host tier in the
@@ -159,7 +175,9 @@ MOE_API int moe_recalibrate(moe_ctx *ctx);
  * traffic whose popularity has drifted.  Synchronises the device. */
 MOE_API int moe_set_router_bias(moe_ctx *ctx, int32_t layer, const float *bias);
 
-/* One decode step (one token through all L layers) as one graph launch on stream:
+/* One decode step (one token through all L layers) as one graph launch on stream (the
+ * write-up's fused token, theneuralfeed.com key components item 3: one graph instead of
+ * 40 per-layer graphs; the cache of items 1 and 2 decides where each expert is read):
  * reads x_dev [H] fp32, writes y_dev [H] fp32 (h_L of the stack, or MoE(x) when
  * use_rmsnorm = 0).  Routing, the histogram, the cache and the event log advance.
  * Asynchronous: device-side failures surface at moe_sync / moe_stats.
@@ -177,7 +195,9 @@ MOE_API int moe_decode_step_host(moe_ctx *ctx, const float *x_host, float *y_hos
 
 /* Batched prefill: n_tokens tokens through the whole stack at once, x_dev [T][H] ->
  * y_dev [T][H] (fp32, device, caller-owned, may not overlap), enqueued on stream.
- * The pages describe decode; this is the same layer computed for a batch: per layer,
+ * The pages describe decode only; this is the same layer computed for a batch of tokens
+ * (a 2048-token prompt through the 40-layer stack is the workload it is sized for), the
+ * one place where the expert FFNs are dense contractions: per layer,
  * each token's top-k is the one the canonical fp32 logits give, as in decode (found
  * from tensor-core approximate logits, certified against exact canonical logits of the
  * candidates), so it agrees with a decode of the same hidden state; the routing
@@ -210,7 +230,10 @@ MOE_API int moe_sync(moe_ctx *ctx);
  * may be torn), resynchronises the miss queue and the grid barrier. */
 MOE_API int moe_clear_error(moe_ctx *ctx);
 
-/* Counters, histogram and event log.  Synchronises the device.  hist_out: [L][E] or
+/* Counters, histogram and event log: the routing-frequency histogram that calibrated
+ * placement accumulates (theneuralfeed.com key components item 1) and the hit / miss /
+ * eviction record behind the write-up's cold-hit rate (items 1 and 2, the 36% -> 7%
+ * figure).  Synchronises the device.  hist_out: [L][E] or
  * NULL.  log_out: room for log_cap events or NULL; receives the events of the steps
  * not yet read, oldest first, and *log_n their count.  reset != 0 zeroes the counters
  * and the histogram after reading. */
@@ -222,14 +245,42 @@ MOE_API int moe_stats(moe_ctx *ctx, moe_stats_t *out, uint32_t *hist_out, moe_ev
  * the routing weights.  Pass NULLs to stop.  Device pointers owned by the caller. */
 MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
 
-/* Phase timing: when stamps_dev ([(L+1)][32] + [L][n_sm][4] uint64, device) is non-NULL, every decode
- * step writes the GPU global timer (ns) of CTA 0 at its phase boundaries: per layer l,
- * [l][0] layer start, [1] logits ready, [2] routing and cache decided, [3] gate/up done
- * (this CTA), [4] all gate/up done, [5] down done (this CTA), [6] layer done, [7..31]
- * finer marks inside routing, gate/up and the down phase; [L][0] kernel start, [L][1] prologue
- * done, [L][2] kernel end.  Then, for every layer and every CTA (one per SM): [0] routing
- * done, [1] gate/up published, [2] down done, [3] barrier passed.  NULL stops it. */
-MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev);
+/* Phase timing: when stamps_dev is non-NULL, every decode step writes GPU global-timer
+ * values (ns) there.  The buffer holds n_words uint64 and must hold at least
+ * (L + 1) * 32 + L * n_sm * 4 words (n_sm = the device's SM count, one CTA per SM):
+ * else MOE_ERR_INVALID and nothing changes.  Layout: first [(L+1)][32] marks of CTA 0;
+ * per layer l: [l][0] layer start, [1] the previous layer's output complete, [2] h
+ * updated, [3] own logits published and input quantised, [4] all logits read, [5]
+ * routing and cache decided, [6] unit loads issued, [7] gate/up computed, [8] units
+ * done, [9] arrival posted; [L][0] kernel start, [L][1] prologue done, [L][2] kernel
+ * end.  Then [L][n_sm][4] marks of every CTA: [0] routing decided, [1] units done,
+ * [2] arrival posted, [3] unused.  NULL stops it (n_words ignored). */
+MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev, size_t n_words);
+
+/* Miss path (the survey's next-row variants of key components item 2): with
+ * MOE_MISS_COPY_ENGINE (the default) the kernel posts a cold expert to a host-mapped
+ * mailbox, the library's proxy thread copies it pinned host -> ring slot with
+ * cudaMemcpyAsync on a side stream and signals the kernel through a stream memory write;
+ * with MOE_MISS_SM_PULL the CTAs that compute the expert read it themselves from the
+ * mapped pinned host tier and write the ring slot, with no host thread involved.  Both
+ * give the same routing, event log and outputs.  Other values: MOE_ERR_INVALID. */
+MOE_API int moe_set_miss_path(moe_ctx *ctx, int32_t mode);
+
+/* Speculative L2 prefetch: at the start of every layer, while the layer's routing is
+ * computed and the HBM would otherwise idle, the kernel prefetches into L2 the slots of
+ * the n_experts pinned experts that the placement histogram (decayed by recalibration)
+ * routes to most often; the expert loads that follow routing then hit L2 for the
+ * predicted experts.  Changes no result, only where bytes come from; mispredicted
+ * prefetches cost HBM bandwidth that would otherwise be idle.  0 (the default) turns it
+ * off; at most 16.  Synchronises the device. */
+MOE_API int moe_set_prefetch(moe_ctx *ctx, int32_t n_experts);
+
+/* Host-to-device rate of the miss path's own copy: n_copies expert slots copied back to
+ * back from the library's pinned host tier into device slots with cudaMemcpyAsync on the
+ * side stream the proxy uses (after one untimed pass), timed with CUDA events.  *gbs =
+ * n_copies * slot bytes / elapsed, in GB/s (1e9 B/s).  Needs a residency; synchronises
+ * the device; do not call it while a decode step is in flight. */
+MOE_API int moe_measure_h2d(moe_ctx *ctx, int32_t n_copies, double *gbs);
 
 /* Fault injection for tests: the miss proxy issues the next n copies but never
  * signals them, so the kernel's bounded wait runs out (no GPU fault involved).  The
@@ -241,15 +292,15 @@ MOE_API int moe_debug_drop_signals(moe_ctx *ctx, int32_t n);
  * resident, in the library's own layouts (a byte regrouping of the canonical Q4_0
  * blocks, values unchanged):
  *   experts_dev: [L][E] routed experts, one slot each, slots slot_bytes(I) apart, where
- *     slot_bytes(W) = 3 * H * W * 9 / 16 rounded up to a multiple of 256.  A slot is a
- *     run of tiles; a tile is 16 matrix rows stored as [16 rows x K/32 blocks x 16
- *     nibble bytes] followed by [16 rows x K/32 fp16 scales].  First, for each 32-row
- *     block rb of the width W: gate rows 32rb..+15, gate rows 32rb+16..+31, up rows
- *     32rb..+15, up rows 32rb+16..+31 (K = H); then, for each chunk c of 16 rows of H,
- *     down rows 16c..16c+15 (K = W).
+ *     slot_bytes(W) = (W / 32) * 54 * H rounded up to a multiple of 256.  A slot is W/32
+ *     units of 54 H bytes; unit rb holds, in order: four gate/up tiles (gate rows
+ *     32rb..+15, gate rows 32rb+16..+31, up rows 32rb..+15, up rows 32rb+16..+31), each
+ *     [16 rows x H/32 blocks x 16 nibble bytes] then [16 rows x H/32 fp16 scales]; then
+ *     the nibble bytes of Q4_0 block rb of every down row j = 0..H-1 ([H x 16] bytes);
+ *     then the fp16 scales of those blocks ([H] x 2 bytes).
  *   shared_dev: [L] shared experts in the same layout with W = shared_inter, slots
  *     slot_bytes(shared_inter) apart; NULL when shared_inter = 0.
- *   router_dev: [L][H/16][E][16] bf16, i.e. W_r[l][e][16 c + t] at ((l H/16 + c) E + e) 16 + t.
+ *   router_dev: [L][E][H] bf16 bit patterns (the canonical router rows).
  *   bias_dev: [L][E] fp32 or NULL; gain_dev: [L][H] fp32 or NULL. */
 typedef struct {
   const uint8_t *experts_dev;
@@ -266,16 +317,20 @@ typedef struct {
  * corresponds to it; it is a deployment variant of the same kernel and arithmetic.
  *
  * It allocates nothing: no context, no graph, no cudaMalloc / cudaFree.  Its scratch
- * (exchange buffers, grid-barrier word, slot tables, histogram, one step of event log)
- * lives in a static 512 KiB device array that every GPU which loads the library holds
- * until the process exits; the call rejects shapes whose scratch would not fit
- * (MOE_ERR_UNSUPPORTED).  All experts must be resident (no cache, no miss path); cfg's
- * ring_slots and log_steps are ignored.  Reads x_dev [H], writes y_dev [H] on stream
- * (the current device must be cfg->device).  The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress) and sets the kernel's shared-memory
- * limit: make that first call before any stream capture.  Every call shares the array
- * and overwrites it (it is cleared at the start of each call): calls that overlap on
- * the GPU, on any stream, race.  Asynchronous; returns the launch status. */
+ * (control block with the arrival counter and error word, output accumulators,
+ * published logits, slot tables, histogram, one step of event log) lives in a static
+ * 2 MiB device array that every GPU which loads the library holds until the process
+ * exits; the call rejects shapes whose scratch would not fit (MOE_ERR_UNSUPPORTED).  All
+ * experts must be resident (no cache, no miss path); cfg's ring_slots and log_steps are
+ * ignored.  Reads x_dev [H], writes y_dev [H] on stream (the current device must be
+ * cfg->device).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and sets the kernel's shared-memory limit: make that first call
+ * before any stream capture.  Each call resets the parts of the array a step depends on
+ * (control block, accumulators, logit words, slot tables) and leaves the rest (histogram
+ * and event log) as the kernel writes it; every call shares the array, so calls that
+ * overlap on the GPU, on any stream, race.  Asynchronous; returns the launch status.  A
+ * step that fails on the device (a bounded wait that ran out, an out-of-range value)
+ * writes NaN to every element of y_dev, since this entry point has no moe_sync. */
 MOE_API int moe_decode_step_noalloc(const moe_config *cfg, const moe_noalloc_weights *w,
                                     const float *x_dev, float *y_dev, void *stream);
 

@@ -77,7 +77,10 @@ def test_null_arguments_are_rejected(lib):
     assert lib.moe_recalibrate(None) == moe.MOE_ERR_INVALID
     assert lib.moe_set_router_bias(None, 0, None) == moe.MOE_ERR_INVALID
     assert lib.moe_set_prefill_trace(None, None, None) == moe.MOE_ERR_INVALID
-    assert lib.moe_set_phase_trace(None, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_phase_trace(None, None, 0) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_miss_path(None, 0) == moe.MOE_ERR_INVALID
+    assert lib.moe_measure_h2d(None, 1, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_prefetch(None, 0) == moe.MOE_ERR_INVALID
     lib.moe_destroy(None)  # no-op
 
 
@@ -89,7 +92,8 @@ _STRUCTS = {
     "moe_event": ("Event", ["step", "layer", "rank", "expert", "kind", "slot", "evicted"]),
     "moe_stats_t": ("Stats", ["steps", "accesses", "pin_hits", "ring_hits", "misses", "evictions", "bytes_copied",
                               "staged_misses", "log_dropped", "device_error", "n_pinned", "residency", "placement",
-                              "repins", "repin_copies", "miss_requests", "miss_served", "proxy_error"]),
+                              "repins", "repin_copies", "miss_requests", "miss_served", "proxy_error",
+                              "miss_path", "pulled_misses", "copies_timed", "copy_ns_timed"]),
 }
 
 

@@ -134,17 +134,25 @@ def test_stack_teacher_forced_and_free_running():
     _, _, log = m.stats(log_cap=3 * s.n_layers * s.top_k)
     sels = _sels_from_log(log, 3, s)
     _check_teacher_forced(orc, s, xs, ys, hs, ws, sels)
+    compared = 0
     for t, x in enumerate(xs):
         h, sel, _ = orc.decode(x)
+        # a free-running stack may legitimately route differently after a near-tie (the
+        # teacher-forced check above holds every layer exactly); compare where it agreed
         if np.array_equal(sel, sels[t]):
-            assert np.linalg.norm(ys[t] - h) <= STACK_TOL * np.linalg.norm(h)
+            assert np.linalg.norm(ys[t] - h) <= STACK_TOL * np.linalg.norm(h), t
+            compared += 1
+    assert compared >= 1, "no token's free-running routing agreed with the oracle's"
     m.close()
 
 
-def test_residency_levels_bit_identical_and_cache_log_exact():
+@pytest.mark.parametrize("miss_path", ["copy_engine", "sm_pull"])
+def test_residency_levels_bit_identical_and_cache_log_exact(miss_path):
+    import expert_cache_host_router_b200 as moe
     s = STACK
     layers = make_layers(s)
     m = build_gpu(s, layers, log_steps=64)
+    m.set_miss_path(moe.MOE_MISS_SM_PULL if miss_path == "sm_pull" else moe.MOE_MISS_COPY_ENGINE)
     m.set_residency(1.0)
     calib = synthetic.tokens(0, 16, s.hidden, synthetic.SEED_CALIB)
     _run_tokens(m, calib)
@@ -164,6 +172,7 @@ def test_residency_levels_bit_identical_and_cache_log_exact():
         ref_log, _ = oracle_events(s, sels, masks, first_step=int(log["step"][0]))
         assert events_equal(log, ref_log), (frac, place)
         assert st["misses"] == int(np.sum(log["kind"] == 2))
+        assert st["pulled_misses"] == (st["misses"] if miss_path == "sm_pull" else 0)
         outs[(frac, place)] = ys
     base = outs[(1.0, 0)]
     for key, ys in outs.items():
@@ -171,13 +180,16 @@ def test_residency_levels_bit_identical_and_cache_log_exact():
     m.close()
 
 
-def test_ring_smaller_than_top_k_stages_misses():
+@pytest.mark.parametrize("miss_path", ["copy_engine", "sm_pull"])
+def test_ring_smaller_than_top_k_stages_misses(miss_path):
     """R=2 < k=4: a layer can miss more often than it has ring slots; the log still
     follows the oracle's LRU exactly and the output stays bit-identical."""
+    import expert_cache_host_router_b200 as moe
     s = synthetic.Shape(n_layers=2, hidden=512, n_experts=64, top_k=4, inter=256, shared_inter=0,
                         ring_slots=2, use_rmsnorm=1, zipf_s=0.0)
     layers = make_layers(s)
     m = build_gpu(s, layers)
+    m.set_miss_path(moe.MOE_MISS_SM_PULL if miss_path == "sm_pull" else moe.MOE_MISS_COPY_ENGINE)
     m.set_residency(1.0)
     xs = synthetic.tokens(3, 10, s.hidden)
     base, _, _ = _run_tokens(m, xs)
