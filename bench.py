@@ -493,8 +493,8 @@ def run_ours(args):
     layers = [synthetic.layer_weights(l, shape) for l in range(shape.n_layers)]
     gen_s = time.time() - t0
     m = moe.ExpertCacheMoE(shape, device=local, log_steps=max(4096, args.steps + args.warmup + 16))
-    if args.prefetch:
-        m.set_prefetch(args.prefetch)
+    if any(args.prefetch):
+        m.set_prefetch(*args.prefetch)
     t0 = time.time()
     for l in range(shape.n_layers):
         m.load_layer(l, layers[l])
@@ -652,13 +652,13 @@ def run_ours(args):
     if args.prefetch_sweep:
         sweep = []
         m.set_residency(1.0)
-        for n in (0, 4, 8, 12, 16):
-            m.set_prefetch(n)
+        for pre, l2 in ((0, 0), (4, 0), (6, 0), (8, 0), (8, 4), (8, 8), (0, 8)):
+            m.set_prefetch(pre, l2)
             for i in range(args.warmup):
                 m.decode(xs[i], y)
-            sweep.append({"prefetch_experts": n, **decode_point(m, shape, xs[args.warmup:], y, stream,
-                                                                min(64, args.steps))})
-        m.set_prefetch(args.prefetch)
+            sweep.append({"preload": pre, "l2": l2, **decode_point(m, shape, xs[args.warmup:], y, stream,
+                                                                 min(64, args.steps))})
+        m.set_prefetch(*args.prefetch)
         line["prefetch_sweep"] = sweep
     if args.phases == "all" and not args.no_curve:
         line["residency_curve"] = run_residency_curve(m, shape, hist, xs, y, stream, steps=min(128, len(xs)))
@@ -697,7 +697,8 @@ def main():
     ap.add_argument("--no-curve", action="store_true",
                     help="skip the residency curve and the small-shape stack")
     ap.add_argument("--prefill-runs", type=int, default=5, help="timed prefill passes")
-    ap.add_argument("--prefetch", type=int, default=0, help="likely experts prefetched into L2 per layer")
+    ap.add_argument("--prefetch", type=int, nargs=2, default=[0, 0], metavar=("PRELOAD", "L2"),
+                    help="likely experts per layer preloaded into shared memory / prefetched into L2")
     ap.add_argument("--prefetch-sweep", action="store_true", help="decode tok/s at 100%% over prefetch depths")
     ap.add_argument("--phase-trace", default=None, help="write a per-layer phase table (JSON) to this path")
     ap.add_argument("--phases", default="all", choices=["all", "100"],

@@ -105,7 +105,7 @@ _SIGS = {
     "moe_set_phase_trace": (ctypes.c_int, [_P, _P, ctypes.c_size_t]),
     "moe_set_miss_path": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_measure_h2d": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double)]),
-    "moe_set_prefetch": (ctypes.c_int, [_P, ctypes.c_int32]),
+    "moe_set_prefetch": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32]),
     "moe_debug_drop_signals": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_decode_step_noalloc": (ctypes.c_int, [ctypes.POINTER(Config), ctypes.POINTER(NoAllocWeights),
                                                 _P, _P, _P]),
@@ -235,8 +235,8 @@ def moe_set_miss_path(ctx: int, mode: int) -> None:
     _check(lib().moe_set_miss_path(ctx, mode), "moe_set_miss_path")
 
 
-def moe_set_prefetch(ctx: int, n_experts: int) -> None:
-    _check(lib().moe_set_prefetch(ctx, n_experts), "moe_set_prefetch")
+def moe_set_prefetch(ctx: int, n_preload: int, n_l2: int = 0) -> None:
+    _check(lib().moe_set_prefetch(ctx, n_preload, n_l2), "moe_set_prefetch")
 
 
 def moe_measure_h2d(ctx: int, n_copies: int) -> float:
@@ -366,8 +366,8 @@ class ExpertCacheMoE:
     def set_miss_path(self, mode: int) -> None:
         moe_set_miss_path(self.ctx, mode)
 
-    def set_prefetch(self, n_experts: int) -> None:
-        moe_set_prefetch(self.ctx, n_experts)
+    def set_prefetch(self, n_preload: int, n_l2: int = 0) -> None:
+        moe_set_prefetch(self.ctx, n_preload, n_l2)
 
     def measure_h2d(self, n_copies: int = 64) -> float:
         return moe_measure_h2d(self.ctx, n_copies)

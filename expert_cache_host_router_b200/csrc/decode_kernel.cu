@@ -238,11 +238,15 @@ struct Misc {
   uint32_t step, seq_base, n_miss;
   int32_t flag;
   int32_t P_l, base_l;
-  int32_t pre;  // the first unit of the next layer was issued ahead (shared expert)
+  // preload matching of the current layer
+  int32_t lk_e[kMaxPreload];  // expert of each preloaded group (-1: none)
+  int32_t hit[kMaxPreload];   // its rank in the layer's top-k, or -1
+  int32_t unc[kMaxK];         // ranks whose expert no group preloaded, in rank order
+  int32_t n_unc, n_avail;
 };
 
 struct SmemPlan {
-  uint32_t unit, rrows, h, g, up, xcodes, xs, xc, z, pinrow, misc, total;
+  uint32_t unit, rrows, h, g, up, xcodes, xs, xc, z, pinrow, cand, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -267,6 +271,7 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
   s.xc = take(4u * (H / 32));
   s.z = take(4u * E);
   s.pinrow = take(4u * E);
+  s.cand = take(8u * kWarps * kMaxK);
   s.misc = take(sizeof(Misc));
   s.total = align_up(off, 128);
   return s;
@@ -398,7 +403,7 @@ __device__ __noinline__ int topk_large(const DecodeParams& p, const float* zs) {
 // Warp 0: top-k of z (value desc, index asc) and the renormalised softmax weights.
 // Keys live in registers (E <= 256: 8 per lane); each round is a lane-local max and a
 // redux max / min.  Lane i returns the expert of rank i (and m.sel / m.w are set).
-__device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
+__device__ __noinline__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
   const int lane = threadIdx.x & 31;
   const int E = p.E;
   int my_e = -1;
@@ -439,6 +444,53 @@ __device__ int topk_weights(const DecodeParams& p, Misc& m, const float* zs) {
     m.w[lane] = __fdividef(ex, sum);
   }
   __syncwarp();
+  return my_e;
+}
+
+// All threads, E <= 256: the same top-k in two parallel steps.  (1) Warp w ranks its 32
+// experts 32w + lane by 64-bit key (logit desc, index asc) with shuffles; a rank below k
+// makes a candidate, stored at w k + rank.  (2) Each of the 8k candidate slots counts
+// the candidates with larger keys (shared-memory broadcasts): that count is its global
+// rank.  Then warp 0 forms the weights exactly as topk_weights does.  Lane i of warp 0
+// returns the expert of rank i.
+__device__ int topk_parallel(const DecodeParams& p, Misc& m, const float* zs, unsigned long long* cand) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.K;
+  const int e = tid;  // E <= 256 = kThreads
+  const unsigned long long key = e < p.E ? route_key(zs[e], e) : 0ull;
+  int rank = 0;
+#pragma unroll 8
+  for (int off = 1; off < 32; ++off) {
+    const unsigned long long o = shfl_xor_u64(key, off);
+    rank += o > key;
+  }
+  const int nc = kWarps * K;  // candidate slots
+  for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
+  __syncthreads();
+  if (e < p.E && rank < K) cand[warp * K + rank] = key;
+  __syncthreads();
+  for (int t = tid; t < nc; t += kThreads) {
+    const unsigned long long c = cand[t];
+    if (c == 0ull) continue;
+    int r = 0;
+    for (int q = 0; q < nc; ++q) r += cand[q] > c;
+    if (r < K) {
+      m.sel[r] = (int)(~(uint32_t)c);
+      if ((c >> 32) == 0ull) set_error(p.ctrl, MOE_DEVERR_ROUTE);  // a NaN logit was needed
+    }
+  }
+  __syncthreads();
+  int my_e = 0;
+  if (warp == 0) {
+    my_e = lane < K ? m.sel[lane] : 0;
+    if (my_e < 0 || my_e >= p.E) my_e = 0;
+    const float zmax = __shfl_sync(0xffffffffu, zs[my_e], 0);
+    const float ex = lane < K ? expf(zs[my_e] - zmax) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < K) m.w[lane] = __fdividef(ex, sum);
+    __syncwarp();
+  }
   return my_e;
 }
 
@@ -612,7 +664,7 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
 // Thread 0: bulk-load a unit (src = its first byte in a slot) into the unit buffer:
 // four gate/up tiles on bar_u[0..3] and, unless the down part comes later, the down
 // nibbles and scales (one run of 18H bytes) on bar_d.
-__device__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src) {
+__device__ __noinline__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src) {
   const uint32_t tb = 9u * p.H;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {
@@ -625,9 +677,22 @@ __device__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const 
   }
 }
 
+// All threads: wait until a unit issued ahead has landed (its copies complete the
+// current phase of the unit barriers), then advance the parities past it.
+__device__ __noinline__ bool drain_unit(const DecodeParams& p, Misc& m, uint32_t (&par_u)[4], uint32_t& par_d) {
+  bool ok = true;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) ok = ok && mbar_wait(p, &m.bar_u[st], par_u[st]);
+  if (!p.down_late) ok = ok && mbar_wait(p, &m.bar_d, par_d);
+#pragma unroll
+  for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
+  if (!p.down_late) par_d ^= 1u;
+  return ok;
+}
+
 // All threads: copy a unit from the mapped pinned host tier into its slot (pull mode),
 // then order those writes before the bulk copies that read the slot back.
-__device__ void pull_unit(const DecodeParams& p, const uint8_t* host, uint8_t* dst) {
+__device__ __noinline__ void pull_unit(const DecodeParams& p, const uint8_t* host, uint8_t* dst) {
   const uint4* s = reinterpret_cast<const uint4*>(host);
   uint4* d = reinterpret_cast<uint4*>(dst);
   const uint32_t n16 = (uint32_t)(p.unit_bytes / 16);
@@ -651,8 +716,8 @@ __device__ void pull_unit(const DecodeParams& p, const uint8_t* host, uint8_t* d
 // One thread: this CTA's share of a layer's speculative prefetch: the slots of the
 // layer's most frequently routed pinned experts (slots, loaded beforehand), as one byte
 // range split evenly over the grid.
-__device__ void prefetch_likely(const DecodeParams& p, const int32_t (&slots)[kMaxLikely]) {
-  const uint64_t sb = p.slot_bytes, total = (uint64_t)p.n_likely * sb;
+__device__ __noinline__ void prefetch_likely(const DecodeParams& p, const int32_t (&slots)[kMaxLikely]) {
+  const uint64_t sb = p.slot_bytes, total = (uint64_t)p.n_l2 * sb;
   const uint64_t per = ((total + gridDim.x - 1) / gridDim.x + 255) / 256 * 256;
   uint64_t lo = (uint64_t)blockIdx.x * per;
   const uint64_t hi = lo + per < total ? lo + per : total;
@@ -662,10 +727,91 @@ __device__ void prefetch_likely(const DecodeParams& p, const int32_t (&slots)[kM
     int32_t slot = -1;
 #pragma unroll
     for (int q = 0; q < kMaxLikely; ++q)
-      if (q == m) slot = slots[q];
+      if (q == m + p.n_pre) slot = slots[q];
     if (slot >= 0) bulk_prefetch_l2(p.pool + (size_t)slot * sb + in, (uint32_t)(end - lo));
     lo = end;
   }
+}
+
+// The k-th unit of CTA b in this layer: rank i (K = the shared expert), block rb, and
+// whether its bytes are already in flight (issued ahead).  With at least one CTA per
+// unit: CTAs [0, n_pre Ur) hold a preload of unit b mod Ur of likely expert b / Ur and
+// compute it if that expert was routed (any rank); CTAs [routed, n_units) own the
+// shared expert's units; every other CTA (a wrong preload, no preload, no unit) is
+// "available" and the j-th of them takes the j-th unit of the ranks no preload covered,
+// in rank order.  Every CTA derives the same assignment from the same routing.
+struct UnitRef {
+  int i, rb;
+  bool shared, issued;
+};
+
+__device__ __forceinline__ bool unit_of(const DecodeParams& p, const Misc& m, bool pre, int b, int G, int k,
+                                        UnitRef& u) {
+  const int Ur = p.I / 32, routed = p.K * Ur;
+  if (G < p.n_units) {  // fewer CTAs than units: round robin, no preload
+    const int uu = b + k * G;
+    if (uu >= p.n_units) return false;
+    u.shared = uu >= routed;
+    u.i = u.shared ? p.K : uu / Ur;
+    u.rb = u.shared ? uu - routed : uu % Ur;
+    u.issued = k == 0 && pre && u.shared;
+    return true;
+  }
+  const int npc = p.n_pre * Ur;
+  if (b >= routed && b < p.n_units) {
+    if (k > 0) return false;
+    u.shared = true;
+    u.i = p.K;
+    u.rb = b - routed;
+    u.issued = pre;
+    return true;
+  }
+  if (b < npc && m.hit[b / Ur] >= 0) {
+    if (k > 0) return false;
+    u.shared = false;
+    u.i = m.hit[b / Ur];
+    u.rb = b % Ur;
+    u.issued = true;
+    return true;
+  }
+  // available CTAs in order: those without a unit (no preload to wait for), those that
+  // preloaded nothing, then those whose preload was not routed
+  int a;
+  const int idle = max(G - p.n_units, 0);
+  if (b >= p.n_units) {
+    a = b - p.n_units;
+  } else if (b >= npc) {
+    a = idle + (b - npc);
+  } else {
+    a = idle + (routed - npc) + b % Ur;
+    for (int q = 0; q < b / Ur; ++q)
+      if (m.hit[q] < 0) a += Ur;
+  }
+  const int j = a + k * m.n_avail;
+  if (j >= m.n_unc * Ur) return false;
+  u.shared = false;
+  u.i = m.unc[j / Ur];
+  u.rb = j % Ur;
+  u.issued = false;
+  return true;
+}
+
+// All threads of every CTA: the deferred ring fills (staging slot -> ring slot), split
+// over the grid.
+__device__ __noinline__ void ring_fills(const DecodeParams& p, const Misc& m) {
+  const size_t n16 = p.slot_bytes / 16;
+  for (int f = 0; f < m.n_fix; ++f) {
+    const uint4* s = reinterpret_cast<const uint4*>(p.pool + (size_t)m.fix_src[f] * p.slot_bytes);
+    uint4* d = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) + (size_t)m.fix_dst[f] * p.slot_bytes);
+    for (size_t t = (size_t)blockIdx.x * kThreads + threadIdx.x; t < n16; t += (size_t)gridDim.x * kThreads)
+      d[t] = __ldcg(s + t);
+  }
+}
+
+// One thread: the pool slots of layer l's likely experts.
+__device__ __noinline__ void load_likely(const DecodeParams& p, int l, int32_t (&lk)[kMaxLikely]) {
+#pragma unroll
+  for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely_slot + (size_t)l * kMaxLikely + q);
 }
 
 // All threads: h += y (or h = y without the residual) from a layer's accumulator; all of
@@ -673,21 +819,23 @@ __device__ void prefetch_likely(const DecodeParams& p, const int32_t (&slots)[kM
 // per element).  trace: where to write the new h, or null.
 __device__ __forceinline__ void add_layer_output(const DecodeParams& p, const unsigned long long* acc, float* hs,
                                                  float* trace) {
-  constexpr int kPer = kMaxH / kThreads;  // 16
-  long long v[kPer];
+  constexpr int kPer = 8;
+  for (int j0 = 0; j0 < p.H; j0 += kPer * kThreads) {
+    long long v[kPer];
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int j = threadIdx.x + k * kThreads;
-    v[k] = j < p.H ? (long long)__ldcg(acc + j) : 0;
-  }
+    for (int k = 0; k < kPer; ++k) {
+      const int j = j0 + threadIdx.x + k * kThreads;
+      v[k] = j < p.H ? (long long)__ldcg(acc + j) : 0;
+    }
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int j = threadIdx.x + k * kThreads;
-    if (j < p.H) {
-      const float y = __ll2float_rn(v[k]) * kAccInvScale;
-      const float hn = p.use_norm ? __fadd_rn(hs[j], y) : y;
-      hs[j] = hn;
-      if (trace) trace[j] = hn;
+    for (int k = 0; k < kPer; ++k) {
+      const int j = j0 + threadIdx.x + k * kThreads;
+      if (j < p.H) {
+        const float y = __ll2float_rn(v[k]) * kAccInvScale;
+        const float hn = p.use_norm ? __fadd_rn(hs[j], y) : y;
+        hs[j] = hn;
+        if (trace) trace[j] = hn;
+      }
     }
   }
 }
@@ -709,6 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   int32_t* xc = reinterpret_cast<int32_t*>(smem + S.xc);
   float* zs = reinterpret_cast<float*>(smem + S.z);
   int32_t* pinrow = reinterpret_cast<int32_t*>(smem + S.pinrow);
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + S.cand);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, b = blockIdx.x;
@@ -717,6 +866,12 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   const bool has_gain = p.use_norm && p.gain;
   const int nrx = b < p.E ? min(p.rx_per_cta, (p.E - b + G - 1) / G) : 0;  // my router experts b, b+G, ...
   const bool first_shared = b < p.n_units && b >= routed;  // my first unit does not depend on routing
+  const int Ur = p.I / 32;
+  const int npc = p.n_pre * Ur;  // CTAs that preload a likely expert's unit
+  // a unit was issued ahead for the current layer (the shared expert's, or a preload);
+  // every thread keeps the same value
+  bool pre = first_shared;
+  int32_t pre_slot = -1;  // the slot this layer's preload reads (issued at the counter), or -1
   const uint32_t gbase = 0;  // arrival counter starts at 0 every launch
   uint32_t par_u[4] = {0, 0, 0, 0}, par_d = 0, par_r = 0;  // mbarrier parities (uniform)
   bool ok = true;
@@ -730,7 +885,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     m.seq_base = *reinterpret_cast<volatile uint32_t*>(&p.ctrl->req_seq);
     m.n_miss = 0;
     m.n_fix = 0;
-    m.pre = 0;
   }
   stamp(p, p.L, 0);
   if (!cta_ok(p, true)) goto fail;
@@ -746,15 +900,18 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         bulk_g2s_stream(const_cast<uint16_t*>(rrows) + (size_t)k * H, p.router + (size_t)(b + k * G) * H, 2u * H,
                         &m.bar_r);
     }
-    if (first_shared) {
-      issue_unit(p, m, ubuf, p.shared_pool + (size_t)(b - routed) * p.unit_bytes);
-      m.pre = 1;
+    if (first_shared) issue_unit(p, m, ubuf, p.shared_pool + (size_t)(b - routed) * p.unit_bytes);
+  }
+  if (b < npc) {  // preload: unit b mod Ur of layer 0's likely expert b / Ur
+    const int32_t slot = __ldg(p.likely_slot + b / Ur);
+    if (slot >= 0) {
+      if (tid == 0) issue_unit(p, m, ubuf, p.pool + (size_t)slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
+      pre = true;
     }
   }
   int32_t lk[kMaxLikely];  // thread 32: the likely experts' slots of the current layer
-  if (tid == 32 && p.n_likely > 0) {
-#pragma unroll
-    for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely + q);
+  if (tid == 32 && p.n_l2 > 0) {
+    load_likely(p, 0, lk);
     prefetch_likely(p, lk);
   }
   if (b == 0 && p.h_trace)
@@ -787,17 +944,22 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (tid == kThreads - 2) m.P_l = __ldg(p.n_pinned + l);
       if (tid == kThreads - 3) m.base_l = __ldg(p.layer_base + l);
       if (tid < nrx) m.bias[tid] = p.bias ? __ldg(p.bias + (size_t)l * p.E + b + tid * G) : 0.0f;
-      if (tid == 32 && p.n_likely > 0 && l > 0) {
-#pragma unroll
-        for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely + (size_t)l * kMaxLikely + q);
-      }
+      if (tid == 32 && p.n_l2 > 0 && l > 0) load_likely(p, l, lk);
+      if (tid < p.n_pre) m.lk_e[tid] = __ldg(p.likely_e + (size_t)l * kMaxLikely + tid);
+      pre_slot = (l > 0 && b < npc) ? __ldg(p.likely_slot + (size_t)l * kMaxLikely + b / Ur) : -1;
     }
     if (l > 0) {
       // ---------------------------------------------------------------- h += y(l - 1)
-      if (tid == 0) ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G);
+      if (tid == 0) {
+        ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G);
+        // every unit of layer l - 1 is done: the HBM is free for this layer's guess
+        if (ok && pre_slot >= 0)
+          issue_unit(p, m, ubuf, p.pool + (size_t)pre_slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
+      }
+      if (pre_slot >= 0) pre = true;
       // the HBM is idle until this layer's routing is known: fetch its likely experts
       // (a thread off the critical path, after the wait)
-      if (tid == 32 && p.n_likely > 0) {
+      if (tid == 32 && p.n_l2 > 0) {
         if (wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G)) prefetch_likely(p, lk);
       }
       if (!cta_ok(p, ok)) goto fail;
@@ -806,12 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
                        (b == 0 && p.h_trace) ? p.h_trace + (size_t)l * H : nullptr);
       // deferred ring fills of layer l - 1 (a layer that missed more often than it has
       // ring slots): its readers are done
-      for (int f = 0; f < m.n_fix; ++f) {
-        const uint4* s = reinterpret_cast<const uint4*>(p.pool + (size_t)m.fix_src[f] * p.slot_bytes);
-        uint4* d = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) + (size_t)m.fix_dst[f] * p.slot_bytes);
-        const size_t n16 = p.slot_bytes / 16;
-        for (size_t t = (size_t)b * kThreads + tid; t < n16; t += (size_t)G * kThreads) d[t] = __ldcg(s + t);
-      }
+      if (m.n_fix > 0) ring_fills(p, m);
       // the accumulator of layer l + 1 was last read at the start of layer l - 1, by CTAs
       // that have all published layer l - 1's logits since
       if (next) {
@@ -978,11 +1135,33 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     }
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 4);
+    int my_e = 0;
+    if (p.E <= kThreads) {
+      my_e = topk_parallel(p, m, zs, cand);
+    } else if (warp == 0) {
+      my_e = topk_weights(p, m, zs);
+    }
     if (warp == 0) {
-      const int my_e = topk_weights(p, m, zs);
       stamp(p, l, 13);
       const bool fast = cache_all_pinned(p, m, l, pinrow, my_e);
       if (lane == 0 && !fast) cache_decide(p, m, l, pinrow);
+      if (lane == 0) {  // preload matching: which group holds which rank, which ranks are left
+        uint32_t covered = 0;
+        int wrong = 0;
+        for (int q = 0; q < p.n_pre; ++q) {
+          int r = -1;
+          for (int i = 0; i < p.K; ++i)
+            if (m.sel[i] == m.lk_e[q]) r = i;
+          m.hit[q] = r;
+          if (r >= 0) covered |= 1u << r;
+          else ++wrong;
+        }
+        int nu = 0;
+        for (int i = 0; i < p.K; ++i)
+          if (!((covered >> i) & 1u)) m.unc[nu++] = i;
+        m.n_unc = nu;
+        m.n_avail = wrong * Ur + (routed - npc) + max(G - p.n_units, 0);
+      }
       stamp(p, l, 14);
     }
     __syncthreads();
@@ -1017,14 +1196,19 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         }
       }
       unsigned long long* acc_l = p.acc + (size_t)(l % kAccBufs) * H;
-      for (int u = b, k = 0; u < p.n_units; u += G, ++k) {
-        const bool shared = u >= routed;
-        const int i = shared ? p.K : u / (p.I / 32);
-        const int rb = shared ? u - routed : u % (p.I / 32);
+      UnitRef ur;
+      for (int k = 0; unit_of(p, m, pre, b, G, k, ur); ++k) {
+        const bool shared = ur.shared;
+        const int i = ur.i, rb = ur.rb;
         const float wi = shared ? 1.0f : m.w[i];
         const uint8_t* usrc = (shared ? p.shared_pool + (size_t)l * p.shared_slot_bytes : m.src[i]) +
                               (size_t)rb * p.unit_bytes;
-        if (!(k == 0 && m.pre)) {
+        if (!ur.issued) {
+          if (pre) {  // a preload that routing did not use: let it land before the buffer is reused
+            ok = drain_unit(p, m, par_u, par_d);
+            if (!cta_ok(p, ok)) goto fail;
+            pre = false;
+          }
           if (!shared && m.pull[i] >= 0) {  // pull mode miss: this CTA fills its unit of the slot
             pull_unit(p, p.host_tier + m.pull[i] + (size_t)rb * p.unit_bytes, const_cast<uint8_t*>(usrc));
             __syncthreads();
@@ -1129,15 +1313,23 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
 #pragma unroll
         for (int st = 0; st < 4; ++st) par_u[st] ^= 1u;
         par_d ^= 1u;
-        if (tid == 0) m.pre = 0;
+        pre = false;
       }
+    }
+    if (pre) {  // a preload left unused (no unit for this CTA): let it land
+      ok = drain_unit(p, m, par_u, par_d);
+      if (!cta_ok(p, ok)) goto fail;
+      pre = false;
     }
     stamp(p, l, 8);
     cta_stamp(p, l, 1);
-    // the next layer's shared-expert unit does not depend on routing: load it now
-    if (first_shared && next && tid == 0) {
-      issue_unit(p, m, ubuf, p.shared_pool + (size_t)(l + 1) * p.shared_slot_bytes + (size_t)(b - routed) * p.unit_bytes);
-      m.pre = 1;
+    // the next layer's shared-expert unit does not depend on routing, and a likely
+    // expert's unit is worth guessing: load them now
+    if (next && first_shared) {
+      if (tid == 0)
+        issue_unit(p, m, ubuf,
+                   p.shared_pool + (size_t)(l + 1) * p.shared_slot_bytes + (size_t)(b - routed) * p.unit_bytes);
+      pre = true;
     }
     __syncthreads();
     if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
@@ -1154,12 +1346,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (j0 + tid < H) p.y[j0 + tid] = hs[j0 + tid];
     if (b == 0 && p.h_trace)
       for (int j = tid; j < H; j += kThreads) p.h_trace[(size_t)p.L * H + j] = hs[j];
-    for (int f = 0; f < m.n_fix; ++f) {
-      const uint4* s = reinterpret_cast<const uint4*>(p.pool + (size_t)m.fix_src[f] * p.slot_bytes);
-      uint4* d = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) + (size_t)m.fix_dst[f] * p.slot_bytes);
-      const size_t n16 = p.slot_bytes / 16;
-      for (size_t t = (size_t)b * kThreads + tid; t < n16; t += (size_t)G * kThreads) d[t] = __ldcg(s + t);
-    }
+    if (m.n_fix > 0) ring_fills(p, m);
   }
   stamp(p, p.L, 2);
   if (b == 0 && tid == 0) {

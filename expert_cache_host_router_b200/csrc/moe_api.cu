@@ -65,8 +65,8 @@ struct moe_ctx {
   uint32_t *ring_stamp = nullptr, *ring_clock = nullptr;
   unsigned long long* acc = nullptr;  // [kAccBufs][H] fixed-point layer outputs
   unsigned long long* zll = nullptr;  // [E] published logits
-  int32_t* likely = nullptr;          // [L][kMaxLikely] pool slots of the likeliest pinned experts
-  int n_likely = 0;
+  int32_t* likely = nullptr;  // [2][L][kMaxLikely]: pool slots, then expert ids, of the likeliest pinned experts
+  int n_pre = 0, n_l2 = 0;
   uint32_t* hist = nullptr;
   int32_t* log = nullptr;
   int log_steps = 0;
@@ -88,6 +88,8 @@ struct moe_ctx {
   // streams and graphs
   cudaStream_t side = nullptr, own = nullptr;
   cudaGraphExec_t g_dev = nullptr, g_host = nullptr;
+  cudaGraph_t gr_dev = nullptr;       // the graph g_dev was instantiated from (kept for its node)
+  cudaGraphNode_t kn_dev = nullptr;   // its kernel node: new x / y pointers update it in place
   const float* g_x = nullptr;
   float* g_y = nullptr;
   // proxy
@@ -251,13 +253,18 @@ static DecodeParams make_params(const moe_ctx* c, const float* x, float* y) {
   p.host_tier = c->host_tier_dev;
   p.timeout_ns = (unsigned long long)c->cfg.wait_timeout_ms * 1000000ull;
   p.phase_trace = c->phase_trace;
-  p.likely = c->likely;
-  p.n_likely = c->n_likely;
+  p.likely_slot = c->likely;
+  p.likely_e = c->likely + (size_t)c->L * kMaxLikely;
+  p.n_pre = c->n_pre;
+  p.n_l2 = c->n_l2;
   return p;
 }
 
 static void drop_graphs(moe_ctx* c) {
   if (c->g_dev) cudaGraphExecDestroy(c->g_dev);
+  if (c->gr_dev) cudaGraphDestroy(c->gr_dev);
+  c->gr_dev = nullptr;
+  c->kn_dev = nullptr;
   if (c->g_host) cudaGraphExecDestroy(c->g_host);
   if (c->g_pf) cudaGraphExecDestroy(c->g_pf);
   c->g_dev = c->g_host = c->g_pf = nullptr;
@@ -266,7 +273,9 @@ static void drop_graphs(moe_ctx* c) {
 }
 
 // Capture one token: [optional H2D of x] -> decode kernel -> [optional D2H of y, error].
-static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cudaGraphExec_t* out) {
+// keep, when non-null, receives the captured graph (not destroyed) and knode its kernel node.
+static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cudaGraphExec_t* out,
+                         cudaGraph_t* keep = nullptr, cudaGraphNode_t* knode = nullptr) {
   cudaGraph_t graph = nullptr;
   CK(cudaStreamBeginCapture(c->own, cudaStreamCaptureModeThreadLocal));
   cudaError_t e = cudaSuccess;
@@ -285,6 +294,25 @@ static int capture_token(moe_ctx* c, const float* x, float* y, bool host_io, cud
   }
   if (e2 != cudaSuccess) return cuda_fail(e2);
   e = cudaGraphInstantiate(out, graph, 0);
+  if (e == cudaSuccess && keep) {
+    size_t n = 0;
+    e = cudaGraphGetNodes(graph, nullptr, &n);
+    std::vector<cudaGraphNode_t> nodes(n);
+    if (e == cudaSuccess && n) e = cudaGraphGetNodes(graph, nodes.data(), &n);
+    *knode = nullptr;
+    for (size_t i = 0; i < n && e == cudaSuccess; ++i) {
+      cudaGraphNodeType t;
+      e = cudaGraphNodeGetType(nodes[i], &t);
+      if (e == cudaSuccess && t == cudaGraphNodeTypeKernel) *knode = nodes[i];
+    }
+    if (e == cudaSuccess && !*knode) e = cudaErrorInvalidValue;
+    if (e == cudaSuccess) {
+      *keep = graph;
+      return MOE_OK;
+    }
+    cudaGraphExecDestroy(*out);
+    *out = nullptr;
+  }
   cudaGraphDestroy(graph);
   if (e != cudaSuccess) return cuda_fail(e);
   return MOE_OK;
@@ -356,20 +384,27 @@ static int empty_rings(moe_ctx* c, cudaStream_t s) {
   return MOE_OK;
 }
 
-// Speculative-prefetch table from the recalibration score (the placement histogram,
-// decayed): per layer, the pool slots of the n_likely pinned experts with the highest
-// counts (ties -> lower index).
+// Speculative-load table from the recalibration score (the placement histogram,
+// decayed): per layer, the pool slots and ids of the n_pre + n_l2 pinned experts with the
+// highest counts (ties -> lower index); unused entries -1.
 static int upload_likely(moe_ctx* c, cudaStream_t s) {
-  std::vector<int32_t> t((size_t)c->L * kMaxLikely, -1);
+  const size_t n = (size_t)c->L * kMaxLikely;
+  std::vector<int32_t> t(2 * n, -1);
   std::vector<int> order(c->E);
-  for (int l = 0; l < c->L && c->n_likely > 0; ++l) {
+  const int want = c->n_pre + c->n_l2;
+  for (int l = 0; l < c->L && want > 0; ++l) {
     const uint32_t* cnt = c->score.data() + (size_t)l * c->E;
     const int32_t* row = c->pin_host.data() + (size_t)l * c->E;
     for (int e = 0; e < c->E; ++e) order[e] = e;
     std::stable_sort(order.begin(), order.end(), [cnt](int a, int b) { return cnt[a] > cnt[b]; });
-    int n = 0;
-    for (int k = 0; k < c->E && n < c->n_likely; ++k)
-      if (row[order[k]] >= 0) t[(size_t)l * kMaxLikely + n++] = l * (c->P + c->R) + (row[order[k]] & 0xffff);
+    int k = 0;
+    for (int q = 0; q < c->E && k < want; ++q) {
+      const int e = order[q];
+      if (row[e] < 0) continue;
+      t[(size_t)l * kMaxLikely + k] = l * (c->P + c->R) + (row[e] & 0xffff);
+      t[n + (size_t)l * kMaxLikely + k] = e;
+      ++k;
+    }
   }
   CK(cudaMemcpyAsync(c->likely, t.data(), t.size() * 4, cudaMemcpyHostToDevice, s));
   return cudaStreamSynchronize(s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -563,7 +598,7 @@ int moe_create(const moe_config* cfg_in, const moe_weights* w, moe_ctx** out) {
   CKC(dalloc(&c->ring_clock, (size_t)2 * c->L));
   CKC(dalloc(&c->acc, (size_t)kAccBufs * c->H));
   CKC(dalloc(&c->zll, c->E));
-  CKC(dalloc(&c->likely, (size_t)c->L * kMaxLikely));
+  CKC(dalloc(&c->likely, (size_t)2 * c->L * kMaxLikely));
   CKC(dalloc(&c->hist, (size_t)c->L * c->E));
   CKC(dalloc(&c->log, (size_t)c->log_steps * c->L * c->K * 7));
   CKC(dalloc(&c->ctrl, 1));
@@ -688,11 +723,20 @@ int moe_set_residency(moe_ctx* c, float fraction, const uint32_t* hist, int32_t 
 int moe_decode_step(moe_ctx* c, const float* x_dev, float* y_dev, void* stream) {
   if (!c || !x_dev || !y_dev) return MOE_ERR_INVALID;
   if (!c->resident) return MOE_ERR_STATE;
-  if (!c->g_dev || c->g_x != x_dev || c->g_y != y_dev) {
-    if (c->g_dev) cudaGraphExecDestroy(c->g_dev);
-    c->g_dev = nullptr;
-    const int st = capture_token(c, x_dev, y_dev, false, &c->g_dev);
+  if (!c->g_dev) {
+    const int st = capture_token(c, x_dev, y_dev, false, &c->g_dev, &c->gr_dev, &c->kn_dev);
     if (st != MOE_OK) return st;
+    c->g_x = x_dev;
+    c->g_y = y_dev;
+  } else if (c->g_x != x_dev || c->g_y != y_dev) {
+    // other buffers: the same graph with the kernel node's x / y updated in place
+    DecodeParams p = make_params(c, x_dev, y_dev);
+    cudaKernelNodeParams kp;
+    CK(cudaGraphKernelNodeGetParams(c->kn_dev, &kp));
+    void* args[1] = {&p};
+    kp.kernelParams = args;
+    kp.extra = nullptr;
+    CK(cudaGraphExecKernelNodeSetParams(c->g_dev, c->kn_dev, &kp));
     c->g_x = x_dev;
     c->g_y = y_dev;
   }
@@ -1012,11 +1056,15 @@ int moe_recalibrate(moe_ctx* c) {
   return upload_likely(c, c->own);
 }
 
-int moe_set_prefetch(moe_ctx* c, int32_t n_experts) {
-  if (!c || n_experts < 0 || n_experts > kMaxLikely) return MOE_ERR_INVALID;
+int moe_set_prefetch(moe_ctx* c, int32_t n_preload, int32_t n_l2) {
+  if (!c || n_preload < 0 || n_l2 < 0 || n_preload > std::min(c->K, kMaxPreload) || n_preload + n_l2 > kMaxLikely)
+    return MOE_ERR_INVALID;
   CK(cudaSetDevice(c->cfg.device));
   CK(cudaDeviceSynchronize());
-  c->n_likely = n_experts;
+  // the preload needs one CTA per unit (a CTA guessing wrong takes another unit)
+  const int n_units = c->K * (c->I / 32) + c->Is / 32;
+  c->n_pre = c->grid >= n_units ? n_preload : 0;
+  c->n_l2 = n_l2;
   drop_graphs(c);
   return c->resident ? upload_likely(c, c->own) : MOE_OK;
 }

@@ -31,7 +31,8 @@ constexpr int kMaxR = 32;
 constexpr int kMaxH = 4096;
 constexpr int kMboxCap = 256;  // miss-request mailbox entries
 constexpr int kAccBufs = 3;    // rotating per-layer output accumulators
-constexpr int kMaxLikely = 16; // experts per layer the kernel may prefetch into L2 ahead of routing
+constexpr int kMaxLikely = 32; // likely experts per layer the kernel may load ahead of routing
+constexpr int kMaxPreload = 16;  // of which preloaded into shared memory
 // Fixed-point scale of the per-layer output accumulator: every unit adds its share of
 // y as round(v * 2^28) into 64-bit integers, so the sum does not depend on the order in
 // which units finish.  A share must satisfy |v| < 2^26 (else MOE_DEVERR_RANGE).
@@ -133,10 +134,13 @@ struct DecodeParams {
   const uint8_t* host_tier;      // device view of the mapped pinned host tier (pull mode)
   unsigned long long timeout_ns;
   unsigned long long* phase_trace;  // see moe_set_phase_trace, or null
-  // speculative L2 prefetch: per layer, pool slots of the n_likely most frequently routed
-  // pinned experts ([L][kMaxLikely], -1 = none), fetched while the layer's routing runs
-  const int32_t* likely;
-  int n_likely;
+  // speculative loads while a layer's routing runs, from its most frequently routed
+  // pinned experts in order ([L][kMaxLikely] pool slots and expert ids, -1 = none): the
+  // first n_pre are preloaded unit by unit into the shared memory of CTAs 0..n_pre*I/32-1,
+  // the next n_l2 are prefetched into L2
+  const int32_t* likely_slot;
+  const int32_t* likely_e;
+  int n_pre, n_l2;
 };
 
 // Words of the phase trace for L layers on a grid of n CTAs.

@@ -161,8 +161,10 @@ extern "C" int moe_decode_step_noalloc(const moe_config* cfg, const moe_noalloc_
   p.host_tier = nullptr;
   p.timeout_ns = (unsigned long long)(cfg->wait_timeout_ms ? cfg->wait_timeout_ms : 2000) * 1000000ull;
   p.phase_trace = nullptr;
-  p.likely = nullptr;
-  p.n_likely = 0;
+  p.likely_slot = nullptr;
+  p.likely_e = nullptr;
+  p.n_pre = 0;
+  p.n_l2 = 0;
 
   // a clean start every call: control block (step 0, no error, counter 0), accumulators,
   // logit words and tables

@@ -266,14 +266,19 @@ MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev, size_t n_wor
  * give the same routing, event log and outputs.  Other values: MOE_ERR_INVALID. */
 MOE_API int moe_set_miss_path(moe_ctx *ctx, int32_t mode);
 
-/* Speculative L2 prefetch: at the start of every layer, while the layer's routing is
- * computed and the HBM would otherwise idle, the kernel prefetches into L2 the slots of
- * the n_experts pinned experts that the placement histogram (decayed by recalibration)
- * routes to most often; the expert loads that follow routing then hit L2 for the
- * predicted experts.  Changes no result, only where bytes come from; mispredicted
- * prefetches cost HBM bandwidth that would otherwise be idle.  0 (the default) turns it
- * off; at most 16.  Synchronises the device. */
-MOE_API int moe_set_prefetch(moe_ctx *ctx, int32_t n_experts);
+/* Speculative loads while a layer's routing is computed (the HBM would otherwise idle):
+ * the layer's pinned experts ordered by the placement histogram (decayed by
+ * recalibration), most frequently routed first.  The units of the first n_preload are
+ * loaded straight into the shared memory of the CTAs that will compute them if they are
+ * routed (n_preload x inter/32 CTAs, one unit each); after routing, every CTA derives
+ * the same assignment: a preloaded unit whose expert was routed is computed at once,
+ * and the CTAs that guessed wrong take the units of the other routed experts.  The next
+ * n_l2 experts are prefetched into L2 only.  Changes no result, only where and when bytes
+ * are read; wrong guesses cost HBM bandwidth that routing leaves idle.  n_preload <=
+ * min(top_k, 16) and n_preload + n_l2 <= 32, else MOE_ERR_INVALID; (0, 0), the default,
+ * turns it off.  n_preload is taken as 0 when the device has fewer SMs than a layer has
+ * units.  Synchronises the device. */
+MOE_API int moe_set_prefetch(moe_ctx *ctx, int32_t n_preload, int32_t n_l2);
 
 /* Host-to-device rate of the miss path's own copy: n_copies expert slots copied back to
  * back from the library's pinned host tier into device slots with cudaMemcpyAsync on the

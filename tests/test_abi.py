@@ -80,7 +80,7 @@ def test_null_arguments_are_rejected(lib):
     assert lib.moe_set_phase_trace(None, None, 0) == moe.MOE_ERR_INVALID
     assert lib.moe_set_miss_path(None, 0) == moe.MOE_ERR_INVALID
     assert lib.moe_measure_h2d(None, 1, None) == moe.MOE_ERR_INVALID
-    assert lib.moe_set_prefetch(None, 0) == moe.MOE_ERR_INVALID
+    assert lib.moe_set_prefetch(None, 0, 0) == moe.MOE_ERR_INVALID
     lib.moe_destroy(None)  # no-op
 
 

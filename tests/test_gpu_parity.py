@@ -265,3 +265,31 @@ def test_invalid_calls_on_a_live_context():
         moe.moe_prefill(m.ctx, x.data_ptr(), 0, x.data_ptr(), 0)
     assert ei.value.status == moe.MOE_ERR_INVALID
     m.close()
+
+
+@pytest.mark.parametrize("frac", [1.0, 0.6])
+def test_speculative_loads_change_nothing(frac):
+    """Preloading likely experts into shared memory (and prefetching more into L2) only
+    moves where and when bytes are read: outputs bit-identical, the same event log."""
+    s = STACK
+    layers = make_layers(s, gain_kind="random")
+    m = build_gpu(s, layers, log_steps=64)
+    m.set_residency(1.0)
+    calib = synthetic.tokens(0, 16, s.hidden, synthetic.SEED_CALIB)
+    _run_tokens(m, calib)
+    _, hist, _ = m.stats(log_cap=16 * s.n_layers * s.top_k, reset=True)
+    xs = synthetic.tokens(40, 8, s.hidden)
+    outs, logs = {}, {}
+    for pre, l2 in [(0, 0), (8, 0), (4, 6), (8, 8)]:
+        m.set_prefetch(pre, l2)
+        m.set_residency(frac, hist)
+        ys, _, _ = _run_tokens(m, xs)
+        _, _, log = m.stats(log_cap=8 * s.n_layers * s.top_k, reset=True)
+        outs[(pre, l2)] = ys
+        logs[(pre, l2)] = log
+    base = outs[(0, 0)]
+    for key, ys in outs.items():
+        assert np.array_equal(ys.view(np.uint32), base.view(np.uint32)), key
+        for f in ("layer", "rank", "expert", "kind", "slot", "evicted"):
+            assert np.array_equal(logs[key][f], logs[(0, 0)][f]), (key, f)
+    m.close()
