@@ -427,16 +427,16 @@ def decode_precision(m, shape, layers, dev):
             "sample": "decode: one token, prefill: two of 16 tokens; every layer, teacher-forced"}
 
 
-def write_phase_table(m, shape, xs, y, path, n_tokens=8):
-    """Per-layer phase times of CTA 0 (median over n_tokens full-residency tokens) from
-    the kernel's global-timer stamps, written as JSON to path."""
+def write_phase_table(m, shape, xs, y, path, n_tokens=8, residency=1.0, hist=None):
+    """Per-layer phase times of CTA 0 (median over n_tokens tokens at the given residency)
+    from the kernel's marks, plus every CTA's skew, written as JSON to path."""
     import torch
 
     import expert_cache_host_router_b200 as moe
     n_sm = torch.cuda.get_device_properties(y.device).multi_processor_count
     words = moe.phase_trace_words(shape.n_layers, n_sm)
     st = torch.zeros(words, dtype=torch.int64, device=y.device)
-    m.set_residency(1.0)
+    m.set_residency(residency, hist)
     m.set_phase_trace(st)
     runs = []
     for i in range(n_tokens):
@@ -446,6 +446,8 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8):
     m.set_phase_trace(None)
     L = shape.n_layers
     marks = np.stack([r[: (L + 1) * 32].reshape(L + 1, 32) for r in runs]).astype(np.float64)
+    # CTA 0's marks are SM cycles; the kernel's start and end on both clocks give ns per cycle
+    ns_per_cycle = float(np.median((marks[:, L, 5] - marks[:, L, 4]) / (marks[:, L, 2] - marks[:, L, 0])))
     names = {1: "prev_layer_output", 2: "h_updated", 10: "norm_u", 11: "own_logit", 12: "x_quantised",
              3: "logits_published", 4: "logits_read", 13: "topk", 14: "cache", 5: "routed", 15: "loads_issued_t0",
              6: "loads_issued", 7: "gateup_done", 16: "swiglu", 17: "down_landed", 18: "down_adds", 19: "fence",
@@ -454,13 +456,24 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8):
     for l in range(L):
         row = {"layer": l}
         for k, n in names.items():
-            row[n] = float(np.median(marks[:, l, k] - marks[:, l, 0])) / 1e3
+            row[n] = float(np.median(marks[:, l, k] - marks[:, l, 0])) * ns_per_cycle / 1e3
         nxt = marks[:, l + 1, 0] if l + 1 < L else marks[:, L, 2]
-        row["layer_us"] = float(np.median(nxt - marks[:, l, 0])) / 1e3
+        row["layer_us"] = float(np.median(nxt - marks[:, l, 0])) * ns_per_cycle / 1e3
         table.append(row)
-    total = float(np.median(marks[:, L, 2] - marks[:, L, 0])) / 1e3
+    total = float(np.median(marks[:, L, 5] - marks[:, L, 4])) / 1e3
+    raw = [float(np.median(marks[:, 1:L, k] - marks[:, 1:L, 0])) * ns_per_cycle / 1e3 for k in range(32)]
+    # every CTA's global-timer marks: [0] routing decided, [1] units done, [2] arrival posted
+    cta = np.stack([r[(L + 1) * 32:].reshape(L, n_sm, 4) for r in runs]).astype(np.float64)  # [tok][L][cta][4]
+    rt, ud, ar = cta[..., 0], cta[..., 1], cta[..., 2]
+    work = ud - rt  # per CTA: routing decided -> its units done
+    cta_stats = {"routed_spread_us": float(np.median(rt.max(axis=2) - rt.min(axis=2))) / 1e3,
+                 "units_median_us": float(np.median(np.median(work, axis=2))) / 1e3,
+                 "units_max_us": float(np.median(work.max(axis=2))) / 1e3,
+                 "arrival_spread_us": float(np.median(ar.max(axis=2) - ar.min(axis=2))) / 1e3,
+                 "last_arrival_after_first_routed_us": float(np.median(ar.max(axis=2) - rt.min(axis=2))) / 1e3}
     with open(path, "w") as f:
         json.dump({"unit": "us since layer start (CTA 0), median over tokens", "tokens": n_tokens,
+                   "ns_per_cycle": ns_per_cycle, "raw_slots_us": raw, "cta_stats": cta_stats,
                    "kernel_us": total, "layers": table}, f, indent=1)
 
 
@@ -649,6 +662,10 @@ def run_ours(args):
         line["precision"] = precision
     if args.phase_trace:
         write_phase_table(m, shape, xs, y, args.phase_trace)
+        if args.phases == "all":  # where the misses of the 60% placement stall a layer
+            write_phase_table(m, shape, xs, y, args.phase_trace.replace(".json", "_60.json"), n_tokens=32,
+                              residency=0.6, hist=hist)
+            m.set_residency(1.0)
     if args.prefetch_sweep:
         sweep = []
         m.set_residency(1.0)

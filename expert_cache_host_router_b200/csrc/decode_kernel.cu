@@ -271,7 +271,7 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
   s.xc = take(4u * (H / 32));
   s.z = take(4u * E);
   s.pinrow = take(4u * E);
-  s.cand = take(8u * kWarps * kMaxK);
+  s.cand = take(8u * kWarps * kMaxK + 8u * kThreads);
   s.misc = take(sizeof(Misc));
   s.total = align_up(off, 128);
   return s;
@@ -364,8 +364,17 @@ __device__ __forceinline__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, 
 // no global memory here.
 __device__ __forceinline__ bool cta_ok(const DecodeParams&, bool ok) { return __syncthreads_and(ok) != 0; }
 
+// CTA 0's marks are SM clock cycles (clock64: fine-grained, one SM); the kernel's start
+// and end are also taken on the global timer so that cycles convert to ns.
 __device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = gtimer();
+  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = clock64();
+}
+
+__device__ __forceinline__ void stamp_both(const DecodeParams& p, int k_clock, int k_timer) {
+  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) {
+    p.phase_trace[p.L * 32 + k_clock] = clock64();
+    p.phase_trace[p.L * 32 + k_timer] = gtimer();
+  }
 }
 
 // Per-CTA marks (every CTA, thread 0): after [(L+1)][32] come [L][gridDim][4] stamps.
@@ -457,13 +466,22 @@ __device__ int topk_parallel(const DecodeParams& p, Misc& m, const float* zs, un
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.K;
   const int e = tid;  // E <= 256 = kThreads
   const unsigned long long key = e < p.E ? route_key(zs[e], e) : 0ull;
-  int rank = 0;
-#pragma unroll 8
-  for (int off = 1; off < 32; ++off) {
-    const unsigned long long o = shfl_xor_u64(key, off);
-    rank += o > key;
-  }
+  unsigned long long* keys = cand + kWarps * kMaxK;  // [256] after the candidate slots
+  keys[e] = key;
   const int nc = kWarps * K;  // candidate slots
+  __syncthreads();
+  int rank = 0;  // among this warp's 32 keys, read as broadcasts
+  {
+    const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + warp * 32);
+#pragma unroll
+    for (int q = 0; q < 16; q += 4) {
+      ulonglong2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = k2[q + u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) rank += (v[u].x > key) + (v[u].y > key);
+    }
+  }
   for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
   __syncthreads();
   if (e < p.E && rank < K) cand[warp * K + rank] = key;
@@ -472,7 +490,14 @@ __device__ int topk_parallel(const DecodeParams& p, Misc& m, const float* zs, un
     const unsigned long long c = cand[t];
     if (c == 0ull) continue;
     int r = 0;
-    for (int q = 0; q < nc; ++q) r += cand[q] > c;
+    const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(cand);  // nc is even
+    for (int q = 0; q < nc / 2; q += 4) {  // four independent 16-byte loads per step
+      ulonglong2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = q + u < nc / 2 ? c2[q + u] : make_ulonglong2(0ull, 0ull);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) r += (v[u].x > c) + (v[u].y > c);
+    }
     if (r < K) {
       m.sel[r] = (int)(~(uint32_t)c);
       if ((c >> 32) == 0ull) set_error(p.ctrl, MOE_DEVERR_ROUTE);  // a NaN logit was needed
@@ -886,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     m.n_miss = 0;
     m.n_fix = 0;
   }
-  stamp(p, p.L, 0);
+  stamp_both(p, 0, 4);
   if (!cta_ok(p, true)) goto fail;
 
   // ---- prologue: accumulators 0 and 1 and the logit words zeroed, h = x, first loads
@@ -985,6 +1010,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       float inv = 1.0f;
       if (p.use_norm) {
         float acc = 0.0f;
+#pragma unroll 4
         for (int c = lane; c < nch; c += 32) {
           const float4* h4 = reinterpret_cast<const float4*>(hs + c * kChunk);
           float pc = 0.0f;
@@ -1018,6 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (ok) {
         const uint16_t* wr = rrows + (size_t)warp * H;
         float acc = 0.0f;
+#pragma unroll 4
         for (int mm = 0; mm * 32 < nch; ++mm) {
           const int c = lane + 32 * mm;
           if (c < nch) {
@@ -1094,8 +1121,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         }
         csum += __shfl_xor_sync(0xffffffffu, csum, 1);
         csum += __shfl_xor_sync(0xffffffffu, csum, 2);
-        if (b0 < nb) {
-          reinterpret_cast<uint4*>(xcodes + bb * 32)[j4] =
+        if (b0 < nb) {  // quarter-major ([4][nb] x 16 B): a warp's reads of one quarter are contiguous
+          reinterpret_cast<uint4*>(xcodes)[j4 * nb + bb] =
               make_uint4(((uint32_t)c[0] & 0xffffu) | ((uint32_t)c[1] << 16),
                          ((uint32_t)c[2] & 0xffffu) | ((uint32_t)c[3] << 16),
                          ((uint32_t)c[4] & 0xffffu) | ((uint32_t)c[5] << 16),
@@ -1182,11 +1209,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       for (int mb = 0; mb < BPL; ++mb) {
         const int bb = g + GS * mb;
         if (bb < nb) {
-          const int4* src = reinterpret_cast<const int4*>(xcodes + bb * 32);
-          xq[mb][0] = src[0];
-          xq[mb][1] = src[1];
-          xq[mb][2] = src[2];
-          xq[mb][3] = src[3];
+          const int4* src = reinterpret_cast<const int4*>(xcodes);
+          xq[mb][0] = src[bb];
+          xq[mb][1] = src[nb + bb];
+          xq[mb][2] = src[2 * nb + bb];
+          xq[mb][3] = src[3 * nb + bb];
           xsc[mb] = xs[bb];
           xsum[mb] = xc[bb];
         } else {
@@ -1306,7 +1333,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           }
           if (!range_ok) set_error(p.ctrl, MOE_DEVERR_RANGE);
           stamp(p, l, 18);
-          __threadfence();  // this thread's adds, before the CTA's arrival below
           stamp(p, l, 19);
         }
         if (!cta_ok(p, ok)) goto fail;
@@ -1348,7 +1374,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       for (int j = tid; j < H; j += kThreads) p.h_trace[(size_t)p.L * H + j] = hs[j];
     if (m.n_fix > 0) ring_fills(p, m);
   }
-  stamp(p, p.L, 2);
+  stamp_both(p, 2, 5);
   if (b == 0 && tid == 0) {
     p.ctrl->step = m.step + 1;
     p.ctrl->req_seq = m.seq_base + m.n_miss;

@@ -245,19 +245,23 @@ MOE_API int moe_stats(moe_ctx *ctx, moe_stats_t *out, uint32_t *hist_out, moe_ev
  * the routing weights.  Pass NULLs to stop.  Device pointers owned by the caller. */
 MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
 
-/* Phase timing: when stamps_dev is non-NULL, every decode step writes GPU global-timer
- * values (ns) there.  The buffer holds n_words uint64 and must hold at least
+/* Phase timing: when stamps_dev is non-NULL, every decode step writes timing marks
+ * there.  The buffer holds n_words uint64 and must hold at least
  * (L + 1) * 32 + L * n_sm * 4 words (n_sm = the device's SM count, one CTA per SM):
- * else MOE_ERR_INVALID and nothing changes.  Layout: first [(L+1)][32] marks of CTA 0;
- * per layer l: [l][0] layer start, [1] the previous layer's output complete, [2] h
- * updated, [3] own logits published and input quantised, [4] all logits read, [5]
- * routing and cache decided, [6] unit loads issued, [7] gate/up computed, [8] units
- * done, [9] arrival posted; [L][0] kernel start, [L][1] prologue done, [L][2] kernel
- * end.  Then [L][n_sm][4] marks of every CTA: [0] routing decided, [1] units done,
- * [2] arrival posted, [3] unused.  NULL stops it (n_words ignored). */
+ * else MOE_ERR_INVALID and nothing changes.  Layout: first [(L+1)][32] marks of CTA 0 in
+ * SM clock cycles (clock64); per layer l: [l][0] layer start, [1] the previous layer's
+ * output complete, [2] h updated, [3] own logits published and input quantised, [4] all
+ * logits read, [5] routing and cache decided, [6] unit loads issued, [7] gate/up
+ * computed, [8] units done, [9] arrival posted, [10..19] finer marks (norm, own logit,
+ * input quantised, top-k, cache, loads issued by thread 0, SwiGLU, down part landed,
+ * down adds issued, fence); [L][0] kernel start and [L][2] kernel end in cycles, [L][4]
+ * and [L][5] the same two instants on the global timer (ns), which converts cycles to
+ * ns; [L][1] prologue done (cycles).  Then [L][n_sm][4] global-timer marks (ns) of every
+ * CTA: [0] routing decided, [1] units done, [2] arrival posted, [3] unused.  NULL stops
+ * it (n_words ignored). */
 MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev, size_t n_words);
 
-/* Miss path (the survey's next-row variants of key components item 2): with
+/* Miss path (how a cold expert crosses PCIe; theneuralfeed.com, key components item 2): with
  * MOE_MISS_COPY_ENGINE (the default) the kernel posts a cold expert to a host-mapped
  * mailbox, the library's proxy thread copies it pinned host -> ring slot with
  * cudaMemcpyAsync on a side stream and signals the kernel through a stream memory write;
