@@ -243,10 +243,11 @@ struct Misc {
   int32_t hit[kMaxPreload];   // its rank in the layer's top-k, or -1
   int32_t unc[kMaxK];         // ranks whose expert no group preloaded, in rank order
   int32_t n_unc, n_avail;
+  int32_t early;  // 1: this layer's first unit was issued as soon as routing was known
 };
 
 struct SmemPlan {
-  uint32_t unit, rrows, h, g, up, xcodes, xs, xc, z, pinrow, cand, misc, total;
+  uint32_t unit, rrows, h, g, pc, xcodes, xs, xc, z, pinrow, cand, misc, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -265,7 +266,7 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
   s.rrows = take(2u * H * (uint32_t)rx);
   s.h = take(4u * H);
   s.g = take(4u * H);
-  s.up = take(4u * kChunk * 32u * ((nch + 31) / 32));
+  s.pc = take(4u * nch * (1u + (uint32_t)rx));  // chunk partials: the norm's, then one row per router expert
   s.xcodes = take(2u * H);
   s.xs = take(4u * (H / 32));
   s.xc = take(4u * (H / 32));
@@ -456,21 +457,23 @@ __device__ __noinline__ int topk_weights(const DecodeParams& p, Misc& m, const f
   return my_e;
 }
 
-// All threads, E <= 256: the same top-k in two parallel steps.  (1) Warp w ranks its 32
-// experts 32w + lane by 64-bit key (logit desc, index asc) with shuffles; a rank below k
-// makes a candidate, stored at w k + rank.  (2) Each of the 8k candidate slots counts
-// the candidates with larger keys (shared-memory broadcasts): that count is its global
-// rank.  Then warp 0 forms the weights exactly as topk_weights does.  Lane i of warp 0
-// returns the expert of rank i.
-__device__ int topk_parallel(const DecodeParams& p, Misc& m, const float* zs, unsigned long long* cand) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.K;
+// All threads, E <= 256: the top-k of topk_weights (m.sel only) in two parallel steps.
+// (1) Warp w ranks its 32 experts 32w + lane by 64-bit key (logit desc, index asc),
+// reading the warp's keys as shared-memory broadcasts; a rank below k makes a
+// candidate, stored at w k + rank.  (2) A candidate's global rank is the number of
+// larger candidates over the 8 warps' lists (a list with k larger keys puts it out of
+// the top k, as its count shows): 256 / (8k) threads per candidate, rounded down to a
+// power of two, each count some of the lists and add up with shuffles.
+__device__ void topk_select(const DecodeParams& p, Misc& m, const float* zs, unsigned long long* cand) {
+  const int tid = threadIdx.x, warp = tid >> 5, K = p.K;
   const int e = tid;  // E <= 256 = kThreads
   const unsigned long long key = e < p.E ? route_key(zs[e], e) : 0ull;
   unsigned long long* keys = cand + kWarps * kMaxK;  // [256] after the candidate slots
   keys[e] = key;
   const int nc = kWarps * K;  // candidate slots
+  for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
   __syncthreads();
-  int rank = 0;  // among this warp's 32 keys, read as broadcasts
+  int rank = 0;  // among this warp's 32 keys
   {
     const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + warp * 32);
 #pragma unroll
@@ -482,41 +485,41 @@ __device__ int topk_parallel(const DecodeParams& p, Misc& m, const float* zs, un
       for (int u = 0; u < 4; ++u) rank += (v[u].x > key) + (v[u].y > key);
     }
   }
-  for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
-  __syncthreads();
   if (e < p.E && rank < K) cand[warp * K + rank] = key;
   __syncthreads();
-  for (int t = tid; t < nc; t += kThreads) {
-    const unsigned long long c = cand[t];
-    if (c == 0ull) continue;
+  int tpc = 1;  // threads per candidate: a power of two, at most 8 (one list each)
+  while (tpc < kWarps && 2 * tpc * nc <= kThreads) tpc <<= 1;
+  const int lpt = kWarps / tpc;  // lists per thread
+  const int ci = tid / tpc, sub = tid % tpc;
+#pragma unroll 1
+  for (int c0 = 0; c0 < nc; c0 += kThreads / tpc) {  // one pass unless k > 16
+    const int cc = c0 + ci;
+    const unsigned long long c = cc < nc ? cand[cc] : 0ull;
     int r = 0;
-    const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(cand);  // nc is even
-    for (int q = 0; q < nc / 2; q += 4) {  // four independent 16-byte loads per step
-      ulonglong2 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = q + u < nc / 2 ? c2[q + u] : make_ulonglong2(0ull, 0ull);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) r += (v[u].x > c) + (v[u].y > c);
+#pragma unroll 1
+    for (int w = sub * lpt; w < (sub + 1) * lpt; ++w) {
+      const unsigned long long* lw = cand + w * K;
+      for (int q = 0; q < K; ++q) r += lw[q] > c;
     }
-    if (r < K) {
+    for (int off = 1; off < tpc; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+    if (sub == 0 && c != 0ull && r < K) {
       m.sel[r] = (int)(~(uint32_t)c);
       if ((c >> 32) == 0ull) set_error(p.ctrl, MOE_DEVERR_ROUTE);  // a NaN logit was needed
     }
   }
   __syncthreads();
-  int my_e = 0;
-  if (warp == 0) {
-    my_e = lane < K ? m.sel[lane] : 0;
-    if (my_e < 0 || my_e >= p.E) my_e = 0;
-    const float zmax = __shfl_sync(0xffffffffu, zs[my_e], 0);
-    const float ex = lane < K ? expf(zs[my_e] - zmax) : 0.0f;
-    float sum = ex;
+}
+
+// Warp 0, after topk_select: the renormalised softmax weights of the selected experts
+// (lane i: rank i), exactly as topk_weights forms them.
+__device__ __forceinline__ void route_weights(const DecodeParams& p, Misc& m, const float* zs, int my_e) {
+  const int lane = threadIdx.x & 31;
+  const float zmax = __shfl_sync(0xffffffffu, zs[my_e], 0);
+  const float ex = lane < p.K ? expf(zs[my_e] - zmax) : 0.0f;
+  float sum = ex;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane < K) m.w[lane] = __fdividef(ex, sum);
-    __syncwarp();
-  }
-  return my_e;
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < p.K) m.w[lane] = __fdividef(ex, sum);
 }
 
 // Thread 0 of every CTA: the cache decision for layer l (identical in all CTAs), from
@@ -645,29 +648,40 @@ __device__ __noinline__ void cache_decide(const DecodeParams& p, Misc& m, int l,
 }
 
 // Warp 0: the common case where every selected expert is pinned; lane i handles rank
-// i.  Returns false (nothing written) when some expert is not pinned.
-__device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow, int my_e) {
+// i.  Returns false (nothing written) when some expert is not pinned; else the slots are
+// set and cache_pinned_commit records the layer.
+__device__ __forceinline__ bool cache_pinned_lookup(const DecodeParams& p, Misc& m, const int32_t* pinrow, int my_e) {
   const int lane = threadIdx.x & 31;
   const int ps = lane < p.K ? pinrow[my_e] : 0;
   if (!__all_sync(0xffffffffu, ps >= 0)) return false;
-  const bool commit = blockIdx.x == 0;
   if (lane < p.K) {
     m.src[lane] = p.pool + (size_t)(m.base_l + (ps & 0xffff)) * p.slot_bytes;
     m.miss_seq[lane] = 0;
     m.pull[lane] = -1;
-    if (commit) {
-      int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * p.K + lane) * 7;
-      ev[0] = (int32_t)m.step;
-      ev[1] = l;
-      ev[2] = lane;
-      ev[3] = my_e;
-      ev[4] = MOE_PIN_HIT;
-      ev[5] = ps >> 16;
-      ev[6] = -1;
-      atomicAdd(p.hist + (size_t)l * p.E + my_e, 1u);
-    }
   }
-  if (commit && lane < p.R) {  // the ring is untouched: carry it to the next token's copy
+  __syncwarp();
+  return true;
+}
+
+// Warp 0, after cache_pinned_lookup: CTA 0 writes the event log, histogram and counters
+// and carries the untouched ring to the next token's copy; every CTA has no ring fill.
+__device__ __noinline__ void cache_pinned_commit(const DecodeParams& p, Misc& m, int l, const int32_t* pinrow,
+                                                 int my_e) {
+  const int lane = threadIdx.x & 31;
+  const bool commit = blockIdx.x == 0;
+  if (commit && lane < p.K) {
+    const int ps = pinrow[my_e];
+    int32_t* ev = p.log + (((size_t)(m.step % (uint32_t)p.log_steps) * p.L + l) * p.K + lane) * 7;
+    ev[0] = (int32_t)m.step;
+    ev[1] = l;
+    ev[2] = lane;
+    ev[3] = my_e;
+    ev[4] = MOE_PIN_HIT;
+    ev[5] = ps >> 16;
+    ev[6] = -1;
+    atomicAdd(p.hist + (size_t)l * p.E + my_e, 1u);
+  }
+  if (commit && lane < p.R) {
     const int par = m.step & 1;
     const size_t ws = ((size_t)(par ^ 1) * p.L + l) * p.R;
     p.ring_owner[ws + lane] = m.ring_owner[lane];
@@ -681,7 +695,6 @@ __device__ bool cache_all_pinned(const DecodeParams& p, Misc& m, int l, const in
     }
   }
   __syncwarp();
-  return true;
 }
 
 // ------------------------------------------------------------------ units
@@ -839,6 +852,98 @@ __device__ __noinline__ void load_likely(const DecodeParams& p, int l, int32_t (
   for (int q = 0; q < kMaxLikely; ++q) lk[q] = __ldg(p.likely_slot + (size_t)l * kMaxLikely + q);
 }
 
+// All threads: the layer's input h (h += y of the previous layer from its accumulator,
+// or h = y without the residual; acc null: h as it is) and, per 16-column chunk c, the
+// canonical partials of the norm and of my router rows: plain fmaf chains over the
+// chunk's columns in order from +0, of h^2 into pc[c] and of w_k * u (u = g * h, or h
+// without the norm) into pc[(1 + k) nch + c].  A chunk is two lanes of 8 columns; the
+// even lane's chain carries on in the odd lane, which makes it the one sequential chain
+// over the 16 columns.
+__device__ __forceinline__ void head_pass(const DecodeParams& p, const unsigned long long* acc, float* hs,
+                                          const float* gs, const uint16_t* rrows, int nrx, float* pc, float* trace) {
+  const int H = p.H, nch = H / kChunk, n8 = H / 8;
+  const int lane = threadIdx.x & 31;
+  const bool odd = lane & 1;
+  for (int q0 = threadIdx.x & ~31; q0 < n8; q0 += kThreads) {  // warp-uniform: the shuffles need every lane
+    const int q = q0 + lane;
+    const bool live = q < n8;  // n8 is even: both lanes of a chunk are live or neither
+    const int qq = live ? q : n8 - 1;
+    float h[8];
+    {
+      const float4* h4 = reinterpret_cast<const float4*>(hs + 8 * qq);
+      const float4 a = h4[0], c = h4[1];
+      h[0] = a.x; h[1] = a.y; h[2] = a.z; h[3] = a.w;
+      h[4] = c.x; h[5] = c.y; h[6] = c.z; h[7] = c.w;
+    }
+    if (acc) {
+      const ulonglong2* a2 = reinterpret_cast<const ulonglong2*>(acc + 8 * qq);
+      ulonglong2 v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = __ldcg(a2 + k);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float y0 = __ll2float_rn((long long)v[k].x) * kAccInvScale;
+        const float y1 = __ll2float_rn((long long)v[k].y) * kAccInvScale;
+        h[2 * k] = p.use_norm ? __fadd_rn(h[2 * k], y0) : y0;
+        h[2 * k + 1] = p.use_norm ? __fadd_rn(h[2 * k + 1], y1) : y1;
+      }
+      if (live) {
+        float4* h4 = reinterpret_cast<float4*>(hs + 8 * q);
+        h4[0] = make_float4(h[0], h[1], h[2], h[3]);
+        h4[1] = make_float4(h[4], h[5], h[6], h[7]);
+        if (trace) {
+          float4* t4 = reinterpret_cast<float4*>(trace + 8 * q);
+          t4[0] = make_float4(h[0], h[1], h[2], h[3]);
+          t4[1] = make_float4(h[4], h[5], h[6], h[7]);
+        }
+      }
+    }
+    if (p.use_norm) {
+      float s = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s = fmaf(h[i], h[i], s);
+      float t = __shfl_up_sync(0xffffffffu, s, 1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t = fmaf(h[i], h[i], t);
+      if (live && odd) pc[q >> 1] = t;
+    }
+    if (nrx > 0) {
+      float u[8];
+      if (p.use_norm) {
+        const float4* g4 = reinterpret_cast<const float4*>(gs + 8 * qq);
+        const float4 a = g4[0], c = g4[1];
+        u[0] = __fmul_rn(a.x, h[0]); u[1] = __fmul_rn(a.y, h[1]);
+        u[2] = __fmul_rn(a.z, h[2]); u[3] = __fmul_rn(a.w, h[3]);
+        u[4] = __fmul_rn(c.x, h[4]); u[5] = __fmul_rn(c.y, h[5]);
+        u[6] = __fmul_rn(c.z, h[6]); u[7] = __fmul_rn(c.w, h[7]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) u[i] = h[i];
+      }
+      for (int k = 0; k < nrx; ++k) {
+        const uint4 w = *reinterpret_cast<const uint4*>(rrows + (size_t)k * H + 8 * qq);
+        const float wf[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                             bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+        float s = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s = fmaf(wf[i], u[i], s);
+        float t = __shfl_up_sync(0xffffffffu, s, 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t = fmaf(wf[i], u[i], t);
+        if (live && odd) pc[(1 + k) * nch + (q >> 1)] = t;
+      }
+    }
+  }
+}
+
+// One warp: the canonical fold of a row of chunk partials: lane l adds chunks l, l + 32,
+// ... in order from +0, then the xor butterfly (16, 8, 4, 2, 1); every lane gets the sum.
+__device__ __forceinline__ float fold_chunks(const float* pc, int nch) {
+  float acc = 0.0f;
+  for (int c = threadIdx.x & 31; c < nch; c += 32) acc = __fadd_rn(acc, pc[c]);
+  return butterfly_sum(acc);
+}
+
 // All threads: h += y (or h = y without the residual) from a layer's accumulator; all of
 // a thread's loads are issued before any of them is used (one L2 round trip, not one
 // per element).  trace: where to write the new h, or null.
@@ -876,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
   const uint16_t* rrows = reinterpret_cast<const uint16_t*>(smem + S.rrows);
   float* hs = reinterpret_cast<float*>(smem + S.h);
   float* gs = reinterpret_cast<float*>(smem + S.g);
-  float* up = reinterpret_cast<float*>(smem + S.up);
+  float* pcs = reinterpret_cast<float*>(smem + S.pc);
   int16_t* xcodes = reinterpret_cast<int16_t*>(smem + S.xcodes);
   float* xs = reinterpret_cast<float*>(smem + S.xs);
   int32_t* xc = reinterpret_cast<int32_t*>(smem + S.xc);
@@ -1005,86 +1110,28 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     stamp(p, l, 2);
 
     // ---------------------------------------------------------------- norm and router
-    // inv = 1 / sqrt(ss / H + eps), ss folded canonically from 16-column fmaf chunks
-    if (warp == 0) {
-      float inv = 1.0f;
-      if (p.use_norm) {
-        float acc = 0.0f;
-#pragma unroll 4
-        for (int c = lane; c < nch; c += 32) {
-          const float4* h4 = reinterpret_cast<const float4*>(hs + c * kChunk);
-          float pc = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 v = h4[q];
-            pc = fmaf(v.x, v.x, pc);
-            pc = fmaf(v.y, v.y, pc);
-            pc = fmaf(v.z, v.z, pc);
-            pc = fmaf(v.w, v.w, pc);
-          }
-          acc = __fadd_rn(acc, pc);
-        }
-        const float ss = butterfly_sum(acc);
-        inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), p.eps)));
-      }
-      if (lane == 0) m.inv = inv;
-    }
-    // router input u = g * h in the lane-major order the canonical fold reads: column
-    // 16 c + 4 q + r, c = lane + 32 m, at float4 (4 m + q) * 32 + lane, component r
-    for (int j = tid; j < H; j += kThreads) {
-      const int c = j >> 4, t = j & 15;
-      const float u = p.use_norm ? __fmul_rn(gs[j], hs[j]) : hs[j];
-      up[((((c >> 5) * 4 + (t >> 2)) * 32 + (c & 31)) << 2) + (t & 3)] = u;
-    }
+    // chunk partials of the norm and of my router rows (this layer's rows landed during
+    // the previous layer), then the canonical folds
+    if (nrx > 0 && !__all_sync(0xffffffffu, ok && mbar_wait(p, &m.bar_r, par_r))) ok = false;
+    head_pass(p, nullptr, hs, gs, rrows, nrx, pcs, nullptr);
     __syncthreads();
+    // inv = 1 / sqrt(ss / H + eps), folded by every warp (the same bits everywhere)
+    const float inv =
+        p.use_norm ? __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(fold_chunks(pcs, nch), (float)H), p.eps))) : 1.0f;
     stamp(p, l, 10);
-    // logits of my experts: warp k folds expert b + k G in the canonical order
+    // logits of my experts: warp k folds expert b + k G
     if (warp < nrx) {
-      if (!__all_sync(0xffffffffu, ok && mbar_wait(p, &m.bar_r, par_r))) ok = false;
-      if (ok) {
-        const uint16_t* wr = rrows + (size_t)warp * H;
-        float acc = 0.0f;
-#pragma unroll 4
-        for (int mm = 0; mm * 32 < nch; ++mm) {
-          const int c = lane + 32 * mm;
-          if (c < nch) {
-            const uint4 w0 = *reinterpret_cast<const uint4*>(wr + c * kChunk);
-            const uint4 w1 = *reinterpret_cast<const uint4*>(wr + c * kChunk + 8);
-            const float4* u4 = reinterpret_cast<const float4*>(up) + (mm * 4) * 32 + lane;
-            const float4 u0 = u4[0], u1 = u4[32], u2 = u4[64], u3 = u4[96];
-            float pc = 0.0f;
-            pc = fmaf(bf16_lo(w0.x), u0.x, pc);
-            pc = fmaf(bf16_hi(w0.x), u0.y, pc);
-            pc = fmaf(bf16_lo(w0.y), u0.z, pc);
-            pc = fmaf(bf16_hi(w0.y), u0.w, pc);
-            pc = fmaf(bf16_lo(w0.z), u1.x, pc);
-            pc = fmaf(bf16_hi(w0.z), u1.y, pc);
-            pc = fmaf(bf16_lo(w0.w), u1.z, pc);
-            pc = fmaf(bf16_hi(w0.w), u1.w, pc);
-            pc = fmaf(bf16_lo(w1.x), u2.x, pc);
-            pc = fmaf(bf16_hi(w1.x), u2.y, pc);
-            pc = fmaf(bf16_lo(w1.y), u2.z, pc);
-            pc = fmaf(bf16_hi(w1.y), u2.w, pc);
-            pc = fmaf(bf16_lo(w1.z), u3.x, pc);
-            pc = fmaf(bf16_hi(w1.z), u3.y, pc);
-            pc = fmaf(bf16_lo(w1.w), u3.z, pc);
-            pc = fmaf(bf16_hi(w1.w), u3.w, pc);
-            acc = __fadd_rn(acc, pc);
-          }
-        }
-        const float S_e = butterfly_sum(acc);
-        if (lane == 0) {
-          const int e = b + warp * G;
-          const float z = fmaf(S_e, m.inv, m.bias[warp]);
-          st_relaxed_u64(p.zll + e, ((unsigned long long)(uint32_t)(l + 1) << 32) | __float_as_uint(z));
-          if (warp == 0) stamp(p, l, 11);
-        }
+      const float S_e = fold_chunks(pcs + (size_t)(1 + warp) * nch, nch);
+      if (lane == 0 && ok) {
+        const int e = b + warp * G;
+        const float z = fmaf(S_e, inv, m.bias[warp]);
+        st_relaxed_u64(p.zll + e, ((unsigned long long)(uint32_t)(l + 1) << 32) | __float_as_uint(z));
+        if (warp == 0) stamp(p, l, 11);
       }
     }
     // quantised expert input x = RMSNorm(h) (or h): four lanes per 32-block, each lane 8
     // values; the block's largest |x| and code sum combine over the four lanes
     {
-      const float inv = m.inv;
       const int j4 = tid & 3;
       for (int b0 = tid >> 2; b0 < ((nb + 63) / 64) * 64; b0 += kThreads / 4) {
         const int bb = b0 < nb ? b0 : nb - 1;  // lanes past the end repeat a block, write nothing
@@ -1162,33 +1209,51 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     }
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 4);
-    int my_e = 0;
-    if (p.E <= kThreads) {
-      my_e = topk_parallel(p, m, zs, cand);
-    } else if (warp == 0) {
-      my_e = topk_weights(p, m, zs);
-    }
     if (warp == 0) {
+      const int my_e = topk_weights(p, m, zs);
       stamp(p, l, 13);
-      const bool fast = cache_all_pinned(p, m, l, pinrow, my_e);
-      if (lane == 0 && !fast) cache_decide(p, m, l, pinrow);
-      if (lane == 0) {  // preload matching: which group holds which rank, which ranks are left
-        uint32_t covered = 0;
-        int wrong = 0;
-        for (int q = 0; q < p.n_pre; ++q) {
-          int r = -1;
-          for (int i = 0; i < p.K; ++i)
-            if (m.sel[i] == m.lk_e[q]) r = i;
-          m.hit[q] = r;
-          if (r >= 0) covered |= 1u << r;
-          else ++wrong;
+      if (lane == 0) m.early = 0;
+      const bool fast = cache_pinned_lookup(p, m, pinrow, my_e);
+      if (fast && p.n_pre == 0) {
+        // no preloads: every rank is uncovered, and one unit per CTA is known now; its
+        // loads go out before the rest of the bookkeeping
+        if (lane < p.K) m.unc[lane] = lane;
+        if (lane == 0) {
+          m.n_unc = p.K;
+          m.n_avail = routed + max(G - p.n_units, 0);
         }
-        int nu = 0;
-        for (int i = 0; i < p.K; ++i)
-          if (!((covered >> i) & 1u)) m.unc[nu++] = i;
-        m.n_unc = nu;
-        m.n_avail = wrong * Ur + (routed - npc) + max(G - p.n_units, 0);
+        __syncwarp();
+        if (lane == 0 && G >= p.n_units) {
+          UnitRef ur;
+          if (unit_of(p, m, pre, b, G, 0, ur) && !ur.issued && !ur.shared) {
+            issue_unit(p, m, ubuf, m.src[ur.i] + (size_t)ur.rb * p.unit_bytes);
+            m.early = 1;
+          }
+        }
       }
+      stamp(p, l, 15);
+      if (fast) cache_pinned_commit(p, m, l, pinrow, my_e);
+      else if (lane == 0) cache_decide(p, m, l, pinrow);
+      if (!(fast && p.n_pre == 0)) {
+        if (lane == 0) {  // preload matching: which group holds which rank, which ranks are left
+          uint32_t covered = 0;
+          int wrong = 0;
+          for (int q = 0; q < p.n_pre; ++q) {
+            int r = -1;
+            for (int i = 0; i < p.K; ++i)
+              if (m.sel[i] == m.lk_e[q]) r = i;
+            m.hit[q] = r;
+            if (r >= 0) covered |= 1u << r;
+            else ++wrong;
+          }
+          int nu = 0;
+          for (int i = 0; i < p.K; ++i)
+            if (!((covered >> i) & 1u)) m.unc[nu++] = i;
+          m.n_unc = nu;
+          m.n_avail = wrong * Ur + (routed - npc) + max(G - p.n_units, 0);
+        }
+      }
+      __syncwarp();
       stamp(p, l, 14);
     }
     __syncthreads();
@@ -1223,6 +1288,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         }
       }
       unsigned long long* acc_l = p.acc + (size_t)(l % kAccBufs) * H;
+      const bool early = m.early != 0;
       UnitRef ur;
       for (int k = 0; unit_of(p, m, pre, b, G, k, ur); ++k) {
         const bool shared = ur.shared;
@@ -1230,7 +1296,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         const float wi = shared ? 1.0f : m.w[i];
         const uint8_t* usrc = (shared ? p.shared_pool + (size_t)l * p.shared_slot_bytes : m.src[i]) +
                               (size_t)rb * p.unit_bytes;
-        if (!ur.issued) {
+        if (!ur.issued && !(k == 0 && early)) {
           if (pre) {  // a preload that routing did not use: let it land before the buffer is reused
             ok = drain_unit(p, m, par_u, par_d);
             if (!cta_ok(p, ok)) goto fail;
@@ -1243,7 +1309,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           if (tid == 0) {
             ok = shared || wait_miss(p, m.miss_seq[i]);
             if (ok) issue_unit(p, m, ubuf, usrc);
-            stamp(p, l, 15);
           }
           if (!cta_ok(p, ok)) goto fail;
         }
