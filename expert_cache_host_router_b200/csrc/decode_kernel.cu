@@ -247,7 +247,7 @@ struct Misc {
 };
 
 struct SmemPlan {
-  uint32_t unit, rrows, h, g, pc, xcodes, xs, xc, z, pinrow, cand, misc, total;
+  uint32_t unit, rrows, h, g, pc, xcodes, xs, xc, z, pinrow, cand, misc, params, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
@@ -274,6 +274,7 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
   s.pinrow = take(4u * E);
   s.cand = take(8u * kWarps * kMaxK + 8u * kThreads);
   s.misc = take(sizeof(Misc));
+  s.params = take(sizeof(DecodeParams));
   s.total = align_up(off, 128);
   return s;
 }
@@ -285,13 +286,13 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
 // enough for the SM instruction cache.
 
 // Spin until *count >= target (acquire), with back-off; false on timeout / error.
-__device__ __noinline__ bool spin_count(const DecodeParams& p, const uint32_t* count, uint32_t target) {
+__device__ __noinline__ bool spin_count(const uint32_t* count, uint32_t target, uint64_t timeout_ns, Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
   for (uint32_t polls = 1; ld_acquire(count) < target; ++polls) {
     if ((polls & 15u) == 0) {
-      if (has_error(p.ctrl)) return false;
-      if (gtimer() - t0 > p.timeout_ns) {
-        set_error(p.ctrl, MOE_DEVERR_BARRIER);
+      if (has_error(ctrl)) return false;
+      if (gtimer() - t0 > timeout_ns) {
+        set_error(ctrl, MOE_DEVERR_BARRIER);
         return false;
       }
     }
@@ -300,36 +301,34 @@ __device__ __noinline__ bool spin_count(const DecodeParams& p, const uint32_t* c
 }
 
 __device__ __forceinline__ bool wait_count(const DecodeParams& p, const uint32_t* count, uint32_t target) {
-  return ld_acquire(count) >= target || spin_count(p, count, target);
+  return ld_acquire(count) >= target || spin_count(count, target, p.timeout_ns, p.ctrl);
 }
 
-// Spin until the published logit word carries epoch; false on timeout / error.
-__device__ __noinline__ bool spin_logit(const DecodeParams& p, const unsigned long long* w, uint32_t epoch,
-                                        unsigned long long* out) {
+// Spin until the published logit word carries epoch (>= 1) and return it; 0 on timeout
+// / error (a published word is never 0).
+__device__ __noinline__ unsigned long long spin_logit(const unsigned long long* w, uint32_t epoch, uint64_t timeout_ns,
+                                                      Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
   for (uint32_t polls = 1;; ++polls) {
     const unsigned long long v = ld_relaxed_u64(w);
-    if ((uint32_t)(v >> 32) == epoch) {
-      *out = v;
-      return true;
-    }
+    if ((uint32_t)(v >> 32) == epoch) return v;
     if ((polls & 15u) == 0) {
-      if (has_error(p.ctrl)) return false;
-      if (gtimer() - t0 > p.timeout_ns) {
-        set_error(p.ctrl, MOE_DEVERR_BARRIER);
-        return false;
+      if (has_error(ctrl)) return 0ull;
+      if (gtimer() - t0 > timeout_ns) {
+        set_error(ctrl, MOE_DEVERR_BARRIER);
+        return 0ull;
       }
     }
   }
 }
 
 // Thread 0: wait until the proxy has signalled miss copy seq (0: nothing to wait for).
-__device__ __noinline__ bool spin_miss(const DecodeParams& p, uint32_t seq) {
+__device__ __noinline__ bool spin_miss(const uint32_t* done_seq, uint32_t seq, uint64_t timeout_ns, Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
-  while ((int32_t)(ld_acquire(p.done_seq) - seq) < 0) {
-    if (has_error(p.ctrl)) return false;
-    if (gtimer() - t0 > p.timeout_ns) {
-      set_error(p.ctrl, MOE_DEVERR_MISS);
+  while ((int32_t)(ld_acquire(done_seq) - seq) < 0) {
+    if (has_error(ctrl)) return false;
+    if (gtimer() - t0 > timeout_ns) {
+      set_error(ctrl, MOE_DEVERR_MISS);
       return false;
     }
   }
@@ -338,17 +337,17 @@ __device__ __noinline__ bool spin_miss(const DecodeParams& p, uint32_t seq) {
 
 __device__ __forceinline__ bool wait_miss(const DecodeParams& p, uint32_t seq) {
   if (seq == 0) return true;
-  if ((int32_t)(ld_acquire(p.done_seq) - seq) < 0 && !spin_miss(p, seq)) return false;
+  if ((int32_t)(ld_acquire(p.done_seq) - seq) < 0 && !spin_miss(p.done_seq, seq, p.timeout_ns, p.ctrl)) return false;
   fence_proxy_async();  // the copy engine's writes, then bulk-copy reads of the same slot
   return true;
 }
 
 // Wait for the bulk copies counted on bar to land (bounded).
-__device__ __noinline__ bool spin_mbar(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
+__device__ __noinline__ bool spin_mbar(uint64_t* bar, uint32_t parity, uint64_t timeout_ns, Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (gtimer() - t0 > p.timeout_ns) {
-      set_error(p.ctrl, MOE_DEVERR_TMA);
+    if (gtimer() - t0 > timeout_ns) {
+      set_error(ctrl, MOE_DEVERR_TMA);
       return false;
     }
   }
@@ -356,7 +355,7 @@ __device__ __noinline__ bool spin_mbar(const DecodeParams& p, uint64_t* bar, uin
 }
 
 __device__ __forceinline__ bool mbar_wait(const DecodeParams& p, uint64_t* bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity) || spin_mbar(p, bar, parity);
+  return mbar_try_wait(bar, parity) || spin_mbar(bar, parity, p.timeout_ns, p.ctrl);
 }
 
 // Barrier + agreement: true when every thread of the CTA passed ok, so that the CTA
@@ -717,7 +716,7 @@ __device__ __noinline__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t*
 
 // All threads: wait until a unit issued ahead has landed (its copies complete the
 // current phase of the unit barriers), then advance the parities past it.
-__device__ __noinline__ bool drain_unit(const DecodeParams& p, Misc& m, uint32_t (&par_u)[4], uint32_t& par_d) {
+__device__ __forceinline__ bool drain_unit(const DecodeParams& p, Misc& m, uint32_t (&par_u)[4], uint32_t& par_d) {
   bool ok = true;
 #pragma unroll
   for (int st = 0; st < 4; ++st) ok = ok && mbar_wait(p, &m.bar_u[st], par_u[st]);
@@ -970,13 +969,23 @@ __device__ __forceinline__ void add_layer_output(const DecodeParams& p, const un
   }
 }
 
+// a[i] of a 4-element register array for a run-time i (selects, no local memory)
+__device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int i) {
+  return i == 0 ? a[0] : i == 1 ? a[1] : i == 2 ? a[2] : a[3];
+}
+
 // ------------------------------------------------------------------ the kernel
 
 template <int BPL>
-__global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const SmemPlan S = smem_plan(p.H, p.E, p.rx_per_cta, p.down_late);
   Misc& m = *reinterpret_cast<Misc*>(smem + S.misc);
+  // a shared-memory copy of the parameters for the out-of-line helpers (a reference to
+  // it is a plain shared address; the kernel body reads the parameters directly)
+  DecodeParams& sp = *reinterpret_cast<DecodeParams*>(smem + S.params);
+  for (int i = threadIdx.x; i < (int)(sizeof(DecodeParams) / 4); i += kThreads)
+    reinterpret_cast<uint32_t*>(&sp)[i] = reinterpret_cast<const uint32_t*>(&p)[i];
   uint8_t* ubuf = smem + S.unit;
   const uint16_t* rrows = reinterpret_cast<const uint16_t*>(smem + S.rrows);
   float* hs = reinterpret_cast<float*>(smem + S.h);
@@ -1030,19 +1039,19 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         bulk_g2s_stream(const_cast<uint16_t*>(rrows) + (size_t)k * H, p.router + (size_t)(b + k * G) * H, 2u * H,
                         &m.bar_r);
     }
-    if (first_shared) issue_unit(p, m, ubuf, p.shared_pool + (size_t)(b - routed) * p.unit_bytes);
+    if (first_shared) issue_unit(sp, m, ubuf, p.shared_pool + (size_t)(b - routed) * p.unit_bytes);
   }
   if (b < npc) {  // preload: unit b mod Ur of layer 0's likely expert b / Ur
     const int32_t slot = __ldg(p.likely_slot + b / Ur);
     if (slot >= 0) {
-      if (tid == 0) issue_unit(p, m, ubuf, p.pool + (size_t)slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
+      if (tid == 0) issue_unit(sp, m, ubuf, p.pool + (size_t)slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
       pre = true;
     }
   }
   int32_t lk[kMaxLikely];  // thread 32: the likely experts' slots of the current layer
   if (tid == 32 && p.n_l2 > 0) {
-    load_likely(p, 0, lk);
-    prefetch_likely(p, lk);
+    load_likely(sp, 0, lk);
+    prefetch_likely(sp, lk);
   }
   if (b == 0 && p.h_trace)
     for (int j = tid; j < H; j += kThreads) p.h_trace[j] = hs[j];
@@ -1074,7 +1083,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (tid == kThreads - 2) m.P_l = __ldg(p.n_pinned + l);
       if (tid == kThreads - 3) m.base_l = __ldg(p.layer_base + l);
       if (tid < nrx) m.bias[tid] = p.bias ? __ldg(p.bias + (size_t)l * p.E + b + tid * G) : 0.0f;
-      if (tid == 32 && p.n_l2 > 0 && l > 0) load_likely(p, l, lk);
+      if (tid == 32 && p.n_l2 > 0 && l > 0) load_likely(sp, l, lk);
       if (tid < p.n_pre) m.lk_e[tid] = __ldg(p.likely_e + (size_t)l * kMaxLikely + tid);
       pre_slot = (l > 0 && b < npc) ? __ldg(p.likely_slot + (size_t)l * kMaxLikely + b / Ur) : -1;
     }
@@ -1084,13 +1093,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G);
         // every unit of layer l - 1 is done: the HBM is free for this layer's guess
         if (ok && pre_slot >= 0)
-          issue_unit(p, m, ubuf, p.pool + (size_t)pre_slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
+          issue_unit(sp, m, ubuf, p.pool + (size_t)pre_slot * p.slot_bytes + (size_t)(b % Ur) * p.unit_bytes);
       }
       if (pre_slot >= 0) pre = true;
       // the HBM is idle until this layer's routing is known: fetch its likely experts
       // (a thread off the critical path, after the wait)
       if (tid == 32 && p.n_l2 > 0) {
-        if (wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G)) prefetch_likely(p, lk);
+        if (wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G)) prefetch_likely(sp, lk);
       }
       if (!cta_ok(p, ok)) goto fail;
       stamp(p, l, 1);
@@ -1098,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
                        (b == 0 && p.h_trace) ? p.h_trace + (size_t)l * H : nullptr);
       // deferred ring fills of layer l - 1 (a layer that missed more often than it has
       // ring slots): its readers are done
-      if (m.n_fix > 0) ring_fills(p, m);
+      if (m.n_fix > 0) ring_fills(sp, m);
       // the accumulator of layer l + 1 was last read at the start of layer l - 1, by CTAs
       // that have all published layer l - 1's logits since
       if (next) {
@@ -1200,7 +1209,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       const uint32_t epoch = (uint32_t)(l + 1);
       for (int e = tid; e < p.E; e += kThreads) {
         unsigned long long v = ld_relaxed_u64(p.zll + e);
-        if ((uint32_t)(v >> 32) != epoch && !spin_logit(p, p.zll + e, epoch, &v)) {
+        if ((uint32_t)(v >> 32) != epoch) v = spin_logit(p.zll + e, epoch, p.timeout_ns, p.ctrl);
+        if (v == 0ull) {
           ok = false;
           break;
         }
@@ -1210,7 +1220,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 4);
     if (warp == 0) {
-      const int my_e = topk_weights(p, m, zs);
+      const int my_e = topk_weights(sp, m, zs);
       stamp(p, l, 13);
       if (lane == 0) m.early = 0;
       const bool fast = cache_pinned_lookup(p, m, pinrow, my_e);
@@ -1226,14 +1236,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
         if (lane == 0 && G >= p.n_units) {
           UnitRef ur;
           if (unit_of(p, m, pre, b, G, 0, ur) && !ur.issued && !ur.shared) {
-            issue_unit(p, m, ubuf, m.src[ur.i] + (size_t)ur.rb * p.unit_bytes);
+            issue_unit(sp, m, ubuf, m.src[ur.i] + (size_t)ur.rb * p.unit_bytes);
             m.early = 1;
           }
         }
       }
       stamp(p, l, 15);
-      if (fast) cache_pinned_commit(p, m, l, pinrow, my_e);
-      else if (lane == 0) cache_decide(p, m, l, pinrow);
+      if (fast) cache_pinned_commit(sp, m, l, pinrow, my_e);
+      else if (lane == 0) cache_decide(sp, m, l, pinrow);
       if (!(fast && p.n_pre == 0)) {
         if (lane == 0) {  // preload matching: which group holds which rank, which ranks are left
           uint32_t covered = 0;
@@ -1298,17 +1308,17 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
                               (size_t)rb * p.unit_bytes;
         if (!ur.issued && !(k == 0 && early)) {
           if (pre) {  // a preload that routing did not use: let it land before the buffer is reused
-            ok = drain_unit(p, m, par_u, par_d);
+            ok = drain_unit(sp, m, par_u, par_d);
             if (!cta_ok(p, ok)) goto fail;
             pre = false;
           }
           if (!shared && m.pull[i] >= 0) {  // pull mode miss: this CTA fills its unit of the slot
-            pull_unit(p, p.host_tier + m.pull[i] + (size_t)rb * p.unit_bytes, const_cast<uint8_t*>(usrc));
+            pull_unit(sp, p.host_tier + m.pull[i] + (size_t)rb * p.unit_bytes, const_cast<uint8_t*>(usrc));
             __syncthreads();
           }
           if (tid == 0) {
             ok = shared || wait_miss(p, m.miss_seq[i]);
-            if (ok) issue_unit(p, m, ubuf, usrc);
+            if (ok) issue_unit(sp, m, ubuf, usrc);
           }
           if (!cta_ok(p, ok)) goto fail;
         }
@@ -1319,8 +1329,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
           const int rows[2] = {rw + sub, rw + sub + rstep};
           const bool live0 = rows[0] < 2 * kUnitRows, live1 = rows[1] < 2 * kUnitRows;
           bool w_ok = ok;
-          if (w_ok && live0) w_ok = mbar_wait(p, &m.bar_u[rows[0] / 16], par_u[rows[0] / 16]);
-          if (w_ok && live1) w_ok = mbar_wait(p, &m.bar_u[rows[1] / 16], par_u[rows[1] / 16]);
+          if (w_ok && live0) w_ok = mbar_wait(p, &m.bar_u[rows[0] / 16], pick4(par_u, rows[0] / 16));
+          if (w_ok && live1) w_ok = mbar_wait(p, &m.bar_u[rows[1] / 16], pick4(par_u, rows[1] / 16));
           if (!__all_sync(0xffffffffu, w_ok)) {
             ok = false;
             break;
@@ -1408,7 +1418,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       }
     }
     if (pre) {  // a preload left unused (no unit for this CTA): let it land
-      ok = drain_unit(p, m, par_u, par_d);
+      ok = drain_unit(sp, m, par_u, par_d);
       if (!cta_ok(p, ok)) goto fail;
       pre = false;
     }
@@ -1418,7 +1428,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
     // expert's unit is worth guessing: load them now
     if (next && first_shared) {
       if (tid == 0)
-        issue_unit(p, m, ubuf,
+        issue_unit(sp, m, ubuf,
                    p.shared_pool + (size_t)(l + 1) * p.shared_slot_bytes + (size_t)(b - routed) * p.unit_bytes);
       pre = true;
     }
@@ -1437,7 +1447,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const DecodePar
       if (j0 + tid < H) p.y[j0 + tid] = hs[j0 + tid];
     if (b == 0 && p.h_trace)
       for (int j = tid; j < H; j += kThreads) p.h_trace[(size_t)p.L * H + j] = hs[j];
-    if (m.n_fix > 0) ring_fills(p, m);
+    if (m.n_fix > 0) ring_fills(sp, m);
   }
   stamp_both(p, 2, 5);
   if (b == 0 && tid == 0) {
