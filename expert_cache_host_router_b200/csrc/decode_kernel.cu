@@ -858,9 +858,9 @@ __device__ __noinline__ void load_likely(const DecodeParams& p, int l, int32_t (
 // without the norm) into pc[(1 + k) nch + c].  A chunk is two lanes of 8 columns; the
 // even lane's chain carries on in the odd lane, which makes it the one sequential chain
 // over the 16 columns.
-__device__ __forceinline__ void head_pass(const DecodeParams& p, const unsigned long long* acc, float* hs,
+__device__ __forceinline__ void head_pass(const DecodeParams& p, int H, const unsigned long long* acc, float* hs,
                                           const float* gs, const uint16_t* rrows, int nrx, float* pc, float* trace) {
-  const int H = p.H, nch = H / kChunk, n8 = H / 8;
+  const int nch = H / kChunk, n8 = H / 8;
   const int lane = threadIdx.x & 31;
   const bool odd = lane & 1;
   for (int q0 = threadIdx.x & ~31; q0 < n8; q0 += kThreads) {  // warp-uniform: the shuffles need every lane
@@ -946,20 +946,20 @@ __device__ __forceinline__ float fold_chunks(const float* pc, int nch) {
 // All threads: h += y (or h = y without the residual) from a layer's accumulator; all of
 // a thread's loads are issued before any of them is used (one L2 round trip, not one
 // per element).  trace: where to write the new h, or null.
-__device__ __forceinline__ void add_layer_output(const DecodeParams& p, const unsigned long long* acc, float* hs,
+__device__ __forceinline__ void add_layer_output(const DecodeParams& p, int H, const unsigned long long* acc, float* hs,
                                                  float* trace) {
   constexpr int kPer = 8;
-  for (int j0 = 0; j0 < p.H; j0 += kPer * kThreads) {
+  for (int j0 = 0; j0 < H; j0 += kPer * kThreads) {
     long long v[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int j = j0 + threadIdx.x + k * kThreads;
-      v[k] = j < p.H ? (long long)__ldcg(acc + j) : 0;
+      v[k] = j < H ? (long long)__ldcg(acc + j) : 0;
     }
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
       const int j = j0 + threadIdx.x + k * kThreads;
-      if (j < p.H) {
+      if (j < H) {
         const float y = __ll2float_rn(v[k]) * kAccInvScale;
         const float hn = p.use_norm ? __fadd_rn(hs[j], y) : y;
         hs[j] = hn;
@@ -976,10 +976,15 @@ __device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int i) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int BPL>
+// BPL: Q4_0 blocks of a gate/up row per lane (ceil(H / 1024), at least 1).  HC: the
+// hidden size when it is 1024 BPL (a lane holds blocks lane + 32 mb exactly; every size
+// and offset below is then a compile-time constant), else 0 (sizes read at run time).
+template <int BPL, int HC>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ DecodeParams p) {
+  static_assert(HC == 0 || HC == 1024 * BPL, "HC is 0 or 1024 BPL");
   extern __shared__ __align__(128) uint8_t smem[];
-  const SmemPlan S = smem_plan(p.H, p.E, p.rx_per_cta, p.down_late);
+  const int H = HC ? HC : p.H;
+  const SmemPlan S = smem_plan(H, p.E, p.rx_per_cta, p.down_late);
   Misc& m = *reinterpret_cast<Misc*>(smem + S.misc);
   // a shared-memory copy of the parameters for the out-of-line helpers (a reference to
   // it is a plain shared address; the kernel body reads the parameters directly)
@@ -1000,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, b = blockIdx.x;
-  const int H = p.H, nb = H / 32, nch = H / kChunk;
+  const int nb = H / 32, nch = H / kChunk;
   const int routed = p.K * (p.I / 32);
   const bool has_gain = p.use_norm && p.gain;
   const int nrx = b < p.E ? min(p.rx_per_cta, (p.E - b + G - 1) / G) : 0;  // my router experts b, b+G, ...
@@ -1103,7 +1108,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       }
       if (!cta_ok(p, ok)) goto fail;
       stamp(p, l, 1);
-      add_layer_output(p, p.acc + (size_t)((l - 1) % kAccBufs) * H, hs,
+      add_layer_output(p, H, p.acc + (size_t)((l - 1) % kAccBufs) * H, hs,
                        (b == 0 && p.h_trace) ? p.h_trace + (size_t)l * H : nullptr);
       // deferred ring fills of layer l - 1 (a layer that missed more often than it has
       // ring slots): its readers are done
@@ -1122,7 +1127,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     // chunk partials of the norm and of my router rows (this layer's rows landed during
     // the previous layer), then the canonical folds
     if (nrx > 0 && !__all_sync(0xffffffffu, ok && mbar_wait(p, &m.bar_r, par_r))) ok = false;
-    head_pass(p, nullptr, hs, gs, rrows, nrx, pcs, nullptr);
+    head_pass(p, H, nullptr, hs, gs, rrows, nrx, pcs, nullptr);
     __syncthreads();
     // inv = 1 / sqrt(ss / H + eps), folded by every warp (the same bits everywhere)
     const float inv =
@@ -1323,41 +1328,80 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           if (!cta_ok(p, ok)) goto fail;
         }
         stamp(p, l, 6);
-        // gate/up: rows r = gate 0..31, up 0..31 of the unit, tile r / 16; two rows at a
-        // time per lane group, in tile order
-        for (int rw = warp * RPW; rw < 2 * kUnitRows; rw += 2 * rstep) {  // warp-uniform
-          const int rows[2] = {rw + sub, rw + sub + rstep};
-          const bool live0 = rows[0] < 2 * kUnitRows, live1 = rows[1] < 2 * kUnitRows;
-          bool w_ok = ok;
-          if (w_ok && live0) w_ok = mbar_wait(p, &m.bar_u[rows[0] / 16], pick4(par_u, rows[0] / 16));
-          if (w_ok && live1) w_ok = mbar_wait(p, &m.bar_u[rows[1] / 16], pick4(par_u, rows[1] / 16));
-          if (!__all_sync(0xffffffffu, w_ok)) {
-            ok = false;
-            break;
-          }
-          float acc[2] = {0.0f, 0.0f};
-#pragma unroll
-          for (int mb = 0; mb < BPL; ++mb) {
-            const int bb = g + GS * mb;
-            if (bb >= nb) continue;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if ((q == 0 && !live0) || (q == 1 && !live1)) continue;
-              const int r = rows[q];
-              const uint8_t* tile = ubuf + (r / 16) * 9u * H;
-              const uint4 qv = *reinterpret_cast<const uint4*>(tile + ((size_t)(r % 16) * nb + bb) * 16);
-              const float d = __half2float(reinterpret_cast<const __half*>(tile + 8u * H)[(r % 16) * nb + bb]);
-              const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
-              acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
+        // gate/up: rows r = gate 0..31, up 0..31 of the unit, tile r / 16; warp w takes rows
+        // w + 8 j (j = 0..7: tile j / 2, row w + 8 (j % 2) of it)
+        if constexpr (HC != 0) {
+          // lane l holds blocks l + 32 mb; four rows (two tiles) per pass
+          constexpr int NB = HC / 32;
+#pragma unroll 1
+          for (int j0 = 0; j0 < 8; j0 += 4) {
+            bool w_ok = ok;
+            w_ok = w_ok && mbar_wait(p, &m.bar_u[j0 / 2], pick4(par_u, j0 / 2));
+            w_ok = w_ok && mbar_wait(p, &m.bar_u[j0 / 2 + 1], pick4(par_u, j0 / 2 + 1));
+            if (!__all_sync(0xffffffffu, w_ok)) {
+              ok = false;
+              break;
             }
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int j = j0 + q;
+              const uint8_t* tile = ubuf + (j / 2) * 9u * HC;
+              const int rt = warp + 8 * (j % 2);  // row in the tile
+              const uint8_t* nib = tile + (size_t)rt * NB * 16;
+              const __half* dsc = reinterpret_cast<const __half*>(tile + 8u * HC) + rt * NB;
+#pragma unroll
+              for (int mb = 0; mb < BPL; ++mb) {
+                const int bb = lane + 32 * mb;
+                const uint4 qv = *reinterpret_cast<const uint4*>(nib + bb * 16);
+                const float d = __half2float(dsc[bb]);
+                const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
+                acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
+              }
+            }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
+            if (lane == 0)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) m.gu[warp + 8 * (j0 + q)] = acc[q];
           }
-          for (int off = GS / 2; off >= 1; off >>= 1) {
-            acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
-            acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], off);
-          }
-          if (g == 0) {
-            if (live0) m.gu[rows[0]] = acc[0];
-            if (live1) m.gu[rows[1]] = acc[1];
+        } else {
+          for (int rw = warp * RPW; rw < 2 * kUnitRows; rw += 2 * rstep) {  // warp-uniform
+            const int rows[2] = {rw + sub, rw + sub + rstep};
+            const bool live0 = rows[0] < 2 * kUnitRows, live1 = rows[1] < 2 * kUnitRows;
+            bool w_ok = ok;
+            if (w_ok && live0) w_ok = mbar_wait(p, &m.bar_u[rows[0] / 16], pick4(par_u, rows[0] / 16));
+            if (w_ok && live1) w_ok = mbar_wait(p, &m.bar_u[rows[1] / 16], pick4(par_u, rows[1] / 16));
+            if (!__all_sync(0xffffffffu, w_ok)) {
+              ok = false;
+              break;
+            }
+            float acc[2] = {0.0f, 0.0f};
+#pragma unroll
+            for (int mb = 0; mb < BPL; ++mb) {
+              const int bb = g + GS * mb;
+              if (bb >= nb) continue;
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                if ((q == 0 && !live0) || (q == 1 && !live1)) continue;
+                const int r = rows[q];
+                const uint8_t* tile = ubuf + (r / 16) * 9u * H;
+                const uint4 qv = *reinterpret_cast<const uint4*>(tile + ((size_t)(r % 16) * nb + bb) * 16);
+                const float d = __half2float(reinterpret_cast<const __half*>(tile + 8u * H)[(r % 16) * nb + bb]);
+                const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
+                acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
+              }
+            }
+            for (int off = GS / 2; off >= 1; off >>= 1) {
+              acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+              acc[1] += __shfl_xor_sync(0xffffffffu, acc[1], off);
+            }
+            if (g == 0) {
+              if (live0) m.gu[rows[0]] = acc[0];
+              if (live1) m.gu[rows[1]] = acc[1];
+            }
           }
         }
         if (!cta_ok(p, ok)) goto fail;
@@ -1442,7 +1486,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
   if (tid == 0) ok = wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(p.L + 1) * G);
   if (!cta_ok(p, ok)) goto fail;
   {
-    add_layer_output(p, p.acc + (size_t)((p.L - 1) % kAccBufs) * H, hs, nullptr);
+    add_layer_output(p, H, p.acc + (size_t)((p.L - 1) % kAccBufs) * H, hs, nullptr);
     for (int j0 = b * kThreads; j0 < H; j0 += G * kThreads)
       if (j0 + tid < H) p.y[j0 + tid] = hs[j0 + tid];
     if (b == 0 && p.h_trace)
@@ -1474,11 +1518,18 @@ static int bpl_of(int H) {
 
 template <typename F>
 static cudaError_t with_kernel(int H, F f) {
+  switch (H) {  // the hidden sizes with a compile-time instance
+    case 1024: return f(moe_decode_kernel<1, 1024>);
+    case 2048: return f(moe_decode_kernel<2, 2048>);
+    case 3072: return f(moe_decode_kernel<3, 3072>);
+    case 4096: return f(moe_decode_kernel<4, 4096>);
+    default: break;
+  }
   switch (bpl_of(H)) {
-    case 1: return f(moe_decode_kernel<1>);
-    case 2: return f(moe_decode_kernel<2>);
-    case 3: return f(moe_decode_kernel<3>);
-    default: return f(moe_decode_kernel<4>);
+    case 1: return f(moe_decode_kernel<1, 0>);
+    case 2: return f(moe_decode_kernel<2, 0>);
+    case 3: return f(moe_decode_kernel<3, 0>);
+    default: return f(moe_decode_kernel<4, 0>);
   }
 }
 
@@ -1506,10 +1557,14 @@ bool decode_plan(int H, int E, int grid, int smem_optin, int* rx, int* down_late
 cudaError_t decode_configure(int limit) {
   cudaError_t e = cudaSuccess;
   auto set = [&](auto kern) { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, limit); };
-  if (e == cudaSuccess) e = set(moe_decode_kernel<1>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<2>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<3>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<4>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<1, 0>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<2, 0>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<3, 0>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<4, 0>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<1, 1024>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<2, 2048>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<3, 3072>);
+  if (e == cudaSuccess) e = set(moe_decode_kernel<4, 4096>);
   return e;
 }
 
