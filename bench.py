@@ -462,7 +462,8 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8, residency=1.0, hist=Non
         table.append(row)
     total = float(np.median(marks[:, L, 5] - marks[:, L, 4])) / 1e3
     raw = [float(np.median(marks[:, 1:L, k] - marks[:, 1:L, 0])) * ns_per_cycle / 1e3 for k in range(32)]
-    # every CTA's global-timer marks: [0] routing decided, [1] units done, [2] arrival posted
+    # every CTA's global-timer marks: [0] routing decided, [1] units done, [2] arrival posted,
+    # [3] own logits published
     cta = np.stack([r[(L + 1) * 32:].reshape(L, n_sm, 4) for r in runs]).astype(np.float64)  # [tok][L][cta][4]
     rt, ud, ar = cta[..., 0], cta[..., 1], cta[..., 2]
     work = ud - rt  # per CTA: routing decided -> its units done
@@ -470,7 +471,10 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8, residency=1.0, hist=Non
                  "units_median_us": float(np.median(np.median(work, axis=2))) / 1e3,
                  "units_max_us": float(np.median(work.max(axis=2))) / 1e3,
                  "arrival_spread_us": float(np.median(ar.max(axis=2) - ar.min(axis=2))) / 1e3,
-                 "last_arrival_after_first_routed_us": float(np.median(ar.max(axis=2) - rt.min(axis=2))) / 1e3}
+                 "last_arrival_after_first_routed_us": float(np.median(ar.max(axis=2) - rt.min(axis=2))) / 1e3,
+                 "publish_spread_us": float(np.median(cta[..., 3].max(axis=2) - cta[..., 3].min(axis=2))) / 1e3,
+                 "last_publishers": [int(c) for c in np.argsort(-np.bincount(
+                     cta[..., 3].argmax(axis=2).ravel(), minlength=n_sm))[:6]]}
     with open(path, "w") as f:
         json.dump({"unit": "us since layer start (CTA 0), median over tokens", "tokens": n_tokens,
                    "ns_per_cycle": ns_per_cycle, "raw_slots_us": raw, "cta_stats": cta_stats,

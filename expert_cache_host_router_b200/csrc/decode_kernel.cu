@@ -456,50 +456,51 @@ __device__ __noinline__ int topk_weights(const DecodeParams& p, Misc& m, const f
   return my_e;
 }
 
-// All threads, E <= 256: the top-k of topk_weights (m.sel only) in two parallel steps.
-// (1) Warp w ranks its 32 experts 32w + lane by 64-bit key (logit desc, index asc),
-// reading the warp's keys as shared-memory broadcasts; a rank below k makes a
-// candidate, stored at w k + rank.  (2) A candidate's global rank is the number of
-// larger candidates over the 8 warps' lists (a list with k larger keys puts it out of
-// the top k, as its count shows): 256 / (8k) threads per candidate, rounded down to a
-// power of two, each count some of the lists and add up with shuffles.
-__device__ void topk_select(const DecodeParams& p, Misc& m, const float* zs, unsigned long long* cand) {
-  const int tid = threadIdx.x, warp = tid >> 5, K = p.K;
+// All threads, E <= 256 and k = K (compile time): the top-k of topk_weights (m.sel
+// only) in two parallel steps.  (1) Warp w ranks its 32 experts 32w + lane by 64-bit key
+// (logit desc, index asc), reading the warp's keys as shared-memory broadcasts; a rank
+// below K makes a candidate, stored at w K + rank.  (2) A candidate's global rank is the
+// number of larger candidates over the 8 warps' lists (a list with K larger keys puts it
+// out of the top K, as its count shows): 256 / (8 K) threads per candidate, at most 8,
+// each count some of the lists and add up with shuffles.
+template <int K>
+__device__ __forceinline__ void topk_select(const DecodeParams& p, Misc& m, const float* zs,
+                                            unsigned long long* cand) {
+  static_assert(K >= 1 && K <= 32, "k");
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int e = tid;  // E <= 256 = kThreads
   const unsigned long long key = e < p.E ? route_key(zs[e], e) : 0ull;
   unsigned long long* keys = cand + kWarps * kMaxK;  // [256] after the candidate slots
   keys[e] = key;
-  const int nc = kWarps * K;  // candidate slots
+  constexpr int nc = kWarps * K;  // candidate slots
   for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
   __syncthreads();
   int rank = 0;  // among this warp's 32 keys
   {
     const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + warp * 32);
+    ulonglong2 v[16];
 #pragma unroll
-    for (int q = 0; q < 16; q += 4) {
-      ulonglong2 v[4];
+    for (int u = 0; u < 16; ++u) v[u] = k2[u];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = k2[q + u];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) rank += (v[u].x > key) + (v[u].y > key);
-    }
+    for (int u = 0; u < 16; ++u) rank += (v[u].x > key) + (v[u].y > key);
   }
   if (e < p.E && rank < K) cand[warp * K + rank] = key;
   __syncthreads();
-  int tpc = 1;  // threads per candidate: a power of two, at most 8 (one list each)
-  while (tpc < kWarps && 2 * tpc * nc <= kThreads) tpc <<= 1;
-  const int lpt = kWarps / tpc;  // lists per thread
+  constexpr int tpc = kThreads / nc >= 8 ? 8 : kThreads / nc >= 4 ? 4 : kThreads / nc >= 2 ? 2 : 1;
+  constexpr int lpt = kWarps / tpc;  // lists per thread
   const int ci = tid / tpc, sub = tid % tpc;
-#pragma unroll 1
-  for (int c0 = 0; c0 < nc; c0 += kThreads / tpc) {  // one pass unless k > 16
+#pragma unroll
+  for (int c0 = 0; c0 < nc; c0 += kThreads / tpc) {  // one pass unless K > 16
     const int cc = c0 + ci;
     const unsigned long long c = cc < nc ? cand[cc] : 0ull;
     int r = 0;
-#pragma unroll 1
-    for (int w = sub * lpt; w < (sub + 1) * lpt; ++w) {
-      const unsigned long long* lw = cand + w * K;
+#pragma unroll
+    for (int w = 0; w < lpt; ++w) {
+      const unsigned long long* lw = cand + (sub * lpt + w) * K;
+#pragma unroll
       for (int q = 0; q < K; ++q) r += lw[q] > c;
     }
+#pragma unroll
     for (int off = 1; off < tpc; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
     if (sub == 0 && c != 0ull && r < K) {
       m.sel[r] = (int)(~(uint32_t)c);
@@ -1198,6 +1199,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     stamp(p, l, 12);
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 3);
+    cta_stamp(p, l, 3);
     // this layer's router rows are read: the buffer takes the next layer's
     if (nrx > 0) {
       if (tid == 0 && next) {
@@ -1224,8 +1226,17 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     }
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 4);
+    // top-k: all threads for the common k = 8 over at most 256 experts, else warp 0
+    const bool topk8 = p.E <= kThreads && p.K == 8;
+    if (topk8) topk_select<8>(p, m, zs, cand);
     if (warp == 0) {
-      const int my_e = topk_weights(sp, m, zs);
+      int my_e;
+      if (topk8) {
+        my_e = lane < p.K ? m.sel[lane] : 0;
+        if (my_e < 0 || my_e >= p.E) my_e = 0;
+      } else {
+        my_e = topk_weights(sp, m, zs);
+      }
       stamp(p, l, 13);
       if (lane == 0) m.early = 0;
       const bool fast = cache_pinned_lookup(p, m, pinrow, my_e);
@@ -1247,6 +1258,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
       }
       stamp(p, l, 15);
+      if (topk8) route_weights(p, m, zs, my_e);
       if (fast) cache_pinned_commit(sp, m, l, pinrow, my_e);
       else if (lane == 0) cache_decide(sp, m, l, pinrow);
       if (!(fast && p.n_pre == 0)) {

@@ -257,7 +257,8 @@ MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
  * down adds issued, fence); [L][0] kernel start and [L][2] kernel end in cycles, [L][4]
  * and [L][5] the same two instants on the global timer (ns), which converts cycles to
  * ns; [L][1] prologue done (cycles).  Then [L][n_sm][4] global-timer marks (ns) of every
- * CTA: [0] routing decided, [1] units done, [2] arrival posted, [3] unused.  NULL stops
+ * CTA: [0] routing decided, [1] units done, [2] arrival posted, [3] own logits
+ * published.  NULL stops
  * it (n_words ignored). */
 MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev, size_t n_words);
 
