@@ -474,7 +474,10 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8, residency=1.0, hist=Non
                  "last_arrival_after_first_routed_us": float(np.median(ar.max(axis=2) - rt.min(axis=2))) / 1e3,
                  "publish_spread_us": float(np.median(cta[..., 3].max(axis=2) - cta[..., 3].min(axis=2))) / 1e3,
                  "last_publishers": [int(c) for c in np.argsort(-np.bincount(
-                     cta[..., 3].argmax(axis=2).ravel(), minlength=n_sm))[:6]]}
+                     cta[..., 3].argmax(axis=2).ravel(), minlength=n_sm))[:6]],
+                 "last_to_finish_units": [int(c) for c in np.argsort(-np.bincount(
+                     ud.argmax(axis=2).ravel(), minlength=n_sm))[:6]],
+                 "slowest_units": [int(c) for c in np.argsort(-np.median(work, axis=(0, 1)))[:6]]}
     with open(path, "w") as f:
         json.dump({"unit": "us since layer start (CTA 0), median over tokens", "tokens": n_tokens,
                    "ns_per_cycle": ns_per_cycle, "raw_slots_us": raw, "cta_stats": cta_stats,

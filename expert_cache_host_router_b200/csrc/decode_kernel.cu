@@ -289,6 +289,7 @@ __host__ __device__ inline SmemPlan smem_plan(int H, int E, int rx, int down_lat
 __device__ __noinline__ bool spin_count(const uint32_t* count, uint32_t target, uint64_t timeout_ns, Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
   for (uint32_t polls = 1; ld_acquire(count) < target; ++polls) {
+    __nanosleep(32);
     if ((polls & 15u) == 0) {
       if (has_error(ctrl)) return false;
       if (gtimer() - t0 > timeout_ns) {
@@ -312,6 +313,7 @@ __device__ __noinline__ unsigned long long spin_logit(const unsigned long long* 
   for (uint32_t polls = 1;; ++polls) {
     const unsigned long long v = ld_relaxed_u64(w);
     if ((uint32_t)(v >> 32) == epoch) return v;
+    __nanosleep(32);
     if ((polls & 15u) == 0) {
       if (has_error(ctrl)) return 0ull;
       if (gtimer() - t0 > timeout_ns) {
@@ -456,25 +458,24 @@ __device__ __noinline__ int topk_weights(const DecodeParams& p, Misc& m, const f
   return my_e;
 }
 
-// All threads, E <= 256 and k = K (compile time): the top-k of topk_weights (m.sel
-// only) in two parallel steps.  (1) Warp w ranks its 32 experts 32w + lane by 64-bit key
-// (logit desc, index asc), reading the warp's keys as shared-memory broadcasts; a rank
-// below K makes a candidate, stored at w K + rank.  (2) A candidate's global rank is the
-// number of larger candidates over the 8 warps' lists (a list with K larger keys puts it
-// out of the top K, as its count shows): 256 / (8 K) threads per candidate, at most 8,
-// each count some of the lists and add up with shuffles.
+// The top-k of topk_weights (m.sel only) for E <= 256 and k = K (compile time), in two
+// parallel steps.  (1) topk_rank_warp: warp w ranks its 32 experts 32w + lane by 64-bit
+// key (logit desc, index asc), reading the warp's keys as shared-memory broadcasts; a
+// rank below K makes a candidate, stored at w K + rank.  A warp needs only its own 32
+// logits, so it runs as soon as they are there.  (2) topk_rank_candidates, after a CTA
+// barrier: a candidate's global rank is the number of larger candidates over the 8
+// warps' lists (a list with K larger keys puts it out of the top K, as its count shows):
+// 256 / (8 K) threads per candidate, at most 8, each count some of the lists and add up
+// with shuffles.
 template <int K>
-__device__ __forceinline__ void topk_select(const DecodeParams& p, Misc& m, const float* zs,
-                                            unsigned long long* cand) {
+__device__ __forceinline__ void topk_rank_warp(const DecodeParams& p, unsigned long long key,
+                                               unsigned long long* cand) {
   static_assert(K >= 1 && K <= 32, "k");
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int e = tid;  // E <= 256 = kThreads
-  const unsigned long long key = e < p.E ? route_key(zs[e], e) : 0ull;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned long long* keys = cand + kWarps * kMaxK;  // [256] after the candidate slots
-  keys[e] = key;
-  constexpr int nc = kWarps * K;  // candidate slots
-  for (int t = tid; t < nc; t += kThreads) cand[t] = 0ull;
-  __syncthreads();
+  keys[tid] = key;
+  if (lane < K) cand[warp * K + lane] = 0ull;
+  __syncwarp();
   int rank = 0;  // among this warp's 32 keys
   {
     const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + warp * 32);
@@ -484,8 +485,13 @@ __device__ __forceinline__ void topk_select(const DecodeParams& p, Misc& m, cons
 #pragma unroll
     for (int u = 0; u < 16; ++u) rank += (v[u].x > key) + (v[u].y > key);
   }
-  if (e < p.E && rank < K) cand[warp * K + rank] = key;
-  __syncthreads();
+  if (key != 0ull && rank < K) cand[warp * K + rank] = key;
+}
+
+template <int K>
+__device__ __forceinline__ void topk_rank_candidates(const DecodeParams& p, Misc& m, const unsigned long long* cand) {
+  const int tid = threadIdx.x;
+  constexpr int nc = kWarps * K;  // candidate slots
   constexpr int tpc = kThreads / nc >= 8 ? 8 : kThreads / nc >= 4 ? 4 : kThreads / nc >= 2 ? 2 : 1;
   constexpr int lpt = kWarps / tpc;  // lists per thread
   const int ci = tid / tpc, sub = tid % tpc;
@@ -510,7 +516,7 @@ __device__ __forceinline__ void topk_select(const DecodeParams& p, Misc& m, cons
   __syncthreads();
 }
 
-// Warp 0, after topk_select: the renormalised softmax weights of the selected experts
+// Warp 0, after the top-k: the renormalised softmax weights of the selected experts
 // (lane i: rank i), exactly as topk_weights forms them.
 __device__ __forceinline__ void route_weights(const DecodeParams& p, Misc& m, const float* zs, int my_e) {
   const int lane = threadIdx.x & 31;
@@ -1212,6 +1218,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     }
 
     // ---------------------------------------------------------------- routing
+    // top-k: all threads for the common k = 8 over at most 256 experts (each warp ranks
+    // its 32 experts as soon as their logits are in), else warp 0 after all are read
+    const bool topk8 = p.E <= kThreads && p.K == 8;
     {
       const uint32_t epoch = (uint32_t)(l + 1);
       for (int e = tid; e < p.E; e += kThreads) {
@@ -1223,12 +1232,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
         zs[e] = __uint_as_float((uint32_t)v);
       }
+      if (topk8) topk_rank_warp<8>(p, tid < p.E && ok ? route_key(zs[tid], tid) : 0ull, cand);
     }
     if (!cta_ok(p, ok)) goto fail;
     stamp(p, l, 4);
-    // top-k: all threads for the common k = 8 over at most 256 experts, else warp 0
-    const bool topk8 = p.E <= kThreads && p.K == 8;
-    if (topk8) topk_select<8>(p, m, zs, cand);
+    if (topk8) topk_rank_candidates<8>(p, m, cand);
     if (warp == 0) {
       int my_e;
       if (topk8) {
