@@ -708,7 +708,7 @@ __device__ __noinline__ void cache_pinned_commit(const DecodeParams& p, Misc& m,
 // Thread 0: bulk-load a unit (src = its first byte in a slot) into the unit buffer:
 // four gate/up tiles on bar_u[0..3] and, unless the down part comes later, the down
 // nibbles and scales (one run of 18H bytes) on bar_d.
-__device__ __noinline__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src) {
+__device__ __forceinline__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src) {
   const uint32_t tb = 9u * p.H;
 #pragma unroll
   for (int st = 0; st < 4; ++st) {

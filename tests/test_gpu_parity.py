@@ -103,9 +103,14 @@ def test_full_shape_layer_with_shared_expert():
     synthetic.Shape(2, 64, 9, 1, 32, 0, ring_slots=1, use_rmsnorm=1, zipf_s=0.5),
     synthetic.Shape(1, 4096, 33, 32, 32, 96, ring_slots=4, use_rmsnorm=0, zipf_s=1.0),
     synthetic.Shape(2, 544, 70, 5, 96, 0, ring_slots=3, use_rmsnorm=1, zipf_s=1.0),
+    # the compile-time hidden-size instances (1024 and 3072) with the k = 8 top-k over a
+    # ragged expert count
+    synthetic.Shape(2, 3072, 24, 8, 64, 32, ring_slots=2, use_rmsnorm=1, zipf_s=1.0),
+    synthetic.Shape(2, 1024, 200, 8, 96, 0, ring_slots=4, use_rmsnorm=1, zipf_s=1.0),
 ])
 def test_ragged_shapes(shape):
-    """Shapes that leave partial warps, odd block counts and single-block rows."""
+    """Shapes that leave partial warps, odd block counts and single-block rows, and the
+    kernel instances compiled for a fixed hidden size."""
     layers = make_layers(shape, gain_kind="random")
     orc = oracle.Model(shape, layers)
     m = build_gpu(shape, layers)
