@@ -971,13 +971,46 @@ __global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams 
       }
     return warp_max_key(best);
   };
-  // 1. the k-th largest approximate logit
+  // 1. the k-th largest approximate logit.  Fast path (at most 256 experts, no NaN): its
+  //    value by k rounds of warp max over orderable 32-bit keys, each round taking out
+  //    one instance of the maximum, so equal logits count once each; every expert at or
+  //    above it is a candidate below anyway.  Otherwise k rounds over (logit, index) keys.
   float zk_approx = 0.0f;
-  for (int r = 0; r < K; ++r) {
-    const int e = (int)(~(uint32_t)best_left());
-    zk_approx = za[e];
-    if (lane == 0) flag[e] = 1;
-    __syncwarp();
+  bool nan = false;
+  for (int e = lane; e < E; e += 32) nan |= za[e] != za[e];
+  const bool fast = E <= 256 && !__any_sync(0xffffffffu, nan);
+  if (fast) {
+    uint32_t ord[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int e = lane + 32 * k;
+      ord[k] = e < E ? (uint32_t)(logit_key(za[e], e) >> 32) : 0u;
+    }
+    uint32_t gv = 0;
+    for (int r = 0; r < K; ++r) {
+      uint32_t lv = ord[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k) lv = max(lv, ord[k]);
+      gv = __reduce_max_sync(0xffffffffu, lv);
+      const unsigned holders = __ballot_sync(0xffffffffu, lv == gv);
+      if (lane == __ffs(holders) - 1) {
+        bool done = false;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (!done && ord[k] == gv) {
+            ord[k] = 0u;
+            done = true;
+          }
+      }
+    }
+    zk_approx = __uint_as_float((gv & 0x80000000u) ? (gv & 0x7FFFFFFFu) : ~gv);
+  } else {
+    for (int r = 0; r < K; ++r) {
+      const int e = (int)(~(uint32_t)best_left());
+      zk_approx = za[e];
+      if (lane == 0) flag[e] = 1;
+      __syncwarp();
+    }
   }
   // 2. candidates: the k best approximate logits and every expert within 2 delta below
   //    the k-th.  An expert outside has z~ < z~(k) - 2 delta, so its exact logit is below
@@ -997,9 +1030,29 @@ __global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams 
   __syncwarp();
   canonical_logits(p, l, urow, cand, nc, inv, zx, lane);
   __syncwarp();
-  // 3. top-k of the candidates by exact logit; lane r keeps rank r
+  // 3. top-k of the candidates by exact logit; lane r keeps rank r.  Up to 32 candidates:
+  //    each lane ranks its own against all of them (shuffles); else k rounds of warp max.
   int sel_e = -1;
   float sel_z = 0.0f;
+  if (nc <= 32) {
+    const int ce = lane < nc ? (int)cand[lane] : 0;
+    const uint64_t mk = lane < nc ? logit_key(zx[ce], ce) : 0ull;
+    int rank = 0;
+    for (int i = 0; i < nc; ++i) {
+      const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)mk, i);
+      const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(mk >> 32), i);
+      rank += (((uint64_t)hi << 32) | lo) > mk;
+    }
+    int* rsel = reinterpret_cast<int*>(za);  // the approximate logits are no longer read
+    __syncwarp();
+    if (lane < nc && rank < K) rsel[rank] = ce;
+    __syncwarp();
+    if (lane < K) {
+      sel_e = rsel[lane];
+      sel_z = zx[sel_e];
+    }
+    __syncwarp();
+  } else {
   for (int r = 0; r < K; ++r) {
     uint64_t best = 0;
     for (int i = lane; i < nc; i += 32) {
@@ -1018,6 +1071,7 @@ __global__ void __launch_bounds__(kPT) prefill_route_select(const PrefillParams 
     __syncwarp();
     if (lane == 0) flag[e] = 2;
     __syncwarp();
+  }
   }
   if ((logit_key(__shfl_sync(0xffffffffu, sel_z, 0), 0) >> 32) == 0 && lane == 0)
     atomicCAS(p.s.error, 0, MOE_DEVERR_ROUTE);  // a NaN logit won
