@@ -368,24 +368,29 @@ __device__ __forceinline__ bool cta_ok(const DecodeParams&, bool ok) { return __
 
 // CTA 0's marks are SM clock cycles (clock64: fine-grained, one SM); the kernel's start
 // and end are also taken on the global timer so that cycles convert to ns.
+template <bool ON>
 __device__ __forceinline__ void stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = clock64();
+  if (ON && p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) p.phase_trace[l * 32 + k] = clock64();
 }
 
+template <bool ON>
 __device__ __forceinline__ void stamp_both(const DecodeParams& p, int k_clock, int k_timer) {
-  if (p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) {
+  if (ON && p.phase_trace && blockIdx.x == 0 && threadIdx.x == 0) {
     p.phase_trace[p.L * 32 + k_clock] = clock64();
     p.phase_trace[p.L * 32 + k_timer] = gtimer();
   }
 }
 
 // Per-CTA marks (every CTA, thread 0): after [(L+1)][32] come [L][gridDim][4] stamps.
+template <bool ON>
 __device__ __forceinline__ void cta_stamp(const DecodeParams& p, int l, int k) {
-  if (p.phase_trace && threadIdx.x == 0)
+  if (ON && p.phase_trace && threadIdx.x == 0)
     p.phase_trace[(size_t)(p.L + 1) * 32 + ((size_t)l * gridDim.x + blockIdx.x) * 4 + k] = gtimer();
 }
 
 // ------------------------------------------------------------------ routing
+
+__device__ __forceinline__ void issue_unit(const DecodeParams& p, Misc& m, uint8_t* ubuf, const uint8_t* src);
 
 // Top-k for more than 256 experts: keys re-read from shared memory every round.
 __device__ __noinline__ int topk_large(const DecodeParams& p, const float* zs) {
@@ -488,8 +493,14 @@ __device__ __forceinline__ void topk_rank_warp(const DecodeParams& p, unsigned l
   if (key != 0ull && rank < K) cand[warp * K + rank] = key;
 }
 
+//
+// The thread that places the candidate of rank early_rank (>= 0: the rank whose unit this
+// CTA computes first, known before routing) issues that unit's loads at once when the
+// expert is pinned (unit block early_rb), and sets m.early.
 template <int K>
-__device__ __forceinline__ void topk_rank_candidates(const DecodeParams& p, Misc& m, const unsigned long long* cand) {
+__device__ __forceinline__ void topk_rank_candidates(const DecodeParams& p, Misc& m, const unsigned long long* cand,
+                                                     const int32_t* pinrow, uint8_t* ubuf, int early_rank,
+                                                     int early_rb) {
   const int tid = threadIdx.x;
   constexpr int nc = kWarps * K;  // candidate slots
   constexpr int tpc = kThreads / nc >= 8 ? 8 : kThreads / nc >= 4 ? 4 : kThreads / nc >= 2 ? 2 : 1;
@@ -509,8 +520,17 @@ __device__ __forceinline__ void topk_rank_candidates(const DecodeParams& p, Misc
 #pragma unroll
     for (int off = 1; off < tpc; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
     if (sub == 0 && c != 0ull && r < K) {
-      m.sel[r] = (int)(~(uint32_t)c);
+      const int e = (int)(~(uint32_t)c);
+      m.sel[r] = e;
       if ((c >> 32) == 0ull) set_error(p.ctrl, MOE_DEVERR_ROUTE);  // a NaN logit was needed
+      if (r == early_rank) {
+        const int ps = pinrow[e];
+        if (ps >= 0) {
+          issue_unit(p, m, ubuf,
+                     p.pool + (size_t)(m.base_l + (ps & 0xffff)) * p.slot_bytes + (size_t)early_rb * p.unit_bytes);
+          m.early = 1;
+        }
+      }
     }
   }
   __syncthreads();
@@ -789,7 +809,7 @@ struct UnitRef {
   bool shared, issued;
 };
 
-__device__ __forceinline__ bool unit_of(const DecodeParams& p, const Misc& m, bool pre, int b, int G, int k,
+__device__ __forceinline__ bool unit_of(const DecodeParams& p, int n_pre, const Misc& m, bool pre, int b, int G, int k,
                                         UnitRef& u) {
   const int Ur = p.I / 32, routed = p.K * Ur;
   if (G < p.n_units) {  // fewer CTAs than units: round robin, no preload
@@ -801,7 +821,7 @@ __device__ __forceinline__ bool unit_of(const DecodeParams& p, const Misc& m, bo
     u.issued = k == 0 && pre && u.shared;
     return true;
   }
-  const int npc = p.n_pre * Ur;
+  const int npc = n_pre * Ur;
   if (b >= routed && b < p.n_units) {
     if (k > 0) return false;
     u.shared = true;
@@ -986,9 +1006,12 @@ __device__ __forceinline__ uint32_t pick4(const uint32_t (&a)[4], int i) {
 // BPL: Q4_0 blocks of a gate/up row per lane (ceil(H / 1024), at least 1).  HC: the
 // hidden size when it is 1024 BPL (a lane holds blocks lane + 32 mb exactly; every size
 // and offset below is then a compile-time constant), else 0 (sizes read at run time).
-template <int BPL, int HC>
+template <int BPL, int HC, bool FULL>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ DecodeParams p) {
   static_assert(HC == 0 || HC == 1024 * BPL, "HC is 0 or 1024 BPL");
+  // the speculative loads and the phase marks exist only in the FULL instances: the lean
+  // ones leave their code out of the per-layer instruction stream
+  const int n_pre = FULL ? p.n_pre : 0, n_l2 = FULL ? p.n_l2 : 0;
   extern __shared__ __align__(128) uint8_t smem[];
   const int H = HC ? HC : p.H;
   const SmemPlan S = smem_plan(H, p.E, p.rx_per_cta, p.down_late);
@@ -1018,7 +1041,18 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
   const int nrx = b < p.E ? min(p.rx_per_cta, (p.E - b + G - 1) / G) : 0;  // my router experts b, b+G, ...
   const bool first_shared = b < p.n_units && b >= routed;  // my first unit does not depend on routing
   const int Ur = p.I / 32;
-  const int npc = p.n_pre * Ur;  // CTAs that preload a likely expert's unit
+  const int npc = n_pre * Ur;  // CTAs that preload a likely expert's unit
+  // with no preloads and a CTA per unit, the routed unit j this CTA computes is fixed
+  // before routing (the idle CTAs take units 0.., then CTA b < routed unit idle + b):
+  // rank j / Ur, block j % Ur; its loads go out as soon as that rank's expert is known
+  int early_rank = -1, early_rb = 0;
+  if (n_pre == 0 && G >= p.n_units) {
+    const int j = b >= p.n_units ? b - p.n_units : b < routed ? (G - p.n_units) + b : -1;
+    if (j >= 0 && j < routed) {
+      early_rank = j / Ur;
+      early_rb = j % Ur;
+    }
+  }
   // a unit was issued ahead for the current layer (the shared expert's, or a preload);
   // every thread keeps the same value
   bool pre = first_shared;
@@ -1037,7 +1071,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     m.n_miss = 0;
     m.n_fix = 0;
   }
-  stamp_both(p, 0, 4);
+  stamp_both<FULL>(p, 0, 4);
   if (!cta_ok(p, true)) goto fail;
 
   // ---- prologue: accumulators 0 and 1 and the logit words zeroed, h = x, first loads
@@ -1061,7 +1095,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     }
   }
   int32_t lk[kMaxLikely];  // thread 32: the likely experts' slots of the current layer
-  if (tid == 32 && p.n_l2 > 0) {
+  if (tid == 32 && n_l2 > 0) {
     load_likely(sp, 0, lk);
     prefetch_likely(sp, lk);
   }
@@ -1073,10 +1107,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     ok = wait_count(p, &p.ctrl->bar_count, gbase + G);
   }
   if (!cta_ok(p, ok)) goto fail;
-  stamp(p, p.L, 1);
+  stamp<FULL>(p, p.L, 1);
 
   for (int l = 0; l < p.L; ++l) {
-    stamp(p, l, 0);
+    stamp<FULL>(p, l, 0);
     const bool next = l + 1 < p.L;
     // ---------------------------------------------------------------- layer inputs
     // loads that do not depend on the previous layer go out first
@@ -1094,9 +1128,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       if (tid == kThreads - 1) m.ring_clock = __ldcg(p.ring_clock + (size_t)par * p.L + l);
       if (tid == kThreads - 2) m.P_l = __ldg(p.n_pinned + l);
       if (tid == kThreads - 3) m.base_l = __ldg(p.layer_base + l);
+      if (tid == kThreads - 4) m.early = 0;
       if (tid < nrx) m.bias[tid] = p.bias ? __ldg(p.bias + (size_t)l * p.E + b + tid * G) : 0.0f;
-      if (tid == 32 && p.n_l2 > 0 && l > 0) load_likely(sp, l, lk);
-      if (tid < p.n_pre) m.lk_e[tid] = __ldg(p.likely_e + (size_t)l * kMaxLikely + tid);
+      if (tid == 32 && n_l2 > 0 && l > 0) load_likely(sp, l, lk);
+      if (tid < n_pre) m.lk_e[tid] = __ldg(p.likely_e + (size_t)l * kMaxLikely + tid);
       pre_slot = (l > 0 && b < npc) ? __ldg(p.likely_slot + (size_t)l * kMaxLikely + b / Ur) : -1;
     }
     if (l > 0) {
@@ -1110,11 +1145,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       if (pre_slot >= 0) pre = true;
       // the HBM is idle until this layer's routing is known: fetch its likely experts
       // (a thread off the critical path, after the wait)
-      if (tid == 32 && p.n_l2 > 0) {
+      if (tid == 32 && n_l2 > 0) {
         if (wait_count(p, &p.ctrl->bar_count, gbase + (uint32_t)(l + 1) * G)) prefetch_likely(sp, lk);
       }
       if (!cta_ok(p, ok)) goto fail;
-      stamp(p, l, 1);
+      stamp<FULL>(p, l, 1);
       add_layer_output(p, H, p.acc + (size_t)((l - 1) % kAccBufs) * H, hs,
                        (b == 0 && p.h_trace) ? p.h_trace + (size_t)l * H : nullptr);
       // deferred ring fills of layer l - 1 (a layer that missed more often than it has
@@ -1128,7 +1163,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       }
     }
     __syncthreads();
-    stamp(p, l, 2);
+    stamp<FULL>(p, l, 2);
 
     // ---------------------------------------------------------------- norm and router
     // chunk partials of the norm and of my router rows (this layer's rows landed during
@@ -1139,7 +1174,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     // inv = 1 / sqrt(ss / H + eps), folded by every warp (the same bits everywhere)
     const float inv =
         p.use_norm ? __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(fold_chunks(pcs, nch), (float)H), p.eps))) : 1.0f;
-    stamp(p, l, 10);
+    stamp<FULL>(p, l, 10);
     // logits of my experts: warp k folds expert b + k G
     if (warp < nrx) {
       const float S_e = fold_chunks(pcs + (size_t)(1 + warp) * nch, nch);
@@ -1147,7 +1182,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         const int e = b + warp * G;
         const float z = fmaf(S_e, inv, m.bias[warp]);
         st_relaxed_u64(p.zll + e, ((unsigned long long)(uint32_t)(l + 1) << 32) | __float_as_uint(z));
-        if (warp == 0) stamp(p, l, 11);
+        if (warp == 0) stamp<FULL>(p, l, 11);
       }
     }
     // quantised expert input x = RMSNorm(h) (or h): four lanes per 32-block, each lane 8
@@ -1202,10 +1237,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
       }
     }
-    stamp(p, l, 12);
+    stamp<FULL>(p, l, 12);
     if (!cta_ok(p, ok)) goto fail;
-    stamp(p, l, 3);
-    cta_stamp(p, l, 3);
+    stamp<FULL>(p, l, 3);
+    cta_stamp<FULL>(p, l, 3);
     // this layer's router rows are read: the buffer takes the next layer's
     if (nrx > 0) {
       if (tid == 0 && next) {
@@ -1235,8 +1270,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       if (topk8) topk_rank_warp<8>(p, tid < p.E && ok ? route_key(zs[tid], tid) : 0ull, cand);
     }
     if (!cta_ok(p, ok)) goto fail;
-    stamp(p, l, 4);
-    if (topk8) topk_rank_candidates<8>(p, m, cand);
+    stamp<FULL>(p, l, 4);
+    if (topk8) topk_rank_candidates<8>(p, m, cand, pinrow, ubuf, early_rank, early_rb);
     if (warp == 0) {
       int my_e;
       if (topk8) {
@@ -1245,10 +1280,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       } else {
         my_e = topk_weights(sp, m, zs);
       }
-      stamp(p, l, 13);
-      if (lane == 0) m.early = 0;
+      stamp<FULL>(p, l, 13);
       const bool fast = cache_pinned_lookup(p, m, pinrow, my_e);
-      if (fast && p.n_pre == 0) {
+      if (fast && n_pre == 0) {
         // no preloads: every rank is uncovered, and one unit per CTA is known now; its
         // loads go out before the rest of the bookkeeping
         if (lane < p.K) m.unc[lane] = lane;
@@ -1257,23 +1291,23 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           m.n_avail = routed + max(G - p.n_units, 0);
         }
         __syncwarp();
-        if (lane == 0 && G >= p.n_units) {
+        if (lane == 0 && G >= p.n_units && !m.early) {
           UnitRef ur;
-          if (unit_of(p, m, pre, b, G, 0, ur) && !ur.issued && !ur.shared) {
+          if (unit_of(p, n_pre, m, pre, b, G, 0, ur) && !ur.issued && !ur.shared) {
             issue_unit(sp, m, ubuf, m.src[ur.i] + (size_t)ur.rb * p.unit_bytes);
             m.early = 1;
           }
         }
       }
-      stamp(p, l, 15);
+      stamp<FULL>(p, l, 15);
       if (topk8) route_weights(p, m, zs, my_e);
       if (fast) cache_pinned_commit(sp, m, l, pinrow, my_e);
       else if (lane == 0) cache_decide(sp, m, l, pinrow);
-      if (!(fast && p.n_pre == 0)) {
+      if (!(fast && n_pre == 0)) {
         if (lane == 0) {  // preload matching: which group holds which rank, which ranks are left
           uint32_t covered = 0;
           int wrong = 0;
-          for (int q = 0; q < p.n_pre; ++q) {
+          for (int q = 0; q < n_pre; ++q) {
             int r = -1;
             for (int i = 0; i < p.K; ++i)
               if (m.sel[i] == m.lk_e[q]) r = i;
@@ -1289,12 +1323,12 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
       }
       __syncwarp();
-      stamp(p, l, 14);
+      stamp<FULL>(p, l, 14);
     }
     __syncthreads();
     if (b == 0 && p.w_trace && tid < p.K) p.w_trace[(size_t)l * p.K + tid] = m.w[tid];
-    stamp(p, l, 5);
-    cta_stamp(p, l, 0);
+    stamp<FULL>(p, l, 5);
+    cta_stamp<FULL>(p, l, 0);
 
     // ---------------------------------------------------------------- units
     {
@@ -1325,7 +1359,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       unsigned long long* acc_l = p.acc + (size_t)(l % kAccBufs) * H;
       const bool early = m.early != 0;
       UnitRef ur;
-      for (int k = 0; unit_of(p, m, pre, b, G, k, ur); ++k) {
+      for (int k = 0; unit_of(p, n_pre, m, pre, b, G, k, ur); ++k) {
         const bool shared = ur.shared;
         const int i = ur.i, rb = ur.rb;
         const float wi = shared ? 1.0f : m.w[i];
@@ -1347,7 +1381,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           }
           if (!cta_ok(p, ok)) goto fail;
         }
-        stamp(p, l, 6);
+        stamp<FULL>(p, l, 6);
         // gate/up: rows r = gate 0..31, up 0..31 of the unit, tile r / 16; warp w takes rows
         // w + 8 j (j = 0..7: tile j / 2, row w + 8 (j % 2) of it)
         if constexpr (HC != 0) {
@@ -1425,7 +1459,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           }
         }
         if (!cta_ok(p, ok)) goto fail;
-        stamp(p, l, 7);
+        stamp<FULL>(p, l, 7);
         // a = silu(g) * u, quantised as one int16 block
         if (warp == 0) {
           const float gv = m.gu[lane], uv = m.gu[kUnitRows + lane];
@@ -1437,7 +1471,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           if (lane == 0) {
             m.asc = sc;
             m.acs = csum;
-            stamp(p, l, 16);
+            stamp<FULL>(p, l, 16);
           }
         }
         __syncthreads();  // codes ready; the gate/up tiles are no longer read
@@ -1447,7 +1481,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           bulk_g2s_stream(ubuf, usrc + 36u * H, 18u * H, &m.bar_d);
         }
         if (!mbar_wait(p, &m.bar_d, par_d)) ok = false;
-        stamp(p, l, 17);
+        stamp<FULL>(p, l, 17);
         if (ok) {
           // down: output row j against the unit's activation block; the weighted share
           // w_i * d_j * scale * dot goes into the accumulator as round(v * 2^28)
@@ -1471,8 +1505,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
             red_add_u64(acc_l + j, (unsigned long long)qf);
           }
           if (!range_ok) set_error(p.ctrl, MOE_DEVERR_RANGE);
-          stamp(p, l, 18);
-          stamp(p, l, 19);
+          stamp<FULL>(p, l, 18);
+          stamp<FULL>(p, l, 19);
         }
         if (!cta_ok(p, ok)) goto fail;
 #pragma unroll
@@ -1486,8 +1520,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       if (!cta_ok(p, ok)) goto fail;
       pre = false;
     }
-    stamp(p, l, 8);
-    cta_stamp(p, l, 1);
+    stamp<FULL>(p, l, 8);
+    cta_stamp<FULL>(p, l, 1);
     // the next layer's shared-expert unit does not depend on routing, and a likely
     // expert's unit is worth guessing: load them now
     if (next && first_shared) {
@@ -1498,8 +1532,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     }
     __syncthreads();
     if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
-    stamp(p, l, 9);
-    cta_stamp(p, l, 2);
+    stamp<FULL>(p, l, 9);
+    cta_stamp<FULL>(p, l, 2);
   }
 
   // ---- the last layer's output
@@ -1513,7 +1547,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
       for (int j = tid; j < H; j += kThreads) p.h_trace[(size_t)p.L * H + j] = hs[j];
     if (m.n_fix > 0) ring_fills(sp, m);
   }
-  stamp_both(p, 2, 5);
+  stamp_both<FULL>(p, 2, 5);
   if (b == 0 && tid == 0) {
     p.ctrl->step = m.step + 1;
     p.ctrl->req_seq = m.seq_base + m.n_miss;
@@ -1536,20 +1570,29 @@ static int bpl_of(int H) {
   return nb <= 32 ? 1 : (nb + 31) / 32;
 }
 
+// The instance for hidden size H: compile-time sizes where there is one; the lean
+// instance (no phase marks, no speculative loads) unless full is asked for.
 template <typename F>
-static cudaError_t with_kernel(int H, F f) {
-  switch (H) {  // the hidden sizes with a compile-time instance
-    case 1024: return f(moe_decode_kernel<1, 1024>);
-    case 2048: return f(moe_decode_kernel<2, 2048>);
-    case 3072: return f(moe_decode_kernel<3, 3072>);
-    case 4096: return f(moe_decode_kernel<4, 4096>);
+static cudaError_t with_kernel(int H, bool full, F f) {
+  if (!full) switch (H) {
+      case 1024: return f(moe_decode_kernel<1, 1024, false>);
+      case 2048: return f(moe_decode_kernel<2, 2048, false>);
+      case 3072: return f(moe_decode_kernel<3, 3072, false>);
+      case 4096: return f(moe_decode_kernel<4, 4096, false>);
+      default: break;
+    }
+  switch (H) {
+    case 1024: return f(moe_decode_kernel<1, 1024, true>);
+    case 2048: return f(moe_decode_kernel<2, 2048, true>);
+    case 3072: return f(moe_decode_kernel<3, 3072, true>);
+    case 4096: return f(moe_decode_kernel<4, 4096, true>);
     default: break;
   }
   switch (bpl_of(H)) {
-    case 1: return f(moe_decode_kernel<1, 0>);
-    case 2: return f(moe_decode_kernel<2, 0>);
-    case 3: return f(moe_decode_kernel<3, 0>);
-    default: return f(moe_decode_kernel<4, 0>);
+    case 1: return f(moe_decode_kernel<1, 0, true>);
+    case 2: return f(moe_decode_kernel<2, 0, true>);
+    case 3: return f(moe_decode_kernel<3, 0, true>);
+    default: return f(moe_decode_kernel<4, 0, true>);
   }
 }
 
@@ -1577,19 +1620,13 @@ bool decode_plan(int H, int E, int grid, int smem_optin, int* rx, int* down_late
 cudaError_t decode_configure(int limit) {
   cudaError_t e = cudaSuccess;
   auto set = [&](auto kern) { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, limit); };
-  if (e == cudaSuccess) e = set(moe_decode_kernel<1, 0>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<2, 0>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<3, 0>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<4, 0>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<1, 1024>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<2, 2048>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<3, 3072>);
-  if (e == cudaSuccess) e = set(moe_decode_kernel<4, 4096>);
+  for (int H : {1024, 2048, 3072, 4096, 32, 1056, 2080, 3104})  // every instance
+    for (int full = 0; full < 2 && e == cudaSuccess; ++full) e = with_kernel(H, full != 0, set);
   return e;
 }
 
 cudaError_t decode_max_blocks_per_sm(int H, uint32_t smem, int* out) {
-  return with_kernel(H, [&](auto kern) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, smem); });
+  return with_kernel(H, true, [&](auto kern) { return cudaOccupancyMaxActiveBlocksPerMultiprocessor(out, kern, kThreads, smem); });
 }
 
 cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) {
@@ -1603,7 +1640,8 @@ cudaError_t decode_launch(const DecodeParams& p, int grid, cudaStream_t stream) 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return with_kernel(p.H, [&](auto kern) { return cudaLaunchKernelEx(&cfg, kern, p); });
+  const bool full = p.phase_trace != nullptr || p.n_pre > 0 || p.n_l2 > 0;
+  return with_kernel(p.H, full, [&](auto kern) { return cudaLaunchKernelEx(&cfg, kern, p); });
 }
 
 }  // namespace moe
