@@ -230,9 +230,6 @@ struct Misc {
   uint32_t ring_stamp[kMaxR];
   uint32_t ring_clock;
   float gu[2 * kUnitRows];
-  int4 acodes[4];  // the unit's activation block: 32 int16 codes in pairs
-  float asc;
-  int32_t acs;
   float inv;
   float bias[kWarps];  // router bias of this CTA's experts, current layer
   uint32_t step, seq_base, n_miss;
@@ -1460,21 +1457,30 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
         if (!cta_ok(p, ok)) goto fail;
         stamp<FULL>(p, l, 7);
-        // a = silu(g) * u, quantised as one int16 block
-        if (warp == 0) {
+        // a = silu(g) * u, quantised as one int16 block: every warp forms it (the same
+        // bits in each) and holds the 32 codes in pairs in registers, so the down rows
+        // start without another CTA barrier
+        int4 a0, a1, a2, a3;
+        float asc;
+        int cs128;
+        {
           const float gv = m.gu[lane], uv = m.gu[kUnitRows + lane];
           const float a = __fdividef(gv, 1.0f + __expf(-gv)) * uv;
-          float sc;
           int csum;
-          const int code = quant_block(a, sc, csum);
-          reinterpret_cast<int16_t*>(m.acodes)[lane] = (int16_t)code;
-          if (lane == 0) {
-            m.asc = sc;
-            m.acs = csum;
-            stamp<FULL>(p, l, 16);
-          }
+          const int code = quant_block(a, asc, csum);
+          cs128 = 128 * csum;
+          // pair q = codes 2q (low half) and 2q + 1 (high half)
+          const int nxt = __shfl_down_sync(0xffffffffu, code, 1);
+          const int pk = (int)(((uint32_t)code & 0xffffu) | ((uint32_t)nxt << 16));
+          int pr[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) pr[q] = __shfl_sync(0xffffffffu, pk, 2 * q);
+          a0 = make_int4(pr[0], pr[1], pr[2], pr[3]);
+          a1 = make_int4(pr[4], pr[5], pr[6], pr[7]);
+          a2 = make_int4(pr[8], pr[9], pr[10], pr[11]);
+          a3 = make_int4(pr[12], pr[13], pr[14], pr[15]);
+          if (warp == 0 && lane == 0) stamp<FULL>(p, l, 16);
         }
-        __syncthreads();  // codes ready; the gate/up tiles are no longer read
         const uint8_t* dn = ubuf + (p.down_late ? 0u : 36u * H);
         if (p.down_late && tid == 0) {
           mbar_expect_tx(&m.bar_d, 18u * H);
@@ -1485,9 +1491,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         if (ok) {
           // down: output row j against the unit's activation block; the weighted share
           // w_i * d_j * scale * dot goes into the accumulator as round(v * 2^28)
-          const int4 a0 = m.acodes[0], a1 = m.acodes[1], a2 = m.acodes[2], a3 = m.acodes[3];
-          const float asc = m.asc;
-          const int cs128 = 128 * m.acs;
           const __half* dsc = reinterpret_cast<const __half*>(dn + 16u * H);
           bool range_ok = true;
 #pragma unroll 4
@@ -1530,7 +1533,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
                    p.shared_pool + (size_t)(l + 1) * p.shared_slot_bytes + (size_t)(b - routed) * p.unit_bytes);
       pre = true;
     }
-    __syncthreads();
+    // arrival: the CTA barrier that ended the unit ordered every thread's adds before
+    // this release (a CTA without a unit added nothing)
     if (tid == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&p.ctrl->bar_count) : "memory");
     stamp<FULL>(p, l, 9);
     cta_stamp<FULL>(p, l, 2);
