@@ -35,7 +35,7 @@ FALLBACK_TFLOPS = 1400.0  # sustained dense bf16, an earlier measurement on this
 # DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
 # 4-layer case scaled by 10, valid only for the kernel source it was taken on; any other
 # source reports null.
-TRAFFIC_REF = {"kernel_sha256_prefix": "0977b6aaaebe20c2", "bytes_per_launch": 691.110016e6}
+TRAFFIC_REF = {"kernel_sha256_prefix": "26c2226b2d10beed", "bytes_per_launch": 690.56512e6}
 WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
             "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
             "residency + 8-slot LRU ring (residency_60)")
@@ -477,7 +477,13 @@ def write_phase_table(m, shape, xs, y, path, n_tokens=8, residency=1.0, hist=Non
                      cta[..., 3].argmax(axis=2).ravel(), minlength=n_sm))[:6]],
                  "last_to_finish_units": [int(c) for c in np.argsort(-np.bincount(
                      ud.argmax(axis=2).ravel(), minlength=n_sm))[:6]],
-                 "slowest_units": [int(c) for c in np.argsort(-np.median(work, axis=(0, 1)))[:6]]}
+                 "slowest_units": [int(c) for c in np.argsort(-np.median(work, axis=(0, 1)))[:6]],
+                 # per CTA, median over tokens and layers: how long after the first CTA it
+                 # published its logits / posted its arrival
+                 "publish_late_us": [round(float(v) / 1e3, 3) for v in np.median(
+                     cta[..., 3] - cta[..., 3].min(axis=2, keepdims=True), axis=(0, 1))],
+                 "arrival_late_us": [round(float(v) / 1e3, 3) for v in np.median(
+                     ar - ar.min(axis=2, keepdims=True), axis=(0, 1))]}
     with open(path, "w") as f:
         json.dump({"unit": "us since layer start (CTA 0), median over tokens", "tokens": n_tokens,
                    "ns_per_cycle": ns_per_cycle, "raw_slots_us": raw, "cta_stats": cta_stats,
