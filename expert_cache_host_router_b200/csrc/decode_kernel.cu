@@ -943,7 +943,34 @@ __device__ __forceinline__ void head_pass(const DecodeParams& p, int H, const un
 #pragma unroll
         for (int i = 0; i < 8; ++i) u[i] = h[i];
       }
-      for (int k = 0; k < nrx; ++k) {
+      // rows two at a time (their chains are independent and interleave), then a last one
+      int k = 0;
+      for (; k + 1 < nrx; k += 2) {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(rrows + (size_t)k * H + 8 * qq);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(rrows + (size_t)(k + 1) * H + 8 * qq);
+        const float f0[8] = {bf16_lo(w0.x), bf16_hi(w0.x), bf16_lo(w0.y), bf16_hi(w0.y),
+                             bf16_lo(w0.z), bf16_hi(w0.z), bf16_lo(w0.w), bf16_hi(w0.w)};
+        const float f1[8] = {bf16_lo(w1.x), bf16_hi(w1.x), bf16_lo(w1.y), bf16_hi(w1.y),
+                             bf16_lo(w1.z), bf16_hi(w1.z), bf16_lo(w1.w), bf16_hi(w1.w)};
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          s0 = fmaf(f0[i], u[i], s0);
+          s1 = fmaf(f1[i], u[i], s1);
+        }
+        float t0 = __shfl_up_sync(0xffffffffu, s0, 1);
+        float t1 = __shfl_up_sync(0xffffffffu, s1, 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          t0 = fmaf(f0[i], u[i], t0);
+          t1 = fmaf(f1[i], u[i], t1);
+        }
+        if (live && odd) {
+          pc[(1 + k) * nch + (q >> 1)] = t0;
+          pc[(2 + k) * nch + (q >> 1)] = t1;
+        }
+      }
+      if (k < nrx) {
         const uint4 w = *reinterpret_cast<const uint4*>(rrows + (size_t)k * H + 8 * qq);
         const float wf[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
                              bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
@@ -1382,9 +1409,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         // gate/up: rows r = gate 0..31, up 0..31 of the unit, tile r / 16; warp w takes rows
         // w + 8 j (j = 0..7: tile j / 2, row w + 8 (j % 2) of it)
         if constexpr (HC != 0) {
-          // lane l holds blocks l + 32 mb; four rows (two tiles) per pass
+          // lane l holds blocks l + 32 mb; four rows (two tiles) per pass, one butterfly
+          // for all eight rows at the end
           constexpr int NB = HC / 32;
-#pragma unroll 1
+          float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
           for (int j0 = 0; j0 < 8; j0 += 4) {
             bool w_ok = ok;
             w_ok = w_ok && mbar_wait(p, &m.bar_u[j0 / 2], pick4(par_u, j0 / 2));
@@ -1393,7 +1422,6 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
               ok = false;
               break;
             }
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int j = j0 + q;
@@ -1407,16 +1435,18 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
                 const uint4 qv = *reinterpret_cast<const uint4*>(nib + bb * 16);
                 const float d = __half2float(dsc[bb]);
                 const int v = q4_block_dot16(qv, xq[mb][0], xq[mb][1], xq[mb][2], xq[mb][3]) - 128 * xsum[mb];
-                acc[q] = fmaf(d * xsc[mb], (float)v, acc[q]);
+                acc[j] = fmaf(d * xsc[mb], (float)v, acc[j]);
               }
             }
+          }
+          if (ok) {
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1)
 #pragma unroll
-              for (int q = 0; q < 4; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
+              for (int q = 0; q < 8; ++q) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], off);
             if (lane == 0)
 #pragma unroll
-              for (int q = 0; q < 4; ++q) m.gu[warp + 8 * (j0 + q)] = acc[q];
+              for (int q = 0; q < 8; ++q) m.gu[warp + 8 * q] = acc[q];
           }
         } else {
           for (int rw = warp * RPW; rw < 2 * kUnitRows; rw += 2 * rstep) {  // warp-uniform
