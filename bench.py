@@ -5,7 +5,8 @@ Workload (one "step" = one batch-1 decode token through the whole hot path): a 4
 pre-norm MoE stack, hidden 2048, 256 experts, top-8, SwiGLU 512 plus a 512-wide shared
 expert, GGUF Q4_0 expert weights, Zipf(1.0)-biased router over seeded per-layer
 permutations, tokens x ~ N(0, 1).  Timed at 100% expert residency (the value) and at
-60% residency with the hot set pinned from a 128-token calibration histogram plus an
+60% residency with the hot set pinned from a calibration histogram (2048 tokens of a
+separate stream, the length of the prefill prompt; --calib-steps) plus an
 8-slot LRU ring per layer, cold experts in pinned host memory (Luce Spark write-up,
 theneuralfeed.com, key components), and with a uniform 60% placement for contrast.
 
@@ -35,7 +36,7 @@ FALLBACK_TFLOPS = 1400.0  # sustained dense bf16, an earlier measurement on this
 # DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
 # 4-layer case scaled by 10, valid only for the kernel source it was taken on; any other
 # source reports null.
-TRAFFIC_REF = {"kernel_sha256_prefix": "26c2226b2d10beed", "bytes_per_launch": 690.56512e6}
+TRAFFIC_REF = {"kernel_sha256_prefix": "0c94bdf6be6b0f76", "bytes_per_launch": 691.86304e6}
 WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
             "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
             "residency + 8-slot LRU ring (residency_60)")
@@ -208,16 +209,17 @@ def run_drift(args, shape, layers, local, dev, xs_steps=1024, switch=512, every=
         m.load_layer(l, layers[l])
     new_bias = [synthetic.zipf_bias(l, s.n_experts, s.zipf_s, synthetic.SEED_RESHUFFLE)
                 for l in range(s.n_layers)]
-    calib = torch.from_numpy(synthetic.tokens(0, args.calib_steps, s.hidden, synthetic.SEED_CALIB)).to(dev)
+    n_cal = args.drift_calib_steps
+    calib = torch.from_numpy(synthetic.tokens(0, n_cal, s.hidden, synthetic.SEED_CALIB)).to(dev)
     xs = torch.from_numpy(synthetic.tokens(0, xs_steps, s.hidden)).to(dev)
     y = torch.empty(s.hidden, dtype=torch.float32, device=dev)
     m.set_residency(1.0)
-    for i in range(args.calib_steps):
+    for i in range(n_cal):
         m.decode(calib[i], y)
     m.sync()
-    _, hist, _ = m.stats(reset=True, log_cap=args.calib_steps * s.n_layers * s.top_k)
+    _, hist, _ = m.stats(reset=True, log_cap=n_cal * s.n_layers * s.top_k)
     out = {"residency": fraction, "ring_slots": ring, "steps": xs_steps, "reshuffle_at": switch,
-           "recalibrate_every": every}
+           "recalibrate_every": every, "calibration_tokens": n_cal}
     stream = torch.cuda.current_stream(dev)
     for name, place, recal in (("calibrated_recal", moe.MOE_PLACE_CALIBRATED, True),
                                ("calibrated_static", moe.MOE_PLACE_CALIBRATED, False),
@@ -538,7 +540,7 @@ def run_ours(args):
     xs = torch.from_numpy(synthetic.tokens(0, n_tok, shape.hidden)).to(dev)
     y = torch.empty(shape.hidden, dtype=torch.float32, device=dev)
 
-    # calibration histogram: 128 tokens of a separate stream at full residency
+    # calibration histogram: --calib-steps tokens of a separate stream at full residency
     m.set_residency(1.0)
     calib = torch.from_numpy(synthetic.tokens(0, args.calib_steps, shape.hidden, synthetic.SEED_CALIB)).to(dev)
     for i in range(args.calib_steps):
@@ -717,7 +719,10 @@ def main():
     ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--calib-steps", type=int, default=128)
+    ap.add_argument("--calib-steps", type=int, default=2048,
+                    help="tokens of the calibration stream whose routing histogram picks the pinned set")
+    ap.add_argument("--drift-calib-steps", type=int, default=128,
+                    help="calibration tokens of the drift run (before its recalibrations take over)")
     ap.add_argument("--cpu-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=40, help="stack depth (40 = the benchmark workload)")
