@@ -302,25 +302,6 @@ __device__ __forceinline__ bool wait_count(const DecodeParams& p, const uint32_t
   return ld_acquire(count) >= target || spin_count(count, target, p.timeout_ns, p.ctrl);
 }
 
-// Spin until the published logit word carries epoch (>= 1) and return it; 0 on timeout
-// / error (a published word is never 0).
-__device__ __noinline__ unsigned long long spin_logit(const unsigned long long* w, uint32_t epoch, uint64_t timeout_ns,
-                                                      Ctrl* ctrl) {
-  const uint64_t t0 = gtimer();
-  for (uint32_t polls = 1;; ++polls) {
-    const unsigned long long v = ld_relaxed_u64(w);
-    if ((uint32_t)(v >> 32) == epoch) return v;
-    __nanosleep(32);
-    if ((polls & 15u) == 0) {
-      if (has_error(ctrl)) return 0ull;
-      if (gtimer() - t0 > timeout_ns) {
-        set_error(ctrl, MOE_DEVERR_BARRIER);
-        return 0ull;
-      }
-    }
-  }
-}
-
 // Thread 0: wait until the proxy has signalled miss copy seq (0: nothing to wait for).
 __device__ __noinline__ bool spin_miss(const uint32_t* done_seq, uint32_t seq, uint64_t timeout_ns, Ctrl* ctrl) {
   const uint64_t t0 = gtimer();
@@ -1281,15 +1262,43 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     // its 32 experts as soon as their logits are in), else warp 0 after all are read
     const bool topk8 = p.E <= kThreads && p.K == 8;
     {
+      // a warp polls its 32 words together: one coalesced load per round for the lanes
+      // still missing (per-lane spins would send one request per lane to the few L2
+      // lines that every CTA polls)
       const uint32_t epoch = (uint32_t)(l + 1);
-      for (int e = tid; e < p.E; e += kThreads) {
-        unsigned long long v = ld_relaxed_u64(p.zll + e);
-        if ((uint32_t)(v >> 32) != epoch) v = spin_logit(p.zll + e, epoch, p.timeout_ns, p.ctrl);
-        if (v == 0ull) {
+      for (int e0 = tid & ~31; e0 < p.E; e0 += kThreads) {  // warp-uniform
+        const int e = e0 + lane;
+        const bool mine = e < p.E;
+        unsigned long long v = mine ? ld_relaxed_u64(p.zll + e) : 0ull;
+        bool have = !mine || (uint32_t)(v >> 32) == epoch;
+        if (!__all_sync(0xffffffffu, have)) {
+          const uint64_t t0 = gtimer();
+          for (uint32_t polls = 1;; ++polls) {
+            __nanosleep(32);
+            if (!have) {
+              v = ld_relaxed_u64(p.zll + e);
+              have = (uint32_t)(v >> 32) == epoch;
+            }
+            if (__all_sync(0xffffffffu, have)) break;
+            if ((polls & 15u) == 0) {  // lane 0 decides for the warp
+              int stop = 0;
+              if (lane == 0) {
+                if (has_error(p.ctrl)) {
+                  stop = 1;
+                } else if (gtimer() - t0 > p.timeout_ns) {
+                  set_error(p.ctrl, MOE_DEVERR_BARRIER);
+                  stop = 1;
+                }
+              }
+              if (__shfl_sync(0xffffffffu, stop, 0)) break;
+            }
+          }
+        }
+        if (!__all_sync(0xffffffffu, have)) {
           ok = false;
           break;
         }
-        zs[e] = __uint_as_float((uint32_t)v);
+        if (mine) zs[e] = __uint_as_float((uint32_t)v);
       }
       if (topk8) topk_rank_warp<8>(p, tid < p.E && ok ? route_key(zs[tid], tid) : 0ull, cand);
     }
