@@ -36,7 +36,7 @@ FALLBACK_TFLOPS = 1400.0  # sustained dense bf16, an earlier measurement on this
 # DRAM bytes (read + write) of one 40-layer decode launch, from the ncu capture of the
 # 4-layer case scaled by 10, valid only for the kernel source it was taken on; any other
 # source reports null.
-TRAFFIC_REF = {"kernel_sha256_prefix": "0c94bdf6be6b0f76", "bytes_per_launch": 691.86304e6}
+TRAFFIC_REF = {"kernel_sha256_prefix": "c2b549be9b6e7e69", "bytes_per_launch": 689.78176e6}
 WORKLOAD = ("40-layer MoE decode stack, hidden 2048, 256 experts top-8, SwiGLU 512 + shared 512, "
             "Q4_0, Zipf router; batch-1 tokens; 100% residency (value) and 60% calibrated "
             "residency + 8-slot LRU ring (residency_60)")
