@@ -253,13 +253,14 @@ MOE_API int moe_set_trace(moe_ctx *ctx, float *h_trace_dev, float *w_trace_dev);
  * output complete, [2] h updated, [3] own logits published and input quantised, [4] all
  * logits read, [5] routing and cache decided, [6] unit loads issued, [7] gate/up
  * computed, [8] units done, [9] arrival posted, [10..19] finer marks (norm, own logit,
- * input quantised, top-k, cache, loads issued by thread 0, SwiGLU, down part landed,
- * down adds issued, fence); [L][0] kernel start and [L][2] kernel end in cycles, [L][4]
+ * input quantised, top-k (with this CTA's unit loads issued inside it when its expert
+ * is pinned), cache, warp 0's pinned-slot lookup, SwiGLU, down part landed, down adds
+ * issued, fence); [L][0] kernel start and [L][2] kernel end in cycles, [L][4]
  * and [L][5] the same two instants on the global timer (ns), which converts cycles to
  * ns; [L][1] prologue done (cycles).  Then [L][n_sm][4] global-timer marks (ns) of every
  * CTA: [0] routing decided, [1] units done, [2] arrival posted, [3] own logits
- * published.  NULL stops
- * it (n_words ignored). */
+ * published.  While a buffer is set, steps run the kernel instance that carries these
+ * marks (a few percent slower than the default one).  NULL stops it (n_words ignored). */
 MOE_API int moe_set_phase_trace(moe_ctx *ctx, uint64_t *stamps_dev, size_t n_words);
 
 /* Miss path (how a cold expert crosses PCIe; theneuralfeed.com, key components item 2): with
