@@ -684,7 +684,7 @@ def run_ours(args):
     if args.prefetch_sweep:
         sweep = []
         m.set_residency(1.0)
-        for pre, l2 in ((0, 0), (4, 0), (6, 0), (8, 0), (8, 4), (8, 8), (0, 8)):
+        for pre, l2 in ((0, 0), (0, 2), (0, 4), (0, 8), (0, 12), (4, 0), (8, 0), (0, 0)):
             m.set_prefetch(pre, l2)
             for i in range(args.warmup):
                 m.decode(xs[i], y)
